@@ -1,0 +1,402 @@
+"""Benchmark of the S4 DPLR forward hot path on B200: kernel generation
+(s4_kernel_dplr: Cauchy/Woodbury spectrum + inverse real FFT) followed by the
+zero-padded causal FFT convolution (s4_fft_conv: kernel spectrum + fused
+convolution), on the H=256, N=64, L=4096, batch-16 workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--config 2]
+
+Prints one JSON line. The metric is (batch * H * L) output elements per second
+of the whole forward; the line also carries the roofline of the dominant
+kernel (the convolution, bound by HBM), the Cauchy stage's fraction of the
+FP32 peak, the end-to-end number through the public API with host buffers,
+clocks sampled during the timed region, and the fp64 CPU oracle timed on a
+bounded sample (the reference arm).
+
+Multi-GPU (torchrun, one process per GPU): weak scaling, each rank owns its
+own H-slice of channels (a different seed per rank); the channels are
+independent SSMs, so there is no data-path collective. The timed region is
+bracketed by barriers and the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import s4inputs  # noqa: E402
+
+METRIC = "S4 fwd (batch·H·L) elems/s; Cauchy FP32 % peak; FFT-conv HBM GB/s % peak"
+UNIT = "elem/s"
+FALLBACK_HBM_GBS = 6650.0
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+NOMINAL_SM_MHZ = 1965.0
+# algorithmic FP32 work of the Cauchy stage per (frequency, mode pair): the
+# scaled denominator (2 mul, 1 add/fma, 2 fma for |q|^2 -> 8 flop incl. the
+# two products by 1/|q|^2) and four complex Cauchy sums as 16 FMAs (32 flop)
+CAUCHY_FLOP_PER_TERM = 40
+KERNEL_SOURCES = ["common.cuh", "fft.cuh", "spectral.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fftconv_h256_l4096_b16_traffic.txt")
+
+
+# ----------------------------------------------------------------- helpers --
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), float(d.get("sm_max_mhz", NOMINAL_SM_MHZ)), "measured"
+    return FALLBACK_HBM_GBS, NOMINAL_SM_MHZ, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "structured_state_space_dplr_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """dram bytes per launch of the convolution kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    vals = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1])); smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def physical_gpu(local_rank):
+    """nvidia-smi id of this process's device (CUDA_VISIBLE_DEVICES aware)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in vis.split(",") if v.strip()]
+    if local_rank < len(ids):
+        return ids[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------- workload -----
+def workload(cfg, seed):
+    c = s4inputs.CONFIGS[cfg]
+    return s4inputs.make_inputs(cfg, seed=seed), c
+
+
+def algorithmic(c):
+    H, L, Bt, Nh = c["H"], c["L"], c["Bt"], c["N"] // 2
+    return {
+        "elements": Bt * H * L,
+        # fused convolution: read u, write y, read the kernel spectrum (H x 2L complex)
+        "conv_bytes": 8 * Bt * H * L + 16 * H * L + 4 * H,
+        "cauchy_flop": CAUCHY_FLOP_PER_TERM * H * (L // 2) * Nh,
+    }
+
+
+# --------------------------------------------------------------- GPU arm ----
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import structured_state_space_dplr_b200 as s4
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    cfg = args.config
+    inp, c = workload(cfg, seed=rank)
+    H, L, Bt = c["H"], c["L"], c["Bt"]
+    alg = algorithmic(c)
+    names = ["Lambda", "P", "Q", "B", "C", "log_dt", "D", "u"]
+    base = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(dev) for k in names}
+    ws_bytes = s4.fft_conv_workspace_size(H, L)
+    # rotating input sets: consecutive steps touch different memory, together
+    # well above the 126 MB L2, so every step reads its inputs from HBM
+    set_bytes = (2 * Bt * H * L + H * L) * 4 + ws_bytes
+    nsets = max(2, math.ceil(3 * 126e6 / set_bytes) + 1)
+    sets = []
+    for i in range(nsets):
+        s = {k: v.clone() for k, v in base.items()}
+        s["K"] = torch.empty(H, L, device=dev)
+        s["y"] = torch.empty(Bt, H, L, device=dev)
+        s["ws"] = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        sets.append(s)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(s, ev=None):
+        if ev is not None:
+            ev[0].record()
+        s4.dplr_spectrum(s["Lambda"], s["P"], s["Q"], s["B"], s["C"], s["log_dt"], L, out=s["K"], flags=flags)
+        if ev is not None:
+            ev[1].record()
+        s4.irfft_packed(s["K"])
+        if ev is not None:
+            ev[2].record()
+        s4.fft_conv_prepare(s["K"], workspace=s["ws"])
+        if ev is not None:
+            ev[3].record()
+        s4.fft_conv_apply(s["u"], s["ws"], s["D"], out=s["y"])
+        if ev is not None:
+            ev[4].record()
+
+    launches_per_step = 4 + (1 if L == 65536 else 0)
+    for i in range(args.warmup):
+        step(sets[i % nsets])
+    torch.cuda.synchronize()
+    if int(flags.item()) != 0:
+        raise RuntimeError(f"kernel flags set: {int(flags.item())}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(physical_gpu(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for i in range(args.steps):
+        step(sets[i % nsets], evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    stage = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(4)]
+
+    # end to end through the public API with host buffers (pinned), copies inside
+    host = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory() for k in names}
+    y_host = torch.empty(Bt, H, L, dtype=torch.float32).pin_memory()
+    dsets = sets[0]
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y_host.numel() * 4
+
+    def e2e_step():
+        for k in names:
+            dsets[k].copy_(host[k], non_blocking=True)
+        K = s4.kernel_dplr(dsets["Lambda"], dsets["P"], dsets["Q"], dsets["B"], dsets["C"], dsets["log_dt"], L,
+                           out=dsets["K"])
+        s4.fft_conv(dsets["u"], K, dsets["D"], out=dsets["y"], workspace=dsets["ws"])
+        y_host.copy_(dsets["y"], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    times = torch.tensor([ms, e2e_ms] + stage, device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        dist.destroy_process_group()
+    ms, e2e_ms = float(times[0]), float(times[1])
+    stage = [float(x) for x in times[2:]]
+    if rank != 0:
+        return None
+
+    hbm, sm_max_mhz, peak_src = peaks()
+    total_elems = alg["elements"] * world * args.steps
+    conv_s = stage[3] * 1e-3
+    conv_gbs = alg["conv_bytes"] / conv_s / 1e9
+    cauchy_tflops = alg["cauchy_flop"] / (stage[0] * 1e-3) / 1e12
+    fp32_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+    traffic = recorded_traffic() if cfg == 2 else None
+    line = {
+        "metric": METRIC,
+        "value": total_elems / (ms * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded HiPPO-LegS DPLR parameters, N(0,1) inputs)",
+        "config": {"workload": c["name"], "H": H, "N": c["N"], "L": L, "batch": Bt,
+                   "global_batch": Bt * world, "dt_range": [c["dt_min"], c["dt_max"]],
+                   "parallelism": f"channel shard x{world}, no collective",
+                   "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
+        "stages_ms": {"cauchy_spectrum": stage[0], "irfft": stage[1], "kernel_spectrum": stage[2],
+                      "fft_conv": stage[3]},
+        "roofline": {"kernel": "k_fftconv", "bound": "hbm", "achieved": conv_gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": conv_gbs / hbm, "traffic": traffic,
+                     "peak_source": peak_src, "algorithmic_bytes": alg["conv_bytes"]},
+        "cauchy": {"kernel": "k_cauchy", "bound": "alu", "achieved": cauchy_tflops, "peak": fp32_peak,
+                   "unit": "TFLOP/s", "frac": cauchy_tflops / fp32_peak,
+                   "peak_derivation": f"{SM_COUNT} SM x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max_mhz:.0f} MHz",
+                   "algorithmic_flop": alg["cauchy_flop"]},
+        "e2e": {"value": total_elems / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_budget)
+    return line
+
+
+# ------------------------------------------------------- oracle (CPU) arm ---
+def oracle_sample(inp, channels):
+    """fp64 oracle forward for all rows of the given channels; returns elements."""
+    from oracle import workloads
+    K = workloads.dplr_kernel(inp, channels=channels)
+    rows = [(b, h) for h in channels for b in range(inp["Bt"])]
+    Krows = [K[list(channels).index(h)] for _, h in rows]
+    workloads.conv_rows_at(inp, Krows, rows, np.arange(inp["L"]))
+    return len(rows) * inp["L"]
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, budget_s=10.0, channels_per_chunk=8):
+    os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
+    inp, c = workload(cfg, seed=0)
+    done, elems, t_used = 0, 0, 0.0
+    while done < c["H"] and t_used < budget_s:
+        ch = list(range(done, min(done + channels_per_chunk, c["H"])))
+        t = time.perf_counter()
+        elems += oracle_sample(inp, ch)
+        t_used += time.perf_counter() - t
+        done += len(ch)
+    return {"value": elems / t_used, "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]),
+            "kind": "oracle",
+            "sample": f"channels 0..{done - 1} of {c['H']} (all {c['Bt']} rows each): fp64 dense-power "
+                      f"aliased kernel + direct O(L^2) convolution, {t_used:.1f} s"}
+
+
+def run_reference(args):
+    os.environ.setdefault("OMP_NUM_THREADS", str(cpu_cores()))
+    inp, c = workload(args.config, seed=0)
+    chunk = 4
+    for i in range(args.warmup):
+        oracle_sample(inp, list(range(chunk)))
+    t = time.perf_counter()
+    elems = 0
+    for i in range(args.steps):
+        h0 = (i * chunk) % c["H"]
+        elems += oracle_sample(inp, list(range(h0, min(h0 + chunk, c["H"]))))
+    dt = time.perf_counter() - t
+    v = elems / dt
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded HiPPO-LegS DPLR parameters, N(0,1) inputs)",
+        "config": {"workload": c["name"], "H": c["H"], "N": c["N"], "L": c["L"], "batch": c["Bt"]},
+        "cpu_baseline": {"value": v, "unit": UNIT, "kind": "oracle", "cores": int(os.environ["OMP_NUM_THREADS"]),
+                         "sample": f"each step: {chunk} channels x {c['Bt']} rows of the workload, fp64 "
+                                   "dense-power aliased kernel + direct O(L^2) convolution"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4])
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    line = run_gpu(args, rank, world, local_rank)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

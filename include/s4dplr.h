@@ -1,0 +1,224 @@
+/*
+ * s4dplr.h -- C ABI of libs4dplr.so: the S4 DPLR convolution kernel, the
+ * zero-padded causal FFT convolution, the S4D Vandermonde kernel and the
+ * recurrent (decode) step, on one NVIDIA B200 (sm_100a).
+ *
+ * Sources of the definitions (page title, section):
+ *   [S4K] "The S4 kernel, from scratch": §1 The continuous state-space model,
+ *         §3 Discretization, §4 The convolutional kernel via the generating
+ *         function (and its "Aliasing" paragraph), §5 Two views, kept in sync,
+ *         §6 Trainable layer.
+ *   [S4W] "S4" (wiki page), section "S4D".
+ *
+ * Conventions shared by every entry point
+ *   - All array pointers are DEVICE pointers unless stated otherwise. The
+ *     caller allocates and owns every buffer; the library allocates no device
+ *     memory and keeps no state between calls except per-device kernel
+ *     attributes set once.
+ *   - Arrays are row-major, last index contiguous. Complex numbers are pairs
+ *     of float32 (re, im) -- the real (..., 2) storage of [S4K] §6.
+ *   - Per-channel parameters of the H independent SSMs ([S4K] §1) are [H, Nh]:
+ *     Nh stored modes. The system is conjugate-closed: each stored mode n has
+ *     an implicit partner conj(mode n) (Lambda, P, Q, B and C all
+ *     conjugated), so the full state size is N = 2 Nh and every kernel is real.
+ *   - The step size enters as log_dt[h] (dt = exp(log_dt), [S4K] §6).
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *     Argument checks run on the host BEFORE anything is launched; on any
+ *     error nothing is launched and the status says why. A failing CUDA launch
+ *     returns S4_ERR_CUDA (see s4_last_cuda_error()).
+ *   - Data-dependent conditions never trap: kernels OR bits into *d_flags
+ *     (a device word; may be NULL), which the caller reads after a sync.
+ *   - Calls on different streams may run concurrently as long as their
+ *     output buffers (and workspaces) do not overlap.
+ */
+#ifndef S4DPLR_H
+#define S4DPLR_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct { float re, im; } s4_c32; /* 8 bytes, 8-byte aligned */
+
+typedef enum {
+    S4_OK = 0,
+    S4_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, overlap */
+    S4_ERR_UNSUPPORTED = 2,  /* L not a power of two in [16, 65536], Nh > 256, ... */
+    S4_ERR_WORKSPACE = 3,    /* workspace missing or smaller than the query says */
+    S4_ERR_CUDA = 4          /* a CUDA runtime call or launch failed */
+} s4_status;
+
+/* Bits OR-ed into *d_flags by the kernels. */
+#define S4_FLAG_UNSTABLE  1u  /* some Re(Lambda) >= 0 (or Re(a) >= 0 for S4D)   */
+#define S4_FLAG_NONFINITE 2u  /* a non-finite value was produced                 */
+
+#define S4_MIN_L 16
+#define S4_MAX_L 65536
+#define S4_MAX_NH 256       /* stored modes per channel                          */
+#define S4_MAX_H 65535      /* channels per call (kernel and decode entry points) */
+#define S4_MAX_DENSE_N 128  /* full state size of the dense decode step           */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *s4_status_string(s4_status s);
+
+/* CUDA error code (cudaError_t as int) of the last S4_ERR_CUDA returned on
+ * the calling host thread, 0 if none. */
+int s4_last_cuda_error(void);
+
+/* ABI version, currently 1. */
+int s4_version(void);
+
+/* ------------------------------------------------------------------------
+ * s4_kernel_dplr -- the S4 convolution kernel K[H, L] of a bilinear-
+ * discretised DPLR SSM ([S4K] §3 and §4).
+ *
+ * For each channel h, with dt = exp(log_dt[h]), A = Lambda - P Q^* and the
+ * bilinear rule Abar = (I - dt/2 A)^-1 (I + dt/2 A), Bbar = (I - dt/2 A)^-1
+ * dt B, Cbar = C, K is the ALIASED kernel ([S4K] §4 "Aliasing"):
+ *     K[h, k] = sum_{p >= 0} Cbar Abar^(k + pL) Bbar,   k = 0 .. L-1,
+ * computed as in [S4K] §4: the generating function is evaluated at the L-th
+ * roots of unity z_j = exp(-2 pi i j / L) by four Cauchy sums over the modes
+ * (k00, k01, k10, k11), the rank-1 Woodbury correction and the factor
+ * 2/(1+z); a length-L inverse FFT then gives K. Only j = 0 .. L/2 are
+ * evaluated (conjugate symmetry); j = L/2 (z = -1) uses the limit
+ * dt * Re sum_n C_n B_n.
+ *
+ *   Lambda, P, Q, B, C : [H, Nh] complex, device, 8-byte aligned. Q enters as
+ *                        conj(Q) in k10 and k11 (A = Lambda - P Q^*).
+ *   log_dt             : [H] float, device.
+ *   1 <= H <= 65535, 1 <= Nh <= 256, L a power of two in [16, 65536].
+ *   K                  : [H, L] float out, device, 16-byte aligned. It is also
+ *                        used as scratch (the half spectrum is staged in it).
+ *   d_flags            : device unsigned or NULL; S4_FLAG_UNSTABLE if some
+ *                        Re(Lambda) >= 0 (K is still computed),
+ *                        S4_FLAG_NONFINITE if a spectrum value is not finite.
+ * Errors: S4_ERR_INVALID_ARG (null, H < 1, Nh < 1, misaligned),
+ *         S4_ERR_UNSUPPORTED (L or Nh out of range), S4_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+s4_status s4_kernel_dplr(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                         const s4_c32 *B, const s4_c32 *C, const float *log_dt,
+                         int H, int Nh, int L, float *K, unsigned *d_flags,
+                         cudaStream_t stream);
+
+/* s4_kernel_dplr in two halves (the kernels it runs, in order):
+ * s4_dplr_spectrum writes the generating function at j = 0 .. L/2, times
+ * 1/L, packed into K[h, :] as K[h,0] = K_hat_0 (real), K[h,1] = K_hat_{L/2}
+ * (real), K[h,2j], K[h,2j+1] = Re, Im K_hat_j for 0 < j < L/2 ([S4K] §4,
+ * the four Cauchy sums, Woodbury and 2/(1+z)); s4_irfft_packed turns such a
+ * packed half spectrum into the real kernel, in place ([S4K] §4, "an inverse
+ * FFT returns the time-domain kernel"). Same argument rules as s4_kernel_dplr. */
+s4_status s4_dplr_spectrum(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                           const s4_c32 *B, const s4_c32 *C, const float *log_dt,
+                           int H, int Nh, int L, float *K, unsigned *d_flags,
+                           cudaStream_t stream);
+s4_status s4_irfft_packed(float *K, int H, int L, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * s4_fft_conv -- y = K * u + D u along the last axis, causal, for every row
+ * (b, h) ([S4K] §1 for y = Cx + Du, §5 "fft_conv", zero-padded so the
+ * circular FFT product has no wrap-around):
+ *     y[b, h, t] = sum_{s=0}^{t} K[h, s] u[b, h, t - s] + D[h] u[b, h, t].
+ * Computed with length-2L transforms (input zero-padded to 2L, output
+ * cropped to [0, L)). Two rows of the same channel are transformed together
+ * as one complex signal.
+ *
+ *   u : [Bt, H, L] float, device, 16-byte aligned.   K : [H, L] float, device,
+ *   16-byte aligned.   D : [H] float, device.   y : [Bt, H, L] float out,
+ *   device, 16-byte aligned, must not overlap u, K, D or the workspace.
+ *   Bt, H >= 1; L a power of two in [16, 65536]; Bt*H*L < 2^40.
+ *   workspace : device, 256-byte aligned, at least
+ *               s4_fft_conv_workspace_size(H, L) bytes; holds the spectrum
+ *               of the zero-padded K after the call.
+ * Errors: S4_ERR_INVALID_ARG, S4_ERR_UNSUPPORTED, S4_ERR_WORKSPACE, S4_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+s4_status s4_fft_conv_workspace_size(int H, int L, size_t *bytes);
+
+s4_status s4_fft_conv(const float *u, const float *K, const float *D,
+                      int Bt, int H, int L, float *y,
+                      void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* s4_fft_conv in two halves, for callers that apply one kernel to many
+ * batches: _prepare writes the spectrum of the zero-padded K into the
+ * workspace; _apply runs the convolution of u with that spectrum.
+ * s4_fft_conv(...) == _prepare(...) then _apply(...). Same arguments and
+ * rules as s4_fft_conv; the workspace must come from a _prepare with the same
+ * H and L and must not be written in between. */
+s4_status s4_fft_conv_prepare(const float *K, int H, int L,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream);
+s4_status s4_fft_conv_apply(const float *u, const void *workspace, const float *D,
+                            int Bt, int H, int L, float *y,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * s4d_kernel_vandermonde -- kernel of the diagonal S4D SSM with zero-order
+ * hold ([S4W] "S4D"; ZOH rule of [S4K] §3):
+ *     Abar_n = exp(dt a_n),  Bbar_n = (exp(dt a_n) - 1)/a_n * B_n,
+ *     K[h, k] = 2 Re sum_{n < Nh} C_n Bbar_n Abar_n^k,   k = 0 .. L-1
+ * (the TRUNCATED kernel: no aliasing). Powers are formed from fp64 phase
+ * reductions, so long kernels keep their phase accuracy.
+ *
+ *   A, B, C : [H, Nh] complex, device (A holds the continuous-time a_n).
+ *   log_dt  : [H] float.  K : [H, L] float out, 16-byte aligned.
+ *   1 <= H <= 65535, 1 <= Nh <= 256, L a power of two in [16, 65536].
+ *   d_flags : as above (S4_FLAG_UNSTABLE if some Re(a_n) >= 0).
+ * ------------------------------------------------------------------------ */
+s4_status s4d_kernel_vandermonde(const s4_c32 *A, const s4_c32 *B, const s4_c32 *C,
+                                 const float *log_dt, int H, int Nh, int L, float *K,
+                                 unsigned *d_flags, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Decode set-up ([S4K] §3 and §5, recurrent view).
+ *
+ * s4_dplr_discretize: dense bilinear discretisation of the full
+ * conjugate-closed DPLR system (N = 2 Nh modes, stored modes first, then
+ * their conjugates): A = diag(Lambda_f) - P_f Q_f^*,
+ *     Abar = (I - dt/2 A)^-1 (I + dt/2 A),   Bbar = (I - dt/2 A)^-1 dt B_f,
+ *     Cfull = C_f.
+ * The inverse uses the Sherman-Morrison form of the diagonal-plus-rank-1
+ * matrix I - dt/2 A.
+ *   Abar : [H, N, N] complex out; Bbar, Cfull : [H, N] complex out.
+ *
+ * s4d_discretize_zoh: S4D diagonal ZOH, Abar[h, n] = exp(dt a_n),
+ * Bbar[h, n] = (exp(dt a_n) - 1)/a_n B_n ([S4K] §3 ZOH; cancellation-free
+ * expm1). Abar, Bbar : [H, Nh] complex out.
+ * ------------------------------------------------------------------------ */
+s4_status s4_dplr_discretize(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                             const s4_c32 *B, const s4_c32 *C, const float *log_dt,
+                             int H, int Nh, s4_c32 *Abar, s4_c32 *Bbar, s4_c32 *Cfull,
+                             cudaStream_t stream);
+
+s4_status s4d_discretize_zoh(const s4_c32 *A, const s4_c32 *B, const float *log_dt,
+                             int H, int Nh, s4_c32 *Abar, s4_c32 *Bbar,
+                             cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * s4_recurrent_step -- one token of the recurrence ([S4K] §5):
+ *     x <- Abar x + Bbar u_t,   y_t = Re(C . x) + D u_t        (dense)
+ *     x <- Abar * x + Bbar u_t, y_t = 2 Re(sum_n C_n x_n) + D u_t  (diagonal)
+ * The state x is owned by the caller (a nonzero initial state is allowed).
+ *   mode S4_STEP_DENSE: Abar [H, Ns, Ns], Bbar, C [H, Ns] with Ns = N = 2 Nh
+ *                       (from s4_dplr_discretize), Ns <= 128 (Abar of a
+ *                       channel is staged in shared memory).
+ *   mode S4_STEP_DIAG : Abar, Bbar, C [H, Ns] with Ns = Nh (S4D), Ns <= 256.
+ *   x   : [Bt, H, Ns] complex in/out.   u_t, y_t : [Bt, H] float.  D : [H].
+ *   1 <= H <= 65535; Bt >= 1.
+ * s4_recurrent_scan runs T consecutive steps in one launch:
+ *   u, y : [Bt, H, T] float (token axis last), x in/out as above.
+ * ------------------------------------------------------------------------ */
+typedef enum { S4_STEP_DENSE = 0, S4_STEP_DIAG = 1 } s4_step_mode;
+
+s4_status s4_recurrent_step(s4_step_mode mode, const s4_c32 *Abar, const s4_c32 *Bbar,
+                            const s4_c32 *C, const float *D, int Bt, int H, int Ns,
+                            s4_c32 *x, const float *u_t, float *y_t, cudaStream_t stream);
+
+s4_status s4_recurrent_scan(s4_step_mode mode, const s4_c32 *Abar, const s4_c32 *Bbar,
+                            const s4_c32 *C, const float *D, int Bt, int H, int Ns, int T,
+                            s4_c32 *x, const float *u, float *y, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* S4DPLR_H */

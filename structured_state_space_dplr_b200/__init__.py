@@ -1,0 +1,228 @@
+"""B200 (sm_100a) S4 DPLR kernel generation and FFT convolution.
+
+Thin Python binding over libs4dplr.so (C ABI in include/s4dplr.h). Each
+function only marshals torch CUDA tensors into device pointers and the
+current CUDA stream; all arithmetic runs in the library's CUDA kernels.
+PyTorch provides device memory and streams.
+
+Complex parameters are [H, Nh] complex64 tensors (or [H, Nh, 2] float32, the
+real (..., 2) storage) holding the Nh stored modes of a conjugate-closed
+system (N = 2 Nh).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (S4_FLAG_NONFINITE, S4_FLAG_UNSTABLE, S4_STEP_DENSE, S4_STEP_DIAG,  # noqa: F401
+                   S4Error)
+
+__all__ = [
+    "kernel_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
+    "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
+    "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
+    "S4_STEP_DIAG", "load",
+]
+
+
+def load():
+    """Load libs4dplr.so now (raises if it is missing)."""
+    return _lib.lib()
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _cuda(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _cplx(t, name):
+    """[H, Nh] complex64, or [H, Nh, 2] float32 viewed as complex."""
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float32 and t.dim() >= 1 and t.shape[-1] == 2:
+        t = torch.view_as_complex(t)
+    return _cuda(t, name, torch.complex64)
+
+
+def _flags_ptr(flags):
+    if flags is None:
+        return ctypes.c_void_p(0)
+    _cuda(flags, "flags", torch.int32)
+    return _ptr(flags)
+
+
+def kernel_dplr(Lambda, P, Q, B, C, log_dt, L, *, out=None, flags=None):
+    """Aliased bilinear DPLR kernel K [H, L] (s4_kernel_dplr)."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    for x in (P, Q, B, C):
+        if tuple(x.shape) != (H, Nh):
+            raise ValueError("parameter shapes differ")
+    if out is None:
+        out = torch.empty(H, L, device=Lambda.device, dtype=torch.float32)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_kernel_dplr", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              H, Nh, int(L), _ptr(out), _flags_ptr(flags), _stream())
+    return out
+
+
+def dplr_spectrum(Lambda, P, Q, B, C, log_dt, L, *, out=None, flags=None):
+    """Packed half spectrum of the DPLR kernel, times 1/L (s4_dplr_spectrum)."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    if out is None:
+        out = torch.empty(H, L, device=Lambda.device, dtype=torch.float32)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_dplr_spectrum", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              H, Nh, int(L), _ptr(out), _flags_ptr(flags), _stream())
+    return out
+
+
+def irfft_packed(K):
+    """In place: packed half spectrum [H, L] -> real kernel (s4_irfft_packed)."""
+    K = _cuda(K, "K", torch.float32)
+    H, L = K.shape
+    _lib.call("s4_irfft_packed", _ptr(K), H, L, _stream())
+    return K
+
+
+def fft_conv_workspace_size(H, L) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.call("s4_fft_conv_workspace_size", int(H), int(L), ctypes.byref(n))
+    return n.value
+
+
+def _workspace(H, L, device, workspace):
+    need = fft_conv_workspace_size(H, L)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    _cuda(workspace, "workspace", torch.uint8)
+    return workspace
+
+
+def fft_conv(u, K, D, *, out=None, workspace=None):
+    """y = K * u + D u (causal, zero-padded FFT convolution; s4_fft_conv).
+
+    u: [Bt, H, L] float32; K: [H, L] float32; D: [H] float32."""
+    u = _cuda(u, "u", torch.float32)
+    K = _cuda(K, "K", torch.float32)
+    D = _cuda(D, "D", torch.float32)
+    Bt, H, L = u.shape
+    if tuple(K.shape) != (H, L) or tuple(D.shape) != (H,):
+        raise ValueError("shape mismatch between u, K and D")
+    workspace = _workspace(H, L, u.device, workspace)
+    if out is None:
+        out = torch.empty_like(u)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_fft_conv", _ptr(u), _ptr(K), _ptr(D), Bt, H, L, _ptr(out), _ptr(workspace),
+              workspace.numel(), _stream())
+    return out
+
+
+def fft_conv_prepare(K, workspace=None):
+    """Spectrum of the zero-padded K into a workspace (s4_fft_conv_prepare)."""
+    K = _cuda(K, "K", torch.float32)
+    H, L = K.shape
+    workspace = _workspace(H, L, K.device, workspace)
+    _lib.call("s4_fft_conv_prepare", _ptr(K), H, L, _ptr(workspace), workspace.numel(), _stream())
+    return workspace
+
+
+def fft_conv_apply(u, workspace, D, *, out=None):
+    """Convolution with a prepared spectrum (s4_fft_conv_apply)."""
+    u = _cuda(u, "u", torch.float32)
+    D = _cuda(D, "D", torch.float32)
+    _cuda(workspace, "workspace", torch.uint8)
+    Bt, H, L = u.shape
+    if out is None:
+        out = torch.empty_like(u)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_fft_conv_apply", _ptr(u), _ptr(workspace), _ptr(D), Bt, H, L, _ptr(out),
+              workspace.numel(), _stream())
+    return out
+
+
+def s4d_kernel_vandermonde(A, B, C, log_dt, L, *, out=None, flags=None):
+    """S4D ZOH truncated kernel K [H, L] (s4d_kernel_vandermonde)."""
+    A, B, C = (_cplx(x, n) for x, n in zip((A, B, C), "A B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = A.shape
+    if out is None:
+        out = torch.empty(H, L, device=A.device, dtype=torch.float32)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4d_kernel_vandermonde", _ptr(A), _ptr(B), _ptr(C), _ptr(log_dt), H, Nh, int(L),
+              _ptr(out), _flags_ptr(flags), _stream())
+    return out
+
+
+def dplr_discretize(Lambda, P, Q, B, C, log_dt):
+    """Dense bilinear (Abar [H,N,N], Bbar [H,N], Cfull [H,N]) complex64, N = 2 Nh."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    N = 2 * Nh
+    dev = Lambda.device
+    Ab = torch.empty(H, N, N, dtype=torch.complex64, device=dev)
+    Bb = torch.empty(H, N, dtype=torch.complex64, device=dev)
+    Cf = torch.empty(H, N, dtype=torch.complex64, device=dev)
+    _lib.call("s4_dplr_discretize", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              H, Nh, _ptr(Ab), _ptr(Bb), _ptr(Cf), _stream())
+    return Ab, Bb, Cf
+
+
+def s4d_discretize_zoh(A, B, log_dt):
+    """Diagonal ZOH (Abar, Bbar) [H, Nh] complex64."""
+    A, B = _cplx(A, "A"), _cplx(B, "B")
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = A.shape
+    Ab = torch.empty_like(A)
+    Bb = torch.empty_like(A)
+    _lib.call("s4d_discretize_zoh", _ptr(A), _ptr(B), _ptr(log_dt), H, Nh, _ptr(Ab), _ptr(Bb), _stream())
+    return Ab, Bb
+
+
+def _step_args(Abar, Bbar, C, D, x):
+    Abar, Bbar, C, x = (_cplx(t, n) for t, n in zip((Abar, Bbar, C, x), "Abar Bbar C x".split()))
+    D = _cuda(D, "D", torch.float32)
+    mode = S4_STEP_DENSE if Abar.dim() == 3 else S4_STEP_DIAG
+    Bt, H, Ns = x.shape
+    return mode, Abar, Bbar, C, D, x, Bt, H, Ns
+
+
+def recurrent_step(Abar, Bbar, C, D, x, u_t, *, out=None):
+    """One token: x <- Abar x + Bbar u_t (in place), returns y_t [Bt, H].
+    Dense if Abar is [H, N, N], diagonal (S4D) if Abar is [H, Nh]."""
+    mode, Abar, Bbar, C, D, x, Bt, H, Ns = _step_args(Abar, Bbar, C, D, x)
+    u_t = _cuda(u_t, "u_t", torch.float32)
+    if out is None:
+        out = torch.empty_like(u_t)
+    _lib.call("s4_recurrent_step", mode, _ptr(Abar), _ptr(Bbar), _ptr(C), _ptr(D), Bt, H, Ns,
+              _ptr(x), _ptr(u_t), _ptr(out), _stream())
+    return out
+
+
+def recurrent_scan(Abar, Bbar, C, D, x, u, *, out=None):
+    """T tokens in one launch: u [Bt, H, T] -> y [Bt, H, T]; x updated in place."""
+    mode, Abar, Bbar, C, D, x, Bt, H, Ns = _step_args(Abar, Bbar, C, D, x)
+    u = _cuda(u, "u", torch.float32)
+    T = u.shape[-1]
+    if out is None:
+        out = torch.empty_like(u)
+    _lib.call("s4_recurrent_scan", mode, _ptr(Abar), _ptr(Bbar), _ptr(C), _ptr(D), Bt, H, Ns, T,
+              _ptr(x), _ptr(u), _ptr(out), _stream())
+    return out

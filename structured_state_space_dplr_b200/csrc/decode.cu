@@ -1,0 +1,203 @@
+// decode.cu -- recurrent view ("The S4 kernel, from scratch", §5):
+//   x_t = Abar x_{t-1} + Bbar u_t,   y_t = Re(C x_t) + D u_t   (§1 output map)
+//
+// k_dplr_discretize: bilinear rule of §3 for the full conjugate-closed DPLR
+// system A = diag(Lambda_f) - P_f Q_f^*. With M = I - dt/2 A
+// = diag(d) + (dt/2) P_f Q_f^*, d_i = 1 - dt/2 Lambda_i, Sherman-Morrison gives
+//   M^-1 = diag(1/d) - (alpha beta^T) / s,   alpha_i = (dt/2) P_i / d_i,
+//   beta_j = conj(Q_j) / d_j,  s = 1 + sum_i conj(Q_i) alpha_i,
+// and then Abar = M^-1 (I + dt/2 A) = 2 M^-1 - I, Bbar = dt M^-1 B_f.
+//
+// Steps: dense (O(N^2) per token, N = 2 Nh) and diagonal (S4D, O(Nh)).
+// The scan variants run T tokens in one launch with the state on chip.
+#include "common.cuh"
+#include "launch.h"
+#include "s4dplr.h"
+
+namespace s4 {
+
+// one block per channel, N = 2 Nh threads (N <= 512)
+__global__ void k_dplr_discretize(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
+                                  const float2 *__restrict__ Q, const float2 *__restrict__ B,
+                                  const float2 *__restrict__ C, const float *__restrict__ log_dt, int Nh,
+                                  float2 *__restrict__ Abar, float2 *__restrict__ Bbar,
+                                  float2 *__restrict__ Cfull) {
+    extern __shared__ double2 sd[];          // alpha[N] | beta[N] | red[2 * 32]
+    const int N = 2 * Nh, h = blockIdx.x;
+    const bool live = (int)threadIdx.x < N;   // the block is padded to whole warps
+    const int i = live ? (int)threadIdx.x : 0;
+    double2 *alpha = sd, *beta = sd + N, *red = sd + 2 * N;
+    const double dt = exp((double)__ldg(log_dt + h));
+    const size_t o = (size_t)h * Nh + (i < Nh ? i : i - Nh);
+    const bool cj = i >= Nh;   // conjugate partner
+    auto ld = [&](const float2 *p) {
+        const float2 v = p[o];
+        return live ? make_double2(v.x, cj ? -(double)v.y : (double)v.y) : make_double2(0.0, 0.0);
+    };
+    const double2 lam = ld(Lambda), p = ld(P), q = ld(Q), b = ld(B), c = ld(C);
+    // 1/d with d = 1 - dt/2 lam
+    const double dr = 1.0 - 0.5 * dt * lam.x, di = -0.5 * dt * lam.y;
+    const double dd = dr * dr + di * di;
+    const double2 inv_d = make_double2(dr / dd, -di / dd);
+    const double2 al = make_double2(0.5 * dt * (p.x * inv_d.x - p.y * inv_d.y),
+                                    0.5 * dt * (p.x * inv_d.y + p.y * inv_d.x));
+    const double2 be = make_double2(q.x * inv_d.x + q.y * inv_d.y, q.x * inv_d.y - q.y * inv_d.x); // conj(q)/d
+    if (live) { alpha[i] = al; beta[i] = be; }
+    // sums: s1 = sum conj(q_i) alpha_i ; s2 = sum beta_i b_i
+    double2 s1 = make_double2(q.x * al.x + q.y * al.y, q.x * al.y - q.y * al.x);
+    double2 s2 = make_double2(be.x * b.x - be.y * b.y, be.x * b.y + be.y * b.x);
+    for (int off = 16; off > 0; off >>= 1) {
+        s1.x += __shfl_xor_sync(0xffffffffu, s1.x, off); s1.y += __shfl_xor_sync(0xffffffffu, s1.y, off);
+        s2.x += __shfl_xor_sync(0xffffffffu, s2.x, off); s2.y += __shfl_xor_sync(0xffffffffu, s2.y, off);
+    }
+    if ((threadIdx.x & 31) == 0) { red[2 * (threadIdx.x >> 5)] = s1; red[2 * (threadIdx.x >> 5) + 1] = s2; }
+    __syncthreads();
+    if (!live) return;
+    double2 S1 = make_double2(0, 0), S2 = make_double2(0, 0);
+    for (int w = 0; w < (N + 31) / 32; ++w) {
+        S1.x += red[2 * w].x; S1.y += red[2 * w].y;
+        S2.x += red[2 * w + 1].x; S2.y += red[2 * w + 1].y;
+    }
+    // 1/s, s = 1 + S1
+    const double sr = 1.0 + S1.x, si = S1.y, ss = sr * sr + si * si;
+    const double2 is = make_double2(sr / ss, -si / ss);
+    // Abar row i: 2 (inv_d_i delta_ij - alpha_i beta_j / s) - delta_ij
+    const double2 ai_s = make_double2(al.x * is.x - al.y * is.y, al.x * is.y + al.y * is.x);
+    float2 *Arow = Abar + ((size_t)h * N + i) * N;
+    for (int j = 0; j < N; ++j) {
+        const double2 bj = beta[j];
+        double re = -2.0 * (ai_s.x * bj.x - ai_s.y * bj.y);
+        double im = -2.0 * (ai_s.x * bj.y + ai_s.y * bj.x);
+        if (j == i) { re += 2.0 * inv_d.x - 1.0; im += 2.0 * inv_d.y; }
+        Arow[j] = make_float2((float)re, (float)im);
+    }
+    // Bbar_i = dt (inv_d_i b_i - alpha_i S2 / s)
+    const double2 t = make_double2(ai_s.x * S2.x - ai_s.y * S2.y, ai_s.x * S2.y + ai_s.y * S2.x);
+    Bbar[(size_t)h * N + i] = make_float2((float)(dt * (inv_d.x * b.x - inv_d.y * b.y - t.x)),
+                                          (float)(dt * (inv_d.x * b.y + inv_d.y * b.x - t.y)));
+    Cfull[(size_t)h * N + i] = make_float2((float)c.x, (float)c.y);
+}
+
+// Dense recurrence: block = (channel h, group of rows); Abar[h] staged in
+// shared memory; thread (row r, state i) owns x[r, i]. Each row gets
+// NP = N rounded up to whole warps of threads (lanes i >= N hold zero), so
+// every warp belongs to one row. T tokens per launch.
+__global__ void k_step_dense(const float2 *__restrict__ Abar, const float2 *__restrict__ Bbar,
+                             const float2 *__restrict__ C, const float *__restrict__ D, int Bt, int H,
+                             int N, int T, int rows_per_block, float2 *__restrict__ x,
+                             const float *__restrict__ u, float *__restrict__ y) {
+    extern __shared__ float2 sm[];   // A[N*N] | xs[2][rows*N] | part[rows * wpr]
+    const int NP = (N + 31) / 32 * 32, wpr = NP / 32;
+    const int h = blockIdx.y, i = threadIdx.x % NP, rl = threadIdx.x / NP;
+    const int r = blockIdx.x * rows_per_block + rl;
+    const bool live = r < Bt && i < N;
+    float2 *As = sm, *xs = sm + (size_t)N * N;
+    float *part = reinterpret_cast<float *>(xs + 2 * rows_per_block * N);
+    for (int k = threadIdx.x; k < N * N; k += blockDim.x) As[k] = Abar[(size_t)h * N * N + k];
+    const size_t row = (size_t)(r < Bt ? r : 0) * H + h;
+    const float2 bi = live ? Bbar[(size_t)h * N + i] : make_float2(0.f, 0.f);
+    const float2 ci = live ? C[(size_t)h * N + i] : make_float2(0.f, 0.f);
+    const float Dh = D[h];
+    float2 xi = live ? x[row * N + i] : make_float2(0.f, 0.f);
+    if (i < N) xs[rl * N + i] = xi;
+    __syncthreads();
+    int cur = 0;
+    for (int t = 0; t < T; ++t) {
+        const float ut = (r < Bt) ? u[row * T + t] : 0.f;
+        if (i < N) {
+            const float2 *xc = xs + cur * rows_per_block * N + rl * N;
+            const float2 *Ai = As + (size_t)i * N;
+            float2 acc = make_float2(bi.x * ut, bi.y * ut);
+            for (int j = 0; j < N; ++j) acc = cadd(acc, cmul(Ai[j], xc[j]));
+            xi = acc;
+            xs[(cur ^ 1) * rows_per_block * N + rl * N + i] = xi;
+        }
+        float v = live ? fmaf(ci.x, xi.x, -ci.y * xi.y) : 0.f;   // Re(C_i x_i)
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if ((threadIdx.x & 31) == 0) part[rl * wpr + (i >> 5)] = v;
+        __syncthreads();
+        if (r < Bt && i == 0) {
+            float sum = 0.f;
+            for (int w = 0; w < wpr; ++w) sum += part[rl * wpr + w];
+            y[row * T + t] = fmaf(Dh, ut, sum);
+        }
+        __syncthreads();
+        cur ^= 1;
+    }
+    if (live) x[row * N + i] = xi;
+}
+
+// Diagonal recurrence: one warp per row (b, h); lanes stride over the modes.
+__global__ void k_step_diag(const float2 *__restrict__ Abar, const float2 *__restrict__ Bbar,
+                            const float2 *__restrict__ C, const float *__restrict__ D, int Bt, int H,
+                            int Nh, int T, float2 *__restrict__ x, const float *__restrict__ u,
+                            float *__restrict__ y) {
+    constexpr int MAXM = 8;   // modes per lane (Nh <= 256)
+    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= (long long)Bt * H) return;
+    const int h = (int)(w % H);
+    const size_t po = (size_t)h * Nh;
+    float2 a[MAXM], b[MAXM], c[MAXM], s[MAXM];
+#pragma unroll
+    for (int k = 0; k < MAXM; ++k) {
+        const int n = lane + 32 * k;
+        const bool ok = n < Nh;
+        a[k] = ok ? Abar[po + n] : make_float2(0.f, 0.f);
+        b[k] = ok ? Bbar[po + n] : make_float2(0.f, 0.f);
+        c[k] = ok ? C[po + n] : make_float2(0.f, 0.f);
+        s[k] = ok ? x[(size_t)w * Nh + n] : make_float2(0.f, 0.f);
+    }
+    const float Dh = D[h];
+    for (int t = 0; t < T; ++t) {
+        const float ut = u[(size_t)w * T + t];
+        float v = 0.f;
+#pragma unroll
+        for (int k = 0; k < MAXM; ++k) {
+            if (lane + 32 * k < Nh) {
+                s[k] = cadd(cmul(a[k], s[k]), make_float2(b[k].x * ut, b[k].y * ut));
+                v = fmaf(c[k].x, s[k].x, fmaf(-c[k].y, s[k].y, v));
+            }
+        }
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) y[(size_t)w * T + t] = fmaf(2.f, v, Dh * ut);
+    }
+#pragma unroll
+    for (int k = 0; k < MAXM; ++k)
+        if (lane + 32 * k < Nh) x[(size_t)w * Nh + lane + 32 * k] = s[k];
+}
+
+cudaError_t launch_dplr_discretize(const float2 *Lambda, const float2 *P, const float2 *Q,
+                                   const float2 *B, const float2 *C, const float *log_dt, int H, int Nh,
+                                   float2 *Abar, float2 *Bbar, float2 *Cfull, cudaStream_t st) {
+    const int N = 2 * Nh;
+    const size_t smem = sizeof(double2) * (2 * (size_t)N + 64);
+    k_dplr_discretize<<<H, (N + 31) / 32 * 32, smem, st>>>(Lambda, P, Q, B, C, log_dt, Nh, Abar, Bbar, Cfull);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_step(int mode, const float2 *Abar, const float2 *Bbar, const float2 *C, const float *D,
+                        int Bt, int H, int Ns, int T, float2 *x, const float *u, float *y, cudaStream_t st) {
+    if (mode == S4_STEP_DIAG) {
+        const long long warps = (long long)Bt * H;
+        const int per_block = 8;
+        k_step_diag<<<(unsigned)((warps + per_block - 1) / per_block), 32 * per_block, 0, st>>>(
+            Abar, Bbar, C, D, Bt, H, Ns, T, x, u, y);
+        return cudaGetLastError();
+    }
+    const int NP = (Ns + 31) / 32 * 32;
+    int rows = 1024 / NP;
+    if (rows > Bt) rows = Bt;
+    if (rows < 1) rows = 1;
+    const int wpr = NP / 32;
+    const size_t smem = sizeof(float2) * ((size_t)Ns * Ns + 2 * (size_t)rows * Ns) + sizeof(float) * rows * wpr;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_step_dense, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid((Bt + rows - 1) / rows, H);
+    k_step_dense<<<grid, rows * NP, smem, st>>>(Abar, Bbar, C, D, Bt, H, Ns, T, rows, x, u, y);
+    return cudaGetLastError();
+}
+
+}  // namespace s4

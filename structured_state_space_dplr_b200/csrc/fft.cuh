@@ -1,0 +1,309 @@
+// fft.cuh -- shared-memory mixed-radix FFT building blocks for sm_100a.
+//
+// A CTA holds m = 2^LG complex points in shared memory and transforms them
+// in place with radix-16 passes (plus one radix-8/4 pass when LG is not a
+// multiple of 4), each thread keeping a whole radix group in registers:
+//
+//   forward  = decimation in frequency: natural input -> digit-reversed
+//              output (no reorder pass);
+//   inverse  = decimation in time: digit-reversed input -> natural output.
+//
+// So a convolution needs no permutation at all: transform, multiply by a
+// spectrum stored in the same digit-reversed order, transform back. The last
+// forward pass and the first inverse pass touch the same groups of R
+// consecutive points, so they are fused with the pointwise product and the
+// data stays in registers across them.
+//
+// A length-N transform is split over a cluster of C CTAs (N = C m): CTA c
+// owns the frequencies C f + c. Forward, each CTA forms its own input
+//     v_c[k] = W_N^{k c} sum_r x[k + r m] W_C^{r c}
+// straight from global memory and runs an m-point transform; inverse, each
+// CTA runs an m-point transform and the C partial results are combined over
+// distributed shared memory:
+//     x[k + r m] = sum_c W_C^{-c r} W_N^{-c k} Z_c[k].
+// The twist W_N^{k c} is folded into the first pass: a per-rank constant on
+// each input of a group plus a per-rank first-pass twiddle table.
+//
+// Shared memory is padded by one point every 16 (index i -> i + i/16), which
+// makes every pass conflict-free for 8-byte accesses.
+#pragma once
+#include "common.cuh"
+
+namespace s4 {
+
+// ------------------------------------------------------------------ plan --
+// log2 of the radix of pass s for a 2^lg-point transform.
+__host__ __device__ constexpr int plan_P(int lg) {
+    return lg == 4 ? 2 : (lg % 4 == 0 ? lg / 4 : lg / 4 + 1);
+}
+__host__ __device__ constexpr int plan_lr(int lg, int s) {
+    return lg == 4 ? 2
+         : (lg % 4 == 0) ? 4
+         : (lg % 4 == 1) ? (s < lg / 4 - 1 ? 4 : (s == lg / 4 - 1 ? 3 : 2))
+         : (s < lg / 4 ? 4 : lg % 4);
+}
+// block size of pass s (the sub-transform length it starts)
+__host__ __device__ constexpr int plan_B(int lg, int s) {
+    int b = lg;
+    for (int i = 0; i < s; ++i) b -= plan_lr(lg, i);
+    return 1 << b;
+}
+// twiddle entries of passes 1 .. s-1 (pass 0 has its own table)
+__host__ __device__ constexpr int plan_tw_off(int lg, int s) {
+    int o = 0;
+    for (int i = 1; i < s; ++i) o += plan_B(lg, i);
+    return o;
+}
+// all twiddle entries of passes 1 .. P-2 (the last pass has none)
+__host__ __device__ constexpr int plan_tw_size(int lg) { return plan_tw_off(lg, plan_P(lg) - 1); }
+
+__host__ __device__ constexpr int padded(int m) { return m + m / 16; }
+__device__ __forceinline__ int pidx(int i) { return i + (i >> 4); }
+
+// frequency index held at position p after the forward passes
+template <int LG>
+__device__ __forceinline__ int digrev(int p) {
+    int f = 0;
+    static_for<0, plan_P(LG)>([&](auto sc) {
+        constexpr int s = decltype(sc)::value;
+        constexpr int lr = plan_lr(LG, s);
+        constexpr int lS = ilog2(plan_B(LG, s)) - lr;            // log2 stride
+        constexpr int lw = LG - ilog2(plan_B(LG, s));            // log2(m / B)
+        f |= ((p >> lS) & ((1 << lr) - 1)) << lw;
+    });
+    return f;
+}
+
+// ------------------------------------------------------------ butterflies --
+__host__ __device__ constexpr float cos16(int e) {
+    switch (e & 15) {
+        case 0: return 1.0f;
+        case 1: case 15: return 0.92387953251128674f;
+        case 2: case 14: return 0.70710678118654752f;
+        case 3: case 13: return 0.38268343236508977f;
+        case 4: case 12: return 0.0f;
+        case 5: case 11: return -0.38268343236508977f;
+        case 6: case 10: return -0.70710678118654752f;
+        case 7: case 9: return -0.92387953251128674f;
+        default: return -1.0f;
+    }
+}
+__host__ __device__ constexpr float sin16(int e) { return cos16(e - 4); }
+
+// v * exp(DIR * 2 pi i E / N), N in {2, 4, 8, 16}
+template <int E, int N, int DIR>
+__device__ __forceinline__ float2 rot(float2 v) {
+    constexpr int e = ((E * (16 / N)) % 16 + 16) % 16;
+    if constexpr (e == 0) return v;
+    else if constexpr (e == 4) return mul_i<DIR>(v);
+    else if constexpr (e == 8) return make_float2(-v.x, -v.y);
+    else if constexpr (e == 12) return mul_i<-DIR>(v);
+    else {
+        constexpr float c = cos16(e);
+        constexpr float s = DIR > 0 ? sin16(e) : -sin16(e);
+        if constexpr (e % 2 == 0) {  // (+-1 +- i)/sqrt(2)
+            constexpr float h = 0.70710678118654752f;
+            constexpr float sc = c > 0 ? 1.0f : -1.0f, ss = s > 0 ? 1.0f : -1.0f;
+            float re = sc * v.x - ss * v.y, im = ss * v.x + sc * v.y;
+            return make_float2(h * re, h * im);
+        } else {
+            return make_float2(fmaf(v.x, c, -v.y * s), fmaf(v.x, s, v.y * c));
+        }
+    }
+}
+
+template <int DIR>
+__device__ __forceinline__ void dft4(float2 &x0, float2 &x1, float2 &x2, float2 &x3) {
+    float2 a0 = cadd(x0, x2), a1 = csub(x0, x2), a2 = cadd(x1, x3), a3 = mul_i<DIR>(csub(x1, x3));
+    x0 = cadd(a0, a2); x2 = csub(a0, a2); x1 = cadd(a1, a3); x3 = csub(a1, a3);
+}
+
+// in-register DFT of length R (natural order in and out), kernel exp(DIR 2 pi i n k / R)
+template <int R, int DIR>
+__device__ __forceinline__ void dft(float2 (&x)[R]) {
+    if constexpr (R == 2) {
+        float2 a = x[0]; x[0] = cadd(a, x[1]); x[1] = csub(a, x[1]);
+    } else if constexpr (R == 4) {
+        dft4<DIR>(x[0], x[1], x[2], x[3]);
+    } else {
+        constexpr int R2 = R / 4;   // n = R2 n1 + n2, k = k1 + 4 k2
+        float2 y[R];
+        static_for<0, R2>([&](auto n2c) {
+            constexpr int n2 = decltype(n2c)::value;
+            float2 a0 = x[n2], a1 = x[R2 + n2], a2 = x[2 * R2 + n2], a3 = x[3 * R2 + n2];
+            dft4<DIR>(a0, a1, a2, a3);
+            y[n2 * 4 + 0] = a0;
+            y[n2 * 4 + 1] = rot<n2 * 1, R, DIR>(a1);
+            y[n2 * 4 + 2] = rot<n2 * 2, R, DIR>(a2);
+            y[n2 * 4 + 3] = rot<n2 * 3, R, DIR>(a3);
+        });
+        static_for<0, 4>([&](auto k1c) {
+            constexpr int k1 = decltype(k1c)::value;
+            float2 b[R2];
+            static_for<0, R2>([&](auto n2c) { b[decltype(n2c)::value] = y[decltype(n2c)::value * 4 + k1]; });
+            dft<R2, DIR>(b);
+            static_for<0, R2>([&](auto k2c) { x[k1 + 4 * decltype(k2c)::value] = b[decltype(k2c)::value]; });
+        });
+    }
+}
+
+// ---------------------------------------------------------------- tables --
+// First-pass table of rank c of a C-way split of an N = C m transform:
+//   tw0[q S0 + j] = W_N^{j (C q + c)}     (S0 = m / R0)
+template <int LG>
+__device__ __forceinline__ float2 tw0_entry(int i, int C, int c) {
+    constexpr int m = 1 << LG;
+    constexpr int lS0 = LG - plan_lr(LG, 0);
+    int q = i >> lS0, j = i & ((1 << lS0) - 1);
+    int N = C * m;
+    return unit_root((j * (C * q + c)) & (N - 1), N);
+}
+
+// Fill (with nthreads threads, index tid) the per-CTA tables:
+//   tw0 (pass 0, rank c; skipped when null), tws (passes 1..P-2), pre[p] = W_{C R0}^{p c}.
+template <int LG>
+__device__ void build_tables(float2 *tw0, float2 *tws, float2 *pre, int C, int c, int tid, int nthreads) {
+    constexpr int m = 1 << LG;
+    constexpr int P = plan_P(LG);
+    constexpr int R0 = 1 << plan_lr(LG, 0);
+    if (tw0 != nullptr)
+        for (int i = tid; i < m; i += nthreads) tw0[i] = tw0_entry<LG>(i, C, c);
+    static_for<1, P - 1>([&](auto sc) {
+        constexpr int s = decltype(sc)::value;
+        constexpr int B = plan_B(LG, s);
+        constexpr int lS = ilog2(B) - plan_lr(LG, s);
+        float2 *t = tws + plan_tw_off(LG, s);
+        for (int i = tid; i < B; i += nthreads) {
+            int q = i >> lS, j = i & ((1 << lS) - 1);
+            t[i] = unit_root((j * q) & (B - 1), B);
+        }
+    });
+    for (int p = tid; p < R0; p += nthreads) pre[p] = unit_root((p * c) % (C * R0), C * R0);
+}
+
+// ---------------------------------------------------------------- passes --
+// Middle pass s (1 <= s <= P-1) in decimation-in-frequency form: DFT of each
+// group, then twiddles. DIR = -1 forward, +1 inverse (conjugate twiddles).
+template <int LG, int s, int DIR, int T>
+__device__ __forceinline__ void dif_pass(float2 *buf, const float2 *tws) {
+    constexpr int lr = plan_lr(LG, s), R = 1 << lr;
+    constexpr int B = plan_B(LG, s), S = B / R, G = (1 << LG) / R;
+    constexpr int lS = ilog2(S);
+    const float2 *tw = tws + plan_tw_off(LG, s);
+    for (int g = threadIdx.x; g < G; g += T) {
+        int base = ((g >> lS) << (lS + lr)) + (g & (S - 1));
+        int j = g & (S - 1);
+        float2 x[R];
+        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q * S)]; });
+        dft<R, DIR>(x);
+        if constexpr (S > 1) {
+            static_for<1, R>([&](auto q) { x[q] = ctw<DIR>(x[q], tw[q * S + j]); });
+        }
+        static_for<0, R>([&](auto q) { buf[pidx(base + q * S)] = x[q]; });
+    }
+}
+
+// Middle pass s in decimation-in-time form (the transpose): twiddles, then DFT.
+template <int LG, int s, int DIR, int T>
+__device__ __forceinline__ void dit_pass(float2 *buf, const float2 *tws) {
+    constexpr int lr = plan_lr(LG, s), R = 1 << lr;
+    constexpr int B = plan_B(LG, s), S = B / R, G = (1 << LG) / R;
+    constexpr int lS = ilog2(S);
+    const float2 *tw = tws + plan_tw_off(LG, s);
+    for (int g = threadIdx.x; g < G; g += T) {
+        int base = ((g >> lS) << (lS + lr)) + (g & (S - 1));
+        int j = g & (S - 1);
+        float2 x[R];
+        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q * S)]; });
+        if constexpr (S > 1) {
+            static_for<1, R>([&](auto q) { x[q] = ctw<DIR>(x[q], tw[q * S + j]); });
+        }
+        dft<R, DIR>(x);
+        static_for<0, R>([&](auto q) { buf[pidx(base + q * S)] = x[q]; });
+    }
+}
+
+// Forward passes 1 .. P-2 (pass 0 and the last pass are done by the caller).
+template <int LG, int T>
+__device__ __forceinline__ void forward_middle(float2 *buf, const float2 *tws) {
+    static_for<1, plan_P(LG) - 1>([&](auto sc) {
+        dif_pass<LG, decltype(sc)::value, -1, T>(buf, tws);
+        __syncthreads();
+    });
+}
+// Inverse passes P-2 .. 1.
+template <int LG, int T>
+__device__ __forceinline__ void inverse_middle(float2 *buf, const float2 *tws) {
+    constexpr int P = plan_P(LG);
+    static_for<1, P - 1>([&](auto sc) {
+        dit_pass<LG, P - 1 - decltype(sc)::value, +1, T>(buf, tws);
+        __syncthreads();
+    });
+}
+
+// First forward pass, reading its input through fetch(k) (k in [0, m)):
+// x_p = fetch(j + p S0) * pre[p], DFT, times tw0[q S0 + j], to shared memory.
+template <int LG, int T, class Fetch>
+__device__ __forceinline__ void forward_first(float2 *buf, const float2 *tw0, const float2 *pre, Fetch &&fetch) {
+    constexpr int lr = plan_lr(LG, 0), R = 1 << lr;
+    constexpr int S = (1 << LG) / R;
+    for (int j = threadIdx.x; j < S; j += T) {
+        float2 x[R];
+        static_for<0, R>([&](auto p) {
+            float2 v = fetch(j + p * S);
+            x[p] = (decltype(p)::value == 0) ? v : cmul(v, pre[p]);
+        });
+        dft<R, -1>(x);
+        static_for<0, R>([&](auto q) { buf[pidx(j + q * S)] = cmul(x[q], tw0[q * S + j]); });
+    }
+}
+
+// Last inverse pass: conjugate tw0, inverse DFT, conjugate pre; natural order
+// result W_N^{-c k} Z_c[k] stored at pidx(k).
+template <int LG, int T>
+__device__ __forceinline__ void inverse_last(float2 *buf, const float2 *tw0, const float2 *pre) {
+    constexpr int lr = plan_lr(LG, 0), R = 1 << lr;
+    constexpr int S = (1 << LG) / R;
+    for (int j = threadIdx.x; j < S; j += T) {
+        float2 x[R];
+        static_for<0, R>([&](auto q) { x[q] = cmulc(buf[pidx(j + q * S)], tw0[q * S + j]); });
+        dft<R, +1>(x);
+        static_for<0, R>([&](auto p) {
+            float2 v = (decltype(p)::value == 0) ? x[p] : cmulc(x[p], pre[p]);
+            buf[pidx(j + p * S)] = v;
+        });
+    }
+}
+
+// Fused last forward pass + pointwise product + first inverse pass. The group
+// of R consecutive positions [g R, g R + R) is multiplied by mul(pos0, x).
+template <int LG, int T, class Mul>
+__device__ __forceinline__ void fused_middle(float2 *buf, Mul &&mul) {
+    constexpr int lr = plan_lr(LG, plan_P(LG) - 1), R = 1 << lr;
+    constexpr int G = (1 << LG) / R;
+    for (int g = threadIdx.x; g < G; g += T) {
+        const int base = g * R;
+        float2 x[R];
+        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q)]; });
+        dft<R, -1>(x);
+        mul(base, x);
+        dft<R, +1>(x);
+        static_for<0, R>([&](auto q) { buf[pidx(base + q)] = x[q]; });
+    }
+}
+
+// Last forward pass only, handing each finished group to out(pos0, x).
+template <int LG, int T, class Out>
+__device__ __forceinline__ void forward_last(float2 *buf, Out &&out) {
+    constexpr int lr = plan_lr(LG, plan_P(LG) - 1), R = 1 << lr;
+    constexpr int G = (1 << LG) / R;
+    for (int g = threadIdx.x; g < G; g += T) {
+        const int base = g * R;
+        float2 x[R];
+        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q)]; });
+        dft<R, -1>(x);
+        out(base, x);
+    }
+}
+
+}  // namespace s4

@@ -1,0 +1,38 @@
+// launch.h -- internal host-side launchers (one per kernel family).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+
+namespace s4 {
+
+// ---- spectral.cu: FFT convolution and inverse real FFT ----
+// Cluster split used for the length-2L convolution transforms.
+struct ConvGeom { int C; int lg; bool tw0_global; };
+ConvGeom conv_geom(int L);
+size_t conv_workspace_bytes(int H, int L);
+
+cudaError_t launch_kspec(const float *K, int H, int L, void *ws, cudaStream_t st);
+cudaError_t launch_fftconv(const float *u, const void *ws, const float *D, int Bt, int H, int L,
+                           float *y, cudaStream_t st);
+// in place: K[H, L] holds the packed half spectrum on entry, the real kernel on exit
+cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st);
+
+// ---- cauchy.cu ----
+cudaError_t launch_cauchy(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
+                          const float2 *C, const float *log_dt, int H, int Nh, int L, float *K,
+                          unsigned *flags, cudaStream_t st);
+
+// ---- s4d.cu ----
+cudaError_t launch_vandermonde(const float2 *A, const float2 *B, const float2 *C, const float *log_dt,
+                               int H, int Nh, int L, float *K, unsigned *flags, cudaStream_t st);
+cudaError_t launch_s4d_zoh(const float2 *A, const float2 *B, const float *log_dt, int H, int Nh,
+                           float2 *Abar, float2 *Bbar, cudaStream_t st);
+
+// ---- decode.cu ----
+cudaError_t launch_dplr_discretize(const float2 *Lambda, const float2 *P, const float2 *Q,
+                                   const float2 *B, const float2 *C, const float *log_dt, int H, int Nh,
+                                   float2 *Abar, float2 *Bbar, float2 *Cfull, cudaStream_t st);
+cudaError_t launch_step(int mode, const float2 *Abar, const float2 *Bbar, const float2 *C, const float *D,
+                        int Bt, int H, int Ns, int T, float2 *x, const float *u, float *y, cudaStream_t st);
+
+}  // namespace s4

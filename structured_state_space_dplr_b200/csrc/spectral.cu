@@ -1,0 +1,465 @@
+// spectral.cu -- zero-padded causal FFT convolution and the inverse real FFT
+// that turns the DPLR spectrum into the kernel K.
+//
+// Convolution ("The S4 kernel, from scratch", §5 fft_conv; D u from §1):
+//   y[b,h,t] = sum_{s<=t} K[h,s] u[b,h,t-s] + D[h] u[b,h,t],
+// computed with length N = 2L transforms so the circular product has no
+// wrap-around. Two rows (b, b+1) of one channel are packed as u_b + i u_{b+1}
+// (K is real, so the product keeps the rows apart: real part -> row b,
+// imaginary part -> row b+1). Each length-N transform is split over a
+// cluster of C CTAs (see fft.cuh); because only the first L inputs are
+// nonzero, CTA c reads just C/2 chunks of the input, and because only the
+// first L outputs are kept, the cluster combine produces only C/2 of its
+// C output chunks.
+//
+// k_kspec      : spectrum of the zero-padded K, once per call, shared by all
+//                rows; stored per (h, rank) in the digit-reversed order the
+//                convolution produces, scaled by 1/N.
+// k_fftconv    : persistent clusters; each cluster loops over row pairs:
+//                forward transform, product, inverse transform, combine over
+//                distributed shared memory, + D u, store.
+// k_irfft      : K[h, 0..L) from the packed half spectrum (two channels per
+//                complex transform), in place.
+#include <atomic>
+#include <cooperative_groups.h>
+
+#include "fft.cuh"
+#include "launch.h"
+
+namespace cg = cooperative_groups;
+
+namespace s4 {
+
+template <int LG>
+__host__ __device__ constexpr int threads_for() {
+    return (1 << LG) / 16 < 32 ? 32 : ((1 << LG) / 16 > 512 ? 512 : (1 << LG) / 16);
+}
+
+// dynamic shared memory, in float2: buf | tw0 (unless in global) | tws | pre[16] | wcr[8]
+template <int LG>
+__host__ __device__ constexpr int smem_f2(bool tw0_global) {
+    return padded(1 << LG) + (tw0_global ? 0 : (1 << LG)) + plan_tw_size(LG) + 16 + 8;
+}
+
+struct Smem {
+    float2 *buf, *tw0, *tws, *pre, *wcr;
+};
+template <int LG, bool TW0G>
+__device__ __forceinline__ Smem carve(float2 *sm) {
+    Smem s;
+    s.buf = sm;
+    s.tw0 = TW0G ? nullptr : sm + padded(1 << LG);
+    s.tws = sm + padded(1 << LG) + (TW0G ? 0 : (1 << LG));
+    s.pre = s.tws + plan_tw_size(LG);
+    s.wcr = s.pre + 16;
+    return s;
+}
+
+// ------------------------------------------------------------ tables (global)
+// First-pass tables of all C ranks, for transforms too long to keep them in
+// shared memory next to the data: tw0g[c m + i] = tw0_entry(i, C, c).
+template <int LG>
+__global__ void k_tw0_init(float2 *__restrict__ tw0g, int C) {
+    constexpr int m = 1 << LG;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < C * m; i += gridDim.x * blockDim.x)
+        tw0g[i] = tw0_entry<LG>(i % m, C, i / m);
+}
+
+// ------------------------------------------------------------------ kspec --
+template <int LG, int C, bool TW0G>
+__global__ void __launch_bounds__(threads_for<LG>())
+k_kspec(const float *__restrict__ K, int H, int L, float2 *__restrict__ spec,
+        const float2 *__restrict__ tw0g) {
+    constexpr int m = 1 << LG, T = threads_for<LG>();
+    extern __shared__ float2 sm[];
+    const Smem s = carve<LG, TW0G>(sm);
+    const int c = blockIdx.x % C;
+    const int slot = blockIdx.x / C, nslots = gridDim.x / C;
+    build_tables<LG>(s.tw0, s.tws, s.pre, C, c, threadIdx.x, T);
+    if (threadIdx.x < C / 2) s.wcr[threadIdx.x] = unit_root((threadIdx.x * c) % C, C);
+    const float2 *t0 = TW0G ? tw0g + (size_t)c * m : s.tw0;
+    __syncthreads();
+    const float scale = 1.0f / (float)(C * m);
+    for (int h = slot; h < H; h += nslots) {
+        const float *Kh = K + (size_t)h * L;
+        forward_first<LG, T>(s.buf, t0, s.pre, [&](int k) {
+            float2 v = make_float2(__ldg(Kh + k), 0.0f);
+            static_for<1, C / 2>([&](auto r) {
+                const float kr = __ldg(Kh + k + r * m);
+                const float2 w = s.wcr[r];
+                v.x = fmaf(kr, w.x, v.x);
+                v.y = fmaf(kr, w.y, v.y);
+            });
+            return v;
+        });
+        __syncthreads();
+        forward_middle<LG, T>(s.buf, s.tws);
+        float4 *out = reinterpret_cast<float4 *>(spec + ((size_t)h * C + c) * m);
+        forward_last<LG, T>(s.buf, [&](int base, auto &x) {
+            constexpr int R = sizeof(x) / sizeof(float2);
+            static_for<0, R / 2>([&](auto i) {
+                out[base / 2 + i] = make_float4(x[2 * i].x * scale, x[2 * i].y * scale,
+                                                x[2 * i + 1].x * scale, x[2 * i + 1].y * scale);
+            });
+        });
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- fftconv --
+template <int LG, int C, bool TW0G>
+__global__ void __launch_bounds__(threads_for<LG>())
+k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, const float *__restrict__ D,
+          int Bt, int H, int L, float *__restrict__ y, const float2 *__restrict__ tw0g) {
+    constexpr int m = 1 << LG, T = threads_for<LG>();
+    constexpr int SL = m / C;                     // combine slice per rank
+    extern __shared__ float2 sm[];
+    const Smem s = carve<LG, TW0G>(sm);
+    cg::cluster_group cluster = cg::this_cluster();
+    const int c = (int)cluster.block_rank();
+    const int cl = blockIdx.x / C, ncl = gridDim.x / C;
+    build_tables<LG>(s.tw0, s.tws, s.pre, C, c, threadIdx.x, T);
+    if (threadIdx.x < C / 2) s.wcr[threadIdx.x] = unit_root((threadIdx.x * c) % C, C);
+    const float2 *t0 = TW0G ? tw0g + (size_t)c * m : s.tw0;
+    __syncthreads();
+
+    const int nbp = (Bt + 1) / 2;
+    const long long npairs = (long long)H * nbp;
+    for (long long pr = cl; pr < npairs; pr += ncl) {
+        const int h = (int)(pr / nbp), bp = (int)(pr % nbp);
+        const int b0 = 2 * bp;
+        const bool has1 = (b0 + 1) < Bt;
+        const float *u0 = u + ((size_t)b0 * H + h) * L;
+        const float *u1 = has1 ? u0 + (size_t)H * L : u0;   // not read when !has1
+        // forward: x = u0 + i u1 (zero-padded to 2L), rank c's share
+        forward_first<LG, T>(s.buf, t0, s.pre, [&](int k) {
+            float2 v = make_float2(__ldg(u0 + k), has1 ? __ldg(u1 + k) : 0.0f);
+            static_for<1, C / 2>([&](auto r) {
+                const float a = __ldg(u0 + k + r * m), b = has1 ? __ldg(u1 + k + r * m) : 0.0f;
+                v = cadd(v, cmul(make_float2(a, b), s.wcr[r]));
+            });
+            return v;
+        });
+        __syncthreads();
+        forward_middle<LG, T>(s.buf, s.tws);
+        const float4 *sp = reinterpret_cast<const float4 *>(spec + ((size_t)h * C + c) * m);
+        fused_middle<LG, T>(s.buf, [&](int base, auto &x) {
+            constexpr int R = sizeof(x) / sizeof(float2);
+            static_for<0, R / 2>([&](auto i) {
+                const float4 k2 = __ldg(sp + base / 2 + i);
+                x[2 * i] = cmul(x[2 * i], make_float2(k2.x, k2.y));
+                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k2.z, k2.w));
+            });
+        });
+        __syncthreads();
+        inverse_middle<LG, T>(s.buf, s.tws);
+        inverse_last<LG, T>(s.buf, t0, s.pre);
+        cluster.sync();
+        // combine the C partial transforms; rank c writes t' in [c SL, (c+1) SL)
+        const float Dh = __ldg(D + h);
+        float *y0 = y + ((size_t)b0 * H + h) * L;
+        float *y1 = y0 + (size_t)H * L;
+        for (int i = threadIdx.x; i < SL; i += T) {
+            const int tp = c * SL + i;
+            float2 w[C];
+            static_for<0, C>([&](auto cc) { w[cc] = cluster.map_shared_rank(s.buf, (int)cc)[pidx(tp)]; });
+            static_for<0, C / 2>([&](auto r) {
+                float2 o = w[0];
+                static_for<1, C>([&](auto cc) {
+                    o = cadd(o, rot<decltype(cc)::value * decltype(r)::value, C, +1>(w[cc]));
+                });
+                const int t = tp + r * m;
+                y0[t] = fmaf(Dh, __ldg(u0 + t), o.x);
+                if (has1) y1[t] = fmaf(Dh, __ldg(u1 + t), o.y);
+            });
+        }
+        cluster.sync();
+    }
+}
+
+// ------------------------------------------------------------------ irfft --
+__device__ __forceinline__ float2 half_spec(const float *Kh, int f, int L) {
+    if (f == 0) return make_float2(Kh[0], 0.0f);
+    if (f == L / 2) return make_float2(Kh[1], 0.0f);
+    if (f < L / 2) return make_float2(Kh[2 * f], Kh[2 * f + 1]);
+    const int g = L - f;
+    return make_float2(Kh[2 * g], -Kh[2 * g + 1]);
+}
+
+template <int LG, int C>
+__global__ void __launch_bounds__(threads_for<LG>())
+k_irfft(float *K, int H, int L) {
+    constexpr int m = 1 << LG, T = threads_for<LG>(), P = plan_P(LG);
+    constexpr int SL = m / C;
+    extern __shared__ float2 sm[];
+    const Smem s = carve<LG, false>(sm);
+    int c = 0, cl = blockIdx.x, ncl = gridDim.x;
+    if constexpr (C > 1) {
+        c = (int)cg::this_cluster().block_rank();
+        cl = blockIdx.x / C;
+        ncl = gridDim.x / C;
+    }
+    build_tables<LG>(s.tw0, s.tws, s.pre, C, c, threadIdx.x, T);
+    __syncthreads();
+    const int npairs = (H + 1) / 2;
+    for (int pr = cl; pr < npairs; pr += ncl) {
+        float *K1 = K + (size_t)(2 * pr) * L;
+        const bool has2 = 2 * pr + 1 < H;
+        float *K2 = has2 ? K1 + L : K1;
+        for (int p = threadIdx.x; p < m; p += T) {
+            const int f = C * digrev<LG>(p) + c;
+            const float2 a = half_spec(K1, f, L);
+            const float2 b = has2 ? half_spec(K2, f, L) : make_float2(0.0f, 0.0f);
+            s.buf[pidx(p)] = make_float2(a.x - b.y, a.y + b.x);
+        }
+        __syncthreads();
+        dit_pass<LG, P - 1, +1, T>(s.buf, s.tws);
+        __syncthreads();
+        inverse_middle<LG, T>(s.buf, s.tws);
+        inverse_last<LG, T>(s.buf, s.tw0, s.pre);
+        if constexpr (C > 1) cg::this_cluster().sync(); else __syncthreads();
+        for (int i = threadIdx.x; i < SL; i += T) {
+            const int tp = c * SL + i;
+            float2 w[C];
+            if constexpr (C > 1) {
+                static_for<0, C>([&](auto cc) { w[cc] = cg::this_cluster().map_shared_rank(s.buf, (int)cc)[pidx(tp)]; });
+            } else {
+                w[0] = s.buf[pidx(tp)];
+            }
+            static_for<0, C>([&](auto r) {
+                float2 o = w[0];
+                static_for<1, C>([&](auto cc) {
+                    o = cadd(o, rot<decltype(cc)::value * decltype(r)::value, C, +1>(w[cc]));
+                });
+                K1[tp + r * m] = o.x;
+                if (has2) K2[tp + r * m] = o.y;
+            });
+        }
+        if constexpr (C > 1) cg::this_cluster().sync(); else __syncthreads();
+    }
+}
+
+// =============================================================== host side ==
+namespace {
+
+int device_sms(int dev) {
+    static std::atomic<int> cache[64];
+    int v = cache[dev & 63].load(std::memory_order_relaxed);
+    if (v == 0) {
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev & 63].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+// Per-instantiation, per-device launch facts: smem opt-in done, how many
+// clusters (or CTAs) are co-resident.
+struct LaunchInfo {
+    std::atomic<int> resident[64];
+};
+
+template <class Kern>
+cudaError_t resident_units(Kern kern, LaunchInfo &info, int C, int T, size_t smem, int *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int v = info.resident[dev & 63].load(std::memory_order_relaxed);
+    if (v == 0) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (C > 1) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = C; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(C * 1024); cfg.blockDim = dim3(T); cfg.dynamicSmemBytes = smem;
+            cfg.attrs = at; cfg.numAttrs = 1;
+            e = cudaOccupancyMaxActiveClusters(&v, (void *)kern, &cfg);
+            if (e != cudaSuccess) return e;
+        } else {
+            int per_sm = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, smem);
+            if (e != cudaSuccess) return e;
+            v = per_sm * device_sms(dev);
+        }
+        if (v <= 0) return cudaErrorInvalidConfiguration;
+        info.resident[dev & 63].store(v, std::memory_order_relaxed);
+    }
+    *out = v;
+    return cudaSuccess;
+}
+
+template <class Kern, class... Args>
+cudaError_t launch_clustered(Kern kern, int C, int nclusters, int T, size_t smem, cudaStream_t st,
+                             Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    cfg.gridDim = dim3(C * nclusters);
+    cfg.blockDim = dim3(T);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    if (C > 1) {
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = C; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// ---- convolution / kspec instantiation for one L ----
+template <int LG, int C, bool TW0G>
+struct ConvKernels {
+    static constexpr int T = threads_for<LG>();
+    static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>(TW0G);
+    static LaunchInfo info_conv, info_kspec;
+
+    static cudaError_t kspec(const float *K, int H, int L, void *ws, cudaStream_t st) {
+        float2 *spec = (float2 *)ws;
+        float2 *tw0g = nullptr;
+        if (TW0G) {
+            tw0g = (float2 *)((char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)));
+            k_tw0_init<LG><<<(C * (1 << LG) + 255) / 256, 256, 0, st>>>(tw0g, C);
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        auto kern = k_kspec<LG, C, TW0G>;
+        int res = 0;
+        cudaError_t e = resident_units(kern, info_kspec, 1, T, smem, &res);
+        if (e != cudaSuccess) return e;
+        // whole rank groups: nslots CTAs per rank
+        int nslots = res / C;
+        if (nslots < 1) nslots = 1;
+        if (nslots > H) nslots = H;
+        kern<<<nslots * C, T, smem, st>>>(K, H, L, spec, (const float2 *)tw0g);
+        return cudaGetLastError();
+    }
+
+    static cudaError_t conv(const float *u, const void *ws, const float *D, int Bt, int H, int L,
+                            float *y, cudaStream_t st) {
+        const float2 *spec = (const float2 *)ws;
+        const float2 *tw0g = TW0G
+            ? (const float2 *)((const char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)))
+            : nullptr;
+        auto kern = k_fftconv<LG, C, TW0G>;
+        int res = 0;
+        cudaError_t e = resident_units(kern, info_conv, C, T, smem, &res);
+        if (e != cudaSuccess) return e;
+        const long long npairs = (long long)H * ((Bt + 1) / 2);
+        int ncl = res;
+        if ((long long)ncl > npairs) ncl = (int)npairs;
+        e = launch_clustered(kern, C, ncl, T, smem, st, u, spec, D, Bt, H, L, y, tw0g);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+};
+template <int LG, int C, bool TW0G> LaunchInfo ConvKernels<LG, C, TW0G>::info_conv;
+template <int LG, int C, bool TW0G> LaunchInfo ConvKernels<LG, C, TW0G>::info_kspec;
+
+// ---- irfft instantiation ----
+template <int LG, int C>
+struct IrfftKernels {
+    static constexpr int T = threads_for<LG>();
+    static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>(false);
+    static LaunchInfo info;
+    static cudaError_t run(float *K, int H, int L, cudaStream_t st) {
+        auto kern = k_irfft<LG, C>;
+        int res = 0;
+        cudaError_t e = resident_units(kern, info, C, T, smem, &res);
+        if (e != cudaSuccess) return e;
+        const int npairs = (H + 1) / 2;
+        int ncl = res < npairs ? res : npairs;
+        e = launch_clustered(kern, C, ncl, T, smem, st, K, H, L);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+};
+template <int LG, int C> LaunchInfo IrfftKernels<LG, C>::info;
+
+}  // namespace
+
+// Cluster split of the length-2L convolution transform: C CTAs of m = 2L/C
+// points, m <= 4096 up to L = 16384 (three CTAs fit one SM), longer
+// transforms use m = 8192 / 16384.
+ConvGeom conv_geom(int L) {
+    switch (L) {
+        case 16: return {2, 4, false};
+        case 32: return {2, 5, false};
+        case 64: return {2, 6, false};
+        case 128: return {2, 7, false};
+        case 256: return {2, 8, false};
+        case 512: return {2, 9, false};
+        case 1024: return {2, 10, false};
+        case 2048: return {2, 11, false};
+        case 4096: return {2, 12, false};
+        case 8192: return {4, 12, false};
+        case 16384: return {8, 12, false};
+        case 32768: return {8, 13, false};
+        case 65536: return {8, 14, true};
+        default: return {0, 0, false};
+    }
+}
+
+size_t conv_workspace_bytes(int H, int L) {
+    ConvGeom g = conv_geom(L);
+    size_t b = align256((size_t)H * 2 * L * sizeof(float2));
+    if (g.tw0_global) b += align256((size_t)2 * L * sizeof(float2));
+    return b;
+}
+
+#define S4_CONV_CASES(X)            \
+    X(16, 4, 2, false)              \
+    X(32, 5, 2, false)              \
+    X(64, 6, 2, false)              \
+    X(128, 7, 2, false)             \
+    X(256, 8, 2, false)             \
+    X(512, 9, 2, false)             \
+    X(1024, 10, 2, false)           \
+    X(2048, 11, 2, false)           \
+    X(4096, 12, 2, false)           \
+    X(8192, 12, 4, false)           \
+    X(16384, 12, 8, false)          \
+    X(32768, 13, 8, false)          \
+    X(65536, 14, 8, true)
+
+cudaError_t launch_kspec(const float *K, int H, int L, void *ws, cudaStream_t st) {
+    switch (L) {
+#define X(LL, LG, C, G) case LL: return ConvKernels<LG, C, G>::kspec(K, H, L, ws, st);
+        S4_CONV_CASES(X)
+#undef X
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_fftconv(const float *u, const void *ws, const float *D, int Bt, int H, int L,
+                           float *y, cudaStream_t st) {
+    switch (L) {
+#define X(LL, LG, C, G) case LL: return ConvKernels<LG, C, G>::conv(u, ws, D, Bt, H, L, y, st);
+        S4_CONV_CASES(X)
+#undef X
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st) {
+    switch (L) {
+        case 16: return IrfftKernels<4, 1>::run(K, H, L, st);
+        case 32: return IrfftKernels<5, 1>::run(K, H, L, st);
+        case 64: return IrfftKernels<6, 1>::run(K, H, L, st);
+        case 128: return IrfftKernels<7, 1>::run(K, H, L, st);
+        case 256: return IrfftKernels<8, 1>::run(K, H, L, st);
+        case 512: return IrfftKernels<9, 1>::run(K, H, L, st);
+        case 1024: return IrfftKernels<10, 1>::run(K, H, L, st);
+        case 2048: return IrfftKernels<11, 1>::run(K, H, L, st);
+        case 4096: return IrfftKernels<12, 1>::run(K, H, L, st);
+        case 8192: return IrfftKernels<13, 1>::run(K, H, L, st);
+        case 16384: return IrfftKernels<13, 2>::run(K, H, L, st);
+        case 32768: return IrfftKernels<13, 4>::run(K, H, L, st);
+        case 65536: return IrfftKernels<13, 8>::run(K, H, L, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace s4

@@ -1,0 +1,130 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+entry point include/s4dplr.h declares, and rejects bad arguments on the host
+before any CUDA call (no kernel is launched by these tests)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from structured_state_space_dplr_b200 import _lib
+from structured_state_space_dplr_b200 import build as s4build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "s4dplr.h")
+
+FAKE = 0x7f0000000000          # 256-byte aligned, never dereferenced
+FAKE2 = 0x7f1000000000
+
+
+@pytest.fixture(scope="module")
+def lib():
+    s4build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|s4_status|int)\s*\**\s*(s4\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_expected_calls():
+    names = declared_functions()
+    for must in ("s4_kernel_dplr", "s4_fft_conv", "s4d_kernel_vandermonde", "s4_recurrent_step"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings(lib):
+    assert _lib.status_string(0) == "S4_OK"
+    assert _lib.status_string(3) == "S4_ERR_WORKSPACE"
+    assert lib.s4_version() == 1
+
+
+def p(v):
+    return ctypes.c_void_p(v)
+
+
+def kdplr(lib, H=4, Nh=32, L=1024, ptrs=None, K=FAKE2):
+    ptrs = ptrs or [FAKE + 0x10000 * i for i in range(6)]
+    return lib.s4_kernel_dplr(*(p(x) for x in ptrs), H, Nh, L, p(K), p(0), p(0))
+
+
+def test_kernel_dplr_rejects_bad_arguments(lib):
+    assert kdplr(lib, ptrs=[0, FAKE, FAKE, FAKE, FAKE, FAKE]) == _lib.S4_ERR_INVALID_ARG
+    assert kdplr(lib, K=0) == _lib.S4_ERR_INVALID_ARG
+    assert kdplr(lib, H=0) == _lib.S4_ERR_INVALID_ARG
+    assert kdplr(lib, Nh=0) == _lib.S4_ERR_INVALID_ARG
+    assert kdplr(lib, Nh=257) == _lib.S4_ERR_UNSUPPORTED
+    assert kdplr(lib, H=65536) == _lib.S4_ERR_UNSUPPORTED
+    for L in (0, 8, 1000, 3 * 1024, 131072, -16):
+        assert kdplr(lib, L=L) == _lib.S4_ERR_UNSUPPORTED
+    assert kdplr(lib, K=FAKE2 + 4) == _lib.S4_ERR_INVALID_ARG          # K not 16-byte aligned
+    assert kdplr(lib, ptrs=[FAKE + 4] + [FAKE] * 5) == _lib.S4_ERR_INVALID_ARG   # complex not 8-aligned
+    assert kdplr(lib, K=FAKE) == _lib.S4_ERR_INVALID_ARG               # K overlaps Lambda
+
+
+def test_workspace_size(lib):
+    n = ctypes.c_size_t()
+    assert lib.s4_fft_conv_workspace_size(256, 4096, ctypes.byref(n)) == 0
+    assert n.value >= 256 * 2 * 4096 * 8 and n.value % 256 == 0
+    assert lib.s4_fft_conv_workspace_size(256, 1000, ctypes.byref(n)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_fft_conv_workspace_size(0, 1024, ctypes.byref(n)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_fft_conv_workspace_size(4, 1024, None) == _lib.S4_ERR_INVALID_ARG
+
+
+def conv(lib, u=FAKE, K=FAKE + 0x10000000, D=FAKE + 0x20000000, Bt=2, H=4, L=1024, y=FAKE2,
+         ws=FAKE + 0x30000000, wsb=None):
+    if wsb is None:
+        n = ctypes.c_size_t()
+        lib.s4_fft_conv_workspace_size(H, L, ctypes.byref(n))
+        wsb = n.value
+    return lib.s4_fft_conv(p(u), p(K), p(D), Bt, H, L, p(y), p(ws), wsb, p(0))
+
+
+def test_fft_conv_rejects_bad_arguments(lib):
+    assert conv(lib, u=0) == _lib.S4_ERR_INVALID_ARG
+    assert conv(lib, y=0) == _lib.S4_ERR_INVALID_ARG
+    assert conv(lib, ws=0) == _lib.S4_ERR_INVALID_ARG
+    assert conv(lib, Bt=0) == _lib.S4_ERR_INVALID_ARG
+    assert conv(lib, L=12) == _lib.S4_ERR_UNSUPPORTED
+    assert conv(lib, wsb=1024) == _lib.S4_ERR_WORKSPACE
+    assert conv(lib, ws=FAKE + 0x30000000 + 64) == _lib.S4_ERR_WORKSPACE   # not 256-aligned
+    assert conv(lib, u=FAKE + 8) == _lib.S4_ERR_INVALID_ARG                # u not 16-aligned
+    assert conv(lib, y=FAKE + 4096) == _lib.S4_ERR_INVALID_ARG             # y overlaps u
+    assert conv(lib, Bt=1 << 20, H=1 << 10, L=1 << 16) == _lib.S4_ERR_INVALID_ARG  # >= 2^40 elements
+
+
+def test_steps_reject_bad_arguments(lib):
+    args = [p(FAKE), p(FAKE + 0x1000000), p(FAKE + 0x2000000), p(FAKE + 0x3000000)]
+    x, u, y = p(FAKE + 0x4000000), p(FAKE + 0x5000000), p(FAKE + 0x6000000)
+    assert lib.s4_recurrent_step(7, *args, 2, 4, 64, x, u, y, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_recurrent_step(0, *args, 2, 4, 1024, x, u, y, p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_recurrent_step(0, *args, 2, 4, 256, x, u, y, p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_recurrent_step(1, *args, 2, 4, 300, x, u, y, p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_recurrent_step(1, *args, 0, 4, 32, x, u, y, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_recurrent_scan(1, *args, 2, 4, 32, 0, x, u, y, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_recurrent_step(1, *args, 2, 4, 32, x, u, u, p(0)) == _lib.S4_ERR_INVALID_ARG  # y aliases u
+
+
+def test_vandermonde_and_discretize_reject_bad_arguments(lib):
+    a = [p(FAKE + 0x100000 * i) for i in range(4)]
+    assert lib.s4d_kernel_vandermonde(*a, 4, 32, 1000, p(FAKE2), p(0), p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4d_kernel_vandermonde(p(0), *a[1:], 4, 32, 1024, p(FAKE2), p(0), p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4d_discretize_zoh(*a[:3], 4, 300, p(FAKE2), p(FAKE2 + 0x100000), p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_dplr_discretize(*(p(FAKE + 0x100000 * i) for i in range(6)), 0, 32,
+                                  p(FAKE2), p(FAKE2 + 0x100000), p(FAKE2 + 0x200000), p(0)) == _lib.S4_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    import structured_state_space_dplr_b200 as s4
+    u = torch.zeros(2, 2, 64)
+    with pytest.raises(TypeError):
+        s4.fft_conv(u, torch.zeros(2, 64), torch.zeros(2))
