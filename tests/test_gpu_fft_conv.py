@@ -118,7 +118,10 @@ def test_prepare_apply_matches_one_call():
     y3 = s4.fft_conv_apply(u[:3].contiguous(), ws, D)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
-    assert torch.equal(y1[:3], y3)
+    # rows 0 and 1 form the same packed pair in both calls; row 2 is paired
+    # with row 3 in one call and alone in the other, so it only rounds alike
+    assert torch.equal(y1[:2], y3[:2])
+    assert rel_l2(y3[2].cpu().numpy(), y1[2].cpu().numpy()) <= Y_TOL
 
 
 def test_workspace_too_small_is_rejected():
