@@ -153,6 +153,31 @@ s4_status s4_fft_conv_apply(const float *u, const void *workspace, const float *
                             size_t workspace_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * s4_fft_conv_static -- s4_fft_conv without a caller-provided workspace.
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory: a plugin inside a host application
+ * whose memory pool owns the GPU, or a real-time path where cudaMalloc's
+ * implicit device synchronisation is not allowed. It allocates nothing.
+ *
+ * The workspace is a library-owned device array of S4_STATIC_SCRATCH_BYTES
+ * (32 MiB); every GPU that loads the library keeps it until the process
+ * exits. The first call on a device looks up that array's device address
+ * (with that device current), so make the first call on each device before
+ * any stream capture. All calls share the one array: calls that overlap on
+ * the GPU (other streams, other host threads) race on it and must be
+ * serialised by the caller. Each call overwrites all the scratch it reads, so
+ * nothing in it has to start at zero.
+ *
+ * Arguments, layouts and errors are those of s4_fft_conv; in addition the
+ * call returns S4_ERR_UNSUPPORTED when s4_fft_conv_workspace_size(H, L)
+ * exceeds S4_STATIC_SCRATCH_BYTES (about H * L <= 2 M elements).
+ * ------------------------------------------------------------------------ */
+#define S4_STATIC_SCRATCH_BYTES (32u << 20)
+
+s4_status s4_fft_conv_static(const float *u, const float *K, const float *D,
+                             int Bt, int H, int L, float *y, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * s4d_kernel_vandermonde -- kernel of the diagonal S4D SSM with zero-order
  * hold ([S4W] "S4D"; ZOH rule of [S4K] §3):
  *     Abar_n = exp(dt a_n),  Bbar_n = (exp(dt a_n) - 1)/a_n * B_n,

@@ -21,6 +21,7 @@ from ._lib import (S4_FLAG_NONFINITE, S4_FLAG_UNSTABLE, S4_STEP_DENSE, S4_STEP_D
 
 __all__ = [
     "kernel_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
+    "fft_conv_static",
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
     "S4_STEP_DIAG", "load",
@@ -131,6 +132,23 @@ def fft_conv(u, K, D, *, out=None, workspace=None):
     _cuda(out, "out", torch.float32)
     _lib.call("s4_fft_conv", _ptr(u), _ptr(K), _ptr(D), Bt, H, L, _ptr(out), _ptr(workspace),
               workspace.numel(), _stream())
+    return out
+
+
+def fft_conv_static(u, K, D, *, out=None):
+    """s4_fft_conv with the library's own device scratch (s4_fft_conv_static),
+    for callers that cannot allocate device memory. Calls that overlap on the
+    GPU share that scratch and must be serialised by the caller."""
+    u = _cuda(u, "u", torch.float32)
+    K = _cuda(K, "K", torch.float32)
+    D = _cuda(D, "D", torch.float32)
+    Bt, H, L = u.shape
+    if tuple(K.shape) != (H, L) or tuple(D.shape) != (H,):
+        raise ValueError("shape mismatch between u, K and D")
+    if out is None:
+        out = torch.empty_like(u)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_fft_conv_static", _ptr(u), _ptr(K), _ptr(D), Bt, H, L, _ptr(out), _stream())
     return out
 
 

@@ -60,6 +60,8 @@ s4_status conv_checks(const float *u, const float *D, int Bt, int H, int L, cons
 
 }  // namespace
 
+void s4::record_cuda_error(cudaError_t e) { g_last_cuda_error = (int)e; }
+
 extern "C" {
 
 const char *s4_status_string(s4_status s) {

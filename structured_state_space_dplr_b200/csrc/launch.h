@@ -5,6 +5,9 @@
 
 namespace s4 {
 
+// remember a failing CUDA call for s4_last_cuda_error() (calling host thread)
+void record_cuda_error(cudaError_t e);
+
 // ---- spectral.cu: FFT convolution and inverse real FFT ----
 // Cluster split used for the length-2L convolution transforms.
 struct ConvGeom { int C; int lg; bool tw0_global; };
