@@ -200,10 +200,10 @@ def run_gpu(args, rank, world, local_rank):
         s4.irfft_packed(s["K"])
         if ev is not None:
             ev[2].record()
-        s4.fft_conv_prepare(s["K"], workspace=s["ws"])
+        s4.fft_conv_prepare(s["K"], s["D"], workspace=s["ws"])
         if ev is not None:
             ev[3].record()
-        s4.fft_conv_apply(s["u"], s["ws"], s["D"], out=s["y"])
+        s4.fft_conv_apply(s["u"], s["ws"], out=s["y"])
         if ev is not None:
             ev[4].record()
 

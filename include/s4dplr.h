@@ -131,7 +131,7 @@ s4_status s4_irfft_packed(float *K, int H, int L, cudaStream_t stream);
  *   Bt, H >= 1; L a power of two in [16, 65536]; Bt*H*L < 2^40.
  *   workspace : device, 256-byte aligned, at least
  *               s4_fft_conv_workspace_size(H, L) bytes; holds the spectrum
- *               of the zero-padded K after the call.
+ *               of the zero-padded K + D delta_0 after the call.
  * Errors: S4_ERR_INVALID_ARG, S4_ERR_UNSUPPORTED, S4_ERR_WORKSPACE, S4_ERR_CUDA.
  * ------------------------------------------------------------------------ */
 s4_status s4_fft_conv_workspace_size(int H, int L, size_t *bytes);
@@ -141,14 +141,15 @@ s4_status s4_fft_conv(const float *u, const float *K, const float *D,
                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* s4_fft_conv in two halves, for callers that apply one kernel to many
- * batches: _prepare writes the spectrum of the zero-padded K into the
- * workspace; _apply runs the convolution of u with that spectrum.
- * s4_fft_conv(...) == _prepare(...) then _apply(...). Same arguments and
- * rules as s4_fft_conv; the workspace must come from a _prepare with the same
- * H and L and must not be written in between. */
-s4_status s4_fft_conv_prepare(const float *K, int H, int L,
+ * batches: _prepare writes into the workspace the spectrum of the
+ * zero-padded K + D delta_0 (so the D u term comes out of the same product);
+ * _apply convolves u with that spectrum. s4_fft_conv(...) == _prepare(K, D)
+ * then _apply(u). In _prepare, D may be NULL (no feed-through term). The
+ * workspace must come from a _prepare with the same H and L and must not be
+ * written in between; other rules as for s4_fft_conv. */
+s4_status s4_fft_conv_prepare(const float *K, const float *D, int H, int L,
                               void *workspace, size_t workspace_bytes, cudaStream_t stream);
-s4_status s4_fft_conv_apply(const float *u, const void *workspace, const float *D,
+s4_status s4_fft_conv_apply(const float *u, const void *workspace,
                             int Bt, int H, int L, float *y,
                             size_t workspace_bytes, cudaStream_t stream);
 

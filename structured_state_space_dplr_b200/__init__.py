@@ -152,26 +152,30 @@ def fft_conv_static(u, K, D, *, out=None):
     return out
 
 
-def fft_conv_prepare(K, workspace=None):
-    """Spectrum of the zero-padded K into a workspace (s4_fft_conv_prepare)."""
+def fft_conv_prepare(K, D=None, workspace=None):
+    """Spectrum of the zero-padded K + D delta_0 into a workspace
+    (s4_fft_conv_prepare); D None means no feed-through term."""
     K = _cuda(K, "K", torch.float32)
     H, L = K.shape
+    if D is not None:
+        D = _cuda(D, "D", torch.float32)
+        if tuple(D.shape) != (H,):
+            raise ValueError("D must be [H]")
     workspace = _workspace(H, L, K.device, workspace)
-    _lib.call("s4_fft_conv_prepare", _ptr(K), H, L, _ptr(workspace), workspace.numel(), _stream())
+    _lib.call("s4_fft_conv_prepare", _ptr(K), _ptr(D), H, L, _ptr(workspace), workspace.numel(), _stream())
     return workspace
 
 
-def fft_conv_apply(u, workspace, D, *, out=None):
+def fft_conv_apply(u, workspace, *, out=None):
     """Convolution with a prepared spectrum (s4_fft_conv_apply)."""
     u = _cuda(u, "u", torch.float32)
-    D = _cuda(D, "D", torch.float32)
     _cuda(workspace, "workspace", torch.uint8)
     Bt, H, L = u.shape
     if out is None:
         out = torch.empty_like(u)
     _cuda(out, "out", torch.float32)
-    _lib.call("s4_fft_conv_apply", _ptr(u), _ptr(workspace), _ptr(D), Bt, H, L, _ptr(out),
-              workspace.numel(), _stream())
+    _lib.call("s4_fft_conv_apply", _ptr(u), _ptr(workspace), Bt, H, L, _ptr(out), workspace.numel(),
+              _stream())
     return out
 
 

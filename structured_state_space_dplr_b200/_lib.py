@@ -30,8 +30,8 @@ SIGNATURES = {
     "s4_irfft_packed": (_i, [_p, _i, _i, _p]),
     "s4_fft_conv_workspace_size": (_i, [_i, _i, ctypes.POINTER(_sz)]),
     "s4_fft_conv": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
-    "s4_fft_conv_prepare": (_i, [_p, _i, _i, _p, _sz, _p]),
-    "s4_fft_conv_apply": (_i, [_p, _p, _p, _i, _i, _i, _p, _sz, _p]),
+    "s4_fft_conv_prepare": (_i, [_p, _p, _i, _i, _p, _sz, _p]),
+    "s4_fft_conv_apply": (_i, [_p, _p, _i, _i, _i, _p, _sz, _p]),
     "s4_fft_conv_static": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
     "s4d_kernel_vandermonde": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p, _p]),
     "s4_dplr_discretize": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _p, _p, _p, _p]),

@@ -42,19 +42,26 @@ bool params_aligned(std::initializer_list<const void *> ps) {
     return true;
 }
 
-s4_status conv_checks(const float *u, const float *D, int Bt, int H, int L, const float *y,
-                      const void *ws, size_t ws_bytes) {
-    if (any_null(u, D, y) || ws == nullptr) return S4_ERR_INVALID_ARG;
+s4_status conv_checks(const float *u, int Bt, int H, int L, const float *y, const void *ws, size_t ws_bytes) {
+    if (any_null(u, y) || ws == nullptr) return S4_ERR_INVALID_ARG;
     if (Bt < 1 || H < 1) return S4_ERR_INVALID_ARG;
     if (!pow2_L(L)) return S4_ERR_UNSUPPORTED;
     if ((double)Bt * (double)H * (double)L >= 1099511627776.0) return S4_ERR_INVALID_ARG;   // 2^40
-    if (!aligned(u, 16) || !aligned(y, 16) || !aligned(D, 4)) return S4_ERR_INVALID_ARG;
+    if (!aligned(u, 16) || !aligned(y, 16)) return S4_ERR_INVALID_ARG;
     if (!aligned(ws, 256)) return S4_ERR_WORKSPACE;
     if (ws_bytes < s4::conv_workspace_bytes(H, L)) return S4_ERR_WORKSPACE;
     const size_t nb = (size_t)Bt * H * L * sizeof(float);
-    if (overlap(u, nb, y, nb) || overlap(y, nb, D, (size_t)H * sizeof(float)) ||
-        overlap(y, nb, ws, ws_bytes))
-        return S4_ERR_INVALID_ARG;
+    if (overlap(u, nb, y, nb) || overlap(y, nb, ws, ws_bytes)) return S4_ERR_INVALID_ARG;
+    return S4_OK;
+}
+
+s4_status prepare_checks(const float *K, const float *D, int H, int L, const void *ws, size_t ws_bytes) {
+    if (K == nullptr || ws == nullptr || H < 1) return S4_ERR_INVALID_ARG;
+    if (!pow2_L(L)) return S4_ERR_UNSUPPORTED;
+    if (!aligned(K, 16) || !aligned(D, 4)) return S4_ERR_INVALID_ARG;
+    if (!aligned(ws, 256) || ws_bytes < s4::conv_workspace_bytes(H, L)) return S4_ERR_WORKSPACE;
+    if (overlap(K, (size_t)H * L * sizeof(float), ws, ws_bytes)) return S4_ERR_INVALID_ARG;
+    if (D != nullptr && overlap(D, (size_t)H * sizeof(float), ws, ws_bytes)) return S4_ERR_INVALID_ARG;
     return S4_OK;
 }
 
@@ -130,35 +137,31 @@ s4_status s4_fft_conv_workspace_size(int H, int L, size_t *bytes) {
     return S4_OK;
 }
 
-s4_status s4_fft_conv_prepare(const float *K, int H, int L, void *workspace, size_t workspace_bytes,
-                              cudaStream_t stream) {
-    if (K == nullptr || workspace == nullptr || H < 1) return S4_ERR_INVALID_ARG;
-    if (!pow2_L(L)) return S4_ERR_UNSUPPORTED;
-    if (!aligned(K, 16)) return S4_ERR_INVALID_ARG;
-    if (!aligned(workspace, 256) || workspace_bytes < s4::conv_workspace_bytes(H, L)) return S4_ERR_WORKSPACE;
-    if (overlap(K, (size_t)H * L * sizeof(float), workspace, workspace_bytes)) return S4_ERR_INVALID_ARG;
-    return cuda_status(s4::launch_kspec(K, H, L, workspace, stream));
+s4_status s4_fft_conv_prepare(const float *K, const float *D, int H, int L, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+    s4_status s = prepare_checks(K, D, H, L, workspace, workspace_bytes);
+    if (s != S4_OK) return s;
+    return cuda_status(s4::launch_kspec(K, D, H, L, workspace, stream));
 }
 
-s4_status s4_fft_conv_apply(const float *u, const void *workspace, const float *D, int Bt, int H, int L,
-                            float *y, size_t workspace_bytes, cudaStream_t stream) {
-    s4_status s = conv_checks(u, D, Bt, H, L, y, workspace, workspace_bytes);
+s4_status s4_fft_conv_apply(const float *u, const void *workspace, int Bt, int H, int L, float *y,
+                            size_t workspace_bytes, cudaStream_t stream) {
+    s4_status s = conv_checks(u, Bt, H, L, y, workspace, workspace_bytes);
     if (s != S4_OK) return s;
-    return cuda_status(s4::launch_fftconv(u, workspace, D, Bt, H, L, y, stream));
+    return cuda_status(s4::launch_fftconv(u, workspace, Bt, H, L, y, stream));
 }
 
 s4_status s4_fft_conv(const float *u, const float *K, const float *D, int Bt, int H, int L, float *y,
                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    if (K == nullptr) return S4_ERR_INVALID_ARG;
-    s4_status s = conv_checks(u, D, Bt, H, L, y, workspace, workspace_bytes);
+    if (D == nullptr) return S4_ERR_INVALID_ARG;
+    s4_status s = conv_checks(u, Bt, H, L, y, workspace, workspace_bytes);
+    if (s == S4_OK) s = prepare_checks(K, D, H, L, workspace, workspace_bytes);
     if (s != S4_OK) return s;
-    if (!aligned(K, 16)) return S4_ERR_INVALID_ARG;
     const size_t nb = (size_t)Bt * H * L * sizeof(float);
-    if (overlap(y, nb, K, (size_t)H * L * sizeof(float)) ||
-        overlap(K, (size_t)H * L * sizeof(float), workspace, workspace_bytes))
+    if (overlap(y, nb, K, (size_t)H * L * sizeof(float)) || overlap(y, nb, D, (size_t)H * sizeof(float)))
         return S4_ERR_INVALID_ARG;
-    cudaError_t e = s4::launch_kspec(K, H, L, workspace, stream);
-    if (e == cudaSuccess) e = s4::launch_fftconv(u, workspace, D, Bt, H, L, y, stream);
+    cudaError_t e = s4::launch_kspec(K, D, H, L, workspace, stream);
+    if (e == cudaSuccess) e = s4::launch_fftconv(u, workspace, Bt, H, L, y, stream);
     return cuda_status(e);
 }
 

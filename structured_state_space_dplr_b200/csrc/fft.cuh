@@ -75,33 +75,28 @@ __device__ __forceinline__ int digrev(int p) {
 }
 
 // ------------------------------------------------------------ butterflies --
-__host__ __device__ constexpr float cos16(int e) {
-    switch (e & 15) {
-        case 0: return 1.0f;
-        case 1: case 15: return 0.92387953251128674f;
-        case 2: case 14: return 0.70710678118654752f;
-        case 3: case 13: return 0.38268343236508977f;
-        case 4: case 12: return 0.0f;
-        case 5: case 11: return -0.38268343236508977f;
-        case 6: case 10: return -0.70710678118654752f;
-        case 7: case 9: return -0.92387953251128674f;
-        default: return -1.0f;
-    }
+// cos(2 pi e / 32) for any integer e (values of cos(k pi / 16), k = 0..8)
+__host__ __device__ constexpr float cos32(int e) {
+    constexpr float c[9] = {1.0f, 0.98078528040323043f, 0.92387953251128674f, 0.83146961230254524f,
+                            0.70710678118654752f, 0.55557023301960218f, 0.38268343236508977f,
+                            0.19509032201612827f, 0.0f};
+    const int k = ((e % 32) + 32) % 32;          // angle k pi / 16 in [0, 2 pi)
+    return k <= 8 ? c[k] : (k <= 16 ? -c[16 - k] : (k <= 24 ? -c[k - 16] : c[32 - k]));
 }
-__host__ __device__ constexpr float sin16(int e) { return cos16(e - 4); }
+__host__ __device__ constexpr float sin32(int e) { return cos32(e - 8); }
 
-// v * exp(DIR * 2 pi i E / N), N in {2, 4, 8, 16}
+// v * exp(DIR * 2 pi i E / N), N in {2, 4, 8, 16, 32}
 template <int E, int N, int DIR>
 __device__ __forceinline__ float2 rot(float2 v) {
-    constexpr int e = ((E * (16 / N)) % 16 + 16) % 16;
+    constexpr int e = ((E * (32 / N)) % 32 + 32) % 32;
     if constexpr (e == 0) return v;
-    else if constexpr (e == 4) return mul_i<DIR>(v);
-    else if constexpr (e == 8) return make_float2(-v.x, -v.y);
-    else if constexpr (e == 12) return mul_i<-DIR>(v);
+    else if constexpr (e == 8) return mul_i<DIR>(v);
+    else if constexpr (e == 16) return make_float2(-v.x, -v.y);
+    else if constexpr (e == 24) return mul_i<-DIR>(v);
     else {
-        constexpr float c = cos16(e);
-        constexpr float s = DIR > 0 ? sin16(e) : -sin16(e);
-        if constexpr (e % 2 == 0) {  // (+-1 +- i)/sqrt(2)
+        constexpr float c = cos32(e);
+        constexpr float s = DIR > 0 ? sin32(e) : -sin32(e);
+        if constexpr (e % 4 == 0) {  // (+-1 +- i)/sqrt(2)
             constexpr float h = 0.70710678118654752f;
             constexpr float sc = c > 0 ? 1.0f : -1.0f, ss = s > 0 ? 1.0f : -1.0f;
             float re = sc * v.x - ss * v.y, im = ss * v.x + sc * v.y;
@@ -182,6 +177,12 @@ __device__ void build_tables(float2 *tw0, float2 *tws, float2 *pre, int C, int c
 }
 
 // ---------------------------------------------------------------- passes --
+// In every pass, group member q sits at padded index pidx(base) + off(q S):
+// (base mod 16) + (q S mod 16) < 16 holds for all plans, so the padding term
+// of base + q S splits into that of base plus (q S) / 16 -- a constant.
+template <int QS>
+__host__ __device__ constexpr int poff() { return QS + (QS >> 4); }
+
 // Middle pass s (1 <= s <= P-1) in decimation-in-frequency form: DFT of each
 // group, then twiddles. DIR = -1 forward, +1 inverse (conjugate twiddles).
 template <int LG, int s, int DIR, int T>
@@ -191,15 +192,15 @@ __device__ __forceinline__ void dif_pass(float2 *buf, const float2 *tws) {
     constexpr int lS = ilog2(S);
     const float2 *tw = tws + plan_tw_off(LG, s);
     for (int g = threadIdx.x; g < G; g += T) {
-        int base = ((g >> lS) << (lS + lr)) + (g & (S - 1));
-        int j = g & (S - 1);
+        const int j = g & (S - 1);
+        float2 *p = buf + pidx(((g >> lS) << (lS + lr)) + j);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q * S)]; });
+        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value * S>()]; });
         dft<R, DIR>(x);
         if constexpr (S > 1) {
             static_for<1, R>([&](auto q) { x[q] = ctw<DIR>(x[q], tw[q * S + j]); });
         }
-        static_for<0, R>([&](auto q) { buf[pidx(base + q * S)] = x[q]; });
+        static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
     }
 }
 
@@ -211,15 +212,15 @@ __device__ __forceinline__ void dit_pass(float2 *buf, const float2 *tws) {
     constexpr int lS = ilog2(S);
     const float2 *tw = tws + plan_tw_off(LG, s);
     for (int g = threadIdx.x; g < G; g += T) {
-        int base = ((g >> lS) << (lS + lr)) + (g & (S - 1));
-        int j = g & (S - 1);
+        const int j = g & (S - 1);
+        float2 *p = buf + pidx(((g >> lS) << (lS + lr)) + j);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q * S)]; });
+        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value * S>()]; });
         if constexpr (S > 1) {
             static_for<1, R>([&](auto q) { x[q] = ctw<DIR>(x[q], tw[q * S + j]); });
         }
         dft<R, DIR>(x);
-        static_for<0, R>([&](auto q) { buf[pidx(base + q * S)] = x[q]; });
+        static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
     }
 }
 
@@ -241,20 +242,36 @@ __device__ __forceinline__ void inverse_middle(float2 *buf, const float2 *tws) {
     });
 }
 
-// First forward pass, reading its input through fetch(k) (k in [0, m)):
-// x_p = fetch(j + p S0) * pre[p], DFT, times tw0[q S0 + j], to shared memory.
+// First forward pass of group j, in registers: x_p = fetch(j + p S0) * pre[p],
+// DFT, times tw0[q S0 + j].
+template <int LG, class Fetch>
+__device__ __forceinline__ void first_group(float2 (&x)[1 << plan_lr(LG, 0)], int j, const float2 *tw0,
+                                            const float2 *pre, Fetch &&fetch) {
+    constexpr int R = 1 << plan_lr(LG, 0);
+    constexpr int S = (1 << LG) / R;
+    static_for<0, R>([&](auto p) {
+        const float2 v = fetch(j + p * S);
+        if constexpr (decltype(p)::value == 0) x[p] = v; else x[p] = cmul(v, pre[p]);
+    });
+    dft<R, -1>(x);
+    static_for<0, R>([&](auto q) { x[q] = cmul(x[q], tw0[q * S + j]); });
+}
+template <int LG>
+__device__ __forceinline__ void store_first_group(float2 *buf, const float2 (&x)[1 << plan_lr(LG, 0)], int j) {
+    constexpr int R = 1 << plan_lr(LG, 0);
+    constexpr int S = (1 << LG) / R;
+    float2 *p = buf + pidx(j);
+    static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
+}
+
+// First forward pass over all groups (input through fetch(k), k in [0, m)).
 template <int LG, int T, class Fetch>
 __device__ __forceinline__ void forward_first(float2 *buf, const float2 *tw0, const float2 *pre, Fetch &&fetch) {
-    constexpr int lr = plan_lr(LG, 0), R = 1 << lr;
-    constexpr int S = (1 << LG) / R;
+    constexpr int S = (1 << LG) >> plan_lr(LG, 0);
     for (int j = threadIdx.x; j < S; j += T) {
-        float2 x[R];
-        static_for<0, R>([&](auto p) {
-            float2 v = fetch(j + p * S);
-            x[p] = (decltype(p)::value == 0) ? v : cmul(v, pre[p]);
-        });
-        dft<R, -1>(x);
-        static_for<0, R>([&](auto q) { buf[pidx(j + q * S)] = cmul(x[q], tw0[q * S + j]); });
+        float2 x[1 << plan_lr(LG, 0)];
+        first_group<LG>(x, j, tw0, pre, fetch);
+        store_first_group<LG>(buf, x, j);
     }
 }
 
@@ -265,30 +282,33 @@ __device__ __forceinline__ void inverse_last(float2 *buf, const float2 *tw0, con
     constexpr int lr = plan_lr(LG, 0), R = 1 << lr;
     constexpr int S = (1 << LG) / R;
     for (int j = threadIdx.x; j < S; j += T) {
+        float2 *p = buf + pidx(j);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = cmulc(buf[pidx(j + q * S)], tw0[q * S + j]); });
+        static_for<0, R>([&](auto q) { x[q] = cmulc(p[poff<decltype(q)::value * S>()], tw0[q * S + j]); });
         dft<R, +1>(x);
-        static_for<0, R>([&](auto p) {
-            float2 v = (decltype(p)::value == 0) ? x[p] : cmulc(x[p], pre[p]);
-            buf[pidx(j + p * S)] = v;
+        static_for<0, R>([&](auto q) {
+            if constexpr (decltype(q)::value == 0) p[0] = x[q];
+            else p[poff<decltype(q)::value * S>()] = cmulc(x[q], pre[q]);
         });
     }
 }
 
 // Fused last forward pass + pointwise product + first inverse pass. The group
-// of R consecutive positions [g R, g R + R) is multiplied by mul(pos0, x).
+// of R consecutive positions [g R, g R + R) is multiplied by mul(pos0, x);
+// pre(pos0) runs first (to start loads early).
 template <int LG, int T, class Mul>
 __device__ __forceinline__ void fused_middle(float2 *buf, Mul &&mul) {
     constexpr int lr = plan_lr(LG, plan_P(LG) - 1), R = 1 << lr;
     constexpr int G = (1 << LG) / R;
     for (int g = threadIdx.x; g < G; g += T) {
         const int base = g * R;
+        float2 *p = buf + pidx(base);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q)]; });
+        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value>()]; });
         dft<R, -1>(x);
         mul(base, x);
         dft<R, +1>(x);
-        static_for<0, R>([&](auto q) { buf[pidx(base + q)] = x[q]; });
+        static_for<0, R>([&](auto q) { p[poff<decltype(q)::value>()] = x[q]; });
     }
 }
 
@@ -299,10 +319,99 @@ __device__ __forceinline__ void forward_last(float2 *buf, Out &&out) {
     constexpr int G = (1 << LG) / R;
     for (int g = threadIdx.x; g < G; g += T) {
         const int base = g * R;
+        const float2 *p = buf + pidx(base);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = buf[pidx(base + q)]; });
+        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value>()]; });
         dft<R, -1>(x);
         out(base, x);
+    }
+}
+
+// Gather the input of an inverse transform into digit-reversed positions:
+// position p receives value(f) with f the frequency index held at p.
+template <int LG, int T, class Val>
+__device__ __forceinline__ void gather_digit_reversed(float2 *buf, Val &&value) {
+    for (int p = threadIdx.x; p < (1 << LG); p += T) buf[pidx(p)] = value(digrev<LG>(p));
+}
+
+// ------------------------------------------------- two transforms at once --
+// The same pass applied to the same group of two independent buffers by one
+// thread: twice the independent work per thread (the two halves of a
+// length-2m transform, see k_fftconv_pair).
+template <int LG, int s, int DIR, bool TW_FIRST, int T>
+__device__ __forceinline__ void pass_x2(float2 *b0, float2 *b1, const float2 *tws) {
+    constexpr int lr = plan_lr(LG, s), R = 1 << lr;
+    constexpr int B = plan_B(LG, s), S = B / R, G = (1 << LG) / R;
+    constexpr int lS = ilog2(S);
+    const float2 *tw = tws + plan_tw_off(LG, s);
+    for (int g = threadIdx.x; g < G; g += T) {
+        const int j = g & (S - 1);
+        const int o = pidx(((g >> lS) << (lS + lr)) + j);
+        float2 x[R], z[R];
+        static_for<0, R>([&](auto q) {
+            x[q] = b0[o + poff<decltype(q)::value * S>()];
+            z[q] = b1[o + poff<decltype(q)::value * S>()];
+        });
+        if constexpr (TW_FIRST && S > 1) {
+            static_for<1, R>([&](auto q) {
+                const float2 w = tw[q * S + j];
+                x[q] = ctw<DIR>(x[q], w);
+                z[q] = ctw<DIR>(z[q], w);
+            });
+        }
+        dft<R, DIR>(x);
+        dft<R, DIR>(z);
+        if constexpr (!TW_FIRST && S > 1) {
+            static_for<1, R>([&](auto q) {
+                const float2 w = tw[q * S + j];
+                x[q] = ctw<DIR>(x[q], w);
+                z[q] = ctw<DIR>(z[q], w);
+            });
+        }
+        static_for<0, R>([&](auto q) {
+            b0[o + poff<decltype(q)::value * S>()] = x[q];
+            b1[o + poff<decltype(q)::value * S>()] = z[q];
+        });
+    }
+}
+template <int LG, int T>
+__device__ __forceinline__ void forward_middle_x2(float2 *b0, float2 *b1, const float2 *tws) {
+    static_for<1, plan_P(LG) - 1>([&](auto sc) {
+        pass_x2<LG, decltype(sc)::value, -1, false, T>(b0, b1, tws);
+        __syncthreads();
+    });
+}
+template <int LG, int T>
+__device__ __forceinline__ void inverse_middle_x2(float2 *b0, float2 *b1, const float2 *tws) {
+    constexpr int P = plan_P(LG);
+    static_for<1, P - 1>([&](auto sc) {
+        pass_x2<LG, P - 1 - decltype(sc)::value, +1, true, T>(b0, b1, tws);
+        __syncthreads();
+    });
+}
+// last forward pass, product with the two spectra (mul(pos0, x, z)), first
+// inverse pass, for both buffers
+template <int LG, int T, class Mul>
+__device__ __forceinline__ void fused_middle_x2(float2 *b0, float2 *b1, Mul &&mul) {
+    constexpr int lr = plan_lr(LG, plan_P(LG) - 1), R = 1 << lr;
+    constexpr int G = (1 << LG) / R;
+    for (int g = threadIdx.x; g < G; g += T) {
+        const int base = g * R;
+        const int o = pidx(base);
+        float2 x[R], z[R];
+        static_for<0, R>([&](auto q) {
+            x[q] = b0[o + poff<decltype(q)::value>()];
+            z[q] = b1[o + poff<decltype(q)::value>()];
+        });
+        dft<R, -1>(x);
+        dft<R, -1>(z);
+        mul(base, x, z);
+        dft<R, +1>(x);
+        dft<R, +1>(z);
+        static_for<0, R>([&](auto q) {
+            b0[o + poff<decltype(q)::value>()] = x[q];
+            b1[o + poff<decltype(q)::value>()] = z[q];
+        });
     }
 }
 

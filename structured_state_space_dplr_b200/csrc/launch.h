@@ -14,9 +14,9 @@ struct ConvGeom { int C; int lg; bool tw0_global; };
 ConvGeom conv_geom(int L);
 size_t conv_workspace_bytes(int H, int L);
 
-cudaError_t launch_kspec(const float *K, int H, int L, void *ws, cudaStream_t st);
-cudaError_t launch_fftconv(const float *u, const void *ws, const float *D, int Bt, int H, int L,
-                           float *y, cudaStream_t st);
+// spectrum of K + D delta_0 (D may be null: no feed-through) into ws
+cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st);
+cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st);
 // in place: K[H, L] holds the packed half spectrum on entry, the real kernel on exit
 cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st);
 

@@ -63,8 +63,8 @@ extern "C" s4_status s4_fft_conv_static(const float *u, const float *K, const fl
     if (s4::conv_workspace_bytes(H, L) > (size_t)S4_STATIC_SCRATCH_BYTES) return S4_ERR_UNSUPPORTED;
     void *ws = nullptr;
     cudaError_t e = scratch_of_current_device(&ws);
-    if (e == cudaSuccess) e = s4::launch_kspec(K, H, L, ws, stream);
-    if (e == cudaSuccess) e = s4::launch_fftconv(u, ws, D, Bt, H, L, y, stream);
+    if (e == cudaSuccess) e = s4::launch_kspec(K, D, H, L, ws, stream);
+    if (e == cudaSuccess) e = s4::launch_fftconv(u, ws, Bt, H, L, y, stream);
     if (e != cudaSuccess) {
         s4::record_cuda_error(e);
         return S4_ERR_CUDA;

@@ -36,9 +36,10 @@ __host__ __device__ constexpr int threads_for() {
 }
 
 // dynamic shared memory, in float2: buf | tw0 (unless in global) | tws | pre[16] | wcr[8]
+// (| stage[2][L] floats for the staged convolution, 16-byte aligned)
 template <int LG>
 __host__ __device__ constexpr int smem_f2(bool tw0_global) {
-    return padded(1 << LG) + (tw0_global ? 0 : (1 << LG)) + plan_tw_size(LG) + 16 + 8;
+    return (padded(1 << LG) + (tw0_global ? 0 : (1 << LG)) + plan_tw_size(LG) + 16 + 8 + 1) / 2 * 2;
 }
 
 struct Smem {
@@ -65,10 +66,34 @@ __global__ void k_tw0_init(float2 *__restrict__ tw0g, int C) {
         tw0g[i] = tw0_entry<LG>(i % m, C, i / m);
 }
 
+// ------------------------------------------------------ async copy, cluster --
+__device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+// 16-byte global -> shared copy (zero-filled when !valid; nothing is read then)
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+// cluster barrier halves: release/acquire hand off shared-memory data between
+// the CTAs; a relaxed arrive only says "I am done reading your memory" (every
+// value read was consumed before the arrive issues)
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
+
 // ------------------------------------------------------------------ kspec --
+// spec[h][c][pos] = (FFT_2L(K_h zero-padded)[f] + D_h) / 2L for the frequency
+// f = C f' + c held at pos: the spectrum of K + D delta_0, so the convolution
+// adds the D u term with no extra pass over u.
 template <int LG, int C, bool TW0G>
 __global__ void __launch_bounds__(threads_for<LG>())
-k_kspec(const float *__restrict__ K, int H, int L, float2 *__restrict__ spec,
+k_kspec(const float *__restrict__ K, const float *__restrict__ D, int H, int L, float2 *__restrict__ spec,
         const float2 *__restrict__ tw0g) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
     extern __shared__ float2 sm[];
@@ -82,6 +107,7 @@ k_kspec(const float *__restrict__ K, int H, int L, float2 *__restrict__ spec,
     const float scale = 1.0f / (float)(C * m);
     for (int h = slot; h < H; h += nslots) {
         const float *Kh = K + (size_t)h * L;
+        const float Dh = D != nullptr ? __ldg(D + h) : 0.0f;
         forward_first<LG, T>(s.buf, t0, s.pre, [&](int k) {
             float2 v = make_float2(__ldg(Kh + k), 0.0f);
             static_for<1, C / 2>([&](auto r) {
@@ -98,8 +124,8 @@ k_kspec(const float *__restrict__ K, int H, int L, float2 *__restrict__ spec,
         forward_last<LG, T>(s.buf, [&](int base, auto &x) {
             constexpr int R = sizeof(x) / sizeof(float2);
             static_for<0, R / 2>([&](auto i) {
-                out[base / 2 + i] = make_float4(x[2 * i].x * scale, x[2 * i].y * scale,
-                                                x[2 * i + 1].x * scale, x[2 * i + 1].y * scale);
+                out[base / 2 + i] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
+                                                (x[2 * i + 1].x + Dh) * scale, x[2 * i + 1].y * scale);
             });
         });
         __syncthreads();
@@ -107,40 +133,97 @@ k_kspec(const float *__restrict__ K, int H, int L, float2 *__restrict__ spec,
 }
 
 // ---------------------------------------------------------------- fftconv --
-template <int LG, int C, bool TW0G>
+// STAGE: the input rows of the next row pair are copied to shared memory with
+// cp.async while the current pair is transformed (used when the whole pair,
+// 8 L bytes, fits next to the transform).
+template <int LG, int C, bool TW0G, bool STAGE>
 __global__ void __launch_bounds__(threads_for<LG>())
-k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, const float *__restrict__ D,
-          int Bt, int H, int L, float *__restrict__ y, const float2 *__restrict__ tw0g) {
+k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
+          float *__restrict__ y, const float2 *__restrict__ tw0g) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
     constexpr int SL = m / C;                     // combine slice per rank
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    static_assert(C >= 2, "the convolution uses at least two ranks");
     extern __shared__ float2 sm[];
     const Smem s = carve<LG, TW0G>(sm);
+    float *stage = reinterpret_cast<float *>(sm + smem_f2<LG>(TW0G));   // [2][L] when STAGE
     cg::cluster_group cluster = cg::this_cluster();
     const int c = (int)cluster.block_rank();
     const int cl = blockIdx.x / C, ncl = gridDim.x / C;
+    float2 *rbuf[C];
+    static_for<0, C>([&](auto cc) { rbuf[cc] = cluster.map_shared_rank(s.buf, (int)cc); });
     build_tables<LG>(s.tw0, s.tws, s.pre, C, c, threadIdx.x, T);
     if (threadIdx.x < C / 2) s.wcr[threadIdx.x] = unit_root((threadIdx.x * c) % C, C);
     const float2 *t0 = TW0G ? tw0g + (size_t)c * m : s.tw0;
-    __syncthreads();
 
     const int nbp = (Bt + 1) / 2;
     const long long npairs = (long long)H * nbp;
+    auto rows = [&](long long pr, const float *&u0, const float *&u1, bool &has1, int &h, int &b0) {
+        h = (int)(pr / nbp);
+        b0 = 2 * (int)(pr % nbp);
+        has1 = (b0 + 1) < Bt;
+        u0 = u + ((size_t)b0 * H + h) * L;
+        u1 = has1 ? u0 + (size_t)H * L : u0;
+    };
+    auto stage_rows = [&](long long pr) {   // both rows of pair pr -> stage (cp.async)
+        const float *u0, *u1; bool has1; int h, b0;
+        rows(pr, u0, u1, has1, h, b0);
+        for (int i = threadIdx.x; i < L / 2; i += T) {     // 16-byte chunks, L/4 per row
+            const int row = i >= L / 4, k = (i - row * (L / 4)) * 4;
+            cp_async16(stage + row * L + k, (row ? u1 : u0) + k, !row || has1);
+        }
+        cp_async_commit();
+    };
+    if constexpr (STAGE) {
+        if (cl < npairs) stage_rows(cl);
+    }
+    __syncthreads();
+
+    bool first = true;
     for (long long pr = cl; pr < npairs; pr += ncl) {
-        const int h = (int)(pr / nbp), bp = (int)(pr % nbp);
-        const int b0 = 2 * bp;
-        const bool has1 = (b0 + 1) < Bt;
-        const float *u0 = u + ((size_t)b0 * H + h) * L;
-        const float *u1 = has1 ? u0 + (size_t)H * L : u0;   // not read when !has1
-        // forward: x = u0 + i u1 (zero-padded to 2L), rank c's share
-        forward_first<LG, T>(s.buf, t0, s.pre, [&](int k) {
-            float2 v = make_float2(__ldg(u0 + k), has1 ? __ldg(u1 + k) : 0.0f);
+        const float *u0, *u1; bool has1; int h, b0;
+        rows(pr, u0, u1, has1, h, b0);
+        // ---- forward pass 0: x = u0 + i u1 (zero-padded to 2L), rank c's share
+        if constexpr (STAGE) {
+            cp_async_wait_all();
+            __syncthreads();
+        }
+        auto fetch = [&](int k) {
+            float2 v;
+            if constexpr (STAGE) {
+                v = make_float2(stage[k], stage[L + k]);
+            } else {
+                v = make_float2(__ldg(u0 + k), has1 ? __ldg(u1 + k) : 0.0f);
+            }
             static_for<1, C / 2>([&](auto r) {
-                const float a = __ldg(u0 + k + r * m), b = has1 ? __ldg(u1 + k + r * m) : 0.0f;
+                float a, b;
+                if constexpr (STAGE) {
+                    a = stage[k + r * m];
+                    b = stage[L + k + r * m];
+                } else {
+                    a = __ldg(u0 + k + r * m);
+                    b = has1 ? __ldg(u1 + k + r * m) : 0.0f;
+                }
                 v = cadd(v, cmul(make_float2(a, b), s.wcr[r]));
             });
             return v;
-        });
+        };
+        if constexpr (S0 == T) {
+            // one group per thread: compute it, then wait until the partner
+            // ranks have finished reading this CTA's buffer (previous combine)
+            float2 x[R0];
+            first_group<LG>(x, threadIdx.x, t0, s.pre, fetch);
+            if (!first) cluster_wait();
+            store_first_group<LG>(s.buf, x, threadIdx.x);
+        } else {
+            if (!first) cluster_wait();
+            forward_first<LG, T>(s.buf, t0, s.pre, fetch);
+        }
+        first = false;
         __syncthreads();
+        if constexpr (STAGE) {   // the stage is free again: fetch the next pair
+            if (pr + ncl < npairs) stage_rows(pr + ncl);
+        }
         forward_middle<LG, T>(s.buf, s.tws);
         const float4 *sp = reinterpret_cast<const float4 *>(spec + ((size_t)h * C + c) * m);
         fused_middle<LG, T>(s.buf, [&](int base, auto &x) {
@@ -154,26 +237,168 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, const fl
         __syncthreads();
         inverse_middle<LG, T>(s.buf, s.tws);
         inverse_last<LG, T>(s.buf, t0, s.pre);
-        cluster.sync();
-        // combine the C partial transforms; rank c writes t' in [c SL, (c+1) SL)
-        const float Dh = __ldg(D + h);
+        cluster_arrive_release();
+        cluster_wait();
+        // ---- combine the C partial transforms; rank c writes t' in [c SL, (c+1) SL)
         float *y0 = y + ((size_t)b0 * H + h) * L;
         float *y1 = y0 + (size_t)H * L;
-        for (int i = threadIdx.x; i < SL; i += T) {
-            const int tp = c * SL + i;
-            float2 w[C];
-            static_for<0, C>([&](auto cc) { w[cc] = cluster.map_shared_rank(s.buf, (int)cc)[pidx(tp)]; });
-            static_for<0, C / 2>([&](auto r) {
-                float2 o = w[0];
-                static_for<1, C>([&](auto cc) {
-                    o = cadd(o, rot<decltype(cc)::value * decltype(r)::value, C, +1>(w[cc]));
+        constexpr int PER = SL / T > 0 ? (SL / T < 4 ? SL / T : 4) : 1;   // elements per batch
+        for (int i0 = threadIdx.x; i0 < SL; i0 += T * PER) {
+            float2 w[PER][C];
+            static_for<0, PER>([&](auto e) {
+                const int i = i0 + e * T;
+                static_for<0, C>([&](auto cc) {
+                    w[e][cc] = (i < SL) ? rbuf[cc][pidx(c * SL + i)] : make_float2(0.f, 0.f);
                 });
-                const int t = tp + r * m;
-                y0[t] = fmaf(Dh, __ldg(u0 + t), o.x);
-                if (has1) y1[t] = fmaf(Dh, __ldg(u1 + t), o.y);
+            });
+            static_for<0, PER>([&](auto e) {
+                const int i = i0 + e * T;
+                if (i < SL) {
+                    static_for<0, C / 2>([&](auto r) {
+                        float2 o = w[e][0];
+                        static_for<1, C>([&](auto cc) {
+                            o = cadd(o, rot<decltype(cc)::value * decltype(r)::value, C, +1>(w[e][cc]));
+                        });
+                        const int t = c * SL + i + r * m;
+                        y0[t] = o.x;
+                        if (has1) y1[t] = o.y;
+                    });
+                }
             });
         }
-        cluster.sync();
+        cluster_arrive_relaxed();
+    }
+    // the partners may still read this CTA's buffer: wait before exiting
+    if (!first) cluster_wait();
+}
+
+// ------------------------------------------------------- fftconv, one CTA --
+// L <= 4096: one CTA per row pair holds both halves of the length-2L
+// transform (rank 0: frequencies 2f, rank 1: 2f + 1), m = L points each.
+// Thread j owns group j of both halves in every pass, so the first pass
+// reads its input once for both halves, and the last inverse pass adds the
+// two halves -- the combine of the split transform -- in registers and
+// stores y directly. First-pass twiddles follow a recurrence from two small
+// tables: W_m^{j q} = b_j^q (rank 0) and W_N^{j (2q+1)} = a_j b_j^q (rank 1),
+// a_j = W_N^j, b_j = W_m^j.
+template <int LG>
+__host__ __device__ constexpr int pair_smem_f2() {
+    return (2 * padded(1 << LG) + plan_tw_size(LG) + 2 * ((1 << LG) >> plan_lr(LG, 0)) + 1) / 2 * 2;
+}
+
+template <int LG>
+__global__ void __launch_bounds__(threads_for<LG>(), 2)
+k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
+               float *__restrict__ y) {
+    constexpr int m = 1 << LG, T = threads_for<LG>(), N = 2 * m;
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    extern __shared__ float2 sm[];
+    float2 *b0 = sm, *b1 = sm + padded(m);
+    float2 *tws = b1 + padded(m);
+    float2 *ta = tws + plan_tw_size(LG), *tb = ta + S0;
+    float *stage = reinterpret_cast<float *>(sm + pair_smem_f2<LG>());   // [2][L]
+
+    for (int i = threadIdx.x; i < S0; i += T) {
+        ta[i] = unit_root(i, N);
+        tb[i] = unit_root(i, m);
+    }
+    static_for<1, plan_P(LG) - 1>([&](auto sc) {
+        constexpr int s = decltype(sc)::value;
+        constexpr int B = plan_B(LG, s);
+        constexpr int lS = ilog2(B) - plan_lr(LG, s);
+        float2 *t = tws + plan_tw_off(LG, s);
+        for (int i = threadIdx.x; i < B; i += T) t[i] = unit_root(((i & ((1 << lS) - 1)) * (i >> lS)) & (B - 1), B);
+    });
+
+    const int nbp = (Bt + 1) / 2;
+    const long long npairs = (long long)H * nbp;
+    auto stage_rows = [&](long long pr) {
+        const int h = (int)(pr / nbp), b0r = 2 * (int)(pr % nbp);
+        const bool has1 = (b0r + 1) < Bt;
+        const float *u0 = u + ((size_t)b0r * H + h) * L;
+        const float *u1 = has1 ? u0 + (size_t)H * L : u0;
+        for (int i = threadIdx.x; i < L / 2; i += T) {
+            const int row = i >= L / 4, k = (i - row * (L / 4)) * 4;
+            cp_async16(stage + row * L + k, (row ? u1 : u0) + k, !row || has1);
+        }
+        cp_async_commit();
+    };
+    if ((long long)blockIdx.x < npairs) stage_rows(blockIdx.x);
+
+    for (long long pr = blockIdx.x; pr < npairs; pr += gridDim.x) {
+        const int h = (int)(pr / nbp), bq = 2 * (int)(pr % nbp);
+        const bool has1 = (bq + 1) < Bt;
+        cp_async_wait_all();
+        __syncthreads();   // stage ready; previous pair's buffers no longer read
+        // ---- first forward pass, both halves
+        for (int j = threadIdx.x; j < S0; j += T) {
+            float2 x[R0], z[R0];
+            static_for<0, R0>([&](auto p) {
+                const int k = j + p * S0;
+                const float2 v = make_float2(stage[k], stage[L + k]);
+                x[p] = v;
+                z[p] = rot<decltype(p)::value, 2 * R0, -1>(v);
+            });
+            dft<R0, -1>(x);
+            dft<R0, -1>(z);
+            const float2 a = ta[j], b = tb[j];
+            float2 w = b, v = a;
+            const int o = pidx(j);
+            b0[o] = x[0];
+            b1[o] = cmul(z[0], a);
+            static_for<1, R0>([&](auto q) {
+                v = cmul(v, b);
+                b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+                b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], v);
+                w = cmul(w, b);
+            });
+        }
+        __syncthreads();
+        if (pr + gridDim.x < npairs) stage_rows(pr + gridDim.x);   // stage is free again
+        forward_middle_x2<LG, T>(b0, b1, tws);
+        const float4 *s0 = reinterpret_cast<const float4 *>(spec + (size_t)h * N);
+        const float4 *s1 = s0 + m / 2;
+        fused_middle_x2<LG, T>(b0, b1, [&](int base, auto &x, auto &z) {
+            constexpr int R = sizeof(x) / sizeof(float2);
+            float4 k0[R / 2], k1[R / 2];
+            static_for<0, R / 2>([&](auto i) {
+                k0[i] = __ldg(s0 + base / 2 + i);
+                k1[i] = __ldg(s1 + base / 2 + i);
+            });
+            static_for<0, R / 2>([&](auto i) {
+                x[2 * i] = cmul(x[2 * i], make_float2(k0[i].x, k0[i].y));
+                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k0[i].z, k0[i].w));
+                z[2 * i] = cmul(z[2 * i], make_float2(k1[i].x, k1[i].y));
+                z[2 * i + 1] = cmul(z[2 * i + 1], make_float2(k1[i].z, k1[i].w));
+            });
+        });
+        __syncthreads();
+        inverse_middle_x2<LG, T>(b0, b1, tws);
+        // ---- last inverse pass of both halves + their sum, straight to y
+        float *y0 = y + ((size_t)bq * H + h) * L;
+        float *y1 = y0 + (size_t)H * L;
+        for (int j = threadIdx.x; j < S0; j += T) {
+            float2 x[R0], z[R0];
+            const int o = pidx(j);
+            const float2 a = ta[j], b = tb[j];
+            float2 w = b, v = a;
+            x[0] = b0[o];
+            z[0] = cmulc(b1[o], a);
+            static_for<1, R0>([&](auto q) {
+                v = cmul(v, b);
+                x[q] = cmulc(b0[o + poff<decltype(q)::value * S0>()], w);
+                z[q] = cmulc(b1[o + poff<decltype(q)::value * S0>()], v);
+                w = cmul(w, b);
+            });
+            dft<R0, +1>(x);
+            dft<R0, +1>(z);
+            static_for<0, R0>([&](auto p) {
+                const float2 r = cadd(x[p], rot<decltype(p)::value, 2 * R0, +1>(z[p]));
+                const int t = j + p * S0;
+                y0[t] = r.x;
+                if (has1) y1[t] = r.y;
+            });
+        }
     }
 }
 
@@ -206,12 +431,12 @@ k_irfft(float *K, int H, int L) {
         float *K1 = K + (size_t)(2 * pr) * L;
         const bool has2 = 2 * pr + 1 < H;
         float *K2 = has2 ? K1 + L : K1;
-        for (int p = threadIdx.x; p < m; p += T) {
-            const int f = C * digrev<LG>(p) + c;
+        gather_digit_reversed<LG, T>(s.buf, [&](int fr) {
+            const int f = C * fr + c;
             const float2 a = half_spec(K1, f, L);
             const float2 b = has2 ? half_spec(K2, f, L) : make_float2(0.0f, 0.0f);
-            s.buf[pidx(p)] = make_float2(a.x - b.y, a.y + b.x);
-        }
+            return make_float2(a.x - b.y, a.y + b.x);
+        });
         __syncthreads();
         dit_pass<LG, P - 1, +1, T>(s.buf, s.tws);
         __syncthreads();
@@ -310,13 +535,14 @@ cudaError_t launch_clustered(Kern kern, int C, int nclusters, int T, size_t smem
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 // ---- convolution / kspec instantiation for one L ----
-template <int LG, int C, bool TW0G>
+template <int LG, int C, bool TW0G, bool STAGE>
 struct ConvKernels {
     static constexpr int T = threads_for<LG>();
     static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>(TW0G);
+    static constexpr size_t smem_conv = smem + (STAGE ? 2 * sizeof(float) * (size_t)(C * (1 << LG) / 2) : 0);
     static LaunchInfo info_conv, info_kspec;
 
-    static cudaError_t kspec(const float *K, int H, int L, void *ws, cudaStream_t st) {
+    static cudaError_t kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st) {
         float2 *spec = (float2 *)ws;
         float2 *tw0g = nullptr;
         if (TW0G) {
@@ -333,30 +559,44 @@ struct ConvKernels {
         int nslots = res / C;
         if (nslots < 1) nslots = 1;
         if (nslots > H) nslots = H;
-        kern<<<nslots * C, T, smem, st>>>(K, H, L, spec, (const float2 *)tw0g);
+        kern<<<nslots * C, T, smem, st>>>(K, D, H, L, spec, (const float2 *)tw0g);
         return cudaGetLastError();
     }
 
-    static cudaError_t conv(const float *u, const void *ws, const float *D, int Bt, int H, int L,
-                            float *y, cudaStream_t st) {
+    static LaunchInfo info_pair;
+
+    static cudaError_t conv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st) {
         const float2 *spec = (const float2 *)ws;
+        if constexpr (C == 2 && !TW0G && LG <= 12) {
+            // one CTA per row pair, both halves in one CTA
+            auto kern = k_fftconv_pair<LG>;
+            constexpr size_t psmem = sizeof(float2) * (size_t)pair_smem_f2<LG>() + 2 * sizeof(float) * (1 << LG);
+            int res = 0;
+            cudaError_t e = resident_units(kern, info_pair, 1, T, psmem, &res);
+            if (e != cudaSuccess) return e;
+            const long long npairs = (long long)H * ((Bt + 1) / 2);
+            const int grid = (long long)res < npairs ? res : (int)npairs;
+            kern<<<grid, T, psmem, st>>>(u, spec, Bt, H, L, y);
+            return cudaGetLastError();
+        }
         const float2 *tw0g = TW0G
             ? (const float2 *)((const char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)))
             : nullptr;
-        auto kern = k_fftconv<LG, C, TW0G>;
+        auto kern = k_fftconv<LG, C, TW0G, STAGE>;
         int res = 0;
-        cudaError_t e = resident_units(kern, info_conv, C, T, smem, &res);
+        cudaError_t e = resident_units(kern, info_conv, C, T, smem_conv, &res);
         if (e != cudaSuccess) return e;
         const long long npairs = (long long)H * ((Bt + 1) / 2);
         int ncl = res;
         if ((long long)ncl > npairs) ncl = (int)npairs;
-        e = launch_clustered(kern, C, ncl, T, smem, st, u, spec, D, Bt, H, L, y, tw0g);
+        e = launch_clustered(kern, C, ncl, T, smem_conv, st, u, spec, Bt, H, L, y, tw0g);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
 };
-template <int LG, int C, bool TW0G> LaunchInfo ConvKernels<LG, C, TW0G>::info_conv;
-template <int LG, int C, bool TW0G> LaunchInfo ConvKernels<LG, C, TW0G>::info_kspec;
+template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_conv;
+template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec;
+template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_pair;
 
 // ---- irfft instantiation ----
 template <int LG, int C>
@@ -409,34 +649,40 @@ size_t conv_workspace_bytes(int H, int L) {
     return b;
 }
 
+// Longest L whose convolution stages the next row pair in shared memory
+// (cp.async prefetch; costs 8 L bytes of shared memory per CTA).
+#ifndef S4_CONV_STAGE_MAX_L
+#define S4_CONV_STAGE_MAX_L 4096
+#endif
+#define S4_STG(LL) ((LL) <= S4_CONV_STAGE_MAX_L)
+// (L, log2 m, C, first-pass table in global memory, staged input)
 #define S4_CONV_CASES(X)            \
-    X(16, 4, 2, false)              \
-    X(32, 5, 2, false)              \
-    X(64, 6, 2, false)              \
-    X(128, 7, 2, false)             \
-    X(256, 8, 2, false)             \
-    X(512, 9, 2, false)             \
-    X(1024, 10, 2, false)           \
-    X(2048, 11, 2, false)           \
-    X(4096, 12, 2, false)           \
-    X(8192, 12, 4, false)           \
-    X(16384, 12, 8, false)          \
-    X(32768, 13, 8, false)          \
-    X(65536, 14, 8, true)
+    X(16, 4, 2, false, S4_STG(16))        \
+    X(32, 5, 2, false, S4_STG(32))        \
+    X(64, 6, 2, false, S4_STG(64))        \
+    X(128, 7, 2, false, S4_STG(128))      \
+    X(256, 8, 2, false, S4_STG(256))      \
+    X(512, 9, 2, false, S4_STG(512))      \
+    X(1024, 10, 2, false, S4_STG(1024))   \
+    X(2048, 11, 2, false, S4_STG(2048))   \
+    X(4096, 12, 2, false, S4_STG(4096))   \
+    X(8192, 12, 4, false, false)    \
+    X(16384, 12, 8, false, false)   \
+    X(32768, 13, 8, false, false)   \
+    X(65536, 14, 8, true, false)
 
-cudaError_t launch_kspec(const float *K, int H, int L, void *ws, cudaStream_t st) {
+cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st) {
     switch (L) {
-#define X(LL, LG, C, G) case LL: return ConvKernels<LG, C, G>::kspec(K, H, L, ws, st);
+#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::kspec(K, D, H, L, ws, st);
         S4_CONV_CASES(X)
 #undef X
         default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_fftconv(const float *u, const void *ws, const float *D, int Bt, int H, int L,
-                           float *y, cudaStream_t st) {
+cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st) {
     switch (L) {
-#define X(LL, LG, C, G) case LL: return ConvKernels<LG, C, G>::conv(u, ws, D, Bt, H, L, y, st);
+#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::conv(u, ws, Bt, H, L, y, st);
         S4_CONV_CASES(X)
 #undef X
         default: return cudaErrorInvalidValue;

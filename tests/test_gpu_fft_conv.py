@@ -113,10 +113,13 @@ def test_prepare_apply_matches_one_call():
     K = torch.from_numpy(rng.standard_normal((4, 2048)).astype(np.float32)).cuda()
     D = torch.from_numpy(rng.standard_normal(4).astype(np.float32)).cuda()
     y1 = s4.fft_conv(u, K, D)
-    ws = s4.fft_conv_prepare(K)
-    y2 = s4.fft_conv_apply(u, ws, D)
-    y3 = s4.fft_conv_apply(u[:3].contiguous(), ws, D)
+    ws = s4.fft_conv_prepare(K, D)
+    y2 = s4.fft_conv_apply(u, ws)
+    y3 = s4.fft_conv_apply(u[:3].contiguous(), ws)
+    ws0 = s4.fft_conv_prepare(K)          # no feed-through term
+    y4 = s4.fft_conv_apply(u, ws0)
     torch.cuda.synchronize()
+    assert rel_l2((y4 + D[None, :, None] * u).cpu().numpy(), y1.cpu().numpy()) <= Y_TOL
     assert torch.equal(y1, y2)
     # rows 0 and 1 form the same packed pair in both calls; row 2 is paired
     # with row 3 in one call and alone in the other, so it only rounds alike
