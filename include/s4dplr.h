@@ -154,6 +154,34 @@ s4_status s4_fft_conv_apply(const float *u, const void *workspace,
                             size_t workspace_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The whole forward pass of the layer's convolution view ([S4K] §4, §5).
+ *
+ * s4_kernel_dplr_prepare = s4_kernel_dplr(...) followed by
+ * s4_fft_conv_prepare(K, D, ...): it writes K[H, L] and the convolution
+ * spectrum of K + D delta_0 into the workspace. For L <= 4096 both come out
+ * of a single kernel per channel (the generating function is written
+ * straight into the inverse transform's input order, and the inverse
+ * transform's output starts the zero-padded forward transform). D may be
+ * NULL (no feed-through term).
+ *
+ * s4_forward_dplr = s4_kernel_dplr_prepare followed by s4_fft_conv_apply:
+ * y[Bt, H, L] from the DPLR parameters and u in one call; K and the
+ * workspace are outputs/scratch as above. Argument rules and errors are those
+ * of the calls it is made of (D required here).
+ * ------------------------------------------------------------------------ */
+s4_status s4_kernel_dplr_prepare(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                                 const s4_c32 *B, const s4_c32 *C, const float *log_dt,
+                                 const float *D, int H, int Nh, int L, float *K,
+                                 void *workspace, size_t workspace_bytes, unsigned *d_flags,
+                                 cudaStream_t stream);
+
+s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                          const s4_c32 *B, const s4_c32 *C, const float *log_dt, const float *D,
+                          int Bt, int H, int Nh, int L, float *K, float *y,
+                          void *workspace, size_t workspace_bytes, unsigned *d_flags,
+                          cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * s4_fft_conv_static -- s4_fft_conv without a caller-provided workspace.
  * The pages have no counterpart of this entry point; it exists for callers
  * that cannot allocate device memory: a plugin inside a host application

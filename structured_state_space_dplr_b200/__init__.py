@@ -20,7 +20,7 @@ from ._lib import (S4_FLAG_NONFINITE, S4_FLAG_UNSTABLE, S4_STEP_DENSE, S4_STEP_D
                    S4Error)
 
 __all__ = [
-    "kernel_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
+    "kernel_dplr", "kernel_dplr_prepare", "forward_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
     "fft_conv_static",
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
@@ -176,6 +176,44 @@ def fft_conv_apply(u, workspace, *, out=None):
     _cuda(out, "out", torch.float32)
     _lib.call("s4_fft_conv_apply", _ptr(u), _ptr(workspace), Bt, H, L, _ptr(out), workspace.numel(),
               _stream())
+    return out
+
+
+def kernel_dplr_prepare(Lambda, P, Q, B, C, log_dt, D, L, *, K=None, workspace=None, flags=None):
+    """K and the convolution spectrum of K + D delta_0 (s4_kernel_dplr_prepare).
+    Returns (K, workspace); the workspace feeds fft_conv_apply."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    if D is not None:
+        D = _cuda(D, "D", torch.float32)
+    if K is None:
+        K = torch.empty(H, L, device=Lambda.device, dtype=torch.float32)
+    _cuda(K, "K", torch.float32)
+    workspace = _workspace(H, L, Lambda.device, workspace)
+    _lib.call("s4_kernel_dplr_prepare", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              _ptr(D), H, Nh, int(L), _ptr(K), _ptr(workspace), workspace.numel(), _flags_ptr(flags),
+              _stream())
+    return K, workspace
+
+
+def forward_dplr(u, Lambda, P, Q, B, C, log_dt, D, *, out=None, K=None, workspace=None, flags=None):
+    """y = K * u + D u with K the DPLR kernel, in one call (s4_forward_dplr)."""
+    u = _cuda(u, "u", torch.float32)
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    D = _cuda(D, "D", torch.float32)
+    Bt, H, L = u.shape
+    Nh = Lambda.shape[1]
+    if K is None:
+        K = torch.empty(H, L, device=u.device, dtype=torch.float32)
+    if out is None:
+        out = torch.empty_like(u)
+    _cuda(out, "out", torch.float32)
+    workspace = _workspace(H, L, u.device, workspace)
+    _lib.call("s4_forward_dplr", _ptr(u), _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              _ptr(D), Bt, H, Nh, L, _ptr(K), _ptr(out), _ptr(workspace), workspace.numel(),
+              _flags_ptr(flags), _stream())
     return out
 
 

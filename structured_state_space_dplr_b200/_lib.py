@@ -33,6 +33,8 @@ SIGNATURES = {
     "s4_fft_conv_prepare": (_i, [_p, _p, _i, _i, _p, _sz, _p]),
     "s4_fft_conv_apply": (_i, [_p, _p, _i, _i, _i, _p, _sz, _p]),
     "s4_fft_conv_static": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
+    "s4_kernel_dplr_prepare": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p, _p]),
+    "s4_forward_dplr": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "s4d_kernel_vandermonde": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p, _p]),
     "s4_dplr_discretize": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _p, _p, _p, _p]),
     "s4d_discretize_zoh": (_i, [_p, _p, _p, _i, _i, _p, _p, _p]),

@@ -165,6 +165,37 @@ s4_status s4_fft_conv(const float *u, const float *K, const float *D, int Bt, in
     return cuda_status(e);
 }
 
+s4_status s4_kernel_dplr_prepare(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B,
+                                 const s4_c32 *C, const float *log_dt, const float *D, int H, int Nh, int L,
+                                 float *K, void *workspace, size_t workspace_bytes, unsigned *d_flags,
+                                 cudaStream_t stream) {
+    s4_status s = dplr_checks(Lambda, P, Q, B, C, log_dt, H, Nh, L, K);
+    if (s == S4_OK) s = prepare_checks(K, D, H, L, workspace, workspace_bytes);
+    if (s != S4_OK) return s;
+    for (const void *p : {(const void *)Lambda, (const void *)P, (const void *)Q, (const void *)B,
+                          (const void *)C})
+        if (overlap(workspace, workspace_bytes, p, (size_t)H * Nh * sizeof(s4_c32))) return S4_ERR_INVALID_ARG;
+    return cuda_status(s4::launch_kgen((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q,
+                                       (const float2 *)B, (const float2 *)C, log_dt, D, H, Nh, L, K, workspace,
+                                       d_flags, stream));
+}
+
+s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                          const s4_c32 *B, const s4_c32 *C, const float *log_dt, const float *D, int Bt, int H,
+                          int Nh, int L, float *K, float *y, void *workspace, size_t workspace_bytes,
+                          unsigned *d_flags, cudaStream_t stream) {
+    if (D == nullptr) return S4_ERR_INVALID_ARG;
+    s4_status s = conv_checks(u, Bt, H, L, y, workspace, workspace_bytes);
+    if (s != S4_OK) return s;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float);
+    if (overlap(y, nb, K, (size_t)H * L * sizeof(float)) || overlap(y, nb, D, (size_t)H * sizeof(float)))
+        return S4_ERR_INVALID_ARG;
+    s = s4_kernel_dplr_prepare(Lambda, P, Q, B, C, log_dt, D, H, Nh, L, K, workspace, workspace_bytes, d_flags,
+                               stream);
+    if (s != S4_OK) return s;
+    return cuda_status(s4::launch_fftconv(u, workspace, Bt, H, L, y, stream));
+}
+
 s4_status s4d_kernel_vandermonde(const s4_c32 *A, const s4_c32 *B, const s4_c32 *C, const float *log_dt,
                                  int H, int Nh, int L, float *K, unsigned *d_flags, cudaStream_t stream) {
     if (any_null(A, B, C) || log_dt == nullptr || K == nullptr) return S4_ERR_INVALID_ARG;

@@ -74,6 +74,20 @@ __device__ __forceinline__ int digrev(int p) {
     return f;
 }
 
+// position holding frequency f after the forward passes (inverse of digrev)
+template <int LG>
+__device__ __forceinline__ int digrev_inv(int f) {
+    int p = 0;
+    static_for<0, plan_P(LG)>([&](auto sc) {
+        constexpr int s = decltype(sc)::value;
+        constexpr int lr = plan_lr(LG, s);
+        constexpr int lS = ilog2(plan_B(LG, s)) - lr;
+        constexpr int lw = LG - ilog2(plan_B(LG, s));
+        p |= ((f >> lw) & ((1 << lr) - 1)) << lS;
+    });
+    return p;
+}
+
 // ------------------------------------------------------------ butterflies --
 // cos(2 pi e / 32) for any integer e (values of cos(k pi / 16), k = 0..8)
 __host__ __device__ constexpr float cos32(int e) {

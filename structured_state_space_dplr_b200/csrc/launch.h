@@ -20,6 +20,12 @@ cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L,
 // in place: K[H, L] holds the packed half spectrum on entry, the real kernel on exit
 cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st);
 
+// ---- kgen.cu: K and the convolution spectrum of K + D delta_0 in one launch
+// (L <= 4096; longer L runs k_cauchy, k_irfft and k_kspec) ----
+cudaError_t launch_kgen(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B, const float2 *C,
+                        const float *log_dt, const float *D, int H, int Nh, int L, float *K, void *ws,
+                        unsigned *flags, cudaStream_t st);
+
 // ---- cauchy.cu ----
 cudaError_t launch_cauchy(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
                           const float2 *C, const float *log_dt, int H, int Nh, int L, float *K,

@@ -1,0 +1,64 @@
+"""GPU parity of the fused entry points: s4_kernel_dplr_prepare (K and the
+convolution spectrum of K + D delta_0 in one launch for L <= 4096) and
+s4_forward_dplr (the whole convolution-view forward), against the fp64 oracle
+and against the modular calls."""
+import numpy as np
+import pytest
+
+import s4inputs
+from oracle import workloads
+from gpu_helpers import K_TOL, Y_TOL, kernel_err, rel_l2, sample_times, to_dev, torch_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def _fused(inp):
+    import structured_state_space_dplr_b200 as s4
+    torch = torch_cuda()
+    t = to_dev(inp)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = s4.forward_dplr(t["u"], t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], t["D"], flags=flags)
+    K, ws = s4.kernel_dplr_prepare(t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], t["D"], inp["L"])
+    y2 = s4.fft_conv_apply(t["u"], ws)
+    K3 = s4.kernel_dplr(t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], inp["L"])
+    y3 = s4.fft_conv(t["u"], K3, t["D"])
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    assert torch.equal(y, y2)
+    return K.cpu().numpy(), y.cpu().numpy(), K3.cpu().numpy(), y3.cpu().numpy()
+
+
+@pytest.mark.parametrize("L", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192])
+def test_random_dplr_all_outputs(L):
+    inp = s4inputs.random_dplr(500 + L, H=3, Nh=6, L=L, Bt=3)
+    K, y, K3, y3 = _fused(inp)
+    Kr = workloads.dplr_kernel(inp)
+    yr = workloads.conv_full(inp, Kr)
+    assert kernel_err(K, Kr) <= K_TOL
+    assert rel_l2(y, yr) <= Y_TOL
+    assert kernel_err(K, K3) <= K_TOL
+    assert rel_l2(y, y3) <= Y_TOL
+
+
+def test_cfg1_all_outputs():
+    inp = s4inputs.make_inputs(1)
+    K, y, _, _ = _fused(inp)
+    Kr = workloads.dplr_kernel(inp)
+    assert kernel_err(K, Kr) <= K_TOL
+    assert rel_l2(y, workloads.conv_full(inp, Kr)) <= Y_TOL
+
+
+def test_cfg2_full_size_sampled():
+    """The benchmark's workload and launch (H=256, L=4096, batch 16)."""
+    inp = s4inputs.make_inputs(2)
+    K, y, K3, y3 = _fused(inp)
+    ch = [0, 128, 255]
+    Kr = workloads.dplr_kernel(inp, channels=ch)
+    assert kernel_err(K[ch], Kr) <= K_TOL
+    assert kernel_err(K, K3) <= K_TOL
+    ts = sample_times(inp["L"], 48, seed=22)
+    rows = [(b, h) for h in ch for b in (0, 7, 15)]
+    yr = workloads.conv_rows_at(inp, [Kr[ch.index(h)] for _, h in rows], rows, ts)
+    ys = np.stack([y[b, h][ts] for b, h in rows])
+    assert rel_l2(ys, yr) <= Y_TOL
+    assert rel_l2(y, y3) <= Y_TOL
