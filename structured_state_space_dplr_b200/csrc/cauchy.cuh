@@ -58,13 +58,13 @@ __device__ __forceinline__ void cauchy_eval(const float4 *sp, int Nh, const int 
 #pragma unroll
     for (int f = 0; f < F; ++f) {
         float sn, cs;
-        sincospif((float)j[f] / (float)L, &sn, &cs);
-        t[f] = sn / cs;
+        sincospif((float)j[f] / (float)L, &sn, &cs);   // j/L is exact, cs > 0 for j < L/2
+        t[f] = __fdividef(sn, cs);
         gam[f] = 2.0f * t[f] * inv_dt;
         const float g2 = gam[f] * gam[f];
-        int e;
-        frexpf(g2, &e);
-        sig[f] = e > 0 ? ldexpf(1.0f, -e) : 1.0f;
+        // sigma = 2^-e with 2^(e-1) <= g2 < 2^e when g2 >= 1, else 1 (exact)
+        const int e = ((__float_as_int(g2) >> 23) & 0xff) - 126;
+        sig[f] = e > 0 ? __int_as_float((127 - e) << 23) : 1.0f;
         g2s[f] = g2 * sig[f];
         gs[f] = gam[f] * sig[f];
 #pragma unroll
@@ -102,7 +102,7 @@ __device__ __forceinline__ void cauchy_eval(const float4 *sp, int Nh, const int 
         // Woodbury: k00 - k01 k10 / (1 + k11)
         const float2 den = make_float2(1.0f + k[3].x, k[3].y);
         const float2 num = cmul(k[1], k[2]);
-        const float idn = 1.0f / fmaf(den.x, den.x, den.y * den.y);
+        const float idn = rcp_approx(fmaf(den.x, den.x, den.y * den.y));
         const float2 w = cscale(cmulc(num, den), idn);
         const float2 r = csub(k[0], w);
         // times 2/(1+z) = 1 + i t, and 1/L for the inverse transform

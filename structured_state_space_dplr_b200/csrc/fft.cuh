@@ -48,17 +48,22 @@ __host__ __device__ constexpr int plan_B(int lg, int s) {
     for (int i = 0; i < s; ++i) b -= plan_lr(lg, i);
     return 1 << b;
 }
-// twiddle entries of passes 1 .. s-1 (pass 0 has its own table)
+// Middle passes 1 .. P-2 keep one base twiddle W_B^j per group index j
+// (S_s entries for pass s); the powers W_B^{j q} follow by a recurrence.
+// Offset of pass s's base table (pass 0 has its own tables):
 __host__ __device__ constexpr int plan_tw_off(int lg, int s) {
     int o = 0;
-    for (int i = 1; i < s; ++i) o += plan_B(lg, i);
+    for (int i = 1; i < s; ++i) o += plan_B(lg, i) >> plan_lr(lg, i);
     return o;
 }
-// all twiddle entries of passes 1 .. P-2 (the last pass has none)
+// all base twiddles of passes 1 .. P-2 (the last pass has none)
 __host__ __device__ constexpr int plan_tw_size(int lg) { return plan_tw_off(lg, plan_P(lg) - 1); }
 
-__host__ __device__ constexpr int padded(int m) { return m + m / 16; }
-__device__ __forceinline__ int pidx(int i) { return i + (i >> 4); }
+// Shared-memory padding: two points after every 16. Groups of the strided
+// passes stay conflict-free for 8-byte accesses, and the contiguous groups of
+// the last pass start on 16-byte boundaries, so they move as 16-byte vectors.
+__host__ __device__ constexpr int padded(int m) { return m + m / 8; }
+__device__ __forceinline__ int pidx(int i) { return i + 2 * (i >> 4); }
 
 // frequency index held at position p after the forward passes
 template <int LG>
@@ -168,6 +173,18 @@ __device__ __forceinline__ float2 tw0_entry(int i, int C, int c) {
     return unit_root((j * (C * q + c)) & (N - 1), N);
 }
 
+// Base twiddles of the middle passes: tws[off_s + j] = W_{B_s}^j, j < S_s.
+template <int LG>
+__device__ void build_middle_tables(float2 *tws, int tid, int nthreads) {
+    static_for<1, plan_P(LG) - 1>([&](auto sc) {
+        constexpr int s = decltype(sc)::value;
+        constexpr int B = plan_B(LG, s);
+        constexpr int S = B >> plan_lr(LG, s);
+        float2 *t = tws + plan_tw_off(LG, s);
+        for (int j = tid; j < S; j += nthreads) t[j] = unit_root(j, B);
+    });
+}
+
 // Fill (with nthreads threads, index tid) the per-CTA tables:
 //   tw0 (pass 0, rank c; skipped when null), tws (passes 1..P-2), pre[p] = W_{C R0}^{p c}.
 template <int LG>
@@ -177,16 +194,7 @@ __device__ void build_tables(float2 *tw0, float2 *tws, float2 *pre, int C, int c
     constexpr int R0 = 1 << plan_lr(LG, 0);
     if (tw0 != nullptr)
         for (int i = tid; i < m; i += nthreads) tw0[i] = tw0_entry<LG>(i, C, c);
-    static_for<1, P - 1>([&](auto sc) {
-        constexpr int s = decltype(sc)::value;
-        constexpr int B = plan_B(LG, s);
-        constexpr int lS = ilog2(B) - plan_lr(LG, s);
-        float2 *t = tws + plan_tw_off(LG, s);
-        for (int i = tid; i < B; i += nthreads) {
-            int q = i >> lS, j = i & ((1 << lS) - 1);
-            t[i] = unit_root((j * q) & (B - 1), B);
-        }
-    });
+    build_middle_tables<LG>(tws, tid, nthreads);
     for (int p = tid; p < R0; p += nthreads) pre[p] = unit_root((p * c) % (C * R0), C * R0);
 }
 
@@ -195,63 +203,97 @@ __device__ void build_tables(float2 *tw0, float2 *tws, float2 *pre, int C, int c
 // (base mod 16) + (q S mod 16) < 16 holds for all plans, so the padding term
 // of base + q S splits into that of base plus (q S) / 16 -- a constant.
 template <int QS>
-__host__ __device__ constexpr int poff() { return QS + (QS >> 4); }
+__host__ __device__ constexpr int poff() { return QS + 2 * (QS >> 4); }
+
+// R consecutive points starting at a 16-byte aligned shared address
+template <int R>
+__device__ __forceinline__ void load_contig(const float2 *p, float2 (&x)[R]) {
+    static_for<0, R / 2>([&](auto i) {
+        const float4 v = reinterpret_cast<const float4 *>(p)[i];
+        x[2 * i] = make_float2(v.x, v.y);
+        x[2 * i + 1] = make_float2(v.z, v.w);
+    });
+}
+template <int R>
+__device__ __forceinline__ void store_contig(float2 *p, const float2 (&x)[R]) {
+    static_for<0, R / 2>([&](auto i) {
+        reinterpret_cast<float4 *>(p)[i] = make_float4(x[2 * i].x, x[2 * i].y, x[2 * i + 1].x, x[2 * i + 1].y);
+    });
+}
+// x[q] *= w^q (q >= 1) with the powers of w formed on the fly
+template <int DIR, int R>
+__device__ __forceinline__ void apply_powers(float2 (&x)[R], float2 w) {
+    float2 wq = w;
+    static_for<1, R>([&](auto q) {
+        x[q] = ctw<DIR>(x[q], wq);
+        if constexpr (decltype(q)::value + 1 < R) wq = cmul(wq, w);
+    });
+}
+template <int DIR, int R>
+__device__ __forceinline__ void apply_powers2(float2 (&x)[R], float2 (&z)[R], float2 w) {
+    float2 wq = w;
+    static_for<1, R>([&](auto q) {
+        x[q] = ctw<DIR>(x[q], wq);
+        z[q] = ctw<DIR>(z[q], wq);
+        if constexpr (decltype(q)::value + 1 < R) wq = cmul(wq, w);
+    });
+}
 
 // Middle pass s (1 <= s <= P-1) in decimation-in-frequency form: DFT of each
 // group, then twiddles. DIR = -1 forward, +1 inverse (conjugate twiddles).
 template <int LG, int s, int DIR, int T>
-__device__ __forceinline__ void dif_pass(float2 *buf, const float2 *tws) {
+__device__ __forceinline__ void dif_pass(float2 *buf, const float2 *tws, int tid = threadIdx.x) {
     constexpr int lr = plan_lr(LG, s), R = 1 << lr;
     constexpr int B = plan_B(LG, s), S = B / R, G = (1 << LG) / R;
     constexpr int lS = ilog2(S);
     const float2 *tw = tws + plan_tw_off(LG, s);
-    for (int g = threadIdx.x; g < G; g += T) {
+    for (int g = tid; g < G; g += T) {
         const int j = g & (S - 1);
         float2 *p = buf + pidx(((g >> lS) << (lS + lr)) + j);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value * S>()]; });
+        if constexpr (S == 1) load_contig<R>(p, x);
+        else static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value * S>()]; });
         dft<R, DIR>(x);
-        if constexpr (S > 1) {
-            static_for<1, R>([&](auto q) { x[q] = ctw<DIR>(x[q], tw[q * S + j]); });
-        }
-        static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
+        if constexpr (S > 1) apply_powers<DIR, R>(x, tw[j]);
+        if constexpr (S == 1) store_contig<R>(p, x);
+        else static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
     }
 }
 
 // Middle pass s in decimation-in-time form (the transpose): twiddles, then DFT.
 template <int LG, int s, int DIR, int T>
-__device__ __forceinline__ void dit_pass(float2 *buf, const float2 *tws) {
+__device__ __forceinline__ void dit_pass(float2 *buf, const float2 *tws, int tid = threadIdx.x) {
     constexpr int lr = plan_lr(LG, s), R = 1 << lr;
     constexpr int B = plan_B(LG, s), S = B / R, G = (1 << LG) / R;
     constexpr int lS = ilog2(S);
     const float2 *tw = tws + plan_tw_off(LG, s);
-    for (int g = threadIdx.x; g < G; g += T) {
+    for (int g = tid; g < G; g += T) {
         const int j = g & (S - 1);
         float2 *p = buf + pidx(((g >> lS) << (lS + lr)) + j);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value * S>()]; });
-        if constexpr (S > 1) {
-            static_for<1, R>([&](auto q) { x[q] = ctw<DIR>(x[q], tw[q * S + j]); });
-        }
+        if constexpr (S == 1) load_contig<R>(p, x);
+        else static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value * S>()]; });
+        if constexpr (S > 1) apply_powers<DIR, R>(x, tw[j]);
         dft<R, DIR>(x);
-        static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
+        if constexpr (S == 1) store_contig<R>(p, x);
+        else static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
     }
 }
 
 // Forward passes 1 .. P-2 (pass 0 and the last pass are done by the caller).
 template <int LG, int T>
-__device__ __forceinline__ void forward_middle(float2 *buf, const float2 *tws) {
+__device__ __forceinline__ void forward_middle(float2 *buf, const float2 *tws, int tid = threadIdx.x) {
     static_for<1, plan_P(LG) - 1>([&](auto sc) {
-        dif_pass<LG, decltype(sc)::value, -1, T>(buf, tws);
+        dif_pass<LG, decltype(sc)::value, -1, T>(buf, tws, tid);
         __syncthreads();
     });
 }
 // Inverse passes P-2 .. 1.
 template <int LG, int T>
-__device__ __forceinline__ void inverse_middle(float2 *buf, const float2 *tws) {
+__device__ __forceinline__ void inverse_middle(float2 *buf, const float2 *tws, int tid = threadIdx.x) {
     constexpr int P = plan_P(LG);
     static_for<1, P - 1>([&](auto sc) {
-        dit_pass<LG, P - 1 - decltype(sc)::value, +1, T>(buf, tws);
+        dit_pass<LG, P - 1 - decltype(sc)::value, +1, T>(buf, tws, tid);
         __syncthreads();
     });
 }
@@ -311,18 +353,18 @@ __device__ __forceinline__ void inverse_last(float2 *buf, const float2 *tw0, con
 // of R consecutive positions [g R, g R + R) is multiplied by mul(pos0, x);
 // pre(pos0) runs first (to start loads early).
 template <int LG, int T, class Mul>
-__device__ __forceinline__ void fused_middle(float2 *buf, Mul &&mul) {
+__device__ __forceinline__ void fused_middle(float2 *buf, Mul &&mul, int tid = threadIdx.x) {
     constexpr int lr = plan_lr(LG, plan_P(LG) - 1), R = 1 << lr;
     constexpr int G = (1 << LG) / R;
-    for (int g = threadIdx.x; g < G; g += T) {
+    for (int g = tid; g < G; g += T) {
         const int base = g * R;
         float2 *p = buf + pidx(base);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value>()]; });
+        load_contig<R>(p, x);
         dft<R, -1>(x);
         mul(base, x);
         dft<R, +1>(x);
-        static_for<0, R>([&](auto q) { p[poff<decltype(q)::value>()] = x[q]; });
+        store_contig<R>(p, x);
     }
 }
 
@@ -335,10 +377,22 @@ __device__ __forceinline__ void forward_last(float2 *buf, Out &&out) {
         const int base = g * R;
         const float2 *p = buf + pidx(base);
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value>()]; });
+        load_contig<R>(p, x);
         dft<R, -1>(x);
         out(base, x);
     }
+}
+
+// Storage of a spectrum produced by the last forward pass (one channel and
+// rank): group g of that pass holds the R consecutive positions
+// [g R, g R + R), kept as R/2 float4 words. Word i of every group is stored
+// contiguously (index i G + g, G = m / R), so the consecutive threads of a
+// warp, which own consecutive groups, read and write consecutive words.
+template <int LG>
+__device__ __forceinline__ int spec4_index(int base, int i) {
+    constexpr int R = 1 << plan_lr(LG, plan_P(LG) - 1);
+    constexpr int G = (1 << LG) / R;
+    return i * G + base / R;
 }
 
 // Gather the input of an inverse transform into digit-reversed positions:
@@ -362,30 +416,28 @@ __device__ __forceinline__ void pass_x2(float2 *b0, float2 *b1, const float2 *tw
         const int j = g & (S - 1);
         const int o = pidx(((g >> lS) << (lS + lr)) + j);
         float2 x[R], z[R];
-        static_for<0, R>([&](auto q) {
-            x[q] = b0[o + poff<decltype(q)::value * S>()];
-            z[q] = b1[o + poff<decltype(q)::value * S>()];
-        });
-        if constexpr (TW_FIRST && S > 1) {
-            static_for<1, R>([&](auto q) {
-                const float2 w = tw[q * S + j];
-                x[q] = ctw<DIR>(x[q], w);
-                z[q] = ctw<DIR>(z[q], w);
+        if constexpr (S == 1) {
+            load_contig<R>(b0 + o, x);
+            load_contig<R>(b1 + o, z);
+        } else {
+            static_for<0, R>([&](auto q) {
+                x[q] = b0[o + poff<decltype(q)::value * S>()];
+                z[q] = b1[o + poff<decltype(q)::value * S>()];
             });
         }
+        if constexpr (TW_FIRST && S > 1) apply_powers2<DIR, R>(x, z, tw[j]);
         dft<R, DIR>(x);
         dft<R, DIR>(z);
-        if constexpr (!TW_FIRST && S > 1) {
-            static_for<1, R>([&](auto q) {
-                const float2 w = tw[q * S + j];
-                x[q] = ctw<DIR>(x[q], w);
-                z[q] = ctw<DIR>(z[q], w);
+        if constexpr (!TW_FIRST && S > 1) apply_powers2<DIR, R>(x, z, tw[j]);
+        if constexpr (S == 1) {
+            store_contig<R>(b0 + o, x);
+            store_contig<R>(b1 + o, z);
+        } else {
+            static_for<0, R>([&](auto q) {
+                b0[o + poff<decltype(q)::value * S>()] = x[q];
+                b1[o + poff<decltype(q)::value * S>()] = z[q];
             });
         }
-        static_for<0, R>([&](auto q) {
-            b0[o + poff<decltype(q)::value * S>()] = x[q];
-            b1[o + poff<decltype(q)::value * S>()] = z[q];
-        });
     }
 }
 template <int LG, int T>
@@ -413,19 +465,15 @@ __device__ __forceinline__ void fused_middle_x2(float2 *b0, float2 *b1, Mul &&mu
         const int base = g * R;
         const int o = pidx(base);
         float2 x[R], z[R];
-        static_for<0, R>([&](auto q) {
-            x[q] = b0[o + poff<decltype(q)::value>()];
-            z[q] = b1[o + poff<decltype(q)::value>()];
-        });
+        load_contig<R>(b0 + o, x);
+        load_contig<R>(b1 + o, z);
         dft<R, -1>(x);
         dft<R, -1>(z);
         mul(base, x, z);
         dft<R, +1>(x);
         dft<R, +1>(z);
-        static_for<0, R>([&](auto q) {
-            b0[o + poff<decltype(q)::value>()] = x[q];
-            b1[o + poff<decltype(q)::value>()] = z[q];
-        });
+        store_contig<R>(b0 + o, x);
+        store_contig<R>(b1 + o, z);
     }
 }
 

@@ -45,13 +45,7 @@ k_kgen(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const fl
         ta[i] = unit_root(i, N);
         tb[i] = unit_root(i, m);
     }
-    static_for<1, NP - 1>([&](auto sc) {
-        constexpr int s = decltype(sc)::value;
-        constexpr int Bs = plan_B(LG, s);
-        constexpr int lS = ilog2(Bs) - plan_lr(LG, s);
-        float2 *t = tws + plan_tw_off(LG, s);
-        for (int i = threadIdx.x; i < Bs; i += T) t[i] = unit_root(((i & ((1 << lS) - 1)) * (i >> lS)) & (Bs - 1), Bs);
-    });
+    build_middle_tables<LG>(tws, threadIdx.x, T);
     cauchy_stage_modes(Lambda, P, Q, B, Cc, h, Nh, sp, flags, threadIdx.x, T);
     __syncthreads();
 
@@ -140,16 +134,14 @@ k_kgen(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const fl
     for (int g = threadIdx.x; g < m / R; g += T) {
         const int base = g * R, o = pidx(base);
         float2 x[R], z[R];
-        static_for<0, R>([&](auto q) {
-            x[q] = X[o + poff<decltype(q)::value>()];
-            z[q] = Y[o + poff<decltype(q)::value>()];
-        });
+        load_contig<R>(X + o, x);
+        load_contig<R>(Y + o, z);
         dft<R, -1>(x);
         dft<R, -1>(z);
         static_for<0, R / 2>([&](auto i) {
-            o0[base / 2 + i] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
+            o0[spec4_index<LG>(base, i)] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
                                            (x[2 * i + 1].x + Dh) * scale, x[2 * i + 1].y * scale);
-            o1[base / 2 + i] = make_float4((z[2 * i].x + Dh) * scale, z[2 * i].y * scale,
+            o1[spec4_index<LG>(base, i)] = make_float4((z[2 * i].x + Dh) * scale, z[2 * i].y * scale,
                                            (z[2 * i + 1].x + Dh) * scale, z[2 * i + 1].y * scale);
         });
     }

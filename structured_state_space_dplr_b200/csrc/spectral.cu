@@ -124,7 +124,7 @@ k_kspec(const float *__restrict__ K, const float *__restrict__ D, int H, int L, 
         forward_last<LG, T>(s.buf, [&](int base, auto &x) {
             constexpr int R = sizeof(x) / sizeof(float2);
             static_for<0, R / 2>([&](auto i) {
-                out[base / 2 + i] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
+                out[spec4_index<LG>(base, i)] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
                                                 (x[2 * i + 1].x + Dh) * scale, x[2 * i + 1].y * scale);
             });
         });
@@ -229,7 +229,7 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
         fused_middle<LG, T>(s.buf, [&](int base, auto &x) {
             constexpr int R = sizeof(x) / sizeof(float2);
             static_for<0, R / 2>([&](auto i) {
-                const float4 k2 = __ldg(sp + base / 2 + i);
+                const float4 k2 = __ldg(sp + spec4_index<LG>(base, i));
                 x[2 * i] = cmul(x[2 * i], make_float2(k2.x, k2.y));
                 x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k2.z, k2.w));
             });
@@ -302,13 +302,7 @@ k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int
         ta[i] = unit_root(i, N);
         tb[i] = unit_root(i, m);
     }
-    static_for<1, plan_P(LG) - 1>([&](auto sc) {
-        constexpr int s = decltype(sc)::value;
-        constexpr int B = plan_B(LG, s);
-        constexpr int lS = ilog2(B) - plan_lr(LG, s);
-        float2 *t = tws + plan_tw_off(LG, s);
-        for (int i = threadIdx.x; i < B; i += T) t[i] = unit_root(((i & ((1 << lS) - 1)) * (i >> lS)) & (B - 1), B);
-    });
+    build_middle_tables<LG>(tws, threadIdx.x, T);
 
     const int nbp = (Bt + 1) / 2;
     const long long npairs = (long long)H * nbp;
@@ -362,8 +356,8 @@ k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int
             constexpr int R = sizeof(x) / sizeof(float2);
             float4 k0[R / 2], k1[R / 2];
             static_for<0, R / 2>([&](auto i) {
-                k0[i] = __ldg(s0 + base / 2 + i);
-                k1[i] = __ldg(s1 + base / 2 + i);
+                k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
+                k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
             });
             static_for<0, R / 2>([&](auto i) {
                 x[2 * i] = cmul(x[2 * i], make_float2(k0[i].x, k0[i].y));
@@ -398,6 +392,105 @@ k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int
                 y0[t] = r.x;
                 if (has1) y1[t] = r.y;
             });
+        }
+    }
+}
+
+// Same convolution with one half per thread: 2 x threads_for<LG> threads,
+// about half the registers each (twice the warps per SM), the two halves
+// summed through shared memory at the end.
+template <int LG>
+__global__ void __launch_bounds__(2 * threads_for<LG>(), 2)
+k_fftconv_wide(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
+               float *__restrict__ y) {
+    constexpr int m = 1 << LG, TH = threads_for<LG>(), T = 2 * TH, N = 2 * m;
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    extern __shared__ float2 sm[];
+    float2 *b0 = sm, *b1 = sm + padded(m);
+    float2 *tws = b1 + padded(m);
+    float2 *ta = tws + plan_tw_size(LG), *tb = ta + S0;
+    float *stage = reinterpret_cast<float *>(sm + pair_smem_f2<LG>());   // [2][L]
+    const int half = threadIdx.x >= TH, tid = threadIdx.x - half * TH;
+    float2 *buf = half ? b1 : b0;
+
+    for (int i = threadIdx.x; i < S0; i += T) {
+        ta[i] = unit_root(i, N);
+        tb[i] = unit_root(i, m);
+    }
+    build_middle_tables<LG>(tws, threadIdx.x, T);
+
+    const int nbp = (Bt + 1) / 2;
+    const long long npairs = (long long)H * nbp;
+    auto stage_rows = [&](long long pr) {
+        const int h = (int)(pr / nbp), b0r = 2 * (int)(pr % nbp);
+        const bool has1 = (b0r + 1) < Bt;
+        const float *u0 = u + ((size_t)b0r * H + h) * L;
+        const float *u1 = has1 ? u0 + (size_t)H * L : u0;
+        for (int i = threadIdx.x; i < L / 2; i += T) {
+            const int row = i >= L / 4, k = (i - row * (L / 4)) * 4;
+            cp_async16(stage + row * L + k, (row ? u1 : u0) + k, !row || has1);
+        }
+        cp_async_commit();
+    };
+    if ((long long)blockIdx.x < npairs) stage_rows(blockIdx.x);
+
+    for (long long pr = blockIdx.x; pr < npairs; pr += gridDim.x) {
+        const int h = (int)(pr / nbp), bq = 2 * (int)(pr % nbp);
+        const bool has1 = (bq + 1) < Bt;
+        cp_async_wait_all();
+        __syncthreads();
+        for (int j = tid; j < S0; j += TH) {   // first forward pass of this thread's half
+            float2 x[R0];
+            static_for<0, R0>([&](auto p) {
+                const int k = j + p * S0;
+                const float2 v = make_float2(stage[k], stage[L + k]);
+                x[p] = half ? rot<decltype(p)::value, 2 * R0, -1>(v) : v;
+            });
+            dft<R0, -1>(x);
+            const float2 b = tb[j];
+            float2 w = half ? ta[j] : make_float2(1.0f, 0.0f);
+            const int o = pidx(j);
+            static_for<0, R0>([&](auto q) {
+                buf[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+                if constexpr (decltype(q)::value + 1 < R0) w = cmul(w, b);
+            });
+        }
+        __syncthreads();
+        if (pr + gridDim.x < npairs) stage_rows(pr + gridDim.x);
+        forward_middle<LG, TH>(buf, tws, tid);
+        const float4 *sp = reinterpret_cast<const float4 *>(spec + (size_t)h * N + half * m);
+        fused_middle<LG, TH>(buf, [&](int base, auto &x) {
+            constexpr int R = sizeof(x) / sizeof(float2);
+            float4 k[R / 2];
+            static_for<0, R / 2>([&](auto i) { k[i] = __ldg(sp + spec4_index<LG>(base, i)); });
+            static_for<0, R / 2>([&](auto i) {
+                x[2 * i] = cmul(x[2 * i], make_float2(k[i].x, k[i].y));
+                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k[i].z, k[i].w));
+            });
+        }, tid);
+        __syncthreads();
+        inverse_middle<LG, TH>(buf, tws, tid);
+        for (int j = tid; j < S0; j += TH) {   // last inverse pass, natural order back to buf
+            float2 x[R0];
+            const int o = pidx(j);
+            const float2 b = tb[j];
+            float2 w = half ? ta[j] : make_float2(1.0f, 0.0f);
+            static_for<0, R0>([&](auto q) {
+                x[q] = cmulc(buf[o + poff<decltype(q)::value * S0>()], w);
+                if constexpr (decltype(q)::value + 1 < R0) w = cmul(w, b);
+            });
+            dft<R0, +1>(x);
+            static_for<0, R0>([&](auto p) {
+                buf[o + poff<decltype(p)::value * S0>()] = half ? rot<decltype(p)::value, 2 * R0, +1>(x[p]) : x[p];
+            });
+        }
+        __syncthreads();
+        float *y0 = y + ((size_t)bq * H + h) * L;
+        float *y1 = y0 + (size_t)H * L;
+        for (int t = threadIdx.x; t < L; t += T) {
+            const float2 r = cadd(b0[pidx(t)], b1[pidx(t)]);
+            y0[t] = r.x;
+            if (has1) y1[t] = r.y;
         }
     }
 }
@@ -569,14 +662,20 @@ struct ConvKernels {
         const float2 *spec = (const float2 *)ws;
         if constexpr (C == 2 && !TW0G && LG <= 12) {
             // one CTA per row pair, both halves in one CTA
+#if S4_CONV_WIDE
+            auto kern = k_fftconv_wide<LG>;
+            constexpr int TT = 2 * T;
+#else
             auto kern = k_fftconv_pair<LG>;
+            constexpr int TT = T;
+#endif
             constexpr size_t psmem = sizeof(float2) * (size_t)pair_smem_f2<LG>() + 2 * sizeof(float) * (1 << LG);
             int res = 0;
-            cudaError_t e = resident_units(kern, info_pair, 1, T, psmem, &res);
+            cudaError_t e = resident_units(kern, info_pair, 1, TT, psmem, &res);
             if (e != cudaSuccess) return e;
             const long long npairs = (long long)H * ((Bt + 1) / 2);
             const int grid = (long long)res < npairs ? res : (int)npairs;
-            kern<<<grid, T, psmem, st>>>(u, spec, Bt, H, L, y);
+            kern<<<grid, TT, psmem, st>>>(u, spec, Bt, H, L, y);
             return cudaGetLastError();
         }
         const float2 *tw0g = TW0G
@@ -649,6 +748,11 @@ size_t conv_workspace_bytes(int H, int L) {
     return b;
 }
 
+// Convolution kernel for L <= 4096: 0 = both halves per thread
+// (k_fftconv_pair), 1 = one half per thread (k_fftconv_wide).
+#ifndef S4_CONV_WIDE
+#define S4_CONV_WIDE 0
+#endif
 // Longest L whose convolution stages the next row pair in shared memory
 // (cp.async prefetch; costs 8 L bytes of shared memory per CTA).
 #ifndef S4_CONV_STAGE_MAX_L
