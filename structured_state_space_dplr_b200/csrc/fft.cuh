@@ -457,19 +457,20 @@ __device__ __forceinline__ void inverse_middle_x2(float2 *b0, float2 *b1, const 
 }
 // last forward pass, product with the two spectra (mul(pos0, x, z)), first
 // inverse pass, for both buffers
-template <int LG, int T, class Mul>
-__device__ __forceinline__ void fused_middle_x2(float2 *b0, float2 *b1, Mul &&mul) {
+template <int LG, int T, class Fetch, class Mul>
+__device__ __forceinline__ void fused_middle_x2(float2 *b0, float2 *b1, Fetch &&fetch, Mul &&mul) {
     constexpr int lr = plan_lr(LG, plan_P(LG) - 1), R = 1 << lr;
     constexpr int G = (1 << LG) / R;
     for (int g = threadIdx.x; g < G; g += T) {
         const int base = g * R;
         const int o = pidx(base);
+        auto spec = fetch(base);   // issued before the transforms that hide its latency
         float2 x[R], z[R];
         load_contig<R>(b0 + o, x);
         load_contig<R>(b1 + o, z);
         dft<R, -1>(x);
         dft<R, -1>(z);
-        mul(base, x, z);
+        mul(spec, x, z);
         dft<R, +1>(x);
         dft<R, +1>(z);
         store_contig<R>(b0 + o, x);

@@ -352,18 +352,21 @@ k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int
         forward_middle_x2<LG, T>(b0, b1, tws);
         const float4 *s0 = reinterpret_cast<const float4 *>(spec + (size_t)h * N);
         const float4 *s1 = s0 + m / 2;
-        fused_middle_x2<LG, T>(b0, b1, [&](int base, auto &x, auto &z) {
-            constexpr int R = sizeof(x) / sizeof(float2);
-            float4 k0[R / 2], k1[R / 2];
-            static_for<0, R / 2>([&](auto i) {
-                k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
-                k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
+        constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
+        struct SpecWords { float4 k0[RL / 2], k1[RL / 2]; };
+        fused_middle_x2<LG, T>(b0, b1, [&](int base) {
+            SpecWords w;
+            static_for<0, RL / 2>([&](auto i) {
+                w.k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
+                w.k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
             });
-            static_for<0, R / 2>([&](auto i) {
-                x[2 * i] = cmul(x[2 * i], make_float2(k0[i].x, k0[i].y));
-                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k0[i].z, k0[i].w));
-                z[2 * i] = cmul(z[2 * i], make_float2(k1[i].x, k1[i].y));
-                z[2 * i + 1] = cmul(z[2 * i + 1], make_float2(k1[i].z, k1[i].w));
+            return w;
+        }, [&](const SpecWords &w, auto &x, auto &z) {
+            static_for<0, RL / 2>([&](auto i) {
+                x[2 * i] = cmul(x[2 * i], make_float2(w.k0[i].x, w.k0[i].y));
+                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(w.k0[i].z, w.k0[i].w));
+                z[2 * i] = cmul(z[2 * i], make_float2(w.k1[i].x, w.k1[i].y));
+                z[2 * i + 1] = cmul(z[2 * i + 1], make_float2(w.k1[i].z, w.k1[i].w));
             });
         });
         __syncthreads();
