@@ -141,6 +141,30 @@ def physical_gpu(local_rank):
     return str(local_rank)
 
 
+# ------------------------------------------------------------ multi-rank ----
+def rank_shard(cfg, rank, world):
+    """Weak scaling by channel: rank r owns channels [r H, (r + 1) H) of a
+    layer with world * H channels (its inputs drawn with seed r). The
+    channels are independent SSMs, so no data crosses ranks."""
+    H = s4inputs.CONFIGS[cfg]["H"]
+    return {"seed": rank, "channel_begin": rank * H, "channel_end": (rank + 1) * H}
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of per-rank timings (all ranks get the result)."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(elements_per_rank_step, world, steps, max_ms):
+    """Whole-job elements per second: all ranks' elements over the slowest rank's time."""
+    return elements_per_rank_step * world * steps / (max_ms * 1e-3)
+
+
 # ------------------------------------------------------------- workload -----
 def workload(cfg, seed):
     c = s4inputs.CONFIGS[cfg]
@@ -172,7 +196,8 @@ def run_gpu(args, rank, world, local_rank):
                                 device_id=dev)
 
     cfg = args.config
-    inp, c = workload(cfg, seed=rank)
+    shard = rank_shard(cfg, rank, world)
+    inp, c = workload(cfg, seed=shard["seed"])
     H, L, Bt = c["H"], c["L"], c["Bt"]
     alg = algorithmic(c)
     names = ["Lambda", "P", "Q", "B", "C", "log_dt", "D", "u"]
@@ -300,18 +325,18 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
 
-    times = torch.tensor([ms, e2e_ms] + stage, device=dev, dtype=torch.float64)
+    times = max_over_ranks([ms, e2e_ms] + stage, dist, dev)
     if dist is not None:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
         dist.barrier()
+        del gen_graphs, conv_graphs
         dist.destroy_process_group()
-    ms, e2e_ms = float(times[0]), float(times[1])
-    stage = [float(x) for x in times[2:]]
+    ms, e2e_ms = times[0], times[1]
+    stage = times[2:]
     if rank != 0:
         return None
 
     hbm, sm_max_mhz, peak_src = peaks()
-    total_elems = alg["elements"] * world * args.steps
+    total_elems = alg["elements"] * world * args.steps   # job_throughput() numerator
     conv_s = stage[1] * 1e-3
     conv_gbs = alg["conv_bytes"] / conv_s / 1e9
     cauchy_tflops = alg["cauchy_flop"] / (stage[2] * 1e-3) / 1e12
@@ -319,7 +344,7 @@ def run_gpu(args, rank, world, local_rank):
     traffic = recorded_traffic() if cfg == 2 else None
     line = {
         "metric": METRIC,
-        "value": total_elems / (ms * 1e-3),
+        "value": job_throughput(alg["elements"], world, args.steps, ms),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -344,7 +369,8 @@ def run_gpu(args, rank, world, local_rank):
                    "unit": "TFLOP/s", "frac": cauchy_tflops / fp32_peak,
                    "peak_derivation": f"{SM_COUNT} SM x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max_mhz:.0f} MHz",
                    "algorithmic_flop": alg["cauchy_flop"]},
-        "e2e": None if args.no_e2e else {"value": total_elems / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": None if args.no_e2e else {"value": job_throughput(alg["elements"], world, args.steps, e2e_ms),
+                                         "unit": UNIT,
                                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,

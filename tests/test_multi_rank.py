@@ -1,0 +1,55 @@
+"""bench.py's multi-rank logic on CPU with the gloo backend (world size 2):
+disjoint channel shards, distinct seeds, max-over-ranks timing and the
+whole-job throughput computed from it."""
+import json
+import os
+import socket
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    shard = bench.rank_shard(2, rank, world)
+    # each rank reports its own timings; every rank must see the max
+    mine = [10.0 + rank, 5.0 - rank, 1.5 * (rank + 1)]
+    got = bench.max_over_ranks(mine, dist, "cpu")
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"shard": shard, "max": got}, f)
+
+
+def test_two_gloo_ranks(tmp_path):
+    import torch.multiprocessing as mp
+    world = 2
+    port = _free_port()
+    mp.start_processes(_worker, args=(world, port, str(tmp_path)), nprocs=world, start_method="spawn")
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    shards = [r["shard"] for r in res]
+    assert shards[0]["seed"] != shards[1]["seed"]
+    assert shards[0]["channel_end"] == shards[1]["channel_begin"]      # disjoint, adjacent slices
+    assert res[0]["max"] == res[1]["max"] == [11.0, 5.0, 3.0]
+
+
+def test_job_throughput_is_total_over_slowest():
+    sys.path.insert(0, ROOT)
+    import bench
+    # 2 ranks x 3 steps x 1000 elements in 2 ms (the slower rank) -> 3e6 elements/s
+    assert bench.job_throughput(1000, 2, 3, 2.0) == pytest.approx(3.0e6)
+    assert bench.max_over_ranks([1, 2]) == [1.0, 2.0]
