@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libs4dplr.so")
 SOURCES = ["api.cu", "cauchy.cu", "kgen.cu", "spectral.cu", "s4d.cu", "decode.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "fft.cuh", "cauchy.cuh", "launch.h"]
+HEADERS = ["common.cuh", "fft.cuh", "cauchy.cuh", "pairs.cuh", "launch.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -186,14 +186,21 @@ s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P,
                           unsigned *d_flags, cudaStream_t stream) {
     if (D == nullptr) return S4_ERR_INVALID_ARG;
     s4_status s = conv_checks(u, Bt, H, L, y, workspace, workspace_bytes);
+    if (s == S4_OK) s = dplr_checks(Lambda, P, Q, B, C, log_dt, H, Nh, L, K);
+    if (s == S4_OK) s = prepare_checks(K, D, H, L, workspace, workspace_bytes);
     if (s != S4_OK) return s;
-    const size_t nb = (size_t)Bt * H * L * sizeof(float);
-    if (overlap(y, nb, K, (size_t)H * L * sizeof(float)) || overlap(y, nb, D, (size_t)H * sizeof(float)))
+    const size_t nb = (size_t)Bt * H * L * sizeof(float), kb = (size_t)H * L * sizeof(float);
+    if (overlap(y, nb, K, kb) || overlap(y, nb, D, (size_t)H * sizeof(float)) || overlap(u, nb, K, kb))
         return S4_ERR_INVALID_ARG;
-    s = s4_kernel_dplr_prepare(Lambda, P, Q, B, C, log_dt, D, H, Nh, L, K, workspace, workspace_bytes, d_flags,
-                               stream);
-    if (s != S4_OK) return s;
-    return cuda_status(s4::launch_fftconv(u, workspace, Bt, H, L, y, stream));
+    for (const void *p : {(const void *)Lambda, (const void *)P, (const void *)Q, (const void *)B,
+                          (const void *)C})
+        if (overlap(workspace, workspace_bytes, p, (size_t)H * Nh * sizeof(s4_c32)) ||
+            overlap(y, nb, p, (size_t)H * Nh * sizeof(s4_c32)))
+            return S4_ERR_INVALID_ARG;
+    cudaError_t e = s4::launch_kgen((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q, (const float2 *)B,
+                                    (const float2 *)C, log_dt, D, H, Nh, L, K, workspace, d_flags, stream);
+    if (e == cudaSuccess) e = s4::launch_fftconv(u, workspace, Bt, H, L, y, stream);
+    return cuda_status(e);
 }
 
 s4_status s4d_kernel_vandermonde(const s4_c32 *A, const s4_c32 *B, const s4_c32 *C, const float *log_dt,

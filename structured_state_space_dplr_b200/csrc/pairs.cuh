@@ -1,0 +1,315 @@
+// pairs.cuh -- the two units of work of the forward pass for L <= 4096, as
+// device functions shared by the standalone kernels and the persistent
+// forward kernel:
+//
+//   kgen_channel : one channel's kernel K and the spectrum of the zero-padded
+//                  K + D delta_0 ("The S4 kernel, from scratch", §4, §5):
+//                  Cauchy/Woodbury generating function written straight into
+//                  the inverse transform's digit-reversed input, length-L
+//                  inverse transform -> K, whose last pass feeds the first
+//                  pass of the length-2L forward transform;
+//   conv_pair    : one row pair's causal convolution y = K * u + D u ([S4K]
+//                  §5 fft_conv) with the spectrum above.
+//
+// Both run on one CTA of pair_threads<LG>() threads and use the same shared
+// memory layout: two padded m-point buffers (the two halves of the 2L
+// transform: rank 0 holds frequencies 2f, rank 1 frequencies 2f + 1), the
+// middle-pass base twiddles, the first-pass tables a_j = W_2L^j, b_j = W_L^j,
+// and an auxiliary area holding either the staged input rows (convolution)
+// or the per-mode Cauchy constants (generation).
+#pragma once
+#include "cauchy.cuh"
+#include "fft.cuh"
+
+namespace s4 {
+
+template <int LG>
+__host__ __device__ constexpr int pair_threads() { return (1 << LG) / 16 < 32 ? 32 : (1 << LG) / 16; }
+template <int LG>
+__host__ __device__ constexpr int pair_s0() { return (1 << LG) >> plan_lr(LG, 0); }
+// float2 words before the auxiliary area (kept even: the area is 16-byte aligned)
+template <int LG>
+__host__ __device__ constexpr int pair_core_f2() {
+    return (2 * padded(1 << LG) + plan_tw_size(LG) + 2 * pair_s0<LG>() + 1) / 2 * 2;
+}
+template <int LG>
+__host__ __device__ constexpr size_t pair_smem_bytes(int Nh) {
+    return sizeof(float2) * ((size_t)pair_core_f2<LG>() + ((1 << LG) > 6 * Nh ? (1 << LG) : 6 * Nh));
+}
+
+struct PairSmem {
+    float2 *b0, *b1, *tws, *ta, *tb;
+    float *stage;   // [2][L] input rows (convolution)
+    float4 *sp;     // [3 Nh] Cauchy constants (generation)
+};
+
+template <int LG>
+__device__ __forceinline__ PairSmem pair_carve(float2 *sm) {
+    constexpr int m = 1 << LG;
+    PairSmem s;
+    s.b0 = sm;
+    s.b1 = sm + padded(m);
+    s.tws = s.b1 + padded(m);
+    s.ta = s.tws + plan_tw_size(LG);
+    s.tb = s.ta + pair_s0<LG>();
+    s.stage = reinterpret_cast<float *>(sm + pair_core_f2<LG>());
+    s.sp = reinterpret_cast<float4 *>(sm + pair_core_f2<LG>());
+    return s;
+}
+
+template <int LG>
+__device__ __forceinline__ void pair_tables(const PairSmem &s) {
+    constexpr int m = 1 << LG, T = pair_threads<LG>();
+    for (int i = threadIdx.x; i < pair_s0<LG>(); i += T) {
+        s.ta[i] = unit_root(i, 2 * m);
+        s.tb[i] = unit_root(i, m);
+    }
+    build_middle_tables<LG>(s.tws, threadIdx.x, T);
+}
+
+// ------------------------------------------------------------ async copy --
+__device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+// 16-byte global -> shared copy (zero-filled when !valid; nothing is read then)
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Row pair pr = (channel h, rows 2 bp and 2 bp + 1) of u [Bt, H, L].
+struct RowPair {
+    int h, b0;
+    bool has1;
+};
+__device__ __forceinline__ RowPair row_pair(long long pr, int Bt) {
+    const int nbp = (Bt + 1) / 2;
+    RowPair r;
+    r.h = (int)(pr / nbp);
+    r.b0 = 2 * (int)(pr % nbp);
+    r.has1 = r.b0 + 1 < Bt;
+    return r;
+}
+
+// Both rows of pair pr into the stage (cp.async, then committed).
+template <int LG>
+__device__ __forceinline__ void pair_stage_rows(const PairSmem &s, const float *__restrict__ u, int Bt, int H,
+                                                long long pr) {
+    constexpr int L = 1 << LG, T = pair_threads<LG>();
+    const RowPair r = row_pair(pr, Bt);
+    const float *u0 = u + ((size_t)r.b0 * H + r.h) * L;
+    const float *u1 = r.has1 ? u0 + (size_t)H * L : u0;
+    for (int i = threadIdx.x; i < L / 2; i += T) {   // 16-byte chunks, L/4 per row
+        const int row = i >= L / 4, k = (i - row * (L / 4)) * 4;
+        cp_async16(s.stage + row * L + k, (row ? u1 : u0) + k, !row || r.has1);
+    }
+    cp_async_commit();
+}
+
+// ------------------------------------------------------------ convolution --
+// Convolution of the staged row pair (stage ready, all threads synced) with
+// the spectrum spec_h (layout of spec4_index, rank 0 then rank 1). After the
+// first pass, after_first() runs (the stage is free then). COHERENT reads the
+// spectrum through L2 only (it was written earlier in the same launch).
+template <int LG, bool COHERENT, class AfterFirst>
+__device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__restrict__ spec_h, float *y0,
+                                          float *y1, bool has1, AfterFirst &&after_first) {
+    constexpr int m = 1 << LG, L = m, T = pair_threads<LG>();
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    float2 *b0 = s.b0, *b1 = s.b1;
+    const float *stage = s.stage;
+    // ---- first forward pass, both halves
+    for (int j = threadIdx.x; j < S0; j += T) {
+        float2 x[R0], z[R0];
+        static_for<0, R0>([&](auto p) {
+            const int k = j + p * S0;
+            const float2 v = make_float2(stage[k], stage[L + k]);
+            x[p] = v;
+            z[p] = rot<decltype(p)::value, 2 * R0, -1>(v);
+        });
+        dft<R0, -1>(x);
+        dft<R0, -1>(z);
+        const float2 a = s.ta[j], b = s.tb[j];
+        float2 w = b, v = a;
+        const int o = pidx(j);
+        b0[o] = x[0];
+        b1[o] = cmul(z[0], a);
+        static_for<1, R0>([&](auto q) {
+            v = cmul(v, b);
+            b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+            b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], v);
+            w = cmul(w, b);
+        });
+    }
+    __syncthreads();
+    after_first();
+    forward_middle_x2<LG, T>(b0, b1, s.tws);
+    const float4 *s0 = reinterpret_cast<const float4 *>(spec_h);
+    const float4 *s1 = s0 + m / 2;
+    constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
+    struct SpecWords { float4 k0[RL / 2], k1[RL / 2]; };
+    fused_middle_x2<LG, T>(b0, b1, [&](int base) {
+        SpecWords w;
+        static_for<0, RL / 2>([&](auto i) {
+            if constexpr (COHERENT) {
+                w.k0[i] = __ldcg(s0 + spec4_index<LG>(base, i));
+                w.k1[i] = __ldcg(s1 + spec4_index<LG>(base, i));
+            } else {
+                w.k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
+                w.k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
+            }
+        });
+        return w;
+    }, [&](const SpecWords &w, auto &x, auto &z) {
+        static_for<0, RL / 2>([&](auto i) {
+            x[2 * i] = cmul(x[2 * i], make_float2(w.k0[i].x, w.k0[i].y));
+            x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(w.k0[i].z, w.k0[i].w));
+            z[2 * i] = cmul(z[2 * i], make_float2(w.k1[i].x, w.k1[i].y));
+            z[2 * i + 1] = cmul(z[2 * i + 1], make_float2(w.k1[i].z, w.k1[i].w));
+        });
+    });
+    __syncthreads();
+    inverse_middle_x2<LG, T>(b0, b1, s.tws);
+    // ---- last inverse pass of both halves + their sum, straight to y
+    for (int j = threadIdx.x; j < S0; j += T) {
+        float2 x[R0], z[R0];
+        const int o = pidx(j);
+        const float2 a = s.ta[j], b = s.tb[j];
+        float2 w = b, v = a;
+        x[0] = b0[o];
+        z[0] = cmulc(b1[o], a);
+        static_for<1, R0>([&](auto q) {
+            v = cmul(v, b);
+            x[q] = cmulc(b0[o + poff<decltype(q)::value * S0>()], w);
+            z[q] = cmulc(b1[o + poff<decltype(q)::value * S0>()], v);
+            w = cmul(w, b);
+        });
+        dft<R0, +1>(x);
+        dft<R0, +1>(z);
+        static_for<0, R0>([&](auto p) {
+            const float2 r = cadd(x[p], rot<decltype(p)::value, 2 * R0, +1>(z[p]));
+            const int t = j + p * S0;
+            y0[t] = r.x;
+            if (has1) y1[t] = r.y;
+        });
+    }
+}
+
+// ------------------------------------------------------------- generation --
+// Channel h: K[h, :] and spec_h (2L complex, spec4_index layout, scaled by
+// 1/2L, with D added). Tables built, all threads synced on entry.
+template <int LG>
+__device__ __forceinline__ void kgen_channel(const PairSmem &s, const float2 *__restrict__ Lambda,
+                                             const float2 *__restrict__ P, const float2 *__restrict__ Q,
+                                             const float2 *__restrict__ B, const float2 *__restrict__ Cc,
+                                             const float *__restrict__ log_dt, const float *__restrict__ D,
+                                             int Nh, int h, float *__restrict__ K, float2 *__restrict__ spec_h,
+                                             unsigned *__restrict__ flags) {
+    constexpr int m = 1 << LG, L = m, T = pair_threads<LG>(), N = 2 * m;
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0, NP = plan_P(LG);
+    constexpr int F = 4;   // frequencies per thread per round
+    float2 *X = s.b0, *Y = s.b1;
+    float4 *sp = s.sp;
+    cauchy_stage_modes(Lambda, P, Q, B, Cc, h, Nh, sp, flags, threadIdx.x, T);
+    __syncthreads();
+
+    // ---- A: generating function -> X at digit-reversed positions (with mirror)
+    const float ldt = __ldg(log_dt + h);
+    const float inv_dt = expf(-ldt);
+    bool bad = false;
+    for (int f0 = 0; f0 < L / 2; f0 += T * F) {
+        int j[F], jj[F];
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+            j[f] = f0 + f * T + threadIdx.x;
+            jj[f] = j[f] < L / 2 ? j[f] : 0;
+        }
+        float2 kh[F];
+        cauchy_eval<F>(sp, Nh, jj, L, inv_dt, kh);
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+            if (j[f] < L / 2) {
+                bad |= !(isfinite(kh[f].x) && isfinite(kh[f].y));
+                if (j[f] == 0) {
+                    X[pidx(0)] = make_float2(kh[f].x, 0.0f);
+                } else {
+                    X[pidx(digrev_inv<LG>(j[f]))] = kh[f];
+                    X[pidx(digrev_inv<LG>(L - j[f]))] = cconj(kh[f]);
+                }
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        const float nyq = cauchy_nyquist(sp, Nh, expf(ldt), L);
+        bad |= !isfinite(nyq);
+        X[pidx(digrev_inv<LG>(L / 2))] = make_float2(nyq, 0.0f);
+    }
+    if (flags != nullptr && __any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0)
+        atomicOr(flags, S4_FLAG_NONFINITE);
+    __syncthreads();
+
+    // ---- B: inverse transform, passes P-1 .. 1
+    dit_pass<LG, NP - 1, +1, T>(X, s.tws);
+    __syncthreads();
+    inverse_middle<LG, T>(X, s.tws);
+
+    // ---- B/C: last inverse pass -> K (stored), first forward pass of both halves
+    float *Kh = K + (size_t)h * L;
+    for (int j = threadIdx.x; j < S0; j += T) {
+        const int o = pidx(j);
+        const float2 a = s.ta[j], b = s.tb[j];
+        float2 x[R0], z[R0];
+        {
+            float2 w = b;
+            x[0] = X[o];
+            static_for<1, R0>([&](auto q) {
+                x[q] = cmulc(X[o + poff<decltype(q)::value * S0>()], w);
+                w = cmul(w, b);
+            });
+        }
+        dft<R0, +1>(x);
+        static_for<0, R0>([&](auto p) {
+            const float k = x[p].x;   // K is real: the imaginary part is rounding
+            Kh[j + p * S0] = k;
+            x[p] = make_float2(k, 0.0f);
+            z[p] = rot<decltype(p)::value, 2 * R0, -1>(x[p]);
+        });
+        dft<R0, -1>(x);
+        dft<R0, -1>(z);
+        float2 w = b, v = a;
+        X[o] = x[0];
+        Y[o] = cmul(z[0], a);
+        static_for<1, R0>([&](auto q) {
+            v = cmul(v, b);
+            X[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+            Y[o + poff<decltype(q)::value * S0>()] = cmul(z[q], v);
+            w = cmul(w, b);
+        });
+    }
+    __syncthreads();
+
+    // ---- C: forward passes 1 .. P-2, last pass -> (spectrum + D) / 2L
+    forward_middle_x2<LG, T>(X, Y, s.tws);
+    const float Dh = D != nullptr ? __ldg(D + h) : 0.0f;
+    const float scale = 1.0f / (float)N;
+    constexpr int lr = plan_lr(LG, NP - 1), R = 1 << lr;
+    float4 *o0 = reinterpret_cast<float4 *>(spec_h);
+    float4 *o1 = o0 + m / 2;
+    for (int g = threadIdx.x; g < m / R; g += T) {
+        const int base = g * R, o = pidx(base);
+        float2 x[R], z[R];
+        load_contig<R>(X + o, x);
+        load_contig<R>(Y + o, z);
+        dft<R, -1>(x);
+        dft<R, -1>(z);
+        static_for<0, R / 2>([&](auto i) {
+            o0[spec4_index<LG>(base, i)] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
+                                                       (x[2 * i + 1].x + Dh) * scale, x[2 * i + 1].y * scale);
+            o1[spec4_index<LG>(base, i)] = make_float4((z[2 * i].x + Dh) * scale, z[2 * i].y * scale,
+                                                       (z[2 * i + 1].x + Dh) * scale, z[2 * i + 1].y * scale);
+        });
+    }
+}
+
+}  // namespace s4

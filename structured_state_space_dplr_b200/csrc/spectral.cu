@@ -25,6 +25,7 @@
 
 #include "fft.cuh"
 #include "launch.h"
+#include "pairs.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -67,15 +68,6 @@ __global__ void k_tw0_init(float2 *__restrict__ tw0g, int C) {
 }
 
 // ------------------------------------------------------ async copy, cluster --
-__device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
-// 16-byte global -> shared copy (zero-filled when !valid; nothing is read then)
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 // cluster barrier halves: release/acquire hand off shared-memory data between
 // the CTAs; a relaxed arrive only says "I am done reading your memory" (every
 // value read was consumed before the arrive issues)
@@ -274,128 +266,25 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
 
 // ------------------------------------------------------- fftconv, one CTA --
 // L <= 4096: one CTA per row pair holds both halves of the length-2L
-// transform (rank 0: frequencies 2f, rank 1: 2f + 1), m = L points each.
-// Thread j owns group j of both halves in every pass, so the first pass
-// reads its input once for both halves, and the last inverse pass adds the
-// two halves -- the combine of the split transform -- in registers and
-// stores y directly. First-pass twiddles follow a recurrence from two small
-// tables: W_m^{j q} = b_j^q (rank 0) and W_N^{j (2q+1)} = a_j b_j^q (rank 1),
-// a_j = W_N^j, b_j = W_m^j.
+// transform; see conv_pair (pairs.cuh). Persistent: the next row pair is
+// staged with cp.async while the current one is transformed.
 template <int LG>
-__host__ __device__ constexpr int pair_smem_f2() {
-    return (2 * padded(1 << LG) + plan_tw_size(LG) + 2 * ((1 << LG) >> plan_lr(LG, 0)) + 1) / 2 * 2;
-}
-
-template <int LG>
-__global__ void __launch_bounds__(threads_for<LG>(), 2)
+__global__ void __launch_bounds__(pair_threads<LG>(), 2)
 k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
                float *__restrict__ y) {
-    constexpr int m = 1 << LG, T = threads_for<LG>(), N = 2 * m;
-    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     extern __shared__ float2 sm[];
-    float2 *b0 = sm, *b1 = sm + padded(m);
-    float2 *tws = b1 + padded(m);
-    float2 *ta = tws + plan_tw_size(LG), *tb = ta + S0;
-    float *stage = reinterpret_cast<float *>(sm + pair_smem_f2<LG>());   // [2][L]
-
-    for (int i = threadIdx.x; i < S0; i += T) {
-        ta[i] = unit_root(i, N);
-        tb[i] = unit_root(i, m);
-    }
-    build_middle_tables<LG>(tws, threadIdx.x, T);
-
-    const int nbp = (Bt + 1) / 2;
-    const long long npairs = (long long)H * nbp;
-    auto stage_rows = [&](long long pr) {
-        const int h = (int)(pr / nbp), b0r = 2 * (int)(pr % nbp);
-        const bool has1 = (b0r + 1) < Bt;
-        const float *u0 = u + ((size_t)b0r * H + h) * L;
-        const float *u1 = has1 ? u0 + (size_t)H * L : u0;
-        for (int i = threadIdx.x; i < L / 2; i += T) {
-            const int row = i >= L / 4, k = (i - row * (L / 4)) * 4;
-            cp_async16(stage + row * L + k, (row ? u1 : u0) + k, !row || has1);
-        }
-        cp_async_commit();
-    };
-    if ((long long)blockIdx.x < npairs) stage_rows(blockIdx.x);
-
+    const PairSmem s = pair_carve<LG>(sm);
+    pair_tables<LG>(s);
+    const long long npairs = (long long)H * ((Bt + 1) / 2);
+    if ((long long)blockIdx.x < npairs) pair_stage_rows<LG>(s, u, Bt, H, blockIdx.x);
     for (long long pr = blockIdx.x; pr < npairs; pr += gridDim.x) {
-        const int h = (int)(pr / nbp), bq = 2 * (int)(pr % nbp);
-        const bool has1 = (bq + 1) < Bt;
+        const RowPair r = row_pair(pr, Bt);
         cp_async_wait_all();
         __syncthreads();   // stage ready; previous pair's buffers no longer read
-        // ---- first forward pass, both halves
-        for (int j = threadIdx.x; j < S0; j += T) {
-            float2 x[R0], z[R0];
-            static_for<0, R0>([&](auto p) {
-                const int k = j + p * S0;
-                const float2 v = make_float2(stage[k], stage[L + k]);
-                x[p] = v;
-                z[p] = rot<decltype(p)::value, 2 * R0, -1>(v);
-            });
-            dft<R0, -1>(x);
-            dft<R0, -1>(z);
-            const float2 a = ta[j], b = tb[j];
-            float2 w = b, v = a;
-            const int o = pidx(j);
-            b0[o] = x[0];
-            b1[o] = cmul(z[0], a);
-            static_for<1, R0>([&](auto q) {
-                v = cmul(v, b);
-                b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
-                b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], v);
-                w = cmul(w, b);
-            });
-        }
-        __syncthreads();
-        if (pr + gridDim.x < npairs) stage_rows(pr + gridDim.x);   // stage is free again
-        forward_middle_x2<LG, T>(b0, b1, tws);
-        const float4 *s0 = reinterpret_cast<const float4 *>(spec + (size_t)h * N);
-        const float4 *s1 = s0 + m / 2;
-        constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
-        struct SpecWords { float4 k0[RL / 2], k1[RL / 2]; };
-        fused_middle_x2<LG, T>(b0, b1, [&](int base) {
-            SpecWords w;
-            static_for<0, RL / 2>([&](auto i) {
-                w.k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
-                w.k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
-            });
-            return w;
-        }, [&](const SpecWords &w, auto &x, auto &z) {
-            static_for<0, RL / 2>([&](auto i) {
-                x[2 * i] = cmul(x[2 * i], make_float2(w.k0[i].x, w.k0[i].y));
-                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(w.k0[i].z, w.k0[i].w));
-                z[2 * i] = cmul(z[2 * i], make_float2(w.k1[i].x, w.k1[i].y));
-                z[2 * i + 1] = cmul(z[2 * i + 1], make_float2(w.k1[i].z, w.k1[i].w));
-            });
+        float *y0 = y + ((size_t)r.b0 * H + r.h) * L;
+        conv_pair<LG, false>(s, spec + (size_t)r.h * 2 * L, y0, y0 + (size_t)H * L, r.has1, [&] {
+            if (pr + gridDim.x < npairs) pair_stage_rows<LG>(s, u, Bt, H, pr + gridDim.x);
         });
-        __syncthreads();
-        inverse_middle_x2<LG, T>(b0, b1, tws);
-        // ---- last inverse pass of both halves + their sum, straight to y
-        float *y0 = y + ((size_t)bq * H + h) * L;
-        float *y1 = y0 + (size_t)H * L;
-        for (int j = threadIdx.x; j < S0; j += T) {
-            float2 x[R0], z[R0];
-            const int o = pidx(j);
-            const float2 a = ta[j], b = tb[j];
-            float2 w = b, v = a;
-            x[0] = b0[o];
-            z[0] = cmulc(b1[o], a);
-            static_for<1, R0>([&](auto q) {
-                v = cmul(v, b);
-                x[q] = cmulc(b0[o + poff<decltype(q)::value * S0>()], w);
-                z[q] = cmulc(b1[o + poff<decltype(q)::value * S0>()], v);
-                w = cmul(w, b);
-            });
-            dft<R0, +1>(x);
-            dft<R0, +1>(z);
-            static_for<0, R0>([&](auto p) {
-                const float2 r = cadd(x[p], rot<decltype(p)::value, 2 * R0, +1>(z[p]));
-                const int t = j + p * S0;
-                y0[t] = r.x;
-                if (has1) y1[t] = r.y;
-            });
-        }
     }
 }
 
@@ -412,7 +301,7 @@ k_fftconv_wide(const float *__restrict__ u, const float2 *__restrict__ spec, int
     float2 *b0 = sm, *b1 = sm + padded(m);
     float2 *tws = b1 + padded(m);
     float2 *ta = tws + plan_tw_size(LG), *tb = ta + S0;
-    float *stage = reinterpret_cast<float *>(sm + pair_smem_f2<LG>());   // [2][L]
+    float *stage = reinterpret_cast<float *>(sm + pair_core_f2<LG>());   // [2][L]
     const int half = threadIdx.x >= TH, tid = threadIdx.x - half * TH;
     float2 *buf = half ? b1 : b0;
 
@@ -672,7 +561,7 @@ struct ConvKernels {
             auto kern = k_fftconv_pair<LG>;
             constexpr int TT = T;
 #endif
-            constexpr size_t psmem = sizeof(float2) * (size_t)pair_smem_f2<LG>() + 2 * sizeof(float) * (1 << LG);
+            constexpr size_t psmem = pair_smem_bytes<LG>(0);
             int res = 0;
             cudaError_t e = resident_units(kern, info_pair, 1, TT, psmem, &res);
             if (e != cudaSuccess) return e;
