@@ -48,6 +48,7 @@ NOMINAL_SM_MHZ = 1965.0
 # scaled denominator (2 mul, 1 add/fma, 2 fma for |q|^2 -> 8 flop incl. the
 # two products by 1/|q|^2) and four complex Cauchy sums as 16 FMAs (32 flop)
 CAUCHY_FLOP_PER_TERM = 40
+VANDERMONDE_FLOP_PER_TERM = 4
 KERNEL_SOURCES = ["common.cuh", "fft.cuh", "spectral.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fftconv_h256_l4096_b16_traffic.txt")
 
@@ -176,8 +177,11 @@ def algorithmic(c):
     return {
         "elements": Bt * H * L,
         # fused convolution: read u, write y, read the kernel spectrum (H x 2L complex)
-        "conv_bytes": 8 * Bt * H * L + 16 * H * L + 4 * H,
-        "cauchy_flop": CAUCHY_FLOP_PER_TERM * H * (L // 2) * Nh,
+        "conv_bytes": 8 * Bt * H * L + 16 * H * L,
+        # Cauchy sums: per (channel, frequency j < L/2, mode pair); Vandermonde:
+        # 2 FMAs per (channel, k, stored mode)
+        "kernel_flop": (VANDERMONDE_FLOP_PER_TERM * H * L * Nh if c["kind"] == "s4d"
+                        else CAUCHY_FLOP_PER_TERM * H * (L // 2) * Nh),
     }
 
 
@@ -200,7 +204,8 @@ def run_gpu(args, rank, world, local_rank):
     inp, c = workload(cfg, seed=shard["seed"])
     H, L, Bt = c["H"], c["L"], c["Bt"]
     alg = algorithmic(c)
-    names = ["Lambda", "P", "Q", "B", "C", "log_dt", "D", "u"]
+    s4d = c["kind"] == "s4d"
+    names = (["A", "B", "C"] if s4d else ["Lambda", "P", "Q", "B", "C"]) + ["log_dt", "D", "u"]
     base = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(dev) for k in names}
     ws_bytes = s4.fft_conv_workspace_size(H, L)
     # rotating input sets: consecutive steps touch different memory, together
@@ -216,25 +221,34 @@ def run_gpu(args, rank, world, local_rank):
         sets.append(s)
     flags = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def step(s, ev=None):
-        # the forward: K and its convolution spectrum (s4_kernel_dplr_prepare),
-        # then the convolution (s4_fft_conv_apply); = s4_forward_dplr
-        if ev is not None:
-            ev[0].record()
-        s4.kernel_dplr_prepare(s["Lambda"], s["P"], s["Q"], s["B"], s["C"], s["log_dt"], s["D"], L,
-                               K=s["K"], workspace=s["ws"], flags=flags)
-        if ev is not None:
-            ev[1].record()
+    # the forward = stage 1 (kernel K and its convolution spectrum) + stage 2
+    # (the convolution, s4_fft_conv_apply)
+    def gen_stage(s):
+        if s4d:   # S4D: Vandermonde kernel, then the spectrum of K + D delta_0
+            s4.s4d_kernel_vandermonde(s["A"], s["B"], s["C"], s["log_dt"], L, out=s["K"], flags=flags)
+            s4.fft_conv_prepare(s["K"], s["D"], workspace=s["ws"])
+        else:     # S4 DPLR: s4_kernel_dplr_prepare
+            s4.kernel_dplr_prepare(s["Lambda"], s["P"], s["Q"], s["B"], s["C"], s["log_dt"], s["D"], L,
+                                   K=s["K"], workspace=s["ws"], flags=flags)
+
+    def conv_stage(s):
         s4.fft_conv_apply(s["u"], s["ws"], out=s["y"])
-        if ev is not None:
-            ev[2].record()
 
-    def cauchy_only(s):
-        s4.dplr_spectrum(s["Lambda"], s["P"], s["Q"], s["B"], s["C"], s["log_dt"], L, out=s["K"])
+    def kernel_only(s):   # the FP32-bound kernel stage alone: Cauchy sums or Vandermonde
+        if s4d:
+            s4.s4d_kernel_vandermonde(s["A"], s["B"], s["C"], s["log_dt"], L, out=s["K"])
+        else:
+            s4.dplr_spectrum(s["Lambda"], s["P"], s["Q"], s["B"], s["C"], s["log_dt"], L, out=s["K"])
 
-    launches_per_step = 2 if L <= 4096 else (4 + (1 if L == 65536 else 0))
+    conv_launches = 1
+    if s4d:
+        gen_launches = 2 + (1 if L == 65536 else 0)
+    else:
+        gen_launches = 1 if L <= 4096 else (3 + (1 if L == 65536 else 0))
+    launches_per_step = gen_launches + conv_launches
     for i in range(args.warmup):
-        step(sets[i % nsets])
+        gen_stage(sets[i % nsets])
+        conv_stage(sets[i % nsets])
     torch.cuda.synchronize()
     if int(flags.item()) != 0:
         raise RuntimeError(f"kernel flags set: {int(flags.item())}")
@@ -248,10 +262,9 @@ def run_gpu(args, rank, world, local_rank):
         for s in sets:
             g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
             with torch.cuda.graph(g1, stream=cap):
-                s4.kernel_dplr_prepare(s["Lambda"], s["P"], s["Q"], s["B"], s["C"], s["log_dt"], s["D"], L,
-                                       K=s["K"], workspace=s["ws"], flags=flags)
+                gen_stage(s)
             with torch.cuda.graph(g2, stream=cap):
-                s4.fft_conv_apply(s["u"], s["ws"], out=s["y"])
+                conv_stage(s)
             gen_graphs.append(g1)
             conv_graphs.append(g2)
     torch.cuda.current_stream().wait_stream(cap)
@@ -284,14 +297,15 @@ def run_gpu(args, rank, world, local_rank):
     ms = t0.elapsed_time(t1)
     stage = [sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j in range(2)]
 
-    # the Cauchy stage alone (s4_dplr_spectrum), timed separately for its FP32 roofline
+    # the FP32-bound kernel stage alone (Cauchy sums / Vandermonde), timed
+    # separately for its FP32 roofline
     cev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     for i in range(args.warmup):
-        cauchy_only(sets[i % nsets])
+        kernel_only(sets[i % nsets])
     torch.cuda.synchronize()
     cev[0].record()
     for i in range(args.steps):
-        cauchy_only(sets[i % nsets])
+        kernel_only(sets[i % nsets])
     cev[1].record()
     torch.cuda.synchronize()
     stage.append(cev[0].elapsed_time(cev[1]) / args.steps)
@@ -306,8 +320,12 @@ def run_gpu(args, rank, world, local_rank):
     def e2e_step():
         for k in names:
             dsets[k].copy_(host[k], non_blocking=True)
-        s4.forward_dplr(dsets["u"], dsets["Lambda"], dsets["P"], dsets["Q"], dsets["B"], dsets["C"],
-                        dsets["log_dt"], dsets["D"], out=dsets["y"], K=dsets["K"], workspace=dsets["ws"])
+        if s4d:
+            K = s4.s4d_kernel_vandermonde(dsets["A"], dsets["B"], dsets["C"], dsets["log_dt"], L, out=dsets["K"])
+            s4.fft_conv(dsets["u"], K, dsets["D"], out=dsets["y"], workspace=dsets["ws"])
+        else:
+            s4.forward_dplr(dsets["u"], dsets["Lambda"], dsets["P"], dsets["Q"], dsets["B"], dsets["C"],
+                            dsets["log_dt"], dsets["D"], out=dsets["y"], K=dsets["K"], workspace=dsets["ws"])
         y_host.copy_(dsets["y"], non_blocking=True)
 
     e2e_ms = float("nan")
@@ -325,6 +343,41 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
 
+    decode = None
+    if s4d:   # recurrent view (decode) of the same layer: 1024 tokens
+        d = sets[0]
+        Ab, Bb = s4.s4d_discretize_zoh(d["A"], d["B"], d["log_dt"])
+        T = 1024
+        x = torch.zeros(Bt, H, c["N"] // 2, dtype=torch.complex64, device=dev)
+        u_tok = d["u"][:, :, :T].contiguous()
+        y_tok = torch.empty_like(u_tok)
+        u_cols = [u_tok[:, :, k].contiguous() for k in range(T)]
+        y_col = torch.empty(Bt, H, device=dev)
+        g_steps = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            s4.recurrent_step(Ab, Bb, d["C"], d["D"], x, u_cols[0], out=y_col)   # warm-up outside capture
+            with torch.cuda.graph(g_steps, stream=cap):
+                for k in range(T):
+                    s4.recurrent_step(Ab, Bb, d["C"], d["D"], x, u_cols[k], out=y_col)
+        torch.cuda.current_stream().wait_stream(cap)
+        for _ in range(2):
+            s4.recurrent_scan(Ab, Bb, d["C"], d["D"], x, u_tok, out=y_tok)
+            g_steps.replay()
+        torch.cuda.synchronize()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        s4.recurrent_scan(Ab, Bb, d["C"], d["D"], x, u_tok, out=y_tok)
+        e[1].record()
+        e[2].record()
+        g_steps.replay()
+        e[3].record()
+        torch.cuda.synchronize()
+        decode = {"tokens": T, "batch": Bt, "H": H, "state": c["N"] // 2,
+                  "scan_us_per_token": e[0].elapsed_time(e[1]) * 1e3 / T,
+                  "step_us_per_token": e[2].elapsed_time(e[3]) * 1e3 / T,
+                  "step_launch": "1024 s4_recurrent_step launches replayed from one CUDA graph"}
+        del g_steps
+
     times = max_over_ranks([ms, e2e_ms] + stage, dist, dev)
     if dist is not None:
         dist.barrier()
@@ -339,7 +392,7 @@ def run_gpu(args, rank, world, local_rank):
     total_elems = alg["elements"] * world * args.steps   # job_throughput() numerator
     conv_s = stage[1] * 1e-3
     conv_gbs = alg["conv_bytes"] / conv_s / 1e9
-    cauchy_tflops = alg["cauchy_flop"] / (stage[2] * 1e-3) / 1e12
+    cauchy_tflops = alg["kernel_flop"] / (stage[2] * 1e-3) / 1e12
     fp32_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
     traffic = recorded_traffic() if cfg == 2 else None
     line = {
@@ -354,25 +407,28 @@ def run_gpu(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f32",
-        "data": "synthetic (seeded HiPPO-LegS DPLR parameters, N(0,1) inputs)",
+        "data": ("synthetic (S4D-Lin parameters, seeded inputs)" if s4d else
+                 "synthetic (seeded HiPPO-LegS DPLR parameters, seeded inputs)"),
         "config": {"workload": c["name"], "H": H, "N": c["N"], "L": L, "batch": Bt,
                    "global_batch": Bt * world, "dt_range": [c["dt_min"], c["dt_max"]],
                    "parallelism": f"channel shard x{world}, no collective",
                    "launch": "per step: s4_kernel_dplr_prepare + s4_fft_conv_apply, each replayed from a CUDA graph",
                    "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
         "stages_ms": {"kernel_and_spectrum": stage[0], "fft_conv": stage[1],
-                      "cauchy_spectrum_alone": stage[2]},
+                      ("vandermonde_alone" if s4d else "cauchy_spectrum_alone"): stage[2]},
         "roofline": {"kernel": "k_fftconv_pair" if L <= 4096 else "k_fftconv", "bound": "hbm", "achieved": conv_gbs, "peak": hbm,
                      "unit": "GB/s", "frac": conv_gbs / hbm, "traffic": traffic,
                      "peak_source": peak_src, "algorithmic_bytes": alg["conv_bytes"]},
-        "cauchy": {"kernel": "k_cauchy", "bound": "alu", "achieved": cauchy_tflops, "peak": fp32_peak,
+        "cauchy": {"kernel": "k_vandermonde" if s4d else "k_cauchy", "bound": "alu", "achieved": cauchy_tflops,
+                   "peak": fp32_peak,
                    "unit": "TFLOP/s", "frac": cauchy_tflops / fp32_peak,
                    "peak_derivation": f"{SM_COUNT} SM x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max_mhz:.0f} MHz",
-                   "algorithmic_flop": alg["cauchy_flop"]},
+                   "algorithmic_flop": alg["kernel_flop"]},
         "e2e": None if args.no_e2e else {"value": job_throughput(alg["elements"], world, args.steps, e2e_ms),
                                          "unit": UNIT,
                                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
+        "decode": decode,
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -384,7 +440,10 @@ def run_gpu(args, rank, world, local_rank):
 def oracle_sample(inp, channels):
     """fp64 oracle forward for all rows of the given channels; returns elements."""
     from oracle import workloads
-    K = workloads.dplr_kernel(inp, channels=channels)
+    if inp["kind"] == "s4d":
+        K = workloads.s4d_kernel(inp, channels=channels)
+    else:
+        K = workloads.dplr_kernel(inp, channels=channels)
     rows = [(b, h) for h in channels for b in range(inp["Bt"])]
     Krows = [K[list(channels).index(h)] for _, h in rows]
     workloads.conv_rows_at(inp, Krows, rows, np.arange(inp["L"]))
@@ -446,7 +505,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4])
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")

@@ -1,6 +1,6 @@
 // kgen.cu -- the DPLR kernel K and the spectrum of the zero-padded K + D
 // delta_0 in one launch ("The S4 kernel, from scratch", §4 and §5), for
-// L <= 4096. One CTA per channel:
+// L <= 8192. One CTA per channel:
 //   A. the Cauchy/Woodbury generating function at j = 0 .. L/2 (cauchy.cuh),
 //      written with its conjugate mirror straight into the digit-reversed
 //      positions the inverse transform reads;
@@ -16,7 +16,7 @@
 namespace s4 {
 
 template <int LG>
-__global__ void __launch_bounds__(pair_threads<LG>(), 2)
+__global__ void __launch_bounds__(pair_threads<LG>(), pair_min_blocks<LG>())
 k_kgen(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const float2 *__restrict__ Q,
        const float2 *__restrict__ B, const float2 *__restrict__ Cc, const float *__restrict__ log_dt,
        const float *__restrict__ D, int Nh, float *__restrict__ K, float2 *__restrict__ spec,
@@ -62,6 +62,7 @@ cudaError_t launch_kgen(const float2 *Lambda, const float2 *P, const float2 *Q, 
         case 1024: return run_kgen<10>(Lambda, P, Q, B, C, log_dt, D, H, Nh, K, ws, flags, st);
         case 2048: return run_kgen<11>(Lambda, P, Q, B, C, log_dt, D, H, Nh, K, ws, flags, st);
         case 4096: return run_kgen<12>(Lambda, P, Q, B, C, log_dt, D, H, Nh, K, ws, flags, st);
+        case 8192: return run_kgen<13>(Lambda, P, Q, B, C, log_dt, D, H, Nh, K, ws, flags, st);
         default: {
             cudaError_t e = launch_cauchy(Lambda, P, Q, B, C, log_dt, H, Nh, L, K, flags, st);
             if (e == cudaSuccess) e = launch_irfft_packed(K, H, L, st);

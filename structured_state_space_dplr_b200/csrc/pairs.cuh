@@ -1,6 +1,5 @@
-// pairs.cuh -- the two units of work of the forward pass for L <= 4096, as
-// device functions shared by the standalone kernels and the persistent
-// forward kernel:
+// pairs.cuh -- the two units of work of the forward pass for L <= 8192, as
+// device functions of the kernels k_kgen and k_fftconv_pair:
 //
 //   kgen_channel : one channel's kernel K and the spectrum of the zero-padded
 //                  K + D delta_0 ("The S4 kernel, from scratch", §4, §5):
@@ -25,6 +24,10 @@ namespace s4 {
 
 template <int LG>
 __host__ __device__ constexpr int pair_threads() { return (1 << LG) / 16 < 32 ? 32 : (1 << LG) / 16; }
+// CTAs per SM the pair kernels are built for: two up to L = 4096 (about
+// 110 KB of shared memory each), one at L = 8192 (221 KB, 512 threads)
+template <int LG>
+__host__ __device__ constexpr int pair_min_blocks() { return LG <= 12 ? 2 : 1; }
 template <int LG>
 __host__ __device__ constexpr int pair_s0() { return (1 << LG) >> plan_lr(LG, 0); }
 // float2 words before the auxiliary area (kept even: the area is 16-byte aligned)
@@ -110,9 +113,8 @@ __device__ __forceinline__ void pair_stage_rows(const PairSmem &s, const float *
 // ------------------------------------------------------------ convolution --
 // Convolution of the staged row pair (stage ready, all threads synced) with
 // the spectrum spec_h (layout of spec4_index, rank 0 then rank 1). After the
-// first pass, after_first() runs (the stage is free then). COHERENT reads the
-// spectrum through L2 only (it was written earlier in the same launch).
-template <int LG, bool COHERENT, class AfterFirst>
+// first pass, after_first() runs (the stage is free then).
+template <int LG, class AfterFirst>
 __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__restrict__ spec_h, float *y0,
                                           float *y1, bool has1, AfterFirst &&after_first) {
     constexpr int m = 1 << LG, L = m, T = pair_threads<LG>();
@@ -152,13 +154,8 @@ __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__res
     fused_middle_x2<LG, T>(b0, b1, [&](int base) {
         SpecWords w;
         static_for<0, RL / 2>([&](auto i) {
-            if constexpr (COHERENT) {
-                w.k0[i] = __ldcg(s0 + spec4_index<LG>(base, i));
-                w.k1[i] = __ldcg(s1 + spec4_index<LG>(base, i));
-            } else {
-                w.k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
-                w.k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
-            }
+            w.k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
+            w.k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
         });
         return w;
     }, [&](const SpecWords &w, auto &x, auto &z) {

@@ -265,11 +265,11 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
 }
 
 // ------------------------------------------------------- fftconv, one CTA --
-// L <= 4096: one CTA per row pair holds both halves of the length-2L
+// L <= 8192: one CTA per row pair holds both halves of the length-2L
 // transform; see conv_pair (pairs.cuh). Persistent: the next row pair is
 // staged with cp.async while the current one is transformed.
 template <int LG>
-__global__ void __launch_bounds__(pair_threads<LG>(), 2)
+__global__ void __launch_bounds__(pair_threads<LG>(), pair_min_blocks<LG>())
 k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
                float *__restrict__ y) {
     extern __shared__ float2 sm[];
@@ -282,7 +282,7 @@ k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int
         cp_async_wait_all();
         __syncthreads();   // stage ready; previous pair's buffers no longer read
         float *y0 = y + ((size_t)r.b0 * H + r.h) * L;
-        conv_pair<LG, false>(s, spec + (size_t)r.h * 2 * L, y0, y0 + (size_t)H * L, r.has1, [&] {
+        conv_pair<LG>(s, spec + (size_t)r.h * 2 * L, y0, y0 + (size_t)H * L, r.has1, [&] {
             if (pr + gridDim.x < npairs) pair_stage_rows<LG>(s, u, Bt, H, pr + gridDim.x);
         });
     }
@@ -552,7 +552,7 @@ struct ConvKernels {
 
     static cudaError_t conv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st) {
         const float2 *spec = (const float2 *)ws;
-        if constexpr (C == 2 && !TW0G && LG <= 12) {
+        if constexpr (C == 2 && !TW0G && LG <= 13) {
             // one CTA per row pair, both halves in one CTA
 #if S4_CONV_WIDE
             auto kern = k_fftconv_wide<LG>;
@@ -625,7 +625,7 @@ ConvGeom conv_geom(int L) {
         case 1024: return {2, 10, false};
         case 2048: return {2, 11, false};
         case 4096: return {2, 12, false};
-        case 8192: return {4, 12, false};
+        case 8192: return {2, 13, false};
         case 16384: return {8, 12, false};
         case 32768: return {8, 13, false};
         case 65536: return {8, 14, true};
@@ -662,7 +662,7 @@ size_t conv_workspace_bytes(int H, int L) {
     X(1024, 10, 2, false, S4_STG(1024))   \
     X(2048, 11, 2, false, S4_STG(2048))   \
     X(4096, 12, 2, false, S4_STG(4096))   \
-    X(8192, 12, 4, false, false)    \
+    X(8192, 13, 2, false, false)    \
     X(16384, 12, 8, false, false)   \
     X(32768, 13, 8, false, false)   \
     X(65536, 14, 8, true, false)
