@@ -49,7 +49,7 @@ NOMINAL_SM_MHZ = 1965.0
 # two products by 1/|q|^2) and four complex Cauchy sums as 16 FMAs (32 flop)
 CAUCHY_FLOP_PER_TERM = 40
 VANDERMONDE_FLOP_PER_TERM = 4
-KERNEL_SOURCES = ["common.cuh", "fft.cuh", "spectral.cu"]
+KERNEL_SOURCES = ["common.cuh", "fft.cuh", "pairs.cuh", "spectral.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fftconv_h256_l4096_b16_traffic.txt")
 
 
@@ -343,40 +343,45 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
 
-    decode = None
-    if s4d:   # recurrent view (decode) of the same layer: 1024 tokens
-        d = sets[0]
+    # recurrent view (decode) of the same layer: up to 1024 tokens from a zero
+    # state, as one s4_recurrent_scan and as single-token steps from a graph
+    d = sets[0]
+    if s4d:
         Ab, Bb = s4.s4d_discretize_zoh(d["A"], d["B"], d["log_dt"])
-        T = 1024
-        x = torch.zeros(Bt, H, c["N"] // 2, dtype=torch.complex64, device=dev)
-        u_tok = d["u"][:, :, :T].contiguous()
-        y_tok = torch.empty_like(u_tok)
-        u_cols = [u_tok[:, :, k].contiguous() for k in range(T)]
-        y_col = torch.empty(Bt, H, device=dev)
-        g_steps = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(cap):
-            s4.recurrent_step(Ab, Bb, d["C"], d["D"], x, u_cols[0], out=y_col)   # warm-up outside capture
-            with torch.cuda.graph(g_steps, stream=cap):
-                for k in range(T):
-                    s4.recurrent_step(Ab, Bb, d["C"], d["D"], x, u_cols[k], out=y_col)
-        torch.cuda.current_stream().wait_stream(cap)
-        for _ in range(2):
-            s4.recurrent_scan(Ab, Bb, d["C"], d["D"], x, u_tok, out=y_tok)
-            g_steps.replay()
-        torch.cuda.synchronize()
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        e[0].record()
+        step_kind = "diagonal ZOH (S4D), O(Nh) per token"
+    else:
+        Ab, Bb = s4.dplr_discretize_structured(d["Lambda"], d["P"], d["Q"], d["B"], d["log_dt"])
+        step_kind = "structured bilinear DPLR (diagonal + rank 1), O(Nh) per token"
+    T = min(1024, L)
+    x = torch.zeros(Bt, H, c["N"] // 2, dtype=torch.complex64, device=dev)
+    u_tok = d["u"][:, :, :T].contiguous()
+    y_tok = torch.empty_like(u_tok)
+    u_cols = [u_tok[:, :, k].contiguous() for k in range(T)]
+    y_col = torch.empty(Bt, H, device=dev)
+    g_steps = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        s4.recurrent_step(Ab, Bb, d["C"], d["D"], x, u_cols[0], out=y_col)   # warm-up outside capture
+        with torch.cuda.graph(g_steps, stream=cap):
+            for k in range(T):
+                s4.recurrent_step(Ab, Bb, d["C"], d["D"], x, u_cols[k], out=y_col)
+    torch.cuda.current_stream().wait_stream(cap)
+    for _ in range(2):
         s4.recurrent_scan(Ab, Bb, d["C"], d["D"], x, u_tok, out=y_tok)
-        e[1].record()
-        e[2].record()
         g_steps.replay()
-        e[3].record()
-        torch.cuda.synchronize()
-        decode = {"tokens": T, "batch": Bt, "H": H, "state": c["N"] // 2,
-                  "scan_us_per_token": e[0].elapsed_time(e[1]) * 1e3 / T,
-                  "step_us_per_token": e[2].elapsed_time(e[3]) * 1e3 / T,
-                  "step_launch": "1024 s4_recurrent_step launches replayed from one CUDA graph"}
-        del g_steps
+    torch.cuda.synchronize()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    e[0].record()
+    s4.recurrent_scan(Ab, Bb, d["C"], d["D"], x, u_tok, out=y_tok)
+    e[1].record()
+    e[2].record()
+    g_steps.replay()
+    e[3].record()
+    torch.cuda.synchronize()
+    decode = {"tokens": T, "batch": Bt, "H": H, "state": c["N"] // 2, "step": step_kind,
+              "scan_us_per_token": e[0].elapsed_time(e[1]) * 1e3 / T,
+              "step_us_per_token": e[2].elapsed_time(e[3]) * 1e3 / T,
+              "step_launch": f"{T} s4_recurrent_step launches replayed from one CUDA graph"}
+    del g_steps
 
     times = max_over_ranks([ms, e2e_ms] + stage, dist, dev)
     if dist is not None:

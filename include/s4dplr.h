@@ -249,6 +249,23 @@ s4_status s4d_discretize_zoh(const s4_c32 *A, const s4_c32 *B, const float *log_
                              cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * s4_dplr_discretize_structured: the same bilinear DPLR discretisation
+ * ([S4K] §3 rule on the §2 DPLR system) kept in its diagonal-plus-rank-1
+ * form, for the O(Nh) step S4_STEP_DPLR ([S4K] §5 recurrent view). With
+ * d_n = 1 - dt/2 Lambda_n, alpha_n = (dt/2) P_n / d_n, beta_n = conj(Q_n)/d_n
+ * and s = 1 + 2 Re sum_n conj(Q_n) alpha_n (the Sherman-Morrison denominator
+ * of I - dt/2 A over the full conjugate-closed system),
+ *     Abar = diag(a) - g beta^T,  a_n = 2/d_n - 1,  g_n = 2 alpha_n / s,
+ * over the full system; only the stored half is written:
+ *   Astr : [H, Nh, 3] complex out, Astr[h, n] = {a_n, g_n, beta_n};
+ *   Bbar : [H, Nh] complex out, the stored half of s4_dplr_discretize's Bbar.
+ * Computed in fp64, stored as fp32. Errors as s4_dplr_discretize.
+ * ------------------------------------------------------------------------ */
+s4_status s4_dplr_discretize_structured(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                                        const s4_c32 *B, const float *log_dt, int H, int Nh,
+                                        s4_c32 *Astr, s4_c32 *Bbar, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * s4_recurrent_step -- one token of the recurrence ([S4K] §5):
  *     x <- Abar x + Bbar u_t,   y_t = Re(C . x) + D u_t        (dense)
  *     x <- Abar * x + Bbar u_t, y_t = 2 Re(sum_n C_n x_n) + D u_t  (diagonal)
@@ -257,12 +274,20 @@ s4_status s4d_discretize_zoh(const s4_c32 *A, const s4_c32 *B, const float *log_
  *                       (from s4_dplr_discretize), Ns <= 128 (Abar of a
  *                       channel is staged in shared memory).
  *   mode S4_STEP_DIAG : Abar, Bbar, C [H, Ns] with Ns = Nh (S4D), Ns <= 256.
+ *   mode S4_STEP_DPLR : structured DPLR step, O(Nh) per token: Abar = Astr
+ *                       [H, Ns, 3] and Bbar [H, Ns] from
+ *                       s4_dplr_discretize_structured, C [H, Ns] (stored
+ *                       modes), Ns = Nh <= 256. x holds the stored half of a
+ *                       conjugate-symmetric full state (zero, for instance;
+ *                       real inputs keep it so), and
+ *                       y_t = 2 Re(sum_n C_n x_n) + D u_t, which equals the
+ *                       dense step's Re(Cfull . x_full).
  *   x   : [Bt, H, Ns] complex in/out.   u_t, y_t : [Bt, H] float.  D : [H].
  *   1 <= H <= 65535; Bt >= 1.
  * s4_recurrent_scan runs T consecutive steps in one launch:
  *   u, y : [Bt, H, T] float (token axis last), x in/out as above.
  * ------------------------------------------------------------------------ */
-typedef enum { S4_STEP_DENSE = 0, S4_STEP_DIAG = 1 } s4_step_mode;
+typedef enum { S4_STEP_DENSE = 0, S4_STEP_DIAG = 1, S4_STEP_DPLR = 2 } s4_step_mode;
 
 s4_status s4_recurrent_step(s4_step_mode mode, const s4_c32 *Abar, const s4_c32 *Bbar,
                             const s4_c32 *C, const float *D, int Bt, int H, int Ns,

@@ -16,7 +16,7 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (S4_FLAG_NONFINITE, S4_FLAG_UNSTABLE, S4_STEP_DENSE, S4_STEP_DIAG,  # noqa: F401
+from ._lib import (S4_FLAG_NONFINITE, S4_FLAG_UNSTABLE, S4_STEP_DENSE, S4_STEP_DIAG, S4_STEP_DPLR,  # noqa: F401
                    S4Error)
 
 __all__ = [
@@ -24,7 +24,7 @@ __all__ = [
     "fft_conv_static",
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
-    "S4_STEP_DIAG", "load",
+    "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "load",
 ]
 
 
@@ -245,6 +245,20 @@ def dplr_discretize(Lambda, P, Q, B, C, log_dt):
     return Ab, Bb, Cf
 
 
+def dplr_discretize_structured(Lambda, P, Q, B, log_dt):
+    """Bilinear DPLR transition in diagonal-plus-rank-1 form for the O(Nh)
+    step: (Astr [H, Nh, 3] = {a, g, beta}, Bbar [H, Nh]) complex64."""
+    Lambda, P, Q, B = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B), "Lambda P Q B".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    dev = Lambda.device
+    Astr = torch.empty(H, Nh, 3, dtype=torch.complex64, device=dev)
+    Bb = torch.empty(H, Nh, dtype=torch.complex64, device=dev)
+    _lib.call("s4_dplr_discretize_structured", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(log_dt),
+              H, Nh, _ptr(Astr), _ptr(Bb), _stream())
+    return Astr, Bb
+
+
 def s4d_discretize_zoh(A, B, log_dt):
     """Diagonal ZOH (Abar, Bbar) [H, Nh] complex64."""
     A, B = _cplx(A, "A"), _cplx(B, "B")
@@ -256,18 +270,24 @@ def s4d_discretize_zoh(A, B, log_dt):
     return Ab, Bb
 
 
-def _step_args(Abar, Bbar, C, D, x):
+def _step_args(Abar, Bbar, C, D, x, mode):
     Abar, Bbar, C, x = (_cplx(t, n) for t, n in zip((Abar, Bbar, C, x), "Abar Bbar C x".split()))
     D = _cuda(D, "D", torch.float32)
-    mode = S4_STEP_DENSE if Abar.dim() == 3 else S4_STEP_DIAG
     Bt, H, Ns = x.shape
+    if mode is None:   # from the shape of Abar
+        dense = Abar.dim() == 3 and tuple(Abar.shape[1:]) == (Ns, Ns)
+        struct = Abar.dim() == 3 and tuple(Abar.shape[1:]) == (Ns, 3)
+        if dense and struct:
+            raise ValueError("Abar [H, 3, 3] is ambiguous: pass mode=S4_STEP_DENSE or S4_STEP_DPLR")
+        mode = S4_STEP_DENSE if dense else (S4_STEP_DPLR if struct else S4_STEP_DIAG)
     return mode, Abar, Bbar, C, D, x, Bt, H, Ns
 
 
-def recurrent_step(Abar, Bbar, C, D, x, u_t, *, out=None):
+def recurrent_step(Abar, Bbar, C, D, x, u_t, *, out=None, mode=None):
     """One token: x <- Abar x + Bbar u_t (in place), returns y_t [Bt, H].
-    Dense if Abar is [H, N, N], diagonal (S4D) if Abar is [H, Nh]."""
-    mode, Abar, Bbar, C, D, x, Bt, H, Ns = _step_args(Abar, Bbar, C, D, x)
+    Dense if Abar is [H, N, N], structured DPLR if Abar is [H, Nh, 3]
+    (from dplr_discretize_structured), diagonal (S4D) if Abar is [H, Nh]."""
+    mode, Abar, Bbar, C, D, x, Bt, H, Ns = _step_args(Abar, Bbar, C, D, x, mode)
     u_t = _cuda(u_t, "u_t", torch.float32)
     if out is None:
         out = torch.empty_like(u_t)
@@ -276,9 +296,9 @@ def recurrent_step(Abar, Bbar, C, D, x, u_t, *, out=None):
     return out
 
 
-def recurrent_scan(Abar, Bbar, C, D, x, u, *, out=None):
+def recurrent_scan(Abar, Bbar, C, D, x, u, *, out=None, mode=None):
     """T tokens in one launch: u [Bt, H, T] -> y [Bt, H, T]; x updated in place."""
-    mode, Abar, Bbar, C, D, x, Bt, H, Ns = _step_args(Abar, Bbar, C, D, x)
+    mode, Abar, Bbar, C, D, x, Bt, H, Ns = _step_args(Abar, Bbar, C, D, x, mode)
     u = _cuda(u, "u", torch.float32)
     T = u.shape[-1]
     if out is None:

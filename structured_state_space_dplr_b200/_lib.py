@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libs4dplr.so")
 S4_OK, S4_ERR_INVALID_ARG, S4_ERR_UNSUPPORTED, S4_ERR_WORKSPACE, S4_ERR_CUDA = range(5)
 S4_FLAG_UNSTABLE = 1
 S4_FLAG_NONFINITE = 2
-S4_STEP_DENSE, S4_STEP_DIAG = 0, 1
+S4_STEP_DENSE, S4_STEP_DIAG, S4_STEP_DPLR = 0, 1, 2
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int
@@ -37,6 +37,7 @@ SIGNATURES = {
     "s4_forward_dplr": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _sz, _p, _p]),
     "s4d_kernel_vandermonde": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p, _p]),
     "s4_dplr_discretize": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _p, _p, _p, _p]),
+    "s4_dplr_discretize_structured": (_i, [_p, _p, _p, _p, _p, _i, _i, _p, _p, _p]),
     "s4d_discretize_zoh": (_i, [_p, _p, _p, _i, _i, _p, _p, _p]),
     "s4_recurrent_step": (_i, [_i, _p, _p, _p, _p, _i, _i, _i, _p, _p, _p, _p]),
     "s4_recurrent_scan": (_i, [_i, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _p]),

@@ -231,6 +231,18 @@ s4_status s4_dplr_discretize(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32
                                                   (float2 *)Cfull, stream));
 }
 
+s4_status s4_dplr_discretize_structured(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                                        const s4_c32 *B, const float *log_dt, int H, int Nh, s4_c32 *Astr,
+                                        s4_c32 *Bbar, cudaStream_t stream) {
+    if (any_null(Lambda, P, Q, B) || any_null(Astr, Bbar) || log_dt == nullptr) return S4_ERR_INVALID_ARG;
+    s4_status s = check_modes(H, Nh, 0, false);
+    if (s != S4_OK) return s;
+    if (!params_aligned({Lambda, P, Q, B, Astr, Bbar})) return S4_ERR_INVALID_ARG;
+    return cuda_status(s4::launch_dplr_discretize_structured((const float2 *)Lambda, (const float2 *)P,
+                                                             (const float2 *)Q, (const float2 *)B, log_dt, H,
+                                                             Nh, (float2 *)Astr, (float2 *)Bbar, stream));
+}
+
 s4_status s4d_discretize_zoh(const s4_c32 *A, const s4_c32 *B, const float *log_dt, int H, int Nh,
                              s4_c32 *Abar, s4_c32 *Bbar, cudaStream_t stream) {
     if (any_null(A, B) || any_null(Abar, Bbar) || log_dt == nullptr) return S4_ERR_INVALID_ARG;
@@ -249,7 +261,7 @@ static s4_status step_checks(s4_step_mode mode, const s4_c32 *Abar, const s4_c32
     if (H > S4_MAX_H) return S4_ERR_UNSUPPORTED;
     if (mode == S4_STEP_DENSE) {
         if (Ns > S4_MAX_DENSE_N) return S4_ERR_UNSUPPORTED;
-    } else if (mode == S4_STEP_DIAG) {
+    } else if (mode == S4_STEP_DIAG || mode == S4_STEP_DPLR) {
         if (Ns > S4_MAX_NH) return S4_ERR_UNSUPPORTED;
     } else {
         return S4_ERR_INVALID_ARG;

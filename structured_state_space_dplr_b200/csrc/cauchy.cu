@@ -17,7 +17,7 @@ k_cauchy(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const 
          int Nh, int L, float *__restrict__ K, unsigned *__restrict__ flags) {
     extern __shared__ float4 sp[];
     const int h = blockIdx.y;
-    cauchy_stage_modes(Lambda, P, Q, B, Cc, h, Nh, sp, flags, threadIdx.x, T);
+    cauchy_stage_modes<true>(Lambda, P, Q, B, Cc, h, Nh, sp, flags, threadIdx.x, T);
     __syncthreads();
     const float ldt = __ldg(log_dt + h);
     const int half = L >> 1;
@@ -28,7 +28,7 @@ k_cauchy(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const 
         jj[f] = j[f] < half ? j[f] : 0;
     }
     float2 kh[F];
-    cauchy_eval<F>(sp, Nh, jj, L, expf(-ldt), kh);
+    cauchy_eval<F, true>(sp, Nh, jj, L, expf(-ldt), kh);
     bool bad = false;
     float *Kh = K + (size_t)h * L;
 #pragma unroll
@@ -40,7 +40,7 @@ k_cauchy(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const 
         }
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-        const float nyq = cauchy_nyquist(sp, Nh, expf(ldt), L);
+        const float nyq = cauchy_nyquist<true>(sp, Nh, expf(ldt), L);
         Kh[1] = nyq;
         bad |= !isfinite(nyq);
     }
@@ -54,7 +54,7 @@ cudaError_t launch_cauchy(const float2 *Lambda, const float2 *P, const float2 *Q
     constexpr int T = kCauchyThreads, F = kCauchyFreqs;
     const int half = L / 2;
     dim3 grid((half + T * F - 1) / (T * F), H);
-    const size_t smem = sizeof(float4) * 3 * (size_t)Nh;
+    const size_t smem = sizeof(float4) * cauchy_mode_words<true>() * (size_t)Nh;
     k_cauchy<T, F><<<grid, T, smem, st>>>(Lambda, P, Q, B, C, log_dt, Nh, L, K, flags);
     return cudaGetLastError();
 }

@@ -8,8 +8,19 @@
 //   beta_j = conj(Q_j) / d_j,  s = 1 + sum_i conj(Q_i) alpha_i,
 // and then Abar = M^-1 (I + dt/2 A) = 2 M^-1 - I, Bbar = dt M^-1 B_f.
 //
-// Steps: dense (O(N^2) per token, N = 2 Nh) and diagonal (S4D, O(Nh)).
-// The scan variants run T tokens in one launch with the state on chip.
+// Steps: dense (O(N^2) per token, N = 2 Nh), diagonal (S4D, O(Nh)) and
+// structured DPLR (O(Nh)). The scan variants run T tokens in one launch with
+// the state on chip.
+//
+// Structured DPLR step. Abar = 2 M^-1 - I = diag(a) - g beta^T with
+// a_i = 2/d_i - 1 and g_i = 2 alpha_i / s. For a state that is conjugate
+// symmetric (x_{i+Nh} = conj(x_i); real inputs keep it so) every full-system
+// sum over a mode and its partner is twice the real part of the stored term:
+//   t   = beta^T x   = 2 Re sum_n beta_n x_n,
+//   s   = 1 + 2 Re sum_n conj(Q_n) alpha_n,
+//   x_n <- a_n x_n - g_n t + Bbar_n u,
+//   y   = 2 Re sum_n C_n x_n + D u,
+// i.e. the dense step's result from 2 dot products over the Nh stored modes.
 #include "common.cuh"
 #include "launch.h"
 #include "s4dplr.h"
@@ -167,6 +178,124 @@ __global__ void k_step_diag(const float2 *__restrict__ Abar, const float2 *__res
         if (lane + 32 * k < Nh) x[(size_t)w * Nh + lane + 32 * k] = s[k];
 }
 
+// Structured transition of the bilinear DPLR system: one warp per channel,
+// lanes striding over the stored modes, fp64 arithmetic.
+//   Astr[h, n] = {a_n, g_n, beta_n},  Bbar[h, n] (stored half of Bbar).
+__global__ void k_dplr_discretize_structured(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
+                                             const float2 *__restrict__ Q, const float2 *__restrict__ B,
+                                             const float *__restrict__ log_dt, int H, int Nh,
+                                             float2 *__restrict__ Astr, float2 *__restrict__ Bbar) {
+    const int h = (int)((blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (h >= H) return;
+    const double dt = exp((double)__ldg(log_dt + h));
+    const size_t po = (size_t)h * Nh;
+    // pass 1: s - 1 = 2 Re sum conj(Q) alpha, and 2 Re sum beta B (= beta^T B_f)
+    double s1 = 0.0, sb = 0.0;
+    for (int n = lane; n < Nh; n += 32) {
+        const float2 lf = Lambda[po + n], pf = P[po + n], qf = Q[po + n], bf = B[po + n];
+        const double dr = 1.0 - 0.5 * dt * lf.x, di = -0.5 * dt * lf.y, dd = dr * dr + di * di;
+        const double ir = dr / dd, ii = -di / dd;                              // 1/d
+        const double ar = 0.5 * dt * (pf.x * ir - pf.y * ii), ai = 0.5 * dt * (pf.x * ii + pf.y * ir);
+        const double br = qf.x * ir + qf.y * ii, bi = qf.x * ii - qf.y * ir;   // conj(q)/d
+        s1 += qf.x * ar + qf.y * ai;                                           // Re(conj(q) alpha)
+        sb += br * bf.x - bi * bf.y;                                           // Re(beta b)
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+        sb += __shfl_xor_sync(0xffffffffu, sb, off);
+    }
+    const double s = 1.0 + 2.0 * s1, tb = 2.0 * sb;
+    // pass 2: the coefficients
+    for (int n = lane; n < Nh; n += 32) {
+        const float2 lf = Lambda[po + n], pf = P[po + n], qf = Q[po + n], bf = B[po + n];
+        const double dr = 1.0 - 0.5 * dt * lf.x, di = -0.5 * dt * lf.y, dd = dr * dr + di * di;
+        const double ir = dr / dd, ii = -di / dd;
+        const double ar = 0.5 * dt * (pf.x * ir - pf.y * ii), ai = 0.5 * dt * (pf.x * ii + pf.y * ir);
+        const double br = qf.x * ir + qf.y * ii, bi = qf.x * ii - qf.y * ir;
+        float2 *o = Astr + 3 * (po + n);
+        o[0] = make_float2((float)(2.0 * ir - 1.0), (float)(2.0 * ii));       // a = 2/d - 1
+        o[1] = make_float2((float)(2.0 * ar / s), (float)(2.0 * ai / s));      // g = 2 alpha / s
+        o[2] = make_float2((float)br, (float)bi);                              // beta
+        // Bbar = dt (b/d - alpha beta^T B_f / s)
+        Bbar[po + n] = make_float2((float)(dt * (bf.x * ir - bf.y * ii - ar * tb / s)),
+                                   (float)(dt * (bf.x * ii + bf.y * ir - ai * tb / s)));
+    }
+}
+
+// Structured DPLR recurrence: one warp per row (b, h), lanes stride over the
+// stored modes. With the per-channel constants cg = 2 Re sum C g and
+// cb = 2 Re sum C Bbar, the output of the updated state is
+//   y = 2 Re sum C a x - cg t + cb u + D u,
+// so both sums of a token (t and the C a x term) come from the state before
+// the update and share one warp reduction.
+__global__ void k_step_dplr(const float2 *__restrict__ Astr, const float2 *__restrict__ Bbar,
+                            const float2 *__restrict__ C, const float *__restrict__ D, int Bt, int H, int Nh,
+                            int T, float2 *__restrict__ x, const float *__restrict__ u, float *__restrict__ y) {
+    constexpr int MAXM = 8;   // modes per lane (Nh <= 256)
+    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= (long long)Bt * H) return;
+    const int h = (int)(w % H);
+    const size_t po = (size_t)h * Nh;
+    float2 a[MAXM], g[MAXM], be[MAXM], b[MAXM], ca[MAXM], st[MAXM];
+    float cg = 0.f, cb = 0.f;
+#pragma unroll
+    for (int k = 0; k < MAXM; ++k) {
+        const int n = lane + 32 * k;
+        const bool ok = n < Nh;
+        const float2 z = make_float2(0.f, 0.f);
+        a[k] = ok ? Astr[3 * (po + n)] : z;
+        g[k] = ok ? Astr[3 * (po + n) + 1] : z;
+        be[k] = ok ? Astr[3 * (po + n) + 2] : z;
+        b[k] = ok ? Bbar[po + n] : z;
+        const float2 c = ok ? C[po + n] : z;
+        ca[k] = cmul(c, a[k]);
+        cg = fmaf(c.x, g[k].x, fmaf(-c.y, g[k].y, cg));
+        cb = fmaf(c.x, b[k].x, fmaf(-c.y, b[k].y, cb));
+        st[k] = ok ? x[(size_t)w * Nh + n] : z;
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+        cg += __shfl_xor_sync(0xffffffffu, cg, off);
+        cb += __shfl_xor_sync(0xffffffffu, cb, off);
+    }
+    cg *= 2.f;
+    cb *= 2.f;
+    const float Dh = D[h];
+    for (int t = 0; t < T; ++t) {
+        const float ut = u[(size_t)w * T + t];
+        float tv = 0.f, yv = 0.f;   // Re sum beta x, Re sum C a x
+#pragma unroll
+        for (int k = 0; k < MAXM; ++k) {
+            tv = fmaf(be[k].x, st[k].x, fmaf(-be[k].y, st[k].y, tv));
+            yv = fmaf(ca[k].x, st[k].x, fmaf(-ca[k].y, st[k].y, yv));
+        }
+        for (int off = 16; off > 0; off >>= 1) {
+            tv += __shfl_xor_sync(0xffffffffu, tv, off);
+            yv += __shfl_xor_sync(0xffffffffu, yv, off);
+        }
+        const float tt = 2.f * tv;
+#pragma unroll
+        for (int k = 0; k < MAXM; ++k) {   // x <- a x - g t + Bbar u (zero for the padding modes)
+            const float2 ax = cmul(a[k], st[k]);
+            st[k] = make_float2(fmaf(b[k].x, ut, fmaf(-g[k].x, tt, ax.x)), fmaf(b[k].y, ut, fmaf(-g[k].y, tt, ax.y)));
+        }
+        if (lane == 0) y[(size_t)w * T + t] = fmaf(2.f, yv, fmaf(-cg, tt, fmaf(cb + Dh, ut, 0.f)));
+    }
+#pragma unroll
+    for (int k = 0; k < MAXM; ++k)
+        if (lane + 32 * k < Nh) x[(size_t)w * Nh + lane + 32 * k] = st[k];
+}
+
+cudaError_t launch_dplr_discretize_structured(const float2 *Lambda, const float2 *P, const float2 *Q,
+                                              const float2 *B, const float *log_dt, int H, int Nh,
+                                              float2 *Astr, float2 *Bbar, cudaStream_t st) {
+    const int per_block = 8;
+    k_dplr_discretize_structured<<<(H + per_block - 1) / per_block, 32 * per_block, 0, st>>>(
+        Lambda, P, Q, B, log_dt, H, Nh, Astr, Bbar);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_dplr_discretize(const float2 *Lambda, const float2 *P, const float2 *Q,
                                    const float2 *B, const float2 *C, const float *log_dt, int H, int Nh,
                                    float2 *Abar, float2 *Bbar, float2 *Cfull, cudaStream_t st) {
@@ -178,11 +307,14 @@ cudaError_t launch_dplr_discretize(const float2 *Lambda, const float2 *P, const 
 
 cudaError_t launch_step(int mode, const float2 *Abar, const float2 *Bbar, const float2 *C, const float *D,
                         int Bt, int H, int Ns, int T, float2 *x, const float *u, float *y, cudaStream_t st) {
-    if (mode == S4_STEP_DIAG) {
+    if (mode == S4_STEP_DIAG || mode == S4_STEP_DPLR) {
         const long long warps = (long long)Bt * H;
         const int per_block = 8;
-        k_step_diag<<<(unsigned)((warps + per_block - 1) / per_block), 32 * per_block, 0, st>>>(
-            Abar, Bbar, C, D, Bt, H, Ns, T, x, u, y);
+        const unsigned grid = (unsigned)((warps + per_block - 1) / per_block);
+        if (mode == S4_STEP_DIAG)
+            k_step_diag<<<grid, 32 * per_block, 0, st>>>(Abar, Bbar, C, D, Bt, H, Ns, T, x, u, y);
+        else
+            k_step_dplr<<<grid, 32 * per_block, 0, st>>>(Abar, Bbar, C, D, Bt, H, Ns, T, x, u, y);
         return cudaGetLastError();
     }
     const int NP = (Ns + 31) / 32 * 32;

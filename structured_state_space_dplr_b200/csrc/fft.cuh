@@ -24,23 +24,27 @@
 // The twist W_N^{k c} is folded into the first pass: a per-rank constant on
 // each input of a group plus a per-rank first-pass twiddle table.
 //
-// Shared memory is padded by one point every 16 (index i -> i + i/16), which
-// makes every pass conflict-free for 8-byte accesses.
+// Shared memory is padded by two points after every 16 (pidx below): with
+// the pass plan, every pass is free of bank conflicts.
 #pragma once
 #include "common.cuh"
 
 namespace s4 {
 
 // ------------------------------------------------------------------ plan --
-// log2 of the radix of pass s for a 2^lg-point transform.
-__host__ __device__ constexpr int plan_P(int lg) {
-    return lg == 4 ? 2 : (lg % 4 == 0 ? lg / 4 : lg / 4 + 1);
-}
+// log2 of the radix of pass s for a 2^lg-point transform. The first and the
+// last pass are radix 16 (from lg = 8 on); the bits left over go to the
+// middle passes, split as evenly as they allow. Every strided pass then has a
+// stride of at least 16 points and the last pass works on 16 consecutive
+// points (moved as 16-byte pairs), which keeps all of them free of
+// shared-memory bank conflicts with the padding below.
+__host__ __device__ constexpr int plan_P(int lg) { return lg <= 8 ? 2 : (lg + 3) / 4; }
 __host__ __device__ constexpr int plan_lr(int lg, int s) {
-    return lg == 4 ? 2
-         : (lg % 4 == 0) ? 4
-         : (lg % 4 == 1) ? (s < lg / 4 - 1 ? 4 : (s == lg / 4 - 1 ? 3 : 2))
-         : (s < lg / 4 ? 4 : lg % 4);
+    if (lg == 4) return 2;
+    if (lg <= 8) return s == 0 ? lg - 4 : 4;
+    if (s == 0 || s == plan_P(lg) - 1) return 4;
+    const int k = plan_P(lg) - 2, mid = lg - 8;
+    return mid / k + (s - 1 < mid % k ? 1 : 0);
 }
 // block size of pass s (the sub-transform length it starts)
 __host__ __device__ constexpr int plan_B(int lg, int s) {

@@ -37,13 +37,14 @@ __host__ __device__ constexpr int pair_core_f2() {
 }
 template <int LG>
 __host__ __device__ constexpr size_t pair_smem_bytes(int Nh) {
-    return sizeof(float2) * ((size_t)pair_core_f2<LG>() + ((1 << LG) > 6 * Nh ? (1 << LG) : 6 * Nh));
+    constexpr size_t cw = 2 * cauchy_mode_words<false>();   // float2 words of Cauchy constants per mode
+    return sizeof(float2) * ((size_t)pair_core_f2<LG>() + ((size_t)(1 << LG) > cw * Nh ? (size_t)(1 << LG) : cw * Nh));
 }
 
 struct PairSmem {
     float2 *b0, *b1, *tws, *ta, *tb;
     float *stage;   // [2][L] input rows (convolution)
-    float4 *sp;     // [3 Nh] Cauchy constants (generation)
+    float4 *sp;     // [3 Nh] Cauchy constants (generation, scalar form)
 };
 
 template <int LG>
@@ -208,7 +209,7 @@ __device__ __forceinline__ void kgen_channel(const PairSmem &s, const float2 *__
     constexpr int F = 4;   // frequencies per thread per round
     float2 *X = s.b0, *Y = s.b1;
     float4 *sp = s.sp;
-    cauchy_stage_modes(Lambda, P, Q, B, Cc, h, Nh, sp, flags, threadIdx.x, T);
+    cauchy_stage_modes<false>(Lambda, P, Q, B, Cc, h, Nh, sp, flags, threadIdx.x, T);
     __syncthreads();
 
     // ---- A: generating function -> X at digit-reversed positions (with mirror)
@@ -223,7 +224,7 @@ __device__ __forceinline__ void kgen_channel(const PairSmem &s, const float2 *__
             jj[f] = j[f] < L / 2 ? j[f] : 0;
         }
         float2 kh[F];
-        cauchy_eval<F>(sp, Nh, jj, L, inv_dt, kh);
+        cauchy_eval<F, false>(sp, Nh, jj, L, inv_dt, kh);
 #pragma unroll
         for (int f = 0; f < F; ++f) {
             if (j[f] < L / 2) {
@@ -238,7 +239,7 @@ __device__ __forceinline__ void kgen_channel(const PairSmem &s, const float2 *__
         }
     }
     if (threadIdx.x == 0) {
-        const float nyq = cauchy_nyquist(sp, Nh, expf(ldt), L);
+        const float nyq = cauchy_nyquist<false>(sp, Nh, expf(ldt), L);
         bad |= !isfinite(nyq);
         X[pidx(digrev_inv<LG>(L / 2))] = make_float2(nyq, 0.0f);
     }

@@ -111,6 +111,9 @@ def test_steps_reject_bad_arguments(lib):
     assert lib.s4_recurrent_step(1, *args, 0, 4, 32, x, u, y, p(0)) == _lib.S4_ERR_INVALID_ARG
     assert lib.s4_recurrent_scan(1, *args, 2, 4, 32, 0, x, u, y, p(0)) == _lib.S4_ERR_INVALID_ARG
     assert lib.s4_recurrent_step(1, *args, 2, 4, 32, x, u, u, p(0)) == _lib.S4_ERR_INVALID_ARG  # y aliases u
+    assert lib.s4_recurrent_step(2, *args, 2, 4, 257, x, u, y, p(0)) == _lib.S4_ERR_UNSUPPORTED   # structured, Nh > 256
+    assert lib.s4_recurrent_scan(2, *args, 2, 4, 32, 0, x, u, y, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_recurrent_step(2, p(FAKE + 4), *args[1:], 2, 4, 32, x, u, y, p(0)) == _lib.S4_ERR_INVALID_ARG
 
 
 def test_vandermonde_and_discretize_reject_bad_arguments(lib):
@@ -120,6 +123,12 @@ def test_vandermonde_and_discretize_reject_bad_arguments(lib):
     assert lib.s4d_discretize_zoh(*a[:3], 4, 300, p(FAKE2), p(FAKE2 + 0x100000), p(0)) == _lib.S4_ERR_UNSUPPORTED
     assert lib.s4_dplr_discretize(*(p(FAKE + 0x100000 * i) for i in range(6)), 0, 32,
                                   p(FAKE2), p(FAKE2 + 0x100000), p(FAKE2 + 0x200000), p(0)) == _lib.S4_ERR_INVALID_ARG
+    five = [p(FAKE + 0x100000 * i) for i in range(5)]
+    out = [p(FAKE2), p(FAKE2 + 0x100000)]
+    assert lib.s4_dplr_discretize_structured(*five, 4, 257, *out, p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_dplr_discretize_structured(*five, 0, 32, *out, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_dplr_discretize_structured(*five[:4], p(0), 4, 32, *out, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_dplr_discretize_structured(*five, 4, 32, p(FAKE2 + 4), out[1], p(0)) == _lib.S4_ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors():
