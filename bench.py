@@ -49,6 +49,7 @@ NOMINAL_SM_MHZ = 1965.0
 # two products by 1/|q|^2) and four complex Cauchy sums as 16 FMAs (32 flop)
 CAUCHY_FLOP_PER_TERM = 40
 VANDERMONDE_FLOP_PER_TERM = 4
+E2E_CHUNKS = 8   # row-pair chunks of the host-buffer pipeline
 KERNEL_SOURCES = ["common.cuh", "fft.cuh", "pairs.cuh", "spectral.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fftconv_h256_l4096_b16_traffic.txt")
 
@@ -317,16 +318,21 @@ def run_gpu(args, rank, world, local_rank):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = y_host.numel() * 4
 
+    params = [k for k in names if k != "u"]
+
     def e2e_step():
-        for k in names:
+        # the parameters go up as ordinary copies; u goes up and y comes back
+        # in chunks overlapped with the convolution (the host-buffer entry points)
+        for k in params:
             dsets[k].copy_(host[k], non_blocking=True)
         if s4d:
             K = s4.s4d_kernel_vandermonde(dsets["A"], dsets["B"], dsets["C"], dsets["log_dt"], L, out=dsets["K"])
-            s4.fft_conv(dsets["u"], K, dsets["D"], out=dsets["y"], workspace=dsets["ws"])
+            s4.fft_conv_host(host["u"], K, dsets["D"], y_host=y_host, u_dev=dsets["u"], y_dev=dsets["y"],
+                             workspace=dsets["ws"], chunks=E2E_CHUNKS)
         else:
-            s4.forward_dplr(dsets["u"], dsets["Lambda"], dsets["P"], dsets["Q"], dsets["B"], dsets["C"],
-                            dsets["log_dt"], dsets["D"], out=dsets["y"], K=dsets["K"], workspace=dsets["ws"])
-        y_host.copy_(dsets["y"], non_blocking=True)
+            s4.forward_dplr_host(host["u"], dsets["Lambda"], dsets["P"], dsets["Q"], dsets["B"], dsets["C"],
+                                 dsets["log_dt"], dsets["D"], y_host=y_host, K=dsets["K"], u_dev=dsets["u"],
+                                 y_dev=dsets["y"], workspace=dsets["ws"], chunks=E2E_CHUNKS)
 
     e2e_ms = float("nan")
     if not args.no_e2e:
@@ -431,7 +437,11 @@ def run_gpu(args, rank, world, local_rank):
                    "algorithmic_flop": alg["kernel_flop"]},
         "e2e": None if args.no_e2e else {"value": job_throughput(alg["elements"], world, args.steps, e2e_ms),
                                          "unit": UNIT,
-                                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                                         "call": ("s4d_kernel_vandermonde + s4_fft_conv_host" if s4d
+                                                  else "s4_forward_dplr_host")
+                                         + f", pinned host u/y, {E2E_CHUNKS} row-pair chunks, parameters"
+                                         " copied up every step"},
         "gpu_launches": launches_per_step * args.steps,
         "decode": decode,
         "clocks": clk,

@@ -182,6 +182,45 @@ s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P,
                           cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Host-buffer forms: s4_fft_conv and s4_forward_dplr with u and y in HOST
+ * memory, the copies pipelined with the convolution. The batch is cut into
+ * nchunks chunks of whole row pairs; chunk c is uploaded on h2d_stream,
+ * convolved on `stream` once it has arrived, and downloaded on d2h_stream
+ * once convolved, so the upload of one chunk, the convolution of the next
+ * earlier one and the download of the one before overlap (the two copy
+ * directions run on separate copy engines). The kernel spectrum
+ * (s4_fft_conv_host) or the kernel generation (s4_forward_dplr_host) runs
+ * on `stream` first, overlapping the first upload. The uploads wait for the
+ * work already queued on `stream`; `stream` waits for the last download, so
+ * synchronising `stream` completes y_host. Results equal those of the
+ * device-buffer forms.
+ *   u_host, y_host : [Bt, H, L] host memory; page-locked memory
+ *                    (cudaHostAlloc, cudaHostRegister) lets the copies run
+ *                    asynchronously and overlap, pageable memory still works.
+ *   u_dev, y_dev   : [Bt, H, L] device staging buffers owned by the caller
+ *                    (16-byte aligned, not overlapping each other, K, D,
+ *                    the workspace or the parameters).
+ *   nchunks        : >= 1 (clamped to the number of row pairs).
+ *   h2d_stream, d2h_stream : caller-owned streams (may be `stream` itself,
+ *                    which serialises the pipeline).
+ * The call creates and releases a few CUDA events; it allocates no memory.
+ * Errors: as the device-buffer forms; null host pointers, overlapping host
+ * buffers or nchunks < 1 -> S4_ERR_INVALID_ARG.
+ * ------------------------------------------------------------------------ */
+s4_status s4_fft_conv_host(const float *u_host, const float *K, const float *D, int Bt, int H, int L,
+                           float *y_host, float *u_dev, float *y_dev, void *workspace,
+                           size_t workspace_bytes, int nchunks, cudaStream_t stream,
+                           cudaStream_t h2d_stream, cudaStream_t d2h_stream);
+
+s4_status s4_forward_dplr_host(const float *u_host, const s4_c32 *Lambda, const s4_c32 *P,
+                               const s4_c32 *Q, const s4_c32 *B, const s4_c32 *C,
+                               const float *log_dt, const float *D, int Bt, int H, int Nh, int L,
+                               float *y_host, float *K, float *u_dev, float *y_dev, void *workspace,
+                               size_t workspace_bytes, unsigned *d_flags, int nchunks,
+                               cudaStream_t stream, cudaStream_t h2d_stream,
+                               cudaStream_t d2h_stream);
+
+/* ------------------------------------------------------------------------
  * s4_fft_conv_static -- s4_fft_conv without a caller-provided workspace.
  * The pages have no counterpart of this entry point; it exists for callers
  * that cannot allocate device memory: a plugin inside a host application
@@ -247,6 +286,25 @@ s4_status s4_dplr_discretize(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32
 s4_status s4d_discretize_zoh(const s4_c32 *A, const s4_c32 *B, const float *log_dt,
                              int H, int Nh, s4_c32 *Abar, s4_c32 *Bbar,
                              cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * s4_dplr_ctilde: Ctilde = C (I - Abar^L) over the full conjugate-closed
+ * bilinear system (Abar as s4_dplr_discretize). The generating function at
+ * the L-th roots of unity gives the aliased kernel sum_p K_{k + pL}
+ * ([S4K] §4, "Aliasing"); with Ctilde in place of C, s4_kernel_dplr (and
+ * s4_forward_dplr) return the truncated kernel Cbar Abar^k Bbar, k < L,
+ * whose convolution equals the recurrence from a zero state exactly.
+ * c = C_f is carried through L products c <- c Abar in the structured form
+ * of s4_dplr_discretize_structured, in fp64 (O(L Nh) per channel, one warp
+ * per channel; a one-time reparameterisation, not a per-step cost).
+ *   Lambda, P, Q, C : [H, Nh] complex; log_dt : [H]; L >= 1.
+ *   Ctilde : [H, Nh] complex out (stored half); may not alias the inputs.
+ * Errors: null pointers, L < 1, H or Nh < 1 -> S4_ERR_INVALID_ARG;
+ * Nh > S4_MAX_NH or H > S4_MAX_H -> S4_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+s4_status s4_dplr_ctilde(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *C,
+                         const float *log_dt, int H, int Nh, int L, s4_c32 *Ctilde,
+                         cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * s4_dplr_discretize_structured: the same bilinear DPLR discretisation

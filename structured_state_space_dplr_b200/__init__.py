@@ -24,7 +24,8 @@ __all__ = [
     "fft_conv_static",
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
-    "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "load",
+    "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "dplr_ctilde", "forward_dplr_host",
+    "fft_conv_host", "load",
 ]
 
 
@@ -217,6 +218,71 @@ def forward_dplr(u, Lambda, P, Q, B, C, log_dt, D, *, out=None, K=None, workspac
     return out
 
 
+_copy_streams = {}
+
+
+def _host(t, name):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.float32:
+        raise TypeError(f"{name} must be a float32 CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _host_call_buffers(u_host, y_host, u_dev, y_dev, dev):
+    u_host = _host(u_host, "u_host")
+    if y_host is None:
+        y_host = torch.empty(u_host.shape, dtype=torch.float32, pin_memory=u_host.is_pinned())
+    _host(y_host, "y_host")
+    if u_dev is None:
+        u_dev = torch.empty(u_host.shape, dtype=torch.float32, device=dev)
+    if y_dev is None:
+        y_dev = torch.empty(u_host.shape, dtype=torch.float32, device=dev)
+    _cuda(u_dev, "u_dev", torch.float32)
+    _cuda(y_dev, "y_dev", torch.float32)
+    key = torch.cuda.current_device()
+    if key not in _copy_streams:   # one upload and one download stream per device
+        _copy_streams[key] = (torch.cuda.Stream(), torch.cuda.Stream())
+    h2d, d2h = _copy_streams[key]
+    return y_host, u_dev, y_dev, ctypes.c_void_p(h2d.cuda_stream), ctypes.c_void_p(d2h.cuda_stream)
+
+
+def forward_dplr_host(u_host, Lambda, P, Q, B, C, log_dt, D, *, y_host=None, K=None, u_dev=None, y_dev=None,
+                      workspace=None, flags=None, chunks=8):
+    """forward_dplr with u and y in host memory (s4_forward_dplr_host): the
+    uploads, convolutions and downloads of `chunks` row-pair chunks overlap.
+    u_host: float32 CPU tensor [Bt, H, L] (pinned memory for overlap).
+    Returns y_host, complete once torch's current stream is synchronised."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    D = _cuda(D, "D", torch.float32)
+    dev = Lambda.device
+    y_host, u_dev, y_dev, h2d, d2h = _host_call_buffers(u_host, y_host, u_dev, y_dev, dev)
+    Bt, H, L = u_host.shape
+    Nh = Lambda.shape[1]
+    if K is None:
+        K = torch.empty(H, L, device=dev, dtype=torch.float32)
+    workspace = _workspace(H, L, dev, workspace)
+    _lib.call("s4_forward_dplr_host", _ptr(u_host), _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C),
+              _ptr(log_dt), _ptr(D), Bt, H, Nh, L, _ptr(y_host), _ptr(K), _ptr(u_dev), _ptr(y_dev),
+              _ptr(workspace), workspace.numel(), _flags_ptr(flags), int(chunks), _stream(), h2d, d2h)
+    return y_host
+
+
+def fft_conv_host(u_host, K, D, *, y_host=None, u_dev=None, y_dev=None, workspace=None, chunks=8):
+    """fft_conv with u and y in host memory (s4_fft_conv_host); K, D on the
+    device. Returns y_host, complete once torch's current stream is
+    synchronised."""
+    K = _cuda(K, "K", torch.float32)
+    D = _cuda(D, "D", torch.float32)
+    y_host, u_dev, y_dev, h2d, d2h = _host_call_buffers(u_host, y_host, u_dev, y_dev, K.device)
+    Bt, H, L = u_host.shape
+    workspace = _workspace(H, L, K.device, workspace)
+    _lib.call("s4_fft_conv_host", _ptr(u_host), _ptr(K), _ptr(D), Bt, H, L, _ptr(y_host), _ptr(u_dev),
+              _ptr(y_dev), _ptr(workspace), workspace.numel(), int(chunks), _stream(), h2d, d2h)
+    return y_host
+
+
 def s4d_kernel_vandermonde(A, B, C, log_dt, L, *, out=None, flags=None):
     """S4D ZOH truncated kernel K [H, L] (s4d_kernel_vandermonde)."""
     A, B, C = (_cplx(x, n) for x, n in zip((A, B, C), "A B C".split()))
@@ -257,6 +323,18 @@ def dplr_discretize_structured(Lambda, P, Q, B, log_dt):
     _lib.call("s4_dplr_discretize_structured", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(log_dt),
               H, Nh, _ptr(Astr), _ptr(Bb), _stream())
     return Astr, Bb
+
+
+def dplr_ctilde(Lambda, P, Q, C, log_dt, L):
+    """Ctilde = C (I - Abar^L) [H, Nh] complex64: used in place of C, the
+    generated kernel is the truncated one (Cbar Abar^k Bbar, k < L)."""
+    Lambda, P, Q, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, C), "Lambda P Q C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    Ct = torch.empty_like(C)
+    _lib.call("s4_dplr_ctilde", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(C), _ptr(log_dt), H, Nh, int(L),
+              _ptr(Ct), _stream())
+    return Ct
 
 
 def s4d_discretize_zoh(A, B, log_dt):

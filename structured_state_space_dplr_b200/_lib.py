@@ -38,6 +38,10 @@ SIGNATURES = {
     "s4d_kernel_vandermonde": (_i, [_p, _p, _p, _p, _i, _i, _i, _p, _p, _p]),
     "s4_dplr_discretize": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _p, _p, _p, _p]),
     "s4_dplr_discretize_structured": (_i, [_p, _p, _p, _p, _p, _i, _i, _p, _p, _p]),
+    "s4_dplr_ctilde": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
+    "s4_fft_conv_host": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _p, _p, _sz, _i, _p, _p, _p]),
+    "s4_forward_dplr_host": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p,
+                                  _i, _p, _p, _p]),
     "s4d_discretize_zoh": (_i, [_p, _p, _p, _i, _i, _p, _p, _p]),
     "s4_recurrent_step": (_i, [_i, _p, _p, _p, _p, _i, _i, _i, _p, _p, _p, _p]),
     "s4_recurrent_scan": (_i, [_i, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _p]),

@@ -2,6 +2,7 @@
 // documented in include/s4dplr.h). Every argument is checked on the host
 // before anything is launched; nothing here allocates device memory.
 #include <cstdint>
+#include <vector>
 
 #include "launch.h"
 #include "s4dplr.h"
@@ -63,6 +64,63 @@ s4_status prepare_checks(const float *K, const float *D, int H, int L, const voi
     if (overlap(K, (size_t)H * L * sizeof(float), ws, ws_bytes)) return S4_ERR_INVALID_ARG;
     if (D != nullptr && overlap(D, (size_t)H * sizeof(float), ws, ws_bytes)) return S4_ERR_INVALID_ARG;
     return S4_OK;
+}
+
+// The convolution of a batch held in host memory. Chunk c (whole row pairs)
+// is uploaded on h2d, convolved on st once it has arrived and downloaded on
+// d2h once convolved, so uploads, convolutions and downloads of consecutive
+// chunks overlap (the two copy directions use separate copy engines). The
+// uploads start only after the work already queued on st (an earlier call
+// may still read u_dev or write y_dev); st waits for the last download, so a
+// caller that synchronises st sees y_host complete.
+cudaError_t conv_host_pipeline(const float *u_host, const void *ws, int Bt, int H, int L, float *y_host,
+                               float *u_dev, float *y_dev, int nchunks, cudaStream_t st, cudaStream_t h2d,
+                               cudaStream_t d2h, cudaEvent_t start) {
+    const int npairs = (Bt + 1) / 2;
+    if (nchunks > npairs) nchunks = npairs;
+    const int pairs_per_chunk = (npairs + nchunks - 1) / nchunks;
+    nchunks = (npairs + pairs_per_chunk - 1) / pairs_per_chunk;
+    const size_t row = (size_t)H * L;
+    std::vector<cudaEvent_t> ev(2 * (size_t)nchunks + 1, nullptr);
+    cudaError_t e = cudaSuccess;
+    for (auto &x : ev)
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h2d, start, 0);
+    for (int c = 0; c < nchunks && e == cudaSuccess; ++c) {
+        const int b0 = 2 * c * pairs_per_chunk;
+        const int b1 = (b0 + 2 * pairs_per_chunk) < Bt ? b0 + 2 * pairs_per_chunk : Bt;
+        const size_t off = (size_t)b0 * row, bytes = (size_t)(b1 - b0) * row * sizeof(float);
+        e = cudaMemcpyAsync(u_dev + off, u_host + off, bytes, cudaMemcpyHostToDevice, h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[2 * c], h2d);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev[2 * c], 0);
+        if (e == cudaSuccess) e = s4::launch_fftconv(u_dev + off, ws, b1 - b0, H, L, y_dev + off, st);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[2 * c + 1], st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(d2h, ev[2 * c + 1], 0);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(y_host + off, y_dev + off, bytes, cudaMemcpyDeviceToHost, d2h);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev.back(), d2h);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev.back(), 0);
+    for (auto &x : ev)   // released by the runtime once their work completes
+        if (x != nullptr) cudaEventDestroy(x);
+    return e;
+}
+
+// checks shared by the two host-buffer entry points
+s4_status host_buffer_checks(const float *u_host, const float *y_host, const float *u_dev, const float *y_dev,
+                             int Bt, int H, int L, const void *ws, size_t ws_bytes, int nchunks) {
+    if (any_null(u_host, y_host) || nchunks < 1) return S4_ERR_INVALID_ARG;
+    s4_status s = conv_checks(u_dev, Bt, H, L, y_dev, ws, ws_bytes);
+    if (s != S4_OK) return s;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float);
+    if (overlap(u_host, nb, y_host, nb) || overlap(u_dev, nb, ws, ws_bytes)) return S4_ERR_INVALID_ARG;
+    return S4_OK;
+}
+
+// an event marking the work queued on st so far
+cudaError_t mark(cudaStream_t st, cudaEvent_t *ev) {
+    cudaError_t e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(*ev, st);
+    return e;
 }
 
 }  // namespace
@@ -203,6 +261,57 @@ s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P,
     return cuda_status(e);
 }
 
+s4_status s4_fft_conv_host(const float *u_host, const float *K, const float *D, int Bt, int H, int L,
+                           float *y_host, float *u_dev, float *y_dev, void *workspace, size_t workspace_bytes,
+                           int nchunks, cudaStream_t stream, cudaStream_t h2d_stream, cudaStream_t d2h_stream) {
+    if (D == nullptr) return S4_ERR_INVALID_ARG;
+    s4_status s = host_buffer_checks(u_host, y_host, u_dev, y_dev, Bt, H, L, workspace, workspace_bytes, nchunks);
+    if (s == S4_OK) s = prepare_checks(K, D, H, L, workspace, workspace_bytes);
+    if (s != S4_OK) return s;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float), kb = (size_t)H * L * sizeof(float);
+    if (overlap(y_dev, nb, K, kb) || overlap(u_dev, nb, K, kb) || overlap(y_dev, nb, D, (size_t)H * sizeof(float)))
+        return S4_ERR_INVALID_ARG;
+    cudaEvent_t start = nullptr;
+    cudaError_t e = mark(stream, &start);
+    if (e == cudaSuccess) e = s4::launch_kspec(K, D, H, L, workspace, stream);
+    if (e == cudaSuccess)
+        e = conv_host_pipeline(u_host, workspace, Bt, H, L, y_host, u_dev, y_dev, nchunks, stream, h2d_stream,
+                               d2h_stream, start);
+    if (start != nullptr) cudaEventDestroy(start);
+    return cuda_status(e);
+}
+
+s4_status s4_forward_dplr_host(const float *u_host, const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                               const s4_c32 *B, const s4_c32 *C, const float *log_dt, const float *D, int Bt,
+                               int H, int Nh, int L, float *y_host, float *K, float *u_dev, float *y_dev,
+                               void *workspace, size_t workspace_bytes, unsigned *d_flags, int nchunks,
+                               cudaStream_t stream, cudaStream_t h2d_stream, cudaStream_t d2h_stream) {
+    if (D == nullptr) return S4_ERR_INVALID_ARG;
+    s4_status s = host_buffer_checks(u_host, y_host, u_dev, y_dev, Bt, H, L, workspace, workspace_bytes, nchunks);
+    if (s == S4_OK) s = dplr_checks(Lambda, P, Q, B, C, log_dt, H, Nh, L, K);
+    if (s == S4_OK) s = prepare_checks(K, D, H, L, workspace, workspace_bytes);
+    if (s != S4_OK) return s;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float), kb = (size_t)H * L * sizeof(float);
+    if (overlap(y_dev, nb, K, kb) || overlap(u_dev, nb, K, kb) || overlap(y_dev, nb, D, (size_t)H * sizeof(float)))
+        return S4_ERR_INVALID_ARG;
+    for (const void *p : {(const void *)Lambda, (const void *)P, (const void *)Q, (const void *)B,
+                          (const void *)C})
+        if (overlap(workspace, workspace_bytes, p, (size_t)H * Nh * sizeof(s4_c32)) ||
+            overlap(y_dev, nb, p, (size_t)H * Nh * sizeof(s4_c32)) ||
+            overlap(u_dev, nb, p, (size_t)H * Nh * sizeof(s4_c32)))
+            return S4_ERR_INVALID_ARG;
+    cudaEvent_t start = nullptr;
+    cudaError_t e = mark(stream, &start);   // the first upload overlaps the kernel generation
+    if (e == cudaSuccess)
+        e = s4::launch_kgen((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q, (const float2 *)B,
+                            (const float2 *)C, log_dt, D, H, Nh, L, K, workspace, d_flags, stream);
+    if (e == cudaSuccess)
+        e = conv_host_pipeline(u_host, workspace, Bt, H, L, y_host, u_dev, y_dev, nchunks, stream, h2d_stream,
+                               d2h_stream, start);
+    if (start != nullptr) cudaEventDestroy(start);
+    return cuda_status(e);
+}
+
 s4_status s4d_kernel_vandermonde(const s4_c32 *A, const s4_c32 *B, const s4_c32 *C, const float *log_dt,
                                  int H, int Nh, int L, float *K, unsigned *d_flags, cudaStream_t stream) {
     if (any_null(A, B, C) || log_dt == nullptr || K == nullptr) return S4_ERR_INVALID_ARG;
@@ -241,6 +350,17 @@ s4_status s4_dplr_discretize_structured(const s4_c32 *Lambda, const s4_c32 *P, c
     return cuda_status(s4::launch_dplr_discretize_structured((const float2 *)Lambda, (const float2 *)P,
                                                              (const float2 *)Q, (const float2 *)B, log_dt, H,
                                                              Nh, (float2 *)Astr, (float2 *)Bbar, stream));
+}
+
+s4_status s4_dplr_ctilde(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *C,
+                         const float *log_dt, int H, int Nh, int L, s4_c32 *Ctilde, cudaStream_t stream) {
+    if (any_null(Lambda, P, Q, C) || Ctilde == nullptr || log_dt == nullptr) return S4_ERR_INVALID_ARG;
+    if (L < 1) return S4_ERR_INVALID_ARG;
+    s4_status s = check_modes(H, Nh, 0, false);
+    if (s != S4_OK) return s;
+    if (!params_aligned({Lambda, P, Q, C, Ctilde})) return S4_ERR_INVALID_ARG;
+    return cuda_status(s4::launch_dplr_ctilde((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q,
+                                              (const float2 *)C, log_dt, H, Nh, L, (float2 *)Ctilde, stream));
 }
 
 s4_status s4d_discretize_zoh(const s4_c32 *A, const s4_c32 *B, const float *log_dt, int H, int Nh,

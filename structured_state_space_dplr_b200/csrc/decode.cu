@@ -178,6 +178,38 @@ __global__ void k_step_diag(const float2 *__restrict__ Abar, const float2 *__res
         if (lane + 32 * k < Nh) x[(size_t)w * Nh + lane + 32 * k] = s[k];
 }
 
+// Per-mode terms of the Sherman-Morrison inverse of I - dt/2 A, in fp64:
+// 1/d, alpha = (dt/2) P / d, beta = conj(Q) / d, with d = 1 - dt/2 Lambda.
+struct SmTerms {
+    double ir, ii, ar, ai, br, bi;
+};
+__device__ __forceinline__ SmTerms sm_terms(float2 lf, float2 pf, float2 qf, double dt) {
+    SmTerms t;
+    const double dr = 1.0 - 0.5 * dt * lf.x, di = -0.5 * dt * lf.y, dd = dr * dr + di * di;
+    t.ir = dr / dd;
+    t.ii = -di / dd;
+    t.ar = 0.5 * dt * (pf.x * t.ir - pf.y * t.ii);
+    t.ai = 0.5 * dt * (pf.x * t.ii + pf.y * t.ir);
+    t.br = qf.x * t.ir + qf.y * t.ii;
+    t.bi = qf.x * t.ii - qf.y * t.ir;
+    return t;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+// s = 1 + 2 Re sum_n conj(Q_n) alpha_n over channel h's modes (all lanes)
+__device__ __forceinline__ double sm_denominator(const float2 *Lambda, const float2 *P, const float2 *Q,
+                                                 size_t po, int Nh, double dt, int lane) {
+    double s1 = 0.0;
+    for (int n = lane; n < Nh; n += 32) {
+        const float2 qf = Q[po + n];
+        const SmTerms t = sm_terms(Lambda[po + n], P[po + n], qf, dt);
+        s1 += qf.x * t.ar + qf.y * t.ai;
+    }
+    return 1.0 + 2.0 * warp_sum(s1);
+}
+
 // Structured transition of the bilinear DPLR system: one warp per channel,
 // lanes striding over the stored modes, fp64 arithmetic.
 //   Astr[h, n] = {a_n, g_n, beta_n},  Bbar[h, n] (stored half of Bbar).
@@ -190,37 +222,89 @@ __global__ void k_dplr_discretize_structured(const float2 *__restrict__ Lambda, 
     if (h >= H) return;
     const double dt = exp((double)__ldg(log_dt + h));
     const size_t po = (size_t)h * Nh;
-    // pass 1: s - 1 = 2 Re sum conj(Q) alpha, and 2 Re sum beta B (= beta^T B_f)
-    double s1 = 0.0, sb = 0.0;
+    const double s = sm_denominator(Lambda, P, Q, po, Nh, dt, lane);
+    double sb = 0.0;   // Re sum beta B, half of beta^T B_f
     for (int n = lane; n < Nh; n += 32) {
-        const float2 lf = Lambda[po + n], pf = P[po + n], qf = Q[po + n], bf = B[po + n];
-        const double dr = 1.0 - 0.5 * dt * lf.x, di = -0.5 * dt * lf.y, dd = dr * dr + di * di;
-        const double ir = dr / dd, ii = -di / dd;                              // 1/d
-        const double ar = 0.5 * dt * (pf.x * ir - pf.y * ii), ai = 0.5 * dt * (pf.x * ii + pf.y * ir);
-        const double br = qf.x * ir + qf.y * ii, bi = qf.x * ii - qf.y * ir;   // conj(q)/d
-        s1 += qf.x * ar + qf.y * ai;                                           // Re(conj(q) alpha)
-        sb += br * bf.x - bi * bf.y;                                           // Re(beta b)
+        const SmTerms t = sm_terms(Lambda[po + n], P[po + n], Q[po + n], dt);
+        const float2 bf = B[po + n];
+        sb += t.br * bf.x - t.bi * bf.y;
     }
-    for (int off = 16; off > 0; off >>= 1) {
-        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
-        sb += __shfl_xor_sync(0xffffffffu, sb, off);
-    }
-    const double s = 1.0 + 2.0 * s1, tb = 2.0 * sb;
-    // pass 2: the coefficients
+    const double tb = 2.0 * warp_sum(sb);
     for (int n = lane; n < Nh; n += 32) {
-        const float2 lf = Lambda[po + n], pf = P[po + n], qf = Q[po + n], bf = B[po + n];
-        const double dr = 1.0 - 0.5 * dt * lf.x, di = -0.5 * dt * lf.y, dd = dr * dr + di * di;
-        const double ir = dr / dd, ii = -di / dd;
-        const double ar = 0.5 * dt * (pf.x * ir - pf.y * ii), ai = 0.5 * dt * (pf.x * ii + pf.y * ir);
-        const double br = qf.x * ir + qf.y * ii, bi = qf.x * ii - qf.y * ir;
+        const SmTerms t = sm_terms(Lambda[po + n], P[po + n], Q[po + n], dt);
+        const float2 bf = B[po + n];
         float2 *o = Astr + 3 * (po + n);
-        o[0] = make_float2((float)(2.0 * ir - 1.0), (float)(2.0 * ii));       // a = 2/d - 1
-        o[1] = make_float2((float)(2.0 * ar / s), (float)(2.0 * ai / s));      // g = 2 alpha / s
-        o[2] = make_float2((float)br, (float)bi);                              // beta
+        o[0] = make_float2((float)(2.0 * t.ir - 1.0), (float)(2.0 * t.ii));       // a = 2/d - 1
+        o[1] = make_float2((float)(2.0 * t.ar / s), (float)(2.0 * t.ai / s));      // g = 2 alpha / s
+        o[2] = make_float2((float)t.br, (float)t.bi);                              // beta
         // Bbar = dt (b/d - alpha beta^T B_f / s)
-        Bbar[po + n] = make_float2((float)(dt * (bf.x * ir - bf.y * ii - ar * tb / s)),
-                                   (float)(dt * (bf.x * ii + bf.y * ir - ai * tb / s)));
+        Bbar[po + n] = make_float2((float)(dt * (bf.x * t.ir - bf.y * t.ii - t.ar * tb / s)),
+                                   (float)(dt * (bf.x * t.ii + bf.y * t.ir - t.ai * tb / s)));
     }
+}
+
+// Ctilde = C (I - Abar^L): the row vector c = C_f is carried through L
+// products c <- c Abar = c o a - (c . g) beta^T (the transpose of the
+// structured step; c stays conjugate symmetric, so c . g = 2 Re sum_n c_n g_n),
+// in fp64, one warp per channel.
+__global__ void k_dplr_ctilde(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
+                              const float2 *__restrict__ Q, const float2 *__restrict__ C,
+                              const float *__restrict__ log_dt, int H, int Nh, int L,
+                              float2 *__restrict__ Ct) {
+    constexpr int MAXM = 8;   // modes per lane (Nh <= 256)
+    const int h = (int)((blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (h >= H) return;
+    const double dt = exp((double)__ldg(log_dt + h));
+    const size_t po = (size_t)h * Nh;
+    const double s = sm_denominator(Lambda, P, Q, po, Nh, dt, lane);
+    double ar[MAXM], ai[MAXM], gr[MAXM], gi[MAXM], br[MAXM], bi[MAXM], cr[MAXM], ci[MAXM];
+#pragma unroll
+    for (int k = 0; k < MAXM; ++k) {
+        const int n = lane + 32 * k;
+        ar[k] = ai[k] = gr[k] = gi[k] = br[k] = bi[k] = cr[k] = ci[k] = 0.0;
+        if (n < Nh) {
+            const SmTerms t = sm_terms(Lambda[po + n], P[po + n], Q[po + n], dt);
+            ar[k] = 2.0 * t.ir - 1.0;
+            ai[k] = 2.0 * t.ii;
+            gr[k] = 2.0 * t.ar / s;
+            gi[k] = 2.0 * t.ai / s;
+            br[k] = t.br;
+            bi[k] = t.bi;
+            const float2 c = C[po + n];
+            cr[k] = c.x;
+            ci[k] = c.y;
+        }
+    }
+    for (int step = 0; step < L; ++step) {
+        double cg = 0.0;
+#pragma unroll
+        for (int k = 0; k < MAXM; ++k) cg += cr[k] * gr[k] - ci[k] * gi[k];
+        cg = 2.0 * warp_sum(cg);
+#pragma unroll
+        for (int k = 0; k < MAXM; ++k) {
+            const double nr = cr[k] * ar[k] - ci[k] * ai[k] - cg * br[k];
+            const double ni = cr[k] * ai[k] + ci[k] * ar[k] - cg * bi[k];
+            cr[k] = nr;
+            ci[k] = ni;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < MAXM; ++k) {
+        const int n = lane + 32 * k;
+        if (n < Nh) {
+            const float2 c = C[po + n];
+            Ct[po + n] = make_float2((float)((double)c.x - cr[k]), (float)((double)c.y - ci[k]));
+        }
+    }
+}
+
+cudaError_t launch_dplr_ctilde(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *C,
+                               const float *log_dt, int H, int Nh, int L, float2 *Ct, cudaStream_t st) {
+    const int per_block = 4;
+    k_dplr_ctilde<<<(H + per_block - 1) / per_block, 32 * per_block, 0, st>>>(Lambda, P, Q, C, log_dt, H, Nh,
+                                                                            L, Ct);
+    return cudaGetLastError();
 }
 
 // Structured DPLR recurrence: one warp per row (b, h), lanes stride over the

@@ -44,6 +44,8 @@ cudaError_t launch_dplr_discretize(const float2 *Lambda, const float2 *P, const 
 cudaError_t launch_dplr_discretize_structured(const float2 *Lambda, const float2 *P, const float2 *Q,
                                               const float2 *B, const float *log_dt, int H, int Nh,
                                               float2 *Astr, float2 *Bbar, cudaStream_t st);
+cudaError_t launch_dplr_ctilde(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *C,
+                               const float *log_dt, int H, int Nh, int L, float2 *Ct, cudaStream_t st);
 cudaError_t launch_step(int mode, const float2 *Abar, const float2 *Bbar, const float2 *C, const float *D,
                         int Bt, int H, int Ns, int T, float2 *x, const float *u, float *y, cudaStream_t st);
 

@@ -1,0 +1,42 @@
+"""The host-buffer entry points (s4_forward_dplr_host, s4_fft_conv_host):
+chunked uploads, convolutions and downloads give exactly the device-buffer
+results, and the oracle's."""
+import numpy as np
+import pytest
+
+import s4inputs
+from oracle import workloads
+from gpu_helpers import Y_TOL, rel_l2, to_dev, torch_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("Bt,chunks,pinned", [(5, 2, True), (4, 1, False), (3, 8, True), (16, 8, True)])
+def test_forward_dplr_host_equals_device_path(Bt, chunks, pinned):
+    import structured_state_space_dplr_b200 as s4
+    torch = torch_cuda()
+    inp = s4inputs.make_inputs(2, H=16, Bt=Bt, L=512)
+    t = to_dev(inp)
+    y_dev = s4.forward_dplr(t["u"], t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], t["D"])
+    u_host = torch.from_numpy(inp["u"].copy())
+    if pinned:
+        u_host = u_host.pin_memory()
+    y_host = s4.forward_dplr_host(u_host, t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], t["D"],
+                                  chunks=chunks)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(y_host, y_dev.cpu())
+
+
+def test_fft_conv_host_matches_device_path_and_oracle():
+    import structured_state_space_dplr_b200 as s4
+    torch = torch_cuda()
+    inp = s4inputs.make_inputs(1)   # H = 4, L = 1024, batch 2
+    t = to_dev(inp)
+    K = s4.kernel_dplr(t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], inp["L"])
+    y_dev = s4.fft_conv(t["u"], K, t["D"])
+    y_host = s4.fft_conv_host(torch.from_numpy(inp["u"].copy()).pin_memory(), K, t["D"], chunks=3)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(y_host, y_dev.cpu())
+    Kr = workloads.dplr_kernel(inp)
+    yr = workloads.conv_full(inp, Kr)
+    assert rel_l2(y_host.numpy(), yr) <= Y_TOL
