@@ -245,7 +245,7 @@ def run_gpu(args, rank, world, local_rank):
     if s4d:
         gen_launches = 2 + (1 if L == 65536 else 0)
     else:
-        gen_launches = 1 if L <= 4096 else (3 + (1 if L == 65536 else 0))
+        gen_launches = 1 if L <= 8192 else (3 + (1 if L == 65536 else 0))
     launches_per_step = gen_launches + conv_launches
     for i in range(args.warmup):
         gen_stage(sets[i % nsets])
@@ -423,11 +423,13 @@ def run_gpu(args, rank, world, local_rank):
         "config": {"workload": c["name"], "H": H, "N": c["N"], "L": L, "batch": Bt,
                    "global_batch": Bt * world, "dt_range": [c["dt_min"], c["dt_max"]],
                    "parallelism": f"channel shard x{world}, no collective",
-                   "launch": "per step: s4_kernel_dplr_prepare + s4_fft_conv_apply, each replayed from a CUDA graph",
+                   "launch": ("per step: s4d_kernel_vandermonde + s4_fft_conv_prepare" if s4d
+                              else "per step: s4_kernel_dplr_prepare")
+                             + " + s4_fft_conv_apply, each stage replayed from a CUDA graph",
                    "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
         "stages_ms": {"kernel_and_spectrum": stage[0], "fft_conv": stage[1],
                       ("vandermonde_alone" if s4d else "cauchy_spectrum_alone"): stage[2]},
-        "roofline": {"kernel": "k_fftconv_pair" if L <= 4096 else "k_fftconv", "bound": "hbm", "achieved": conv_gbs, "peak": hbm,
+        "roofline": {"kernel": "k_fftconv_pair" if L <= 8192 else "k_fftconv", "bound": "hbm", "achieved": conv_gbs, "peak": hbm,
                      "unit": "GB/s", "frac": conv_gbs / hbm, "traffic": traffic,
                      "peak_source": peak_src, "algorithmic_bytes": alg["conv_bytes"]},
         "cauchy": {"kernel": "k_vandermonde" if s4d else "k_cauchy", "bound": "alu", "achieved": cauchy_tflops,

@@ -111,6 +111,79 @@ __device__ __forceinline__ void pair_stage_rows(const PairSmem &s, const float *
     cp_async_commit();
 }
 
+// ------------------------------------------------------ both halves, pass 0 --
+// First forward pass of group j of both halves of the zero-padded length-2m
+// transform, from the m nonzero inputs v[p] = input point j + p S0: half 0
+// (even frequencies) transforms v as it is, half 1 (odd frequencies) after
+// the twist W_2m^-k, whose in-group share W_2R0^-p is a constant rotation and
+// whose remainder a_j b_j^q is applied with the group twiddles b_j^q.
+template <int LG>
+__device__ __forceinline__ void first_pass_halves(const PairSmem &s, const float2 (&v)[1 << plan_lr(LG, 0)],
+                                                  int j) {
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = (1 << LG) / R0;
+    float2 x[R0], z[R0];
+    static_for<0, R0>([&](auto p) {
+        x[p] = v[p];
+        z[p] = rot<decltype(p)::value, 2 * R0, -1>(v[p]);
+    });
+    dft<R0, -1>(x);
+    dft<R0, -1>(z);
+    const float2 a = s.ta[j], b = s.tb[j];
+    float2 w = b, u = a;
+    const int o = pidx(j);
+    s.b0[o] = x[0];
+    s.b1[o] = cmul(z[0], a);
+    static_for<1, R0>([&](auto q) {
+        u = cmul(u, b);
+        s.b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+        s.b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], u);
+        w = cmul(w, b);
+    });
+}
+
+// After the first pass of both halves (stored, all threads synced): forward
+// passes 1 .. P-1, then (spectrum + D) / 2L to spec_h in spec4_index order,
+// rank 0 then rank 1. Adding D to every frequency adds D delta_0 to K.
+template <int LG>
+__device__ __forceinline__ void spectrum_tail(const PairSmem &s, float Dh, float2 *__restrict__ spec_h) {
+    constexpr int m = 1 << LG, T = pair_threads<LG>();
+    constexpr int R = 1 << plan_lr(LG, plan_P(LG) - 1);
+    forward_middle_x2<LG, T>(s.b0, s.b1, s.tws);
+    const float scale = 1.0f / (float)(2 * m);
+    float4 *o0 = reinterpret_cast<float4 *>(spec_h);
+    float4 *o1 = o0 + m / 2;
+    for (int g = threadIdx.x; g < m / R; g += T) {
+        const int base = g * R, o = pidx(base);
+        float2 x[R], z[R];
+        load_contig<R>(s.b0 + o, x);
+        load_contig<R>(s.b1 + o, z);
+        dft<R, -1>(x);
+        dft<R, -1>(z);
+        static_for<0, R / 2>([&](auto i) {
+            o0[spec4_index<LG>(base, i)] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
+                                                       (x[2 * i + 1].x + Dh) * scale, x[2 * i + 1].y * scale);
+            o1[spec4_index<LG>(base, i)] = make_float4((z[2 * i].x + Dh) * scale, z[2 * i].y * scale,
+                                                       (z[2 * i + 1].x + Dh) * scale, z[2 * i + 1].y * scale);
+        });
+    }
+}
+
+// The same spectrum from K[h, :] in global memory (tables built, all threads
+// synced on entry).
+template <int LG>
+__device__ __forceinline__ void kspec_channel(const PairSmem &s, const float *__restrict__ Kh, float Dh,
+                                              float2 *__restrict__ spec_h) {
+    constexpr int m = 1 << LG, T = pair_threads<LG>();
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    for (int j = threadIdx.x; j < S0; j += T) {
+        float2 v[R0];
+        static_for<0, R0>([&](auto p) { v[p] = make_float2(__ldg(Kh + j + p * S0), 0.0f); });
+        first_pass_halves<LG>(s, v, j);
+    }
+    __syncthreads();
+    spectrum_tail<LG>(s, Dh, spec_h);
+}
+
 // ------------------------------------------------------------ convolution --
 // Convolution of the staged row pair (stage ready, all threads synced) with
 // the spectrum spec_h (layout of spec4_index, rank 0 then rank 1). After the
@@ -122,28 +195,14 @@ __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__res
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     float2 *b0 = s.b0, *b1 = s.b1;
     const float *stage = s.stage;
-    // ---- first forward pass, both halves
+    // ---- first forward pass, both halves: input u0 + i u1
     for (int j = threadIdx.x; j < S0; j += T) {
-        float2 x[R0], z[R0];
+        float2 v[R0];
         static_for<0, R0>([&](auto p) {
             const int k = j + p * S0;
-            const float2 v = make_float2(stage[k], stage[L + k]);
-            x[p] = v;
-            z[p] = rot<decltype(p)::value, 2 * R0, -1>(v);
+            v[p] = make_float2(stage[k], stage[L + k]);
         });
-        dft<R0, -1>(x);
-        dft<R0, -1>(z);
-        const float2 a = s.ta[j], b = s.tb[j];
-        float2 w = b, v = a;
-        const int o = pidx(j);
-        b0[o] = x[0];
-        b1[o] = cmul(z[0], a);
-        static_for<1, R0>([&](auto q) {
-            v = cmul(v, b);
-            b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
-            b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], v);
-            w = cmul(w, b);
-        });
+        first_pass_halves<LG>(s, v, j);
     }
     __syncthreads();
     after_first();
@@ -204,36 +263,52 @@ __device__ __forceinline__ void kgen_channel(const PairSmem &s, const float2 *__
                                              const float *__restrict__ log_dt, const float *__restrict__ D,
                                              int Nh, int h, float *__restrict__ K, float2 *__restrict__ spec_h,
                                              unsigned *__restrict__ flags) {
-    constexpr int m = 1 << LG, L = m, T = pair_threads<LG>(), N = 2 * m;
+    constexpr int m = 1 << LG, L = m, T = pair_threads<LG>();
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0, NP = plan_P(LG);
     constexpr int F = 4;   // frequencies per thread per round
-    float2 *X = s.b0, *Y = s.b1;
+    float2 *X = s.b0;   // the length-L inverse transform
     float4 *sp = s.sp;
     cauchy_stage_modes<false>(Lambda, P, Q, B, Cc, h, Nh, sp, flags, threadIdx.x, T);
     __syncthreads();
 
     // ---- A: generating function -> X at digit-reversed positions (with mirror)
+    // Threads walk the positions that hold frequencies j < L/2 rather than
+    // the frequencies themselves: the top digit of j is the low digit of its
+    // position p (the radix RL of the last pass), so j < L/2 exactly when
+    // p mod RL < RL/2. Slot q goes to p = (q mod RL/2) + RL b', with the
+    // blocks b' of consecutive slots interleaved so that the two 8-lane
+    // halves of a half-warp store 4 blocks (8 bank slots) apart: the stores
+    // of a warp hit distinct banks (their mirrors at most two ways), where
+    // consecutive frequencies would land 256 points apart, all in one bank.
     const float ldt = __ldg(log_dt + h);
     const float inv_dt = expf(-ldt);
+    constexpr int RL = 1 << plan_lr(LG, NP - 1), HB = RL / 2;
+    constexpr bool SPREAD = HB == 8 && (L / RL) % 8 == 0;
+    auto slot_pos = [](int q) {
+        const int b = q / HB;
+        const int bb = SPREAD ? ((b & ~7) | ((b & 1) << 2) | ((b >> 1) & 3)) : b;
+        return q % HB + RL * bb;
+    };
     bool bad = false;
     for (int f0 = 0; f0 < L / 2; f0 += T * F) {
-        int j[F], jj[F];
+        int q[F], pos[F], jj[F];
 #pragma unroll
         for (int f = 0; f < F; ++f) {
-            j[f] = f0 + f * T + threadIdx.x;
-            jj[f] = j[f] < L / 2 ? j[f] : 0;
+            q[f] = f0 + f * T + threadIdx.x;
+            pos[f] = slot_pos(q[f] < L / 2 ? q[f] : 0);
+            jj[f] = digrev<LG>(pos[f]);   // < L/2
         }
         float2 kh[F];
         cauchy_eval<F, false>(sp, Nh, jj, L, inv_dt, kh);
 #pragma unroll
         for (int f = 0; f < F; ++f) {
-            if (j[f] < L / 2) {
+            if (q[f] < L / 2) {
                 bad |= !(isfinite(kh[f].x) && isfinite(kh[f].y));
-                if (j[f] == 0) {
+                if (jj[f] == 0) {
                     X[pidx(0)] = make_float2(kh[f].x, 0.0f);
                 } else {
-                    X[pidx(digrev_inv<LG>(j[f]))] = kh[f];
-                    X[pidx(digrev_inv<LG>(L - j[f]))] = cconj(kh[f]);
+                    X[pidx(pos[f])] = kh[f];
+                    X[pidx(digrev_inv<LG>(L - jj[f]))] = cconj(kh[f]);
                 }
             }
         }
@@ -252,62 +327,31 @@ __device__ __forceinline__ void kgen_channel(const PairSmem &s, const float2 *__
     __syncthreads();
     inverse_middle<LG, T>(X, s.tws);
 
-    // ---- B/C: last inverse pass -> K (stored), first forward pass of both halves
+    // ---- B/C: last inverse pass -> K (stored); its registers start the
+    // first forward pass of both halves (same group, same positions)
     float *Kh = K + (size_t)h * L;
     for (int j = threadIdx.x; j < S0; j += T) {
         const int o = pidx(j);
-        const float2 a = s.ta[j], b = s.tb[j];
-        float2 x[R0], z[R0];
-        {
-            float2 w = b;
-            x[0] = X[o];
-            static_for<1, R0>([&](auto q) {
-                x[q] = cmulc(X[o + poff<decltype(q)::value * S0>()], w);
-                w = cmul(w, b);
-            });
-        }
+        const float2 b = s.tb[j];
+        float2 x[R0];
+        float2 w = b;
+        x[0] = X[o];
+        static_for<1, R0>([&](auto q) {
+            x[q] = cmulc(X[o + poff<decltype(q)::value * S0>()], w);
+            w = cmul(w, b);
+        });
         dft<R0, +1>(x);
         static_for<0, R0>([&](auto p) {
             const float k = x[p].x;   // K is real: the imaginary part is rounding
             Kh[j + p * S0] = k;
             x[p] = make_float2(k, 0.0f);
-            z[p] = rot<decltype(p)::value, 2 * R0, -1>(x[p]);
         });
-        dft<R0, -1>(x);
-        dft<R0, -1>(z);
-        float2 w = b, v = a;
-        X[o] = x[0];
-        Y[o] = cmul(z[0], a);
-        static_for<1, R0>([&](auto q) {
-            v = cmul(v, b);
-            X[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
-            Y[o + poff<decltype(q)::value * S0>()] = cmul(z[q], v);
-            w = cmul(w, b);
-        });
+        first_pass_halves<LG>(s, x, j);
     }
     __syncthreads();
 
-    // ---- C: forward passes 1 .. P-2, last pass -> (spectrum + D) / 2L
-    forward_middle_x2<LG, T>(X, Y, s.tws);
-    const float Dh = D != nullptr ? __ldg(D + h) : 0.0f;
-    const float scale = 1.0f / (float)N;
-    constexpr int lr = plan_lr(LG, NP - 1), R = 1 << lr;
-    float4 *o0 = reinterpret_cast<float4 *>(spec_h);
-    float4 *o1 = o0 + m / 2;
-    for (int g = threadIdx.x; g < m / R; g += T) {
-        const int base = g * R, o = pidx(base);
-        float2 x[R], z[R];
-        load_contig<R>(X + o, x);
-        load_contig<R>(Y + o, z);
-        dft<R, -1>(x);
-        dft<R, -1>(z);
-        static_for<0, R / 2>([&](auto i) {
-            o0[spec4_index<LG>(base, i)] = make_float4((x[2 * i].x + Dh) * scale, x[2 * i].y * scale,
-                                                       (x[2 * i + 1].x + Dh) * scale, x[2 * i + 1].y * scale);
-            o1[spec4_index<LG>(base, i)] = make_float4((z[2 * i].x + Dh) * scale, z[2 * i].y * scale,
-                                                       (z[2 * i + 1].x + Dh) * scale, z[2 * i + 1].y * scale);
-        });
-    }
+    // ---- C: forward passes 1 .. P-1 -> (spectrum + D) / 2L
+    spectrum_tail<LG>(s, D != nullptr ? __ldg(D + h) : 0.0f, spec_h);
 }
 
 }  // namespace s4

@@ -288,6 +288,22 @@ k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int
     }
 }
 
+// The spectrum k_fftconv_pair reads, from K in global memory: one CTA per
+// channel, both halves of the length-2L transform (see kspec_channel).
+template <int LG>
+__global__ void __launch_bounds__(pair_threads<LG>(), pair_min_blocks<LG>())
+k_kspec_pair(const float *__restrict__ K, const float *__restrict__ D, int H, float2 *__restrict__ spec) {
+    extern __shared__ float2 sm[];
+    const PairSmem s = pair_carve<LG>(sm);
+    pair_tables<LG>(s);
+    __syncthreads();
+    for (int h = blockIdx.x; h < H; h += gridDim.x) {
+        kspec_channel<LG>(s, K + (size_t)h * (1 << LG), D != nullptr ? __ldg(D + h) : 0.0f,
+                          spec + (size_t)h * 2 * (1 << LG));
+        __syncthreads();   // the buffers are reused by the next channel
+    }
+}
+
 // Same convolution with one half per thread: 2 x threads_for<LG> threads,
 // about half the registers each (twice the warps per SM), the two halves
 // summed through shared memory at the end.
@@ -527,8 +543,20 @@ struct ConvKernels {
     static constexpr size_t smem_conv = smem + (STAGE ? 2 * sizeof(float) * (size_t)(C * (1 << LG) / 2) : 0);
     static LaunchInfo info_conv, info_kspec;
 
+    static LaunchInfo info_kspec_pair;
+
     static cudaError_t kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st) {
         float2 *spec = (float2 *)ws;
+        if constexpr (C == 2 && !TW0G && LG <= 13) {
+            // the one-CTA convolution's spectrum: persistent, one channel per CTA at a time
+            auto kern = k_kspec_pair<LG>;
+            constexpr size_t psmem = pair_smem_bytes<LG>(0);
+            int res = 0;
+            cudaError_t e = resident_units(kern, info_kspec_pair, 1, pair_threads<LG>(), psmem, &res);
+            if (e != cudaSuccess) return e;
+            kern<<<res < H ? res : H, pair_threads<LG>(), psmem, st>>>(K, D, H, spec);
+            return cudaGetLastError();
+        }
         float2 *tw0g = nullptr;
         if (TW0G) {
             tw0g = (float2 *)((char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)));
@@ -588,6 +616,7 @@ struct ConvKernels {
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_conv;
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec;
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_pair;
+template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec_pair;
 
 // ---- irfft instantiation ----
 template <int LG, int C>

@@ -1,5 +1,5 @@
 """GPU parity of the fused entry points: s4_kernel_dplr_prepare (K and the
-convolution spectrum of K + D delta_0 in one launch for L <= 4096) and
+convolution spectrum of K + D delta_0 in one launch for L <= 8192) and
 s4_forward_dplr (the whole convolution-view forward), against the fp64 oracle
 and against the modular calls."""
 import numpy as np
