@@ -154,6 +154,38 @@ s4_status s4_fft_conv_apply(const float *u, const void *workspace,
                             size_t workspace_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Backward pass of the convolution ([S4K] §5 fft_conv; §6 trains the layer):
+ * for y = K * u + D u and an upstream gradient dy [Bt, H, L],
+ *
+ * s4_fft_conv_apply_adjoint: du = dL/du, the correlation
+ *     du[b,h,s] = sum_{t>=s} K[h,t-s] dy[b,h,t] + D[h] dy[b,h,s],
+ *   with the same workspace as s4_fft_conv_apply (from s4_fft_conv_prepare or
+ *   s4_kernel_dplr_prepare): the forward kernel with the conjugate spectrum.
+ *   Arguments and errors as s4_fft_conv_apply (dy in place of u, du of y).
+ *
+ * s4_fft_conv_kernel_grad: dK = dL/dK [H, L] and dD = dL/dD [H],
+ *     dK[h,k] = sum_b sum_{t>=k} dy[b,h,t] u[b,h,t-k],   dD[h] = dK[h,0],
+ *   for L <= 8192 (longer L -> S4_ERR_UNSUPPORTED). u, dy [Bt, H, L] device,
+ *   16-byte aligned; dK [H, L] out, 16-byte aligned; dD [H] out, nullable.
+ *   Workspace: s4_fft_conv_kernel_grad_workspace_size bytes (= 2 H 2L 8:
+ *   a per-channel accumulator of the spectrum products and a per-channel
+ *   scratch), 256-byte aligned, caller-owned, contents irrelevant on entry.
+ *   Per channel the row pairs are summed in a fixed order (deterministic).
+ *   Errors: null pointers, Bt/H < 1, misalignment, overlapping buffers ->
+ *   S4_ERR_INVALID_ARG; workspace too small or misaligned ->
+ *   S4_ERR_WORKSPACE.
+ * ------------------------------------------------------------------------ */
+s4_status s4_fft_conv_apply_adjoint(const float *dy, const void *workspace,
+                                    int Bt, int H, int L, float *du,
+                                    size_t workspace_bytes, cudaStream_t stream);
+
+s4_status s4_fft_conv_kernel_grad_workspace_size(int H, int L, size_t *bytes);
+
+s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H, int L,
+                                  float *dK, float *dD, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * The whole forward pass of the layer's convolution view ([S4K] §4, §5).
  *
  * s4_kernel_dplr_prepare = s4_kernel_dplr(...) followed by

@@ -168,6 +168,30 @@ def causal_conv(u, K, D):
     return y.reshape(Bt, H, L)
 
 
+def causal_conv_adjoint(dy, K, D):
+    """The adjoint of causal_conv in u, i.e. the gradient of
+    <causal_conv(u, K, D), dy> with respect to u (the backward pass of §5's
+    fft_conv): du[b,h,s] = sum_{t>=s} K[h,t-s] dy[b,h,t] + D[h] dy[b,h,s].
+    Written as the causal sum of the time-reversed dy, reversed back."""
+    dy = np.asarray(dy, np.float64)
+    return np.ascontiguousarray(causal_conv(np.ascontiguousarray(dy[..., ::-1]), K, D)[..., ::-1])
+
+
+def causal_conv_kernel_grad(u, dy):
+    """The gradient of <causal_conv(u, K, D), dy> with respect to K and D:
+    dK[h,k] = sum_b sum_{t>=k} dy[b,h,t] u[b,h,t-k],  dD[h] = sum_b sum_t dy u."""
+    u = np.asarray(u, np.float64)
+    dy = np.asarray(dy, np.float64)
+    Bt, H, L = u.shape
+    dK = np.zeros((H, L))
+    for b in range(Bt):
+        for h in range(H):
+            for k in range(L):
+                dK[h, k] += np.dot(dy[b, h, k:], u[b, h, :L - k])
+    dD = np.einsum("bht,bht->h", dy, u)
+    return dK, dD
+
+
 def causal_conv_rows_at(u_rows, row_h, K, D, ts):
     """The direct sum for selected rows (u_rows [R, L], channel row_h[r]) at
     selected output times ts only."""

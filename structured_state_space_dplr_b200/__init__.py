@@ -25,7 +25,7 @@ __all__ = [
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
     "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "dplr_ctilde", "forward_dplr_host",
-    "fft_conv_host", "load",
+    "fft_conv_host", "fft_conv_apply_adjoint", "fft_conv_kernel_grad", "load",
 ]
 
 
@@ -178,6 +178,42 @@ def fft_conv_apply(u, workspace, *, out=None):
     _lib.call("s4_fft_conv_apply", _ptr(u), _ptr(workspace), Bt, H, L, _ptr(out), workspace.numel(),
               _stream())
     return out
+
+
+def fft_conv_apply_adjoint(dy, workspace, *, out=None):
+    """Backward of fft_conv_apply in u: du = sum_{t>=s} K[t-s] dy[t] + D dy[s]
+    with the same prepared spectrum (s4_fft_conv_apply_adjoint)."""
+    dy = _cuda(dy, "dy", torch.float32)
+    _cuda(workspace, "workspace", torch.uint8)
+    Bt, H, L = dy.shape
+    if out is None:
+        out = torch.empty_like(dy)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_fft_conv_apply_adjoint", _ptr(dy), _ptr(workspace), Bt, H, L, _ptr(out), workspace.numel(),
+              _stream())
+    return out
+
+
+def fft_conv_kernel_grad(u, dy, *, dK=None, dD=None, workspace=None):
+    """Backward of the convolution in K and D (s4_fft_conv_kernel_grad):
+    (dK [H, L], dD [H]) for the batch u, dy [Bt, H, L]; L <= 8192."""
+    u = _cuda(u, "u", torch.float32)
+    dy = _cuda(dy, "dy", torch.float32)
+    Bt, H, L = u.shape
+    if dK is None:
+        dK = torch.empty(H, L, device=u.device, dtype=torch.float32)
+    if dD is None:
+        dD = torch.empty(H, device=u.device, dtype=torch.float32)
+    _cuda(dK, "dK", torch.float32)
+    _cuda(dD, "dD", torch.float32)
+    if workspace is None:
+        n = ctypes.c_size_t()
+        _lib.call("s4_fft_conv_kernel_grad_workspace_size", H, L, ctypes.byref(n))
+        workspace = torch.empty(n.value, dtype=torch.uint8, device=u.device)
+    _cuda(workspace, "workspace", torch.uint8)
+    _lib.call("s4_fft_conv_kernel_grad", _ptr(u), _ptr(dy), Bt, H, L, _ptr(dK), _ptr(dD), _ptr(workspace),
+              workspace.numel(), _stream())
+    return dK, dD
 
 
 def kernel_dplr_prepare(Lambda, P, Q, B, C, log_dt, D, L, *, K=None, workspace=None, flags=None):

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libs4dplr.so")
-SOURCES = ["api.cu", "cauchy.cu", "kgen.cu", "spectral.cu", "s4d.cu", "decode.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "cauchy.cu", "kgen.cu", "spectral.cu", "s4d.cu", "decode.cu", "noalloc.cu", "backward.cu"]
 HEADERS = ["common.cuh", "fft.cuh", "cauchy.cuh", "pairs.cuh", "launch.h"]
 
 NVCC_FLAGS = [

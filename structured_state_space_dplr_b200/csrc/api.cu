@@ -209,6 +209,41 @@ s4_status s4_fft_conv_apply(const float *u, const void *workspace, int Bt, int H
     return cuda_status(s4::launch_fftconv(u, workspace, Bt, H, L, y, stream));
 }
 
+s4_status s4_fft_conv_apply_adjoint(const float *dy, const void *workspace, int Bt, int H, int L, float *du,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+    s4_status s = conv_checks(dy, Bt, H, L, du, workspace, workspace_bytes);
+    if (s != S4_OK) return s;
+    return cuda_status(s4::launch_fftconv(dy, workspace, Bt, H, L, du, stream, true));
+}
+
+s4_status s4_fft_conv_kernel_grad_workspace_size(int H, int L, size_t *bytes) {
+    if (bytes == nullptr || H < 1) return S4_ERR_INVALID_ARG;
+    if (!pow2_L(L) || L > 8192) return S4_ERR_UNSUPPORTED;
+    *bytes = s4::corr_workspace_bytes(H, L);
+    return S4_OK;
+}
+
+s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H, int L, float *dK, float *dD,
+                                  void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (any_null(u, dy, dK) || workspace == nullptr) return S4_ERR_INVALID_ARG;
+    if (Bt < 1 || H < 1) return S4_ERR_INVALID_ARG;
+    if (!pow2_L(L) || L > 8192) return S4_ERR_UNSUPPORTED;
+    if ((double)Bt * (double)H * (double)L >= 1099511627776.0) return S4_ERR_INVALID_ARG;   // 2^40
+    if (!aligned(u, 16) || !aligned(dy, 16) || !aligned(dK, 16) || (dD != nullptr && !aligned(dD, 4)))
+        return S4_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || workspace_bytes < s4::corr_workspace_bytes(H, L)) return S4_ERR_WORKSPACE;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float), kb = (size_t)H * L * sizeof(float);
+    const size_t hb = (size_t)H * sizeof(float);
+    for (const void *p : {(const void *)u, (const void *)dy}) {
+        if (overlap(p, nb, dK, kb) || overlap(p, nb, workspace, workspace_bytes)) return S4_ERR_INVALID_ARG;
+        if (dD != nullptr && overlap(p, nb, dD, hb)) return S4_ERR_INVALID_ARG;
+    }
+    if (overlap(dK, kb, workspace, workspace_bytes)) return S4_ERR_INVALID_ARG;
+    if (dD != nullptr && (overlap(dD, hb, dK, kb) || overlap(dD, hb, workspace, workspace_bytes)))
+        return S4_ERR_INVALID_ARG;
+    return cuda_status(s4::launch_corr(u, dy, Bt, H, L, dK, dD, workspace, stream));
+}
+
 s4_status s4_fft_conv(const float *u, const float *K, const float *D, int Bt, int H, int L, float *y,
                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     if (D == nullptr) return S4_ERR_INVALID_ARG;

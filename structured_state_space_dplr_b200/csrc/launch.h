@@ -16,8 +16,15 @@ size_t conv_workspace_bytes(int H, int L);
 
 // spectrum of K + D delta_0 (D may be null: no feed-through) into ws
 cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st);
-cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st);
+// adjoint: the correlation with the same spectrum (conjugated), y[s] = sum_{t>=s} K[t-s] u[t] + D u[s]
+cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st,
+                           bool adjoint = false);
 // in place: K[H, L] holds the packed half spectrum on entry, the real kernel on exit
+// ---- backward.cu ----
+size_t corr_workspace_bytes(int H, int L);
+cudaError_t launch_corr(const float *u, const float *dy, int Bt, int H, int L, float *dK, float *dD, void *ws,
+                        cudaStream_t st);
+
 cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st);
 
 // ---- kgen.cu: K and the convolution spectrum of K + D delta_0 in one launch

@@ -184,11 +184,42 @@ __device__ __forceinline__ void kspec_channel(const PairSmem &s, const float *__
     spectrum_tail<LG>(s, Dh, spec_h);
 }
 
+// Last inverse pass of both halves (all threads synced on entry): output
+// point t < m of the length-2m inverse is half 0's value plus half 1's, the
+// latter twisted back by W_2m^t (in-group share W_2R0^p); out(t, value)
+// receives each one.
+template <int LG, class Out>
+__device__ __forceinline__ void last_pass_halves_sum(const PairSmem &s, Out &&out) {
+    constexpr int m = 1 << LG, T = pair_threads<LG>();
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    for (int j = threadIdx.x; j < S0; j += T) {
+        float2 x[R0], z[R0];
+        const int o = pidx(j);
+        const float2 a = s.ta[j], b = s.tb[j];
+        float2 w = b, v = a;
+        x[0] = s.b0[o];
+        z[0] = cmulc(s.b1[o], a);
+        static_for<1, R0>([&](auto q) {
+            v = cmul(v, b);
+            x[q] = cmulc(s.b0[o + poff<decltype(q)::value * S0>()], w);
+            z[q] = cmulc(s.b1[o + poff<decltype(q)::value * S0>()], v);
+            w = cmul(w, b);
+        });
+        dft<R0, +1>(x);
+        dft<R0, +1>(z);
+        static_for<0, R0>([&](auto p) {
+            out(j + p * S0, cadd(x[p], rot<decltype(p)::value, 2 * R0, +1>(z[p])));
+        });
+    }
+}
+
 // ------------------------------------------------------------ convolution --
 // Convolution of the staged row pair (stage ready, all threads synced) with
 // the spectrum spec_h (layout of spec4_index, rank 0 then rank 1). After the
-// first pass, after_first() runs (the stage is free then).
-template <int LG, class AfterFirst>
+// first pass, after_first() runs (the stage is free then). CONJ multiplies
+// by the conjugate spectrum instead: the adjoint, a correlation
+// y[s] = sum_{t >= s} K[t - s] u[t] + D u[s] (K and D are real).
+template <int LG, bool CONJ, class AfterFirst>
 __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__restrict__ spec_h, float *y0,
                                           float *y1, bool has1, AfterFirst &&after_first) {
     constexpr int m = 1 << LG, L = m, T = pair_threads<LG>();
@@ -219,38 +250,23 @@ __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__res
         });
         return w;
     }, [&](const SpecWords &w, auto &x, auto &z) {
+        auto mul = [](float2 a, float x0, float x1) {
+            if constexpr (CONJ) return cmulc(a, make_float2(x0, x1)); else return cmul(a, make_float2(x0, x1));
+        };
         static_for<0, RL / 2>([&](auto i) {
-            x[2 * i] = cmul(x[2 * i], make_float2(w.k0[i].x, w.k0[i].y));
-            x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(w.k0[i].z, w.k0[i].w));
-            z[2 * i] = cmul(z[2 * i], make_float2(w.k1[i].x, w.k1[i].y));
-            z[2 * i + 1] = cmul(z[2 * i + 1], make_float2(w.k1[i].z, w.k1[i].w));
+            x[2 * i] = mul(x[2 * i], w.k0[i].x, w.k0[i].y);
+            x[2 * i + 1] = mul(x[2 * i + 1], w.k0[i].z, w.k0[i].w);
+            z[2 * i] = mul(z[2 * i], w.k1[i].x, w.k1[i].y);
+            z[2 * i + 1] = mul(z[2 * i + 1], w.k1[i].z, w.k1[i].w);
         });
     });
     __syncthreads();
     inverse_middle_x2<LG, T>(b0, b1, s.tws);
     // ---- last inverse pass of both halves + their sum, straight to y
-    for (int j = threadIdx.x; j < S0; j += T) {
-        float2 x[R0], z[R0];
-        const int o = pidx(j);
-        const float2 a = s.ta[j], b = s.tb[j];
-        float2 w = b, v = a;
-        x[0] = b0[o];
-        z[0] = cmulc(b1[o], a);
-        static_for<1, R0>([&](auto q) {
-            v = cmul(v, b);
-            x[q] = cmulc(b0[o + poff<decltype(q)::value * S0>()], w);
-            z[q] = cmulc(b1[o + poff<decltype(q)::value * S0>()], v);
-            w = cmul(w, b);
-        });
-        dft<R0, +1>(x);
-        dft<R0, +1>(z);
-        static_for<0, R0>([&](auto p) {
-            const float2 r = cadd(x[p], rot<decltype(p)::value, 2 * R0, +1>(z[p]));
-            const int t = j + p * S0;
-            y0[t] = r.x;
-            if (has1) y1[t] = r.y;
-        });
-    }
+    last_pass_halves_sum<LG>(s, [&](int t, float2 r) {
+        y0[t] = r.x;
+        if (has1) y1[t] = r.y;
+    });
 }
 
 // ------------------------------------------------------------- generation --

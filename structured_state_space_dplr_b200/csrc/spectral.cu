@@ -131,7 +131,7 @@ k_kspec(const float *__restrict__ K, const float *__restrict__ D, int H, int L, 
 template <int LG, int C, bool TW0G, bool STAGE>
 __global__ void __launch_bounds__(threads_for<LG>())
 k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
-          float *__restrict__ y, const float2 *__restrict__ tw0g) {
+          float *__restrict__ y, const float2 *__restrict__ tw0g, float conj_sign) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
     constexpr int SL = m / C;                     // combine slice per rank
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
@@ -222,8 +222,8 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
             constexpr int R = sizeof(x) / sizeof(float2);
             static_for<0, R / 2>([&](auto i) {
                 const float4 k2 = __ldg(sp + spec4_index<LG>(base, i));
-                x[2 * i] = cmul(x[2 * i], make_float2(k2.x, k2.y));
-                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k2.z, k2.w));
+                x[2 * i] = cmul(x[2 * i], make_float2(k2.x, conj_sign * k2.y));
+                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k2.z, conj_sign * k2.w));
             });
         });
         __syncthreads();
@@ -268,7 +268,7 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
 // L <= 8192: one CTA per row pair holds both halves of the length-2L
 // transform; see conv_pair (pairs.cuh). Persistent: the next row pair is
 // staged with cp.async while the current one is transformed.
-template <int LG>
+template <int LG, bool CONJ>
 __global__ void __launch_bounds__(pair_threads<LG>(), pair_min_blocks<LG>())
 k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
                float *__restrict__ y) {
@@ -282,7 +282,7 @@ k_fftconv_pair(const float *__restrict__ u, const float2 *__restrict__ spec, int
         cp_async_wait_all();
         __syncthreads();   // stage ready; previous pair's buffers no longer read
         float *y0 = y + ((size_t)r.b0 * H + r.h) * L;
-        conv_pair<LG>(s, spec + (size_t)r.h * 2 * L, y0, y0 + (size_t)H * L, r.has1, [&] {
+        conv_pair<LG, CONJ>(s, spec + (size_t)r.h * 2 * L, y0, y0 + (size_t)H * L, r.has1, [&] {
             if (pr + gridDim.x < npairs) pair_stage_rows<LG>(s, u, Bt, H, pr + gridDim.x);
         });
     }
@@ -301,105 +301,6 @@ k_kspec_pair(const float *__restrict__ K, const float *__restrict__ D, int H, fl
         kspec_channel<LG>(s, K + (size_t)h * (1 << LG), D != nullptr ? __ldg(D + h) : 0.0f,
                           spec + (size_t)h * 2 * (1 << LG));
         __syncthreads();   // the buffers are reused by the next channel
-    }
-}
-
-// Same convolution with one half per thread: 2 x threads_for<LG> threads,
-// about half the registers each (twice the warps per SM), the two halves
-// summed through shared memory at the end.
-template <int LG>
-__global__ void __launch_bounds__(2 * threads_for<LG>(), 2)
-k_fftconv_wide(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
-               float *__restrict__ y) {
-    constexpr int m = 1 << LG, TH = threads_for<LG>(), T = 2 * TH, N = 2 * m;
-    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
-    extern __shared__ float2 sm[];
-    float2 *b0 = sm, *b1 = sm + padded(m);
-    float2 *tws = b1 + padded(m);
-    float2 *ta = tws + plan_tw_size(LG), *tb = ta + S0;
-    float *stage = reinterpret_cast<float *>(sm + pair_core_f2<LG>());   // [2][L]
-    const int half = threadIdx.x >= TH, tid = threadIdx.x - half * TH;
-    float2 *buf = half ? b1 : b0;
-
-    for (int i = threadIdx.x; i < S0; i += T) {
-        ta[i] = unit_root(i, N);
-        tb[i] = unit_root(i, m);
-    }
-    build_middle_tables<LG>(tws, threadIdx.x, T);
-
-    const int nbp = (Bt + 1) / 2;
-    const long long npairs = (long long)H * nbp;
-    auto stage_rows = [&](long long pr) {
-        const int h = (int)(pr / nbp), b0r = 2 * (int)(pr % nbp);
-        const bool has1 = (b0r + 1) < Bt;
-        const float *u0 = u + ((size_t)b0r * H + h) * L;
-        const float *u1 = has1 ? u0 + (size_t)H * L : u0;
-        for (int i = threadIdx.x; i < L / 2; i += T) {
-            const int row = i >= L / 4, k = (i - row * (L / 4)) * 4;
-            cp_async16(stage + row * L + k, (row ? u1 : u0) + k, !row || has1);
-        }
-        cp_async_commit();
-    };
-    if ((long long)blockIdx.x < npairs) stage_rows(blockIdx.x);
-
-    for (long long pr = blockIdx.x; pr < npairs; pr += gridDim.x) {
-        const int h = (int)(pr / nbp), bq = 2 * (int)(pr % nbp);
-        const bool has1 = (bq + 1) < Bt;
-        cp_async_wait_all();
-        __syncthreads();
-        for (int j = tid; j < S0; j += TH) {   // first forward pass of this thread's half
-            float2 x[R0];
-            static_for<0, R0>([&](auto p) {
-                const int k = j + p * S0;
-                const float2 v = make_float2(stage[k], stage[L + k]);
-                x[p] = half ? rot<decltype(p)::value, 2 * R0, -1>(v) : v;
-            });
-            dft<R0, -1>(x);
-            const float2 b = tb[j];
-            float2 w = half ? ta[j] : make_float2(1.0f, 0.0f);
-            const int o = pidx(j);
-            static_for<0, R0>([&](auto q) {
-                buf[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
-                if constexpr (decltype(q)::value + 1 < R0) w = cmul(w, b);
-            });
-        }
-        __syncthreads();
-        if (pr + gridDim.x < npairs) stage_rows(pr + gridDim.x);
-        forward_middle<LG, TH>(buf, tws, tid);
-        const float4 *sp = reinterpret_cast<const float4 *>(spec + (size_t)h * N + half * m);
-        fused_middle<LG, TH>(buf, [&](int base, auto &x) {
-            constexpr int R = sizeof(x) / sizeof(float2);
-            float4 k[R / 2];
-            static_for<0, R / 2>([&](auto i) { k[i] = __ldg(sp + spec4_index<LG>(base, i)); });
-            static_for<0, R / 2>([&](auto i) {
-                x[2 * i] = cmul(x[2 * i], make_float2(k[i].x, k[i].y));
-                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k[i].z, k[i].w));
-            });
-        }, tid);
-        __syncthreads();
-        inverse_middle<LG, TH>(buf, tws, tid);
-        for (int j = tid; j < S0; j += TH) {   // last inverse pass, natural order back to buf
-            float2 x[R0];
-            const int o = pidx(j);
-            const float2 b = tb[j];
-            float2 w = half ? ta[j] : make_float2(1.0f, 0.0f);
-            static_for<0, R0>([&](auto q) {
-                x[q] = cmulc(buf[o + poff<decltype(q)::value * S0>()], w);
-                if constexpr (decltype(q)::value + 1 < R0) w = cmul(w, b);
-            });
-            dft<R0, +1>(x);
-            static_for<0, R0>([&](auto p) {
-                buf[o + poff<decltype(p)::value * S0>()] = half ? rot<decltype(p)::value, 2 * R0, +1>(x[p]) : x[p];
-            });
-        }
-        __syncthreads();
-        float *y0 = y + ((size_t)bq * H + h) * L;
-        float *y1 = y0 + (size_t)H * L;
-        for (int t = threadIdx.x; t < L; t += T) {
-            const float2 r = cadd(b0[pidx(t)], b1[pidx(t)]);
-            y0[t] = r.x;
-            if (has1) y1[t] = r.y;
-        }
     }
 }
 
@@ -576,22 +477,18 @@ struct ConvKernels {
         return cudaGetLastError();
     }
 
-    static LaunchInfo info_pair;
+    static LaunchInfo info_pair[2];
 
-    static cudaError_t conv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st) {
+    static cudaError_t conv(const float *u, const void *ws, int Bt, int H, int L, float *y, bool adjoint,
+                            cudaStream_t st) {
         const float2 *spec = (const float2 *)ws;
         if constexpr (C == 2 && !TW0G && LG <= 13) {
-            // one CTA per row pair, both halves in one CTA
-#if S4_CONV_WIDE
-            auto kern = k_fftconv_wide<LG>;
-            constexpr int TT = 2 * T;
-#else
-            auto kern = k_fftconv_pair<LG>;
-            constexpr int TT = T;
-#endif
+            // one CTA per row pair, both halves in one CTA; persistent grid
+            auto kern = adjoint ? k_fftconv_pair<LG, true> : k_fftconv_pair<LG, false>;
+            constexpr int TT = pair_threads<LG>();
             constexpr size_t psmem = pair_smem_bytes<LG>(0);
             int res = 0;
-            cudaError_t e = resident_units(kern, info_pair, 1, TT, psmem, &res);
+            cudaError_t e = resident_units(kern, info_pair[adjoint], 1, TT, psmem, &res);
             if (e != cudaSuccess) return e;
             const long long npairs = (long long)H * ((Bt + 1) / 2);
             const int grid = (long long)res < npairs ? res : (int)npairs;
@@ -608,14 +505,14 @@ struct ConvKernels {
         const long long npairs = (long long)H * ((Bt + 1) / 2);
         int ncl = res;
         if ((long long)ncl > npairs) ncl = (int)npairs;
-        e = launch_clustered(kern, C, ncl, T, smem_conv, st, u, spec, Bt, H, L, y, tw0g);
+        e = launch_clustered(kern, C, ncl, T, smem_conv, st, u, spec, Bt, H, L, y, tw0g, adjoint ? -1.0f : 1.0f);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
 };
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_conv;
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec;
-template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_pair;
+template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_pair[2];
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec_pair;
 
 // ---- irfft instantiation ----
@@ -669,11 +566,6 @@ size_t conv_workspace_bytes(int H, int L) {
     return b;
 }
 
-// Convolution kernel for L <= 4096: 0 = both halves per thread
-// (k_fftconv_pair), 1 = one half per thread (k_fftconv_wide).
-#ifndef S4_CONV_WIDE
-#define S4_CONV_WIDE 0
-#endif
 // Longest L whose convolution stages the next row pair in shared memory
 // (cp.async prefetch; costs 8 L bytes of shared memory per CTA).
 #ifndef S4_CONV_STAGE_MAX_L
@@ -705,9 +597,10 @@ cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws,
     }
 }
 
-cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st) {
+cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st,
+                           bool adjoint) {
     switch (L) {
-#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::conv(u, ws, Bt, H, L, y, st);
+#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::conv(u, ws, Bt, H, L, y, adjoint, st);
         S4_CONV_CASES(X)
 #undef X
         default: return cudaErrorInvalidValue;

@@ -131,6 +131,20 @@ def test_vandermonde_and_discretize_reject_bad_arguments(lib):
     assert lib.s4_dplr_discretize_structured(*five, 4, 32, p(FAKE2 + 4), out[1], p(0)) == _lib.S4_ERR_INVALID_ARG
 
 
+def test_backward_entries_reject_bad_arguments(lib):
+    n = ctypes.c_size_t()
+    assert lib.s4_fft_conv_kernel_grad_workspace_size(4, 16384, ctypes.byref(n)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_fft_conv_kernel_grad_workspace_size(4, 4096, ctypes.byref(n)) == _lib.S4_OK
+    assert n.value == 2 * 4 * 2 * 4096 * 8
+    u, dy, dK, dD = p(FAKE), p(FAKE + 0x10000000), p(FAKE2), p(FAKE2 + 0x10000000)
+    ws, wsb = p(FAKE + 0x40000000), n.value
+    assert lib.s4_fft_conv_kernel_grad(p(0), dy, 2, 4, 4096, dK, dD, ws, wsb, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_fft_conv_kernel_grad(u, dy, 2, 4, 1000, dK, dD, ws, wsb, p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_fft_conv_kernel_grad(u, dy, 2, 4, 4096, dK, dD, ws, wsb - 1, p(0)) == _lib.S4_ERR_WORKSPACE
+    assert lib.s4_fft_conv_kernel_grad(u, dy, 2, 4, 4096, p(FAKE + 4096), dD, ws, wsb, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_fft_conv_apply_adjoint(p(0), ws, 2, 4, 4096, dK, wsb, p(0)) == _lib.S4_ERR_INVALID_ARG
+
+
 def test_binding_refuses_cpu_tensors():
     torch = pytest.importorskip("torch")
     import structured_state_space_dplr_b200 as s4

@@ -293,3 +293,34 @@ def test_s4d_kernel_closed_form_and_recurrence():
     yr, _ = ssm.recurrence_diag(Ab, Bb, inp["C"].astype(np.complex128), inp["D"].astype(np.float64), u, hh)
     for i, (b, h) in enumerate(rows):
         assert np.abs(yr[i] - y[b, h]).max() < 1e-11 * np.abs(y[b, h]).max()
+
+
+def test_conv_adjoint_identity_and_kernel_grad_by_basis():
+    """<conv(u), dy> = <u, adjoint(dy)>, and since the convolution is linear
+    in K and D, its derivative along a basis kernel e_{h,k} (or D = e_h) is
+    exactly the inner product with that basis output."""
+    rng = np.random.default_rng(5)
+    Bt, H, L = 3, 2, 40
+    u = rng.standard_normal((Bt, H, L))
+    dy = rng.standard_normal((Bt, H, L))
+    K = rng.standard_normal((H, L))
+    D = rng.standard_normal(H)
+    y = ssm.causal_conv(u, K, D)
+    du = ssm.causal_conv_adjoint(dy, K, D)
+    assert abs(np.sum(y * dy) - np.sum(u * du)) <= 1e-12 * np.sum(np.abs(y * dy))
+    dK, dD = ssm.causal_conv_kernel_grad(u, dy)
+    zero = np.zeros(H)
+    for h, k in [(0, 0), (1, 7), (0, L - 1), (1, 23)]:
+        E = np.zeros((H, L))
+        E[h, k] = 1.0
+        assert abs(np.sum(ssm.causal_conv(u, E, zero) * dy) - dK[h, k]) <= 1e-12 * (1 + abs(dK[h, k]))
+    for h in range(H):
+        e = np.zeros(H)
+        e[h] = 1.0
+        assert abs(np.sum(ssm.causal_conv(u, np.zeros((H, L)), e) * dy) - dD[h]) <= 1e-12 * (1 + abs(dD[h]))
+    # the adjoint is the transpose: du of a unit impulse dy picks one kernel row
+    d1 = np.zeros((1, 1, L))
+    d1[0, 0, 30] = 1.0
+    du1 = ssm.causal_conv_adjoint(d1, K[:1], D[:1])[0, 0]
+    assert np.allclose(du1[:31], K[0, 30::-1] + np.where(np.arange(31) == 30, D[0], 0.0), rtol=0, atol=1e-14)
+    assert np.all(du1[31:] == 0.0)
