@@ -186,6 +186,29 @@ s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H
                                   size_t workspace_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * s4_kernel_dplr_backward: the gradient of a loss through the DPLR kernel
+ * ([S4K] §4 generating function; §6 trains Lambda, P, Q, B, C and log dt)
+ * with respect to the parameters, given dK = dLoss/dK [H, L] (for instance
+ * from s4_fft_conv_kernel_grad). For each complex parameter the result is
+ * dLoss/dRe + i dLoss/dIm of the stored modes (the implicit conjugate modes
+ * are accounted for); dlog_dt is the derivative in log dt. The gradient runs
+ * through DFT(dK) at the same roots of unity and the derivatives of the
+ * four Cauchy sums, the Woodbury correction and the bilinear factor
+ * (squared-denominator Cauchy sums for Lambda and dt), and the closed form at
+ * the Nyquist bin. L <= 8192 (longer -> S4_ERR_UNSUPPORTED).
+ *   Lambda, P, Q, B, C : [H, Nh] complex;  log_dt : [H];  dK : [H, L].
+ *   dLambda, dP, dQ, dB, dC : [H, Nh] complex out;  dlog_dt : [H] out.
+ * Errors: null pointers, misaligned complex arrays, outputs overlapping
+ * inputs or each other -> S4_ERR_INVALID_ARG; L not a power of two in range,
+ * Nh > S4_MAX_NH -> S4_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+s4_status s4_kernel_dplr_backward(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                                  const s4_c32 *B, const s4_c32 *C, const float *log_dt,
+                                  const float *dK, int H, int Nh, int L, s4_c32 *dLambda,
+                                  s4_c32 *dP, s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC,
+                                  float *dlog_dt, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * The whole forward pass of the layer's convolution view ([S4K] §4, §5).
  *
  * s4_kernel_dplr_prepare = s4_kernel_dplr(...) followed by

@@ -82,3 +82,55 @@ def conv_rows_at(inp, K_rows, rows, ts):
     D = np.array([float(inp["D"][h]) for _, h in rows])
     return ssm.causal_conv_rows_at(u, np.arange(len(rows)), np.asarray(K_rows, np.float64), D,
                                    np.asarray(ts, np.int64))
+
+
+# ---------------------------------------------------------------- gradients --
+def fd_gradient(fun, params, keys, eps=1e-6):
+    """Central-difference gradient of the real scalar fun(params) in fp64.
+
+    params: dict of fp64 arrays (not modified); keys: which of them to
+    differentiate. For a complex entry theta the result is
+    d fun / d Re(theta) + i d fun / d Im(theta); for a real entry, the
+    derivative. Steps are eps * max(1, |entry|)."""
+    out = {}
+    for key in keys:
+        base = np.asarray(params[key])
+        g = np.zeros(base.shape, dtype=base.dtype)
+        for idx in np.ndindex(base.shape):
+            step = eps * max(1.0, abs(base[idx]))
+            dirs = (1.0, 1j) if np.iscomplexobj(base) else (1.0,)
+            for d in dirs:
+                vals = []
+                for sgn in (1.0, -1.0):
+                    p = dict(params)
+                    arr = base.copy()
+                    arr[idx] = arr[idx] + sgn * step * d
+                    p[key] = arr
+                    vals.append(fun(p))
+                deriv = (vals[0] - vals[1]) / (2.0 * step)
+                g[idx] += deriv if d == 1.0 else 1j * deriv
+        out[key] = g
+    return out
+
+
+def dplr_kernel_param_grad(inp, dK, channels=None, eps=1e-6):
+    """Gradient of <K, dK> (K = dplr_kernel, the aliased bilinear kernel of
+    "The S4 kernel, from scratch" §3-§4) with respect to each channel's
+    Lambda, P, Q, B, C (complex: d/dRe + i d/dIm) and log_dt, by central
+    differences of the dense fp64 definition. dK: [len(channels), L].
+    Returns a dict of arrays [len(channels), Nh] (log_dt: [len(channels)])."""
+    channels = list(range(inp["H"]) if channels is None else channels)
+    keys = ("Lambda", "P", "Q", "B", "C", "log_dt")
+    res = {k: [] for k in keys}
+    for i, h in enumerate(channels):
+        params = {k: _f64(inp[k])[h:h + 1] for k in keys}
+        dKh = np.asarray(dK[i], np.float64)
+
+        def fun(p):
+            sub = dict(H=1, L=inp["L"], **{k: p[k] for k in keys})
+            return float(np.dot(dplr_kernel(sub, [0])[0], dKh))
+
+        g = fd_gradient(fun, params, keys, eps)
+        for k in keys:
+            res[k].append(g[k][0])
+    return {k: np.array(v) for k, v in res.items()}

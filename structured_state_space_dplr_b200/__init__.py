@@ -25,7 +25,7 @@ __all__ = [
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
     "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "dplr_ctilde", "forward_dplr_host",
-    "fft_conv_host", "fft_conv_apply_adjoint", "fft_conv_kernel_grad", "load",
+    "fft_conv_host", "fft_conv_apply_adjoint", "fft_conv_kernel_grad", "kernel_dplr_backward", "load",
 ]
 
 
@@ -214,6 +214,23 @@ def fft_conv_kernel_grad(u, dy, *, dK=None, dD=None, workspace=None):
     _lib.call("s4_fft_conv_kernel_grad", _ptr(u), _ptr(dy), Bt, H, L, _ptr(dK), _ptr(dD), _ptr(workspace),
               workspace.numel(), _stream())
     return dK, dD
+
+
+def kernel_dplr_backward(Lambda, P, Q, B, C, log_dt, dK):
+    """Gradient through the DPLR kernel (s4_kernel_dplr_backward): given
+    dK = dLoss/dK [H, L], returns dict(Lambda, P, Q, B, C -> complex64
+    [H, Nh] as dLoss/dRe + i dLoss/dIm; log_dt -> float32 [H])."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    dK = _cuda(dK, "dK", torch.float32)
+    H, Nh = Lambda.shape
+    L = dK.shape[-1]
+    out = {k: torch.empty_like(Lambda) for k in ("Lambda", "P", "Q", "B", "C")}
+    out["log_dt"] = torch.empty_like(log_dt)
+    _lib.call("s4_kernel_dplr_backward", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              _ptr(dK), H, Nh, L, _ptr(out["Lambda"]), _ptr(out["P"]), _ptr(out["Q"]), _ptr(out["B"]),
+              _ptr(out["C"]), _ptr(out["log_dt"]), _stream())
+    return out
 
 
 def kernel_dplr_prepare(Lambda, P, Q, B, C, log_dt, D, L, *, K=None, workspace=None, flags=None):

@@ -244,6 +244,34 @@ s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H
     return cuda_status(s4::launch_corr(u, dy, Bt, H, L, dK, dD, workspace, stream));
 }
 
+s4_status s4_kernel_dplr_backward(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B,
+                                  const s4_c32 *C, const float *log_dt, const float *dK, int H, int Nh, int L,
+                                  s4_c32 *dLambda, s4_c32 *dP, s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC,
+                                  float *dlog_dt, cudaStream_t stream) {
+    if (any_null(Lambda, P, Q, B, C) || any_null(dLambda, dP, dQ, dB, dC) || any_null(log_dt, dK, dlog_dt))
+        return S4_ERR_INVALID_ARG;
+    s4_status s = check_modes(H, Nh, L, true);
+    if (s != S4_OK) return s;
+    if (L > 8192) return S4_ERR_UNSUPPORTED;
+    if (!params_aligned({Lambda, P, Q, B, C, dLambda, dP, dQ, dB, dC}) || !aligned(dK, 4)) return S4_ERR_INVALID_ARG;
+    const size_t pb = (size_t)H * Nh * sizeof(s4_c32);
+    const void *outs[] = {dLambda, dP, dQ, dB, dC};
+    const void *ins[] = {Lambda, P, Q, B, C};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 5; ++j) {
+            if (overlap(outs[i], pb, ins[j], pb)) return S4_ERR_INVALID_ARG;
+            if (j > i && overlap(outs[i], pb, outs[j], pb)) return S4_ERR_INVALID_ARG;
+        }
+        if (overlap(outs[i], pb, dK, (size_t)H * L * sizeof(float)) ||
+            overlap(outs[i], pb, dlog_dt, (size_t)H * sizeof(float)))
+            return S4_ERR_INVALID_ARG;
+    }
+    return cuda_status(s4::launch_kgen_backward((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q,
+                                                (const float2 *)B, (const float2 *)C, log_dt, dK, H, Nh, L,
+                                                (float2 *)dLambda, (float2 *)dP, (float2 *)dQ, (float2 *)dB,
+                                                (float2 *)dC, dlog_dt, stream));
+}
+
 s4_status s4_fft_conv(const float *u, const float *K, const float *D, int Bt, int H, int L, float *y,
                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     if (D == nullptr) return S4_ERR_INVALID_ARG;

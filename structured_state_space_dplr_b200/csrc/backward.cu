@@ -122,6 +122,242 @@ k_corr_pair(const float *__restrict__ u, const float *__restrict__ dy, int Bt, i
     }
 }
 
+// ------------------------------------------------------ kernel parameters --
+// Gradient of a loss through K = iDFT(K_hat) with respect to the DPLR
+// parameters ("The S4 kernel, from scratch", §4 generating function, §6
+// trainable parameters), given dK = dLoss/dK [H, L].
+//
+// With G_hat = DFT(dK), the loss moves with K_hat_j (j < L/2, each with its
+// Hermitian partner) through g_j = dLoss/dRe K_hat_j + i dLoss/dIm K_hat_j
+// = (2/L) G_hat_j ((1/L) G_hat_0 at j = 0). K_hat_j = c_j R_j with
+// c_j = 1 + i t_j, R = k00 - k01 k10 / (1 + k11) and
+// k_v = sum_i v_i r_i over the full conjugate-closed system,
+// r_i = 1/(s_j - lambda_i), s_j = i gamma_j. Writing e_v = dK_hat/dk_v
+// (e00 = c, e01 = -c k10/(1+k11), e10 = -c k01/(1+k11),
+// e11 = c k01 k10/(1+k11)^2) and a_v = conj(g_j) e_v, every complex
+// parameter's gradient (d/dRe + i d/dIm) of a stored mode n collects, per v,
+//   S_v  = sum_j a_v r_n' + conj(a_v r_n)         (r_n' = 1/(s - conj lambda_n))
+//   S2_v = sum_j a_v r_n'^2 + conj(a_v r_n^2),
+// and then
+//   dC = conj(B) S00 + conj(P) S01,   dB = conj(C) S00 + Q S10,
+//   dP = conj(C) S01 + Q S11,         dQ = B conj(S10) + P conj(S11),
+//   dLambda = sum_v conj(v_v) S2_v    (v00 = CB, v01 = CP, v10 = conj(Q) B,
+//                                      v11 = conj(Q) P);
+//   dlog_dt = sum_j Re(conj(g_j) s_j sum_v e_v sum_i v_i r_i^2)
+// (s_j scales as 1/dt). The Nyquist bin, K_hat = dt Re sum_n C_n B_n, adds
+// g dt conj(B) to dC, g dt conj(C) to dB and g K_hat to dlog_dt.
+//
+// One CTA per channel (persistent): G_hat by a length-L forward transform in
+// shared memory; then frequencies in chunks of T: each thread forms the four
+// k_v and sum_i v_i r_i^2 of one frequency (its a_v go to shared memory),
+// then thread (n, q) accumulates S_v, S2_v of mode n over every nq-th
+// frequency of the chunk; the nq partial sums of a mode are added at the end.
+constexpr int kBwdThreads = 256;
+constexpr int kModeFloats = 20;   // lambda(2) C(2) B(2) P(2) Q(2) v00..v11(8) -(2)
+
+template <int LG>
+__host__ __device__ constexpr size_t kbwd_smem_bytes(int Nh) {
+    return sizeof(float2) * ((size_t)padded(1 << LG) + plan_tw_size(LG) + ((1 << LG) >> plan_lr(LG, 0))) +
+           sizeof(float) * ((size_t)kModeFloats * Nh + 9 * kBwdThreads + 16 * kBwdThreads + 32);
+}
+
+__device__ __forceinline__ float2 crcp(float2 d) {
+    const float inv = 1.0f / fmaf(d.x, d.x, d.y * d.y);
+    return make_float2(d.x * inv, -d.y * inv);
+}
+
+template <int LG>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const float2 *__restrict__ Q,
+                const float2 *__restrict__ B, const float2 *__restrict__ Cc, const float *__restrict__ log_dt,
+                const float *__restrict__ dK, int H, int Nh, float2 *__restrict__ dLambda,
+                float2 *__restrict__ dP, float2 *__restrict__ dQ, float2 *__restrict__ dB,
+                float2 *__restrict__ dC, float *__restrict__ dlog_dt) {
+    constexpr int m = 1 << LG, L = m, T = kBwdThreads;
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
+    extern __shared__ float2 smb[];
+    float2 *buf = smb, *tws = buf + padded(m), *tb = tws + plan_tw_size(LG);
+    float *md = reinterpret_cast<float *>(tb + S0);         // [Nh][kModeFloats]
+    float *chA = md + kModeFloats * Nh;                      // [T][8]  a_v of the chunk
+    float *chG = chA + 8 * T;                                // [T]     gamma of the chunk
+    float *red = chG + T;                                    // [T][16] partial sums
+    float *red32 = red + 16 * T;                             // [32]
+    const int tid = threadIdx.x;
+    for (int j = tid; j < S0; j += T) tb[j] = unit_root(j, m);
+    build_middle_tables<LG>(tws, tid, T);
+    const int nq = T / Nh;   // frequency slices per mode (Nh <= T)
+    const int my_n = tid % Nh, my_q = tid / Nh;
+
+    for (int h = blockIdx.x; h < H; h += gridDim.x) {
+        const size_t po = (size_t)h * Nh;
+        const float dt = expf(__ldg(log_dt + h));
+        for (int n = tid; n < Nh; n += T) {
+            const float2 lam = Lambda[po + n], c = Cc[po + n], b = B[po + n], p = P[po + n], q = Q[po + n];
+            const float2 v00 = cmul(c, b), v01 = cmul(c, p), v10 = cmulc(b, q), v11 = cmulc(p, q);
+            float *w = md + kModeFloats * n;
+            const float vals[kModeFloats] = {lam.x, lam.y, c.x, c.y, b.x, b.y, p.x, p.y, q.x, q.y,
+                                             v00.x, v00.y, v01.x, v01.y, v10.x, v10.y, v11.x, v11.y, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < kModeFloats; ++i) w[i] = vals[i];
+        }
+        // ---- G_hat = DFT(dK): forward transform, digit-reversed result in buf
+        const float *dKh = dK + (size_t)h * L;
+        for (int j = tid; j < S0; j += T) {
+            float2 x[R0];
+            static_for<0, R0>([&](auto p) { x[p] = make_float2(__ldg(dKh + j + p * S0), 0.0f); });
+            dft<R0, -1>(x);
+            const float2 b = tb[j];
+            float2 w = b;
+            float2 *o = buf + pidx(j);
+            o[0] = x[0];
+            static_for<1, R0>([&](auto q) {
+                o[poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+                w = cmul(w, b);
+            });
+        }
+        __syncthreads();
+        forward_middle<LG, T>(buf, tws);
+        for (int g = tid; g < m / RL; g += T) {
+            float2 x[RL];
+            float2 *o = buf + pidx(g * RL);
+            load_contig<RL>(o, x);
+            dft<RL, -1>(x);
+            store_contig<RL>(o, x);
+        }
+        __syncthreads();
+
+        float ld_acc = 0.0f;
+        float2 S[4], S2[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) S[v] = S2[v] = make_float2(0.f, 0.f);
+        const float2 lam_n = make_float2(md[kModeFloats * my_n], md[kModeFloats * my_n + 1]);
+        for (int j0 = 0; j0 < L / 2; j0 += T) {
+            // ---- per frequency: k_v, e_v, a_v
+            const int j = j0 + tid;
+            float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
+            float gam = 0.0f;
+            if (j < L / 2) {
+                float sn, cs;
+                sincospif((float)j / (float)L, &sn, &cs);
+                const float t = sn / cs;
+                gam = 2.0f * t / dt;
+                float2 k[4], k2[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) k[v] = k2[v] = make_float2(0.f, 0.f);
+                for (int n = 0; n < Nh; ++n) {
+                    const float *w = md + kModeFloats * n;
+                    const float2 r1 = crcp(make_float2(-w[0], gam - w[1]));   // 1/(s - lambda)
+                    const float2 r2 = crcp(make_float2(-w[0], gam + w[1]));   // 1/(s - conj lambda)
+                    const float2 q1 = cmul(r1, r1), q2 = cmul(r2, r2);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float2 vv = make_float2(w[10 + 2 * v], w[11 + 2 * v]);
+                        k[v] = cadd(k[v], cadd(cmul(vv, r1), cmulc(r2, vv)));
+                        k2[v] = cadd(k2[v], cadd(cmul(vv, q1), cmulc(q2, vv)));
+                    }
+                }
+                const float2 c = make_float2(1.0f, t);
+                const float2 iden = crcp(make_float2(1.0f + k[3].x, k[3].y));
+                float2 e[4];
+                e[0] = c;
+                e[1] = cscale(cmul(c, cmul(k[2], iden)), -1.0f);
+                e[2] = cscale(cmul(c, cmul(k[1], iden)), -1.0f);
+                e[3] = cmul(c, cmul(cmul(k[1], k[2]), cmul(iden, iden)));
+                const float2 G = buf[pidx(digrev_inv<LG>(j))];
+                const float wj = (j == 0 ? 1.0f : 2.0f) / (float)L;
+                const float2 gj = make_float2(G.x * wj, G.y * wj);
+                float2 dw = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    a[v] = cmulc(e[v], gj);   // conj(g) e_v
+                    dw = cadd(dw, cmul(e[v], k2[v]));
+                }
+                // dK_hat/dlog_dt = s sum_v e_v sum_i v_i r_i^2, s = i gamma
+                const float2 sdw = make_float2(-gam * dw.y, gam * dw.x);
+                ld_acc = fmaf(gj.x, sdw.x, fmaf(gj.y, sdw.y, ld_acc));   // Re(conj(g) sdw)
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                chA[8 * tid + 2 * v] = a[v].x;
+                chA[8 * tid + 2 * v + 1] = a[v].y;
+            }
+            chG[tid] = gam;
+            __syncthreads();
+            // ---- per mode: S_v, S2_v over this chunk
+            if (my_q < nq) {
+                const int jn = (L / 2 - j0) < T ? (L / 2 - j0) : T;
+                for (int jj = my_q; jj < jn; jj += nq) {
+                    const float g = chG[jj];
+                    const float2 r1 = crcp(make_float2(-lam_n.x, g - lam_n.y));
+                    const float2 r2 = crcp(make_float2(-lam_n.x, g + lam_n.y));
+                    const float2 q1 = cmul(r1, r1), q2 = cmul(r2, r2);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const float2 av = make_float2(chA[8 * jj + 2 * v], chA[8 * jj + 2 * v + 1]);
+                        S[v] = cadd(S[v], cadd(cmul(av, r2), cconj(cmul(av, r1))));
+                        S2[v] = cadd(S2[v], cadd(cmul(av, q2), cconj(cmul(av, q1))));
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        // ---- add the partial sums of each mode; the Nyquist bin; write
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            red[16 * tid + 2 * v] = S[v].x;
+            red[16 * tid + 2 * v + 1] = S[v].y;
+            red[16 * tid + 8 + 2 * v] = S2[v].x;
+            red[16 * tid + 8 + 2 * v + 1] = S2[v].y;
+        }
+        const float gN = buf[pidx(digrev_inv<LG>(L / 2))].x / (float)L;
+        if (tid < Nh) {   // Nyquist share of dlog_dt: gN dt Re(C_n B_n), summed below
+            const float *w = md + kModeFloats * tid;
+            ld_acc = fmaf(gN * dt, w[10], ld_acc);
+        }
+        for (int off = 16; off > 0; off >>= 1) ld_acc += __shfl_xor_sync(0xffffffffu, ld_acc, off);
+        if ((tid & 31) == 0) red32[tid >> 5] = ld_acc;
+        __syncthreads();
+        if (tid == 0) {
+            float sum = 0.0f;
+            for (int i = 0; i < T / 32; ++i) sum += red32[i];
+            dlog_dt[h] = sum;
+        }
+        for (int n = tid; n < Nh; n += T) {
+            float2 Sv[4], S2v[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) Sv[v] = S2v[v] = make_float2(0.f, 0.f);
+            for (int qq = 0; qq < nq; ++qq) {
+                const float *r = red + 16 * (qq * Nh + n);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    Sv[v] = cadd(Sv[v], make_float2(r[2 * v], r[2 * v + 1]));
+                    S2v[v] = cadd(S2v[v], make_float2(r[8 + 2 * v], r[8 + 2 * v + 1]));
+                }
+            }
+            const float *w = md + kModeFloats * n;
+            const float2 c = make_float2(w[2], w[3]), b = make_float2(w[4], w[5]);
+            const float2 p = make_float2(w[6], w[7]), q = make_float2(w[8], w[9]);
+            float2 gC = cadd(cmulc(Sv[0], b), cmulc(Sv[1], p));      // conj(B) S00 + conj(P) S01
+            float2 gB = cadd(cmulc(Sv[0], c), cmul(q, Sv[2]));       // conj(C) S00 + Q S10
+            const float2 gP = cadd(cmulc(Sv[1], c), cmul(q, Sv[3]));  // conj(C) S01 + Q S11
+            const float2 gQ = cadd(cmulc(b, Sv[2]), cmulc(p, Sv[3]));  // B conj(S10) + P conj(S11)
+            float2 gL = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) gL = cadd(gL, cmulc(S2v[v], make_float2(w[10 + 2 * v], w[11 + 2 * v])));
+            gC = cadd(gC, cscale(cconj(b), gN * dt));
+            gB = cadd(gB, cscale(cconj(c), gN * dt));
+            dLambda[po + n] = gL;
+            dP[po + n] = gP;
+            dQ[po + n] = gQ;
+            dB[po + n] = gB;
+            dC[po + n] = gC;
+        }
+        __syncthreads();   // shared memory is reused by the next channel
+    }
+}
+
 namespace {
 struct LaunchCache {
     int resident[64];
@@ -152,6 +388,47 @@ cudaError_t run_corr(const float *u, const float *dy, int Bt, int H, float *dK, 
     return cudaGetLastError();
 }
 }  // namespace
+
+namespace {
+template <int LG>
+cudaError_t run_kgen_backward(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
+                              const float2 *C, const float *log_dt, const float *dK, int H, int Nh,
+                              float2 *dLambda, float2 *dP, float2 *dQ, float2 *dB, float2 *dC, float *dlog_dt,
+                              cudaStream_t st) {
+    const size_t smem = kbwd_smem_bytes<LG>(Nh);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess && smem > 48 * 1024)
+        e = cudaFuncSetAttribute(k_kgen_backward<LG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = H < sms ? H : sms;
+    k_kgen_backward<LG><<<grid, kBwdThreads, smem, st>>>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ,
+                                                         dB, dC, dlog_dt);
+    return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
+                                 const float2 *C, const float *log_dt, const float *dK, int H, int Nh, int L,
+                                 float2 *dLambda, float2 *dP, float2 *dQ, float2 *dB, float2 *dC,
+                                 float *dlog_dt, cudaStream_t st) {
+#define S4_KBWD(LG) run_kgen_backward<LG>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC, dlog_dt, st)
+    switch (L) {
+        case 16: return S4_KBWD(4);
+        case 32: return S4_KBWD(5);
+        case 64: return S4_KBWD(6);
+        case 128: return S4_KBWD(7);
+        case 256: return S4_KBWD(8);
+        case 512: return S4_KBWD(9);
+        case 1024: return S4_KBWD(10);
+        case 2048: return S4_KBWD(11);
+        case 4096: return S4_KBWD(12);
+        case 8192: return S4_KBWD(13);
+        default: return cudaErrorInvalidValue;
+    }
+#undef S4_KBWD
+}
 
 size_t corr_workspace_bytes(int H, int L) {
     return 2 * (((size_t)H * 2 * L * sizeof(float2) + 255) & ~size_t(255));

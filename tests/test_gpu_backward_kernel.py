@@ -1,0 +1,77 @@
+"""GPU parity of the gradient through the DPLR kernel (s4_kernel_dplr_backward;
+"The S4 kernel, from scratch", §4 generating function, §6 trainable
+parameters) against central differences of the oracle's dense fp64 aliased
+kernel, and of the whole layer's backward (kernel + convolution)."""
+import numpy as np
+import pytest
+
+import s4inputs
+from oracle import ssm, workloads
+from gpu_helpers import to_dev, torch_cuda
+
+pytestmark = pytest.mark.gpu
+
+# per parameter array: max |g - g_ref| / max |g_ref|. The GPU sums L/2
+# frequencies x Nh modes of fp32 terms (relative rounding ~6e-8 each, growing
+# like the square root of the term count, with cancellation between a mode
+# and its conjugate partner); the finite differences are good to ~1e-8.
+# Random systems measured at most 2e-5 (L = 16..8192); the HiPPO-LegS modes
+# span a wider range of |Im Lambda| and get a wider bound.
+P_TOL = 2e-4
+P_TOL_HIPPO = 1e-3
+KEYS = ("Lambda", "P", "Q", "B", "C", "log_dt")
+
+
+def _gpu_grad(inp, dK):
+    import structured_state_space_dplr_b200 as s4
+    torch = torch_cuda()
+    t = to_dev(inp, ["Lambda", "P", "Q", "B", "C", "log_dt"])
+    g = s4.kernel_dplr_backward(t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"],
+                                torch.from_numpy(np.ascontiguousarray(dK, np.float32)).cuda())
+    torch.cuda.synchronize()
+    return {k: v.cpu().numpy() for k, v in g.items()}
+
+
+def _check(g, ref, channels, tol=P_TOL):
+    for k in KEYS:
+        a, b = g[k][channels], ref[k]
+        err = np.abs(a - b).max() / np.abs(b).max()
+        assert err <= tol, (k, err)
+
+
+@pytest.mark.parametrize("L", [16, 64, 256, 1024, 4096, 8192])
+def test_random_dplr_parameter_gradients(L):
+    inp = s4inputs.random_dplr(40 + L, H=2, Nh=5, L=L, Bt=1)
+    dK = np.random.default_rng(L).standard_normal((2, L))
+    g = _gpu_grad(inp, dK)
+    ref = workloads.dplr_kernel_param_grad(inp, dK)
+    _check(g, ref, slice(None))
+
+
+def test_hippo_parameter_gradients_one_channel():
+    """HiPPO-LegS modes (Nh = 32, |Im Lambda| up to ~1300), L = 1024."""
+    inp = s4inputs.make_inputs(1, with_u=False)
+    dK = np.random.default_rng(3).standard_normal((inp["H"], inp["L"]))
+    g = _gpu_grad(inp, dK)
+    ref = workloads.dplr_kernel_param_grad(inp, dK[2:3], channels=[2])
+    _check(g, ref, [2], P_TOL_HIPPO)
+
+
+def test_layer_backward_composes_to_finite_differences():
+    """d<y, dy>/dtheta for y = forward_dplr(u; theta): dK from the batch
+    correlation, then the kernel backward; against central differences of
+    the oracle's kernel + direct convolution."""
+    import structured_state_space_dplr_b200 as s4
+    torch = torch_cuda()
+    inp = s4inputs.random_dplr(77, H=2, Nh=4, L=128, Bt=3)
+    dy = np.random.default_rng(9).standard_normal((3, 2, 128)).astype(np.float32)
+    t = to_dev(inp)
+    dK, dD = s4.fft_conv_kernel_grad(t["u"], torch.from_numpy(dy).cuda())
+    g = s4.kernel_dplr_backward(t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], dK)
+    torch.cuda.synchronize()
+    g = {k: v.cpu().numpy() for k, v in g.items()}
+    # oracle: the layer's dK by its definition, then the kernel gradient by differences
+    dKr, dDr = ssm.causal_conv_kernel_grad(inp["u"], dy)
+    ref = workloads.dplr_kernel_param_grad(inp, dKr)
+    _check(g, ref, slice(None))
+    assert np.allclose(dD.cpu().numpy(), dDr, rtol=1e-4, atol=1e-4 * np.abs(dDr).max())

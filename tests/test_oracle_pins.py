@@ -324,3 +324,36 @@ def test_conv_adjoint_identity_and_kernel_grad_by_basis():
     du1 = ssm.causal_conv_adjoint(d1, K[:1], D[:1])[0, 0]
     assert np.allclose(du1[:31], K[0, 30::-1] + np.where(np.arange(31) == 30, D[0], 0.0), rtol=0, atol=1e-14)
     assert np.all(du1[31:] == 0.0)
+
+
+def test_fd_gradient_matches_s4d_closed_form_derivative():
+    """The finite-difference helper behind the kernel-parameter gradients,
+    on the S4D kernel K[k] = 2 Re sum_n C_n Bbar_n Abar_n^k, whose derivative
+    in C is closed form: d<K, G>/dRe C_n + i d<K, G>/dIm C_n
+    = 2 sum_k G[k] conj(Bbar_n Abar_n^k)."""
+    rng = np.random.default_rng(8)
+    Nh, L = 3, 24
+    a = -0.3 - rng.uniform(0, 0.5, Nh) + 1j * np.pi * np.arange(Nh)
+    B = np.ones(Nh, complex)
+    C = rng.standard_normal(Nh) + 1j * rng.standard_normal(Nh)
+    dt = 0.07
+    G = rng.standard_normal(L)
+
+    def fun(p):
+        return float(np.dot(ssm.s4d_kernel(a[None], B[None], p["C"][None], np.array([dt]), L)[0], G))
+
+    g = workloads.fd_gradient(fun, {"C": C}, ["C"])["C"]
+    Ab, Bb = ssm.zoh_diag(a, B, dt)
+    ref = 2.0 * np.array([np.sum(G * np.conj(Bb[n] * Ab[n] ** np.arange(L))) for n in range(Nh)])
+    assert np.abs(g - ref).max() <= 1e-7 * np.abs(ref).max()
+    # a real parameter, log(dt): with Bbar Abar^k = (e^{dt a} - 1)/a B e^{k dt a},
+    # d/d log(dt) = dt B (e^{(k+1) dt a} + k (e^{dt a} - 1) e^{k dt a})
+    def fun_dt(p):
+        return float(np.dot(ssm.s4d_kernel(a[None], B[None], C[None], np.exp(p["ld"]), L)[0], G))
+    g1 = workloads.fd_gradient(fun_dt, {"ld": np.array([np.log(dt)])}, ["ld"])["ld"][0]
+    k = np.arange(L)
+    dK = sum(2.0 * np.real(C[n] * dt * B[n] * (np.exp((k + 1) * dt * a[n])
+                                              + k * (np.exp(dt * a[n]) - 1.0) * np.exp(k * dt * a[n])))
+             for n in range(Nh))
+    ref_dt = float(np.dot(dK, G))
+    assert abs(g1 - ref_dt) <= 1e-7 * abs(ref_dt)
