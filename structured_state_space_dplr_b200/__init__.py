@@ -25,7 +25,8 @@ __all__ = [
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
     "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "dplr_ctilde", "forward_dplr_host",
-    "fft_conv_host", "fft_conv_apply_adjoint", "fft_conv_kernel_grad", "kernel_dplr_backward", "load",
+    "fft_conv_host", "fft_conv_apply_adjoint", "fft_conv_kernel_grad", "fft_conv_kernel_grad_workspace_size",
+    "kernel_dplr_backward", "load",
 ]
 
 
@@ -101,6 +102,13 @@ def irfft_packed(K):
     H, L = K.shape
     _lib.call("s4_irfft_packed", _ptr(K), H, L, _stream())
     return K
+
+
+def fft_conv_kernel_grad_workspace_size(H, L) -> int:
+    """Bytes of workspace fft_conv_kernel_grad needs (L <= 8192)."""
+    n = ctypes.c_size_t()
+    _lib.call("s4_fft_conv_kernel_grad_workspace_size", int(H), int(L), ctypes.byref(n))
+    return n.value
 
 
 def fft_conv_workspace_size(H, L) -> int:
@@ -207,9 +215,7 @@ def fft_conv_kernel_grad(u, dy, *, dK=None, dD=None, workspace=None):
     _cuda(dK, "dK", torch.float32)
     _cuda(dD, "dD", torch.float32)
     if workspace is None:
-        n = ctypes.c_size_t()
-        _lib.call("s4_fft_conv_kernel_grad_workspace_size", H, L, ctypes.byref(n))
-        workspace = torch.empty(n.value, dtype=torch.uint8, device=u.device)
+        workspace = torch.empty(fft_conv_kernel_grad_workspace_size(H, L), dtype=torch.uint8, device=u.device)
     _cuda(workspace, "workspace", torch.uint8)
     _lib.call("s4_fft_conv_kernel_grad", _ptr(u), _ptr(dy), Bt, H, L, _ptr(dK), _ptr(dD), _ptr(workspace),
               workspace.numel(), _stream())

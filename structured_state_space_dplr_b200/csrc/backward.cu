@@ -161,13 +161,15 @@ __host__ __device__ constexpr size_t kbwd_smem_bytes(int Nh) {
            sizeof(float) * ((size_t)kModeFloats * Nh + 9 * kBwdThreads + 16 * kBwdThreads + 32);
 }
 
+// 1/d for complex d (hardware reciprocal of |d|^2; |d| >= |Re lambda| > 0)
 __device__ __forceinline__ float2 crcp(float2 d) {
-    const float inv = 1.0f / fmaf(d.x, d.x, d.y * d.y);
+    float inv;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(fmaf(d.x, d.x, d.y * d.y)));
     return make_float2(d.x * inv, -d.y * inv);
 }
 
 template <int LG>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 2)
 k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const float2 *__restrict__ Q,
                 const float2 *__restrict__ B, const float2 *__restrict__ Cc, const float *__restrict__ log_dt,
                 const float *__restrict__ dK, int H, int Nh, float2 *__restrict__ dLambda,
@@ -396,13 +398,16 @@ cudaError_t run_kgen_backward(const float2 *Lambda, const float2 *P, const float
                               float2 *dLambda, float2 *dP, float2 *dQ, float2 *dB, float2 *dC, float *dlog_dt,
                               cudaStream_t st) {
     const size_t smem = kbwd_smem_bytes<LG>(Nh);
-    int dev = 0, sms = 0;
+    int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess && smem > 48 * 1024)
         e = cudaFuncSetAttribute(k_kgen_backward<LG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_kgen_backward<LG>, kBwdThreads, smem);
     if (e != cudaSuccess) return e;
-    const int grid = H < sms ? H : sms;
+    const int slots = (per_sm > 0 ? per_sm : 1) * sms;
+    const int grid = H < slots ? H : slots;
     k_kgen_backward<LG><<<grid, kBwdThreads, smem, st>>>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ,
                                                          dB, dC, dlog_dt);
     return cudaGetLastError();
