@@ -114,7 +114,7 @@ k_corr_pair(const float *__restrict__ u, const float *__restrict__ dy, int Bt, i
         inverse_middle_x2<LG, T>(s.b0, s.b1, s.tws);
         const float scale = 1.0f / (float)(2 * m);
         float *dKh = dK + (size_t)h * L;
-        last_pass_halves_sum<LG>(s, [&](int t, float2 r) {
+        last_pass_halves_sum<LG>(s, [&](auto, int t, float2 r, float2) {
             dKh[t] = r.x * scale;
             if (t == 0 && dD != nullptr) dD[h] = r.x * scale;
         });

@@ -98,28 +98,31 @@ __device__ __forceinline__ int digrev_inv(int f) {
 }
 
 // ------------------------------------------------------------ butterflies --
-// cos(2 pi e / 32) for any integer e (values of cos(k pi / 16), k = 0..8)
-__host__ __device__ constexpr float cos32(int e) {
-    constexpr float c[9] = {1.0f, 0.98078528040323043f, 0.92387953251128674f, 0.83146961230254524f,
-                            0.70710678118654752f, 0.55557023301960218f, 0.38268343236508977f,
-                            0.19509032201612827f, 0.0f};
-    const int k = ((e % 32) + 32) % 32;          // angle k pi / 16 in [0, 2 pi)
-    return k <= 8 ? c[k] : (k <= 16 ? -c[16 - k] : (k <= 24 ? -c[k - 16] : c[32 - k]));
+// cos(2 pi e / 64) for any integer e (values of cos(k pi / 32), k = 0..16)
+__host__ __device__ constexpr float cos64(int e) {
+    constexpr float c[17] = {1.0f, 0.99518472667219693f, 0.98078528040323043f, 0.95694033573220882f,
+                             0.92387953251128674f, 0.88192126434835505f, 0.83146961230254524f,
+                             0.77301045336273699f, 0.70710678118654752f, 0.63439328416364549f,
+                             0.55557023301960218f, 0.47139673682599781f, 0.38268343236508977f,
+                             0.29028467725446233f, 0.19509032201612827f, 0.09801714032956077f, 0.0f};
+    const int k = ((e % 64) + 64) % 64;          // angle k pi / 32 in [0, 2 pi)
+    return k <= 16 ? c[k] : (k <= 32 ? -c[32 - k] : (k <= 48 ? -c[k - 32] : c[64 - k]));
 }
-__host__ __device__ constexpr float sin32(int e) { return cos32(e - 8); }
+__host__ __device__ constexpr float sin64(int e) { return cos64(e - 16); }
 
-// v * exp(DIR * 2 pi i E / N), N in {2, 4, 8, 16, 32}
+// v * exp(DIR * 2 pi i E / N), N in {2, 4, 8, 16, 32, 64}
 template <int E, int N, int DIR>
 __device__ __forceinline__ float2 rot(float2 v) {
-    constexpr int e = ((E * (32 / N)) % 32 + 32) % 32;
+    static_assert(N >= 2 && N <= 64 && (N & (N - 1)) == 0, "rot: N a power of two up to 64");
+    constexpr int e = ((E * (64 / N)) % 64 + 64) % 64;
     if constexpr (e == 0) return v;
-    else if constexpr (e == 8) return mul_i<DIR>(v);
-    else if constexpr (e == 16) return make_float2(-v.x, -v.y);
-    else if constexpr (e == 24) return mul_i<-DIR>(v);
+    else if constexpr (e == 16) return mul_i<DIR>(v);
+    else if constexpr (e == 32) return make_float2(-v.x, -v.y);
+    else if constexpr (e == 48) return mul_i<-DIR>(v);
     else {
-        constexpr float c = cos32(e);
-        constexpr float s = DIR > 0 ? sin32(e) : -sin32(e);
-        if constexpr (e % 4 == 0) {  // (+-1 +- i)/sqrt(2)
+        constexpr float c = cos64(e);
+        constexpr float s = DIR > 0 ? sin64(e) : -sin64(e);
+        if constexpr (e % 8 == 0) {  // (+-1 +- i)/sqrt(2)
             constexpr float h = 0.70710678118654752f;
             constexpr float sc = c > 0 ? 1.0f : -1.0f, ss = s > 0 ? 1.0f : -1.0f;
             float re = sc * v.x - ss * v.y, im = ss * v.x + sc * v.y;

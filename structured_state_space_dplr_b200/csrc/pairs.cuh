@@ -113,45 +113,62 @@ __device__ __forceinline__ void pair_stage_rows(const PairSmem &s, const float *
 
 // ------------------------------------------------------ both halves, pass 0 --
 // First forward pass of group j of both halves of the zero-padded length-2m
-// transform, from the m nonzero inputs v[p] = input point j + p S0: half 0
-// (even frequencies) transforms v as it is, half 1 (odd frequencies) after
-// the twist W_2m^-k, whose in-group share W_2R0^-p is a constant rotation and
-// whose remainder a_j b_j^q is applied with the group twiddles b_j^q.
-template <int LG>
-__device__ __forceinline__ void first_pass_halves(const PairSmem &s, const float2 (&v)[1 << plan_lr(LG, 0)],
-                                                  int j) {
+// transform: half 0 transforms v0, half 1 transforms v1 after the twist
+// W_2m^-k, whose in-group share W_2R0^-p is a constant rotation and whose
+// remainder a_j b_j^q is applied with the group twiddles b_j^q (v0, v1: the
+// group's inputs, point j + p S0). SCALE also multiplies every output of the
+// group by f (a twist constant over the group).
+template <int LG, bool SCALE>
+__device__ __forceinline__ void first_pass_halves2(const PairSmem &s, const float2 (&v0)[1 << plan_lr(LG, 0)],
+                                                   const float2 (&v1)[1 << plan_lr(LG, 0)], int j, float2 f) {
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = (1 << LG) / R0;
     float2 x[R0], z[R0];
     static_for<0, R0>([&](auto p) {
-        x[p] = v[p];
-        z[p] = rot<decltype(p)::value, 2 * R0, -1>(v[p]);
+        x[p] = v0[p];
+        z[p] = rot<decltype(p)::value, 2 * R0, -1>(v1[p]);
     });
     dft<R0, -1>(x);
     dft<R0, -1>(z);
     const float2 a = s.ta[j], b = s.tb[j];
-    float2 w = b, u = a;
     const int o = pidx(j);
-    s.b0[o] = x[0];
-    s.b1[o] = cmul(z[0], a);
-    static_for<1, R0>([&](auto q) {
-        u = cmul(u, b);
-        s.b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
-        s.b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], u);
-        w = cmul(w, b);
-    });
+    if constexpr (SCALE) {
+        float2 w = f, u = cmul(f, a);
+        s.b0[o] = cmul(x[0], w);
+        s.b1[o] = cmul(z[0], u);
+        static_for<1, R0>([&](auto q) {
+            w = cmul(w, b);
+            u = cmul(u, b);
+            s.b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+            s.b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], u);
+        });
+    } else {
+        float2 w = b, u = a;
+        s.b0[o] = x[0];
+        s.b1[o] = cmul(z[0], a);
+        static_for<1, R0>([&](auto q) {
+            u = cmul(u, b);
+            s.b0[o + poff<decltype(q)::value * S0>()] = cmul(x[q], w);
+            s.b1[o + poff<decltype(q)::value * S0>()] = cmul(z[q], u);
+            w = cmul(w, b);
+        });
+    }
+}
+// both halves from the same m nonzero inputs (the zero-padded length-2m transform)
+template <int LG>
+__device__ __forceinline__ void first_pass_halves(const PairSmem &s, const float2 (&v)[1 << plan_lr(LG, 0)],
+                                                  int j) {
+    first_pass_halves2<LG, false>(s, v, v, j, make_float2(1.0f, 0.0f));
 }
 
 // After the first pass of both halves (stored, all threads synced): forward
-// passes 1 .. P-1, then (spectrum + D) / 2L to spec_h in spec4_index order,
-// rank 0 then rank 1. Adding D to every frequency adds D delta_0 to K.
+// passes 1 .. P-1, then (spectrum + D) * scale in spec4_index order, half 0
+// to o0 and half 1 to o1. Adding D to every frequency adds D delta_0 to K.
 template <int LG>
-__device__ __forceinline__ void spectrum_tail(const PairSmem &s, float Dh, float2 *__restrict__ spec_h) {
+__device__ __forceinline__ void spectrum_tail2(const PairSmem &s, float Dh, float scale, float4 *__restrict__ o0,
+                                               float4 *__restrict__ o1) {
     constexpr int m = 1 << LG, T = pair_threads<LG>();
     constexpr int R = 1 << plan_lr(LG, plan_P(LG) - 1);
     forward_middle_x2<LG, T>(s.b0, s.b1, s.tws);
-    const float scale = 1.0f / (float)(2 * m);
-    float4 *o0 = reinterpret_cast<float4 *>(spec_h);
-    float4 *o1 = o0 + m / 2;
     for (int g = threadIdx.x; g < m / R; g += T) {
         const int base = g * R, o = pidx(base);
         float2 x[R], z[R];
@@ -166,6 +183,13 @@ __device__ __forceinline__ void spectrum_tail(const PairSmem &s, float Dh, float
                                                        (z[2 * i + 1].x + Dh) * scale, z[2 * i + 1].y * scale);
         });
     }
+}
+// the length-2m spectrum of one channel: rank 0 then rank 1, scaled by 1/2m
+template <int LG>
+__device__ __forceinline__ void spectrum_tail(const PairSmem &s, float Dh, float2 *__restrict__ spec_h) {
+    constexpr int m = 1 << LG;
+    float4 *o0 = reinterpret_cast<float4 *>(spec_h);
+    spectrum_tail2<LG>(s, Dh, 1.0f / (float)(2 * m), o0, o0 + m / 2);
 }
 
 // The same spectrum from K[h, :] in global memory (tables built, all threads
@@ -186,8 +210,9 @@ __device__ __forceinline__ void kspec_channel(const PairSmem &s, const float *__
 
 // Last inverse pass of both halves (all threads synced on entry): output
 // point t < m of the length-2m inverse is half 0's value plus half 1's, the
-// latter twisted back by W_2m^t (in-group share W_2R0^p); out(t, value)
-// receives each one.
+// latter twisted back by W_2m^t (in-group share W_2R0^p); out(p, t, sum,
+// diff) receives that sum and the difference (half 0 minus half 1), with p
+// (t = j + p S0) as a compile-time constant.
 template <int LG, class Out>
 __device__ __forceinline__ void last_pass_halves_sum(const PairSmem &s, Out &&out) {
     constexpr int m = 1 << LG, T = pair_threads<LG>();
@@ -208,7 +233,8 @@ __device__ __forceinline__ void last_pass_halves_sum(const PairSmem &s, Out &&ou
         dft<R0, +1>(x);
         dft<R0, +1>(z);
         static_for<0, R0>([&](auto p) {
-            out(j + p * S0, cadd(x[p], rot<decltype(p)::value, 2 * R0, +1>(z[p])));
+            const float2 rz = rot<decltype(p)::value, 2 * R0, +1>(z[p]);
+            out(p, j + p * S0, cadd(x[p], rz), csub(x[p], rz));
         });
     }
 }
@@ -263,7 +289,7 @@ __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__res
     __syncthreads();
     inverse_middle_x2<LG, T>(b0, b1, s.tws);
     // ---- last inverse pass of both halves + their sum, straight to y
-    last_pass_halves_sum<LG>(s, [&](int t, float2 r) {
+    last_pass_halves_sum<LG>(s, [&](auto, int t, float2 r, float2) {
         y0[t] = r.x;
         if (has1) y1[t] = r.y;
     });

@@ -304,6 +304,162 @@ k_kspec_pair(const float *__restrict__ K, const float *__restrict__ D, int H, fl
     }
 }
 
+// ------------------------------------------------ fftconv, cluster of two --
+// L = 16384: the zero-padded length-N = 2L transform split four ways, rank c
+// holding the frequencies 4f + c (m = N/4 = 8192 points each). With the
+// nonzero input in two chunks x0[k] = x[k], x1[k] = x[k + m] (k < m), rank c
+// transforms v_c[k] = W_N^{kc} (x0[k] + (-i)^c x1[k]), and the output points
+// k and k + m are
+//   x[k + r m] = sum_c i^{c r} W_N^{-ck} Z_c[k]     (Z_c: rank c after the
+//                                                    product and the inverse).
+// A cluster of two CTAs takes a row pair; CTA 0 holds ranks 0 and 2, CTA 1
+// ranks 1 and 3, as the two halves of the one-CTA kernel (rank c + 2 is rank
+// c twisted by W_N^{2k} = W_2m^k, the halves' relation there):
+//   CTA 0: halves from x0 + x1 and x0 - x1;
+//   CTA 1: halves from W_N^k (x0 - i x1) and W_N^k (x0 + i x1).
+// The halves' last inverse pass gives each CTA their sum S and difference M
+// at every k, and
+//   x[k] = S_0 + W_N^-k S_1,   x[k + m] = M_0 + i W_N^-k M_1.
+// So CTA 0 keeps S_0 and hands M_0 over, CTA 1 keeps i W_N^-k M_1 and hands
+// W_N^-k S_1 over, through distributed shared memory; CTA 0 writes x[k], CTA 1
+// x[k + m]. The spectrum holds 4 ranks x m points per channel (k_kspec_quad).
+constexpr int kQuadLG = 13;
+
+// the two ranks' inputs of point k = j + p S0 from the chunks a = x0[k], b = x1[k]
+template <int P>
+__device__ __forceinline__ void quad_inputs(int cr, float2 a, float2 b, float2 &v0, float2 &v1) {
+    if (cr == 0) {
+        v0 = cadd(a, b);
+        v1 = csub(a, b);
+    } else {   // W_N^{p S0} = W_64^p inside the group; W_N^j goes with the group twiddles
+        v0 = rot<P, 64, -1>(cadd(a, mul_i<-1>(b)));
+        v1 = rot<P, 64, -1>(cadd(a, mul_i<+1>(b)));
+    }
+}
+
+template <bool CONJ>
+__global__ void __launch_bounds__(pair_threads<kQuadLG>(), 1)
+k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, float *__restrict__ y) {
+    constexpr int LG = kQuadLG, m = 1 << LG, L = 2 * m, T = pair_threads<LG>();
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
+    static_assert(S0 == T, "one first-pass group per thread");
+    extern __shared__ float2 sm[];
+    const PairSmem s = pair_carve<LG>(sm);
+    float2 *tc = reinterpret_cast<float2 *>(s.stage);   // W_N^j (the stage area is free here)
+    cg::cluster_group cluster = cg::this_cluster();
+    const int cr = (int)cluster.block_rank();
+    const float2 *rb0 = cluster.map_shared_rank(s.b0, cr ^ 1);
+    pair_tables<LG>(s);
+    const int j = threadIdx.x;
+    tc[j] = unit_root(j, 2 * L);
+    __syncthreads();
+    const long long npairs = (long long)H * ((Bt + 1) / 2);
+    const long long cl = blockIdx.x / 2, ncl = gridDim.x / 2;
+    bool first = true;
+    for (long long pr = cl; pr < npairs; pr += ncl) {
+        const RowPair r = row_pair(pr, Bt);
+        const float *u0 = u + ((size_t)r.b0 * H + r.h) * L;
+        const float *u1 = u0 + (size_t)H * L;
+        float2 v0[R0], v1[R0];
+        static_for<0, R0>([&](auto p) {
+            const int k = j + p * S0;
+            const float2 a = make_float2(__ldg(u0 + k), r.has1 ? __ldg(u1 + k) : 0.0f);
+            const float2 b = make_float2(__ldg(u0 + k + m), r.has1 ? __ldg(u1 + k + m) : 0.0f);
+            quad_inputs<decltype(p)::value>(cr, a, b, v0[p], v1[p]);
+        });
+        if (!first) cluster_wait();   // the partner has read this CTA's previous hand-over
+        first = false;
+        if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
+        else first_pass_halves2<LG, true>(s, v0, v1, j, tc[j]);
+        __syncthreads();
+        forward_middle_x2<LG, T>(s.b0, s.b1, s.tws);
+        const float2 *sh = spec + (size_t)r.h * 2 * L;
+        const float4 *k0p = reinterpret_cast<const float4 *>(sh + (size_t)cr * m);
+        const float4 *k1p = reinterpret_cast<const float4 *>(sh + (size_t)(cr + 2) * m);
+        struct SpecWords { float4 k0[RL / 2], k1[RL / 2]; };
+        fused_middle_x2<LG, T>(s.b0, s.b1, [&](int base) {
+            SpecWords w;
+            static_for<0, RL / 2>([&](auto i) {
+                w.k0[i] = __ldg(k0p + spec4_index<LG>(base, i));
+                w.k1[i] = __ldg(k1p + spec4_index<LG>(base, i));
+            });
+            return w;
+        }, [&](const SpecWords &w, auto &x, auto &z) {
+            auto mul = [](float2 a, float x0, float x1) {
+                if constexpr (CONJ) return cmulc(a, make_float2(x0, x1)); else return cmul(a, make_float2(x0, x1));
+            };
+            static_for<0, RL / 2>([&](auto i) {
+                x[2 * i] = mul(x[2 * i], w.k0[i].x, w.k0[i].y);
+                x[2 * i + 1] = mul(x[2 * i + 1], w.k0[i].z, w.k0[i].w);
+                z[2 * i] = mul(z[2 * i], w.k1[i].x, w.k1[i].y);
+                z[2 * i + 1] = mul(z[2 * i + 1], w.k1[i].z, w.k1[i].w);
+            });
+        });
+        __syncthreads();
+        inverse_middle_x2<LG, T>(s.b0, s.b1, s.tws);
+        // ---- keep one of (S, M) in b1, hand the other over in b0 (each thread
+        // writes only the positions of its own group, which it has just read)
+        const float2 cj = cconj(tc[j]);   // W_N^-j
+        last_pass_halves_sum<LG>(s, [&](auto pc, int t, float2 S, float2 M) {
+            constexpr int p = decltype(pc)::value;
+            if (cr == 0) {
+                s.b1[pidx(t)] = S;
+                s.b0[pidx(t)] = M;
+            } else {   // W_N^-t = W_N^-j W_64^-p
+                s.b1[pidx(t)] = mul_i<+1>(rot<p, 64, +1>(cmul(M, cj)));
+                s.b0[pidx(t)] = rot<p, 64, +1>(cmul(S, cj));
+            }
+        });
+        cluster_arrive_release();
+        cluster_wait();
+        float *y0 = y + ((size_t)r.b0 * H + r.h) * L + (cr == 0 ? 0 : m);
+        float *y1 = y0 + (size_t)H * L;
+        static_for<0, R0>([&](auto p) {
+            const int t = j + p * S0;
+            const float2 o = cadd(s.b1[pidx(t)], rb0[pidx(t)]);
+            y0[t] = o.x;
+            if (r.has1) y1[t] = o.y;
+        });
+        cluster_arrive_relaxed();
+    }
+    if (!first) cluster_wait();   // the partner may still read this CTA's buffer
+}
+
+// The spectrum k_fftconv_quad reads: per channel 4 ranks x m points in
+// spec4_index order, rank c holding (FFT_N(K + D delta_0))[4f + c] / N. One
+// CTA per (channel, rank pair), persistent; K's two chunks enter as the
+// convolution's input rows do.
+__global__ void __launch_bounds__(pair_threads<kQuadLG>(), 1)
+k_kspec_quad(const float *__restrict__ K, const float *__restrict__ D, int H, float2 *__restrict__ spec) {
+    constexpr int LG = kQuadLG, m = 1 << LG, L = 2 * m;
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    extern __shared__ float2 sm[];
+    const PairSmem s = pair_carve<LG>(sm);
+    float2 *tc = reinterpret_cast<float2 *>(s.stage);
+    pair_tables<LG>(s);
+    const int j = threadIdx.x;
+    tc[j] = unit_root(j, 2 * L);
+    __syncthreads();
+    for (int it = blockIdx.x; it < 2 * H; it += gridDim.x) {
+        const int h = it >> 1, cr = it & 1;
+        const float *Kh = K + (size_t)h * L;
+        float2 v0[R0], v1[R0];
+        static_for<0, R0>([&](auto p) {
+            const int k = j + p * S0;
+            quad_inputs<decltype(p)::value>(cr, make_float2(__ldg(Kh + k), 0.0f),
+                                           make_float2(__ldg(Kh + k + m), 0.0f), v0[p], v1[p]);
+        });
+        if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
+        else first_pass_halves2<LG, true>(s, v0, v1, j, tc[j]);
+        __syncthreads();
+        float4 *sh = reinterpret_cast<float4 *>(spec + (size_t)h * 2 * L);
+        spectrum_tail2<LG>(s, D != nullptr ? __ldg(D + h) : 0.0f, 1.0f / (float)(2 * L), sh + (size_t)cr * (m / 2),
+                           sh + (size_t)(cr + 2) * (m / 2));
+        __syncthreads();
+    }
+}
+
 // ------------------------------------------------------------------ irfft --
 __device__ __forceinline__ float2 half_spec(const float *Kh, int f, int L) {
     if (f == 0) return make_float2(Kh[0], 0.0f);
@@ -588,7 +744,35 @@ size_t conv_workspace_bytes(int H, int L) {
     X(32768, 13, 8, false, false)   \
     X(65536, 14, 8, true, false)
 
+namespace {
+LaunchInfo g_quad_conv[2], g_quad_kspec;
+
+cudaError_t quad_kspec(const float *K, const float *D, int H, void *ws, cudaStream_t st) {
+    constexpr size_t smem = pair_smem_bytes<kQuadLG>(0);
+    int res = 0;
+    cudaError_t e = resident_units(k_kspec_quad, g_quad_kspec, 1, pair_threads<kQuadLG>(), smem, &res);
+    if (e != cudaSuccess) return e;
+    k_kspec_quad<<<res < 2 * H ? res : 2 * H, pair_threads<kQuadLG>(), smem, st>>>(K, D, H, (float2 *)ws);
+    return cudaGetLastError();
+}
+
+cudaError_t quad_conv(const float *u, const void *ws, int Bt, int H, float *y, bool adjoint, cudaStream_t st) {
+    constexpr size_t smem = pair_smem_bytes<kQuadLG>(0);
+    constexpr int T = pair_threads<kQuadLG>();
+    auto kern = adjoint ? k_fftconv_quad<true> : k_fftconv_quad<false>;
+    int res = 0;
+    cudaError_t e = resident_units(kern, g_quad_conv[adjoint], 2, T, smem, &res);
+    if (e != cudaSuccess) return e;
+    const long long npairs = (long long)H * ((Bt + 1) / 2);
+    const int ncl = (long long)res < npairs ? res : (int)npairs;
+    e = launch_clustered(kern, 2, ncl, T, smem, st, u, (const float2 *)ws, Bt, H, y);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st) {
+    if (L == 2 << kQuadLG) return quad_kspec(K, D, H, ws, st);
     switch (L) {
 #define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::kspec(K, D, H, L, ws, st);
         S4_CONV_CASES(X)
@@ -599,6 +783,7 @@ cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws,
 
 cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st,
                            bool adjoint) {
+    if (L == 2 << kQuadLG) return quad_conv(u, ws, Bt, H, y, adjoint, st);
     switch (L) {
 #define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::conv(u, ws, Bt, H, L, y, adjoint, st);
         S4_CONV_CASES(X)

@@ -35,6 +35,24 @@ def test_random_kernel_full_outputs(L, Bt, H):
             assert rel_l2(yg[b, h], yr[b, h]) <= 4 * Y_TOL
 
 
+@pytest.mark.parametrize("Bt,H", [(1, 1), (3, 2), (6, 3)])
+def test_cluster_of_two_full_outputs(Bt, H):
+    """L = 16384 (the transform split four ways over a cluster of two CTAs):
+    every output, unpaired rows, several channels, and more row pairs than
+    one cluster takes in a single pass."""
+    L = 16384
+    rng = np.random.default_rng(1600 + Bt)
+    u = rng.standard_normal((Bt, H, L), dtype=np.float32)
+    K = (rng.standard_normal((H, L)) * np.exp(-np.arange(L) / (L / 4))).astype(np.float32)
+    D = rng.standard_normal(H).astype(np.float32)
+    yg = _conv(u, K, D)
+    yr = ssm.causal_conv(u, K.astype(np.float64), D.astype(np.float64))
+    assert rel_l2(yg, yr) <= Y_TOL
+    for b in range(Bt):
+        for h in range(H):
+            assert rel_l2(yg[b, h], yr[b, h]) <= 4 * Y_TOL
+
+
 @pytest.mark.parametrize("L", [8192, 16384, 32768, 65536])
 def test_long_lengths_sampled(L):
     rng = np.random.default_rng(L)
