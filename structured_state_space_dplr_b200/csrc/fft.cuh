@@ -403,10 +403,12 @@ __device__ __forceinline__ int spec4_index(int base, int i) {
 }
 
 // Gather the input of an inverse transform into digit-reversed positions:
-// position p receives value(f) with f the frequency index held at p.
+// frequency f goes to the position that holds it. Threads take consecutive
+// frequencies, so value(f) may read global memory in order (coalesced); the
+// scattered side is the shared-memory store.
 template <int LG, int T, class Val>
 __device__ __forceinline__ void gather_digit_reversed(float2 *buf, Val &&value) {
-    for (int p = threadIdx.x; p < (1 << LG); p += T) buf[pidx(p)] = value(digrev<LG>(p));
+    for (int f = threadIdx.x; f < (1 << LG); f += T) buf[pidx(digrev_inv<LG>(f))] = value(f);
 }
 
 // ------------------------------------------------- two transforms at once --
