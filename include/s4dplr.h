@@ -54,6 +54,8 @@ typedef enum {
 /* Bits OR-ed into *d_flags by the kernels. */
 #define S4_FLAG_UNSTABLE  1u  /* some Re(Lambda) >= 0 (or Re(a) >= 0 for S4D)   */
 #define S4_FLAG_NONFINITE 2u  /* a non-finite value was produced                 */
+#define S4_FLAG_TIMEOUT   4u  /* a bounded wait for the tensor cores ran out: the
+                                 output is incomplete (not expected in practice) */
 
 #define S4_MIN_L 16
 #define S4_MAX_L 65536

@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libs4dplr.so")
 S4_OK, S4_ERR_INVALID_ARG, S4_ERR_UNSUPPORTED, S4_ERR_WORKSPACE, S4_ERR_CUDA = range(5)
 S4_FLAG_UNSTABLE = 1
 S4_FLAG_NONFINITE = 2
+S4_FLAG_TIMEOUT = 4
 S4_STEP_DENSE, S4_STEP_DIAG, S4_STEP_DPLR = 0, 1, 2
 
 _p = ctypes.c_void_p

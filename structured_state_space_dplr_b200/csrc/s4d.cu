@@ -163,6 +163,228 @@ k_vandermonde(const float2 *__restrict__ A, const float2 *__restrict__ B, const 
     }
 }
 
+// ------------------------------------------------- tensor-core product --
+// For L a multiple of 8192 the product K = 2 Re(G T) runs on the 5th-generation
+// tensor cores: with k = 64 kh + kl,
+//   K[h, 64 kh + kl] = 2 sum_c A[kh, c] B[kl, c],
+//   A[kh, 2n] = Re G[n, kh], A[kh, 2n+1] = -Im G[n, kh],
+//   B[kl, 2n] = Re T[n, kl], B[kl, 2n+1] = Im T[n, kl],
+// a real [128 x 64] x [64 x 64] product per tile of 128 kh rows and 32 modes.
+// The tables come from fp64 power recurrences (T[n, kl] = Abar^kl from
+// Abar^16b, G[n, kh] = CBbar Abar^(64 kh) from Abar^(64 kh0) and Abar^64),
+// each start value evaluated directly with an fp64 phase reduction. The
+// operands are split into two tf32 parts (hi: the top 19 bits, lo: the
+// fp32 remainder) and the product is A_hi B_hi + A_hi B_lo + A_lo B_hi with
+// tcgen05.mma kind::tf32 (fp32 accumulation in tensor memory): fp32-level
+// accuracy. One CTA of 256 threads per (channel, tile of 128 rows) at a
+// time; one thread issues the MMAs, an mbarrier signals their completion
+// (bounded wait), warp w reads rows 32 (w % 4) .. + 31, columns 32 (w / 4) ..
+// + 31 back with tcgen05.ld, and the tile leaves through shared memory as
+// whole rows.
+namespace tc {
+
+constexpr int kM = 128;   // kh rows per tile (tensor-memory lanes)
+constexpr int kN = 64;    // kl columns (KB)
+constexpr int kK = 64;    // 2 x 32 modes per chunk
+constexpr int kThreads = 256;   // 8 warps: all build tables; warp w reads lanes 32 (w % 4).. back
+constexpr int kModes = kK / 2;
+constexpr uint32_t kIdesc = (1u << 4)                          // D: f32
+                          | (2u << 7) | (2u << 10)             // A, B: tf32
+                          | ((uint32_t)(kN >> 3) << 17)        // N
+                          | ((uint32_t)(kM >> 4) << 24);       // M (A and B K-major)
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+__device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// shared-memory matrix descriptor: K-major, no swizzle; element (row r, k)
+// of a tile with `rows` rows at byte (r%8)*16 + (r/8)*128 + (k/4)*lbo + (k%4)*4,
+// lbo = rows/8 * 128 (8-row core matrices of 16 bytes per row)
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+__device__ __forceinline__ int tile_index(int rows, int r, int k) {
+    return ((r & 7) * 16 + (r >> 3) * 128 + (k >> 2) * (rows / 8) * 128 + (k & 3) * 4) >> 2;
+}
+__device__ __forceinline__ void split_tf32(double v, float &hi, float &lo) {
+    const float f = (float)v;
+    hi = __uint_as_float(__float_as_uint(f) & 0xFFFFE000u);
+    lo = f - hi;
+}
+// z^e for complex z = exp(dt a) given as ZohMode, directly (fp64 phase reduction)
+__device__ __forceinline__ double2 zoh_power_d(const ZohMode &z, long long e) {
+    double ph = (double)e * z.kph;
+    ph -= rint(ph);
+    double sn, cs;
+    sincospi(2.0 * ph, &sn, &cs);
+    const double mag = exp((double)e * z.kre);
+    return make_double2(mag * cs, mag * sn);
+}
+__device__ __forceinline__ double2 zmul(double2 a, double2 b) {
+    return make_double2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
+
+}  // namespace tc
+
+__global__ void __launch_bounds__(tc::kThreads, 1)
+k_vandermonde_tc(const float2 *__restrict__ A, const float2 *__restrict__ B, const float2 *__restrict__ Cc,
+                 const float *__restrict__ log_dt, int H, int Nh, int L, float *__restrict__ K,
+                 unsigned *__restrict__ flags) {
+    using namespace tc;
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    float *Ah = reinterpret_cast<float *>(smraw), *Al = Ah + kM * kK;
+    float *Bh = Al + kM * kK, *Bl = Bh + kN * kK;
+    ZohMode *zm = reinterpret_cast<ZohMode *>(Bl + kN * kK);        // [kModes]
+    double2 *cb = reinterpret_cast<double2 *>(zm + kModes);          // [kModes] C Bbar
+    double2 *a8s = cb + kModes;                                      // [kModes] Abar^8
+    double2 *a512s = a8s + kModes;                                   // [kModes] Abar^512
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(a512s + kModes);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);
+    float *out = Ah;   // the finished tile leaves through the A_hi area (kM x kN floats)
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(mbar)));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tslot)),
+                     "r"(kN));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tslot;
+    uint32_t phase = 0;
+    bool ok = true;
+    const int ntiles = L / (kM * kN);
+    for (int item = blockIdx.x; item < H * ntiles && ok; item += gridDim.x) {
+        const int h = item / ntiles, tile = item % ntiles;
+        const double dt = exp((double)__ldg(log_dt + h));
+        const long long kh0 = (long long)tile * kM;
+        for (int n0 = 0; n0 < Nh; n0 += kModes) {
+            const int nc = (Nh - n0) < kModes ? (Nh - n0) : kModes;
+            __syncthreads();   // the previous chunk's tiles and mode constants are free
+            if (tid < kModes) {
+                if (tid < nc) {
+                    const size_t o = (size_t)h * Nh + n0 + tid;
+                    const float2 an = A[o], cn = Cc[o];
+                    zm[tid] = zoh_mode(an, B[o], dt);
+                    cb[tid] = make_double2(cn.x * zm[tid].bbar.x - cn.y * zm[tid].bbar.y,
+                                           cn.x * zm[tid].bbar.y + cn.y * zm[tid].bbar.x);
+                    a8s[tid] = zoh_power_d(zm[tid], 8);
+                    a512s[tid] = zoh_power_d(zm[tid], 8 * kN);
+                    if (flags != nullptr && tile == 0 && !(an.x < 0.0f)) atomicOr(flags, S4_FLAG_UNSTABLE);
+                } else {   // padding modes contribute zero
+                    zm[tid].kre = 0.0; zm[tid].kph = 0.0;
+                    cb[tid] = make_double2(0.0, 0.0);
+                    a8s[tid] = a512s[tid] = make_double2(1.0, 0.0);
+                }
+            }
+            __syncthreads();
+            // Lane (r0, n % 4) of warp w (modes 4w .. 4w + 3) forms the rows r0 + 8 i
+            // of mode n: T[n][r0 + 8i] = Abar^(r0 + 8i), G[n][r0 + 8i]; the (re, im)
+            // pair of a mode sits in one 8-byte slot of the K-major tile, and a
+            // half-warp's 16 slots are distinct banks.
+            {
+                const int lane = tid & 31, r0 = lane & 7, n = 4 * warp + (lane >> 3);
+                const ZohMode &z = zm[n];
+                const double2 a8 = a8s[n], a512 = a512s[n];
+                double2 t = zoh_power_d(z, r0);
+                for (int i = 0; i < kN / 8; ++i) {
+                    float h0, l0, h1, l1;
+                    split_tf32(t.x, h0, l0);
+                    split_tf32(t.y, h1, l1);
+                    const int o = tile_index(kN, r0 + 8 * i, 2 * n);
+                    *reinterpret_cast<float2 *>(Bh + o) = make_float2(h0, h1);
+                    *reinterpret_cast<float2 *>(Bl + o) = make_float2(l0, l1);
+                    t = zmul(t, a8);
+                }
+                double2 g = zmul(cb[n], zoh_power_d(z, (long long)kN * (kh0 + r0)));
+                for (int i = 0; i < kM / 8; ++i) {
+                    float h0, l0, h1, l1;
+                    split_tf32(g.x, h0, l0);
+                    split_tf32(-g.y, h1, l1);
+                    const int o = tile_index(kM, r0 + 8 * i, 2 * n);
+                    *reinterpret_cast<float2 *>(Ah + o) = make_float2(h0, h1);
+                    *reinterpret_cast<float2 *>(Al + o) = make_float2(l0, l1);
+                    g = zmul(g, a512);
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the tiles, to the tensor cores
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncthreads();
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            if (tid == 0) {
+                constexpr uint32_t a_lbo = (kM / 8) * 128, b_lbo = (kN / 8) * 128;
+                const float *As[3] = {Ah, Ah, Al}, *Bs[3] = {Bh, Bl, Bh};
+                for (int pr = 0; pr < 3; ++pr) {
+                    for (int s = 0; s < kK / 8; ++s) {
+                        const uint64_t da = smem_desc(saddr(As[pr]) + s * 2 * a_lbo, a_lbo);
+                        const uint64_t db = smem_desc(saddr(Bs[pr]) + s * 2 * b_lbo, b_lbo);
+                        const uint32_t accumulate = (n0 > 0 || pr > 0 || s > 0) ? 1u : 0u;
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem),
+                            "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+                    }
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 saddr(mbar))
+                             : "memory");
+            }
+            // the MMAs read the tiles: wait before the next chunk or the read-back
+            uint32_t done = 0;
+            for (uint32_t it = 0; it < kSpinLimit && !done; ++it) {
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                    "selp.u32 %0, 1, 0, p;\n\t}\n"
+                    : "=r"(done)
+                    : "r"(saddr(mbar)), "r"(phase)
+                    : "memory");
+            }
+            phase ^= 1u;
+            ok = __syncthreads_and(done) != 0;   // one decision for the whole CTA
+            if (!ok) {   // never expected: report and stop, freeing tensor memory below
+                if (flags != nullptr && tid == 0) atomicOr(flags, S4_FLAG_TIMEOUT);
+                break;
+            }
+        }
+        if (!ok) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        // ---- read back: warp w holds rows 32 (w % 4) + lane, columns 32 (w / 4) .. + 31;
+        // 2x; out through shared memory
+        __syncthreads();   // every thread has passed the wait: the tiles may be overwritten
+        bool bad = false;
+        const int row = 32 * (warp & 3) + (tid & 31), col0 = 32 * (warp >> 2);
+        for (int c0 = col0; c0 < col0 + 32; c0 += 16) {
+            uint32_t v[16];
+            const uint32_t addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0;
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
+                "[%16];"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                : "r"(addr));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float k = 2.0f * __uint_as_float(v[i]);
+                bad |= !isfinite(k);
+                out[row * (kN + 1) + c0 + i] = k;   // padded rows: conflict-free columns
+            }
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        float *Kt = K + (size_t)h * L + (size_t)kh0 * kN;
+        for (int i = tid; i < kM * kN; i += kThreads) Kt[i] = out[(i / kN) * (kN + 1) + i % kN];
+        if (flags != nullptr && __any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(flags, S4_FLAG_NONFINITE);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kN));
+}
+
 __global__ void k_s4d_zoh(const float2 *__restrict__ A, const float2 *__restrict__ B,
                           const float *__restrict__ log_dt, int H, int Nh,
                           float2 *__restrict__ Abar, float2 *__restrict__ Bbar) {
@@ -174,8 +396,35 @@ __global__ void k_s4d_zoh(const float2 *__restrict__ A, const float2 *__restrict
     Bbar[i] = make_float2((float)z.bbar.x, (float)z.bbar.y);
 }
 
+namespace {
+// dynamic shared memory of k_vandermonde_tc: 4 operand tiles, mode constants, mbarrier, TMEM slot
+constexpr size_t kVdmTcSmem = ((sizeof(float) * (2 * tc::kM * tc::kK + 2 * tc::kN * tc::kK) +
+                                (sizeof(ZohMode) + 3 * sizeof(double2)) * tc::kModes + 16) + 127) / 128 * 128;
+int g_vdm_tc_resident[64];
+}  // namespace
+
 cudaError_t launch_vandermonde(const float2 *A, const float2 *B, const float2 *C, const float *log_dt,
                                int H, int Nh, int L, float *K, unsigned *flags, cudaStream_t st) {
+    if (L % (tc::kM * tc::kN) == 0) {   // L a multiple of 8192: the tensor-core product
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        int &res = g_vdm_tc_resident[dev & 63];
+        if (res == 0) {
+            e = cudaFuncSetAttribute(k_vandermonde_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kVdmTcSmem);
+            int per_sm = 0, sms = 0;
+            if (e == cudaSuccess)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_vandermonde_tc, tc::kThreads, kVdmTcSmem);
+            if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            if (per_sm * sms <= 0) return cudaErrorInvalidConfiguration;
+            res = per_sm * sms;
+        }
+        const long long items = (long long)H * (L / (tc::kM * tc::kN));
+        const int grid = (long long)res < items ? res : (int)items;
+        k_vandermonde_tc<<<grid, tc::kThreads, kVdmTcSmem, st>>>(A, B, C, log_dt, H, Nh, L, K, flags);
+        return cudaGetLastError();
+    }
     const int KB = L < kVdmKB ? L : kVdmKB;
     const int nkh = L / KB;
     dim3 grid((nkh + kVdmKH - 1) / kVdmKH, H);

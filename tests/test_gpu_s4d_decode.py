@@ -39,6 +39,22 @@ def test_vandermonde_long_and_many_modes():
     assert kernel_err(_vdm(inp), workloads.s4d_kernel(inp)) <= K_TOL
 
 
+@pytest.mark.parametrize("Nh", [4, 33, 100])
+def test_vandermonde_tensor_core_mode_chunks(Nh):
+    """L = 8192 takes the tensor-core product, 32 modes per chunk: partial and
+    several chunks accumulate in tensor memory; no wait runs out."""
+    torch = torch_cuda()
+    rng = np.random.default_rng(Nh)
+    inp = s4inputs.make_inputs(5, H=3, L=8192, with_u=False)
+    inp["A"] = (-rng.uniform(0.01, 1, (3, Nh)) + 1j * rng.uniform(0, 300, (3, Nh))).astype(np.complex64)
+    inp["B"] = np.ones((3, Nh), np.complex64)
+    inp["C"] = (rng.standard_normal((3, Nh)) + 1j * rng.standard_normal((3, Nh))).astype(np.complex64)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Kg = _vdm(inp, flags=flags)
+    assert int(flags.item()) == 0
+    assert kernel_err(Kg, workloads.s4d_kernel(inp)) <= K_TOL
+
+
 def test_vandermonde_cfg5_full_size_sampled():
     inp = s4inputs.make_inputs(5, with_u=False)
     Kg = _vdm(inp)
