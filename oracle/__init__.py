@@ -11,6 +11,8 @@ Contents:
   ssm        discretisation, generating function, the pages' Cauchy/Woodbury
              formula, aliased kernel by dense powers, direct causal
              convolution, recurrence, S4D kernel (§1, §3-§5; "S4" wiki, S4D)
+  block      the S4Block around the layer: channel layer norm, GLU-gated
+             projection, residual (§6 "Trainable layer")
   workloads  drivers over the seeded workloads in ``s4inputs``
   loops.c    the O(L N^2) / O(L^2) fp64 loops, compiled with gcc
 
@@ -18,5 +20,5 @@ Every function is pinned by a CPU test against something other than itself
 (values printed on the pages, closed forms, invariants, library routines,
 brute force); see tests/test_oracle_*.py. Parity unpinned: none.
 """
-from . import hippo, ssm, workloads  # noqa: F401
+from . import block, hippo, ssm, workloads  # noqa: F401
 from ._cloops import build as build_loops  # noqa: F401

@@ -137,6 +137,23 @@ def make_inputs(cfg: int, seed: int = 0, *, H=None, Bt=None, L=None, with_u=True
     return out
 
 
+def block_params(seed: int, H: int):
+    """Seeded S4Block parameters around an H-channel S4 layer.
+
+    Drawn from ``default_rng([seed, 7])`` (independent of the layer's own
+    draws), in this order: gamma = 1 + 0.1 N(0,1) [H]; beta = 0.1 N(0,1) [H];
+    W = N(0, 1/H) [2H, H] (rows [0, H) project to the GLU value, [H, 2H) to the
+    gate); bias = 0.1 N(0,1) [2H]. eps = 1e-5. All float32.
+    """
+    rng = np.random.default_rng([seed, 7])
+    gamma = 1.0 + 0.1 * rng.standard_normal(H)
+    beta = 0.1 * rng.standard_normal(H)
+    W = rng.standard_normal((2 * H, H)) / math.sqrt(H)
+    bias = 0.1 * rng.standard_normal(2 * H)
+    return dict(gamma=gamma.astype(np.float32), beta=beta.astype(np.float32),
+                W=W.astype(np.float32), bias=bias.astype(np.float32), eps=1e-5)
+
+
 def random_dplr(seed: int, H: int, Nh: int, L: int, Bt: int, *, dt_min=1e-3, dt_max=1e-1,
                 re_min=-2.0, re_max=-0.1, im_max=60.0, lowrank=1.0):
     """Random (non-HiPPO) DPLR systems for generality cases.
