@@ -303,6 +303,66 @@ s4_status s4_fft_conv_static(const float *u, const float *K, const float *D,
                              int Bt, int H, int L, float *y, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The S4Block around the layer ([S4K] §6 "Trainable layer": a pre-norm, a
+ * GLU-gated projection and a residual connection). All tensors [Bt, H, L]
+ * float, device, 16-byte aligned, time (L) contiguous -- the layout of u and
+ * y above. 1 <= Bt, 1 <= H <= 8192, L a power of two in [16, 65536],
+ * Bt * H * L < 2^40.
+ *
+ * s4_layernorm_channels: z[b,h,t] = (x[b,h,t] - mu[b,t]) / sqrt(var[b,t] +
+ *   eps) * gamma[h] + beta[h], mu and var the mean and the biased variance
+ *   of x[b, :, t] over the H channels. gamma, beta: [H] device. eps > 0.
+ *   z may equal x (in place) but must not otherwise overlap it.
+ *
+ * s4_glu_projection_prepare: splits W [2H, H] (device; rows [0, H) give the
+ *   GLU value, rows [H, 2H) the gate) into the operand images the projection
+ *   reads: bf16 high and low parts of every weight, laid out for the tensor
+ *   cores. workspace: s4_glu_projection_workspace_size(H) bytes, device,
+ *   256-byte aligned, caller-owned; valid until W changes.
+ *
+ * s4_glu_projection_residual: out[b,o,t] = x[b,o,t] + p[o] * sigmoid(p[H+o]),
+ *   p = W y[b, :, t] + bias, with W from the prepared workspace and bias
+ *   [2H] device. The product runs on the tensor cores as three bf16 products
+ *   of the split operands with fp32 accumulation (relative error ~1e-5 of
+ *   the sum of |W||y| terms). out may equal x; out must not overlap y or the
+ *   workspace. d_flags (nullable): S4_FLAG_TIMEOUT if a bounded wait for the
+ *   tensor cores ran out (the output is then incomplete).
+ *
+ * s4_block_forward: out = x + GLU(W S4(LN(x)) + bias) in three launches:
+ *   s4_layernorm_channels(x) -> z, s4_fft_conv_apply(z) -> y with the
+ *   prepared convolution workspace of the layer (s4_fft_conv_prepare or
+ *   s4_kernel_dplr_prepare: the spectrum of K + D delta_0), then
+ *   s4_glu_projection_residual(y, x) -> out. z and y are caller-owned
+ *   [Bt, H, L] buffers (they are the activations a backward pass needs);
+ *   out may equal x.
+ *
+ * Errors: null pointers, H > 8192, Bt/H < 1, eps <= 0 or not finite,
+ * misalignment, forbidden overlaps -> S4_ERR_INVALID_ARG; L not a power of
+ * two in range -> S4_ERR_UNSUPPORTED; workspace too small or misaligned ->
+ * S4_ERR_WORKSPACE.
+ * ------------------------------------------------------------------------ */
+#define S4_MAX_BLOCK_H 8192
+
+s4_status s4_layernorm_channels(const float *x, const float *gamma, const float *beta, float eps,
+                                int Bt, int H, int L, float *z, cudaStream_t stream);
+
+s4_status s4_glu_projection_workspace_size(int H, size_t *bytes);
+
+s4_status s4_glu_projection_prepare(const float *W, int H, void *workspace, size_t workspace_bytes,
+                                    cudaStream_t stream);
+
+s4_status s4_glu_projection_residual(const float *y, const float *x, const float *bias,
+                                     const void *workspace, size_t workspace_bytes,
+                                     int Bt, int H, int L, float *out, unsigned *d_flags,
+                                     cudaStream_t stream);
+
+s4_status s4_block_forward(const float *x, const float *gamma, const float *beta, float eps,
+                           const void *conv_workspace, size_t conv_workspace_bytes,
+                           const float *bias, const void *glu_workspace, size_t glu_workspace_bytes,
+                           int Bt, int H, int L, float *z, float *y, float *out, unsigned *d_flags,
+                           cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * s4d_kernel_vandermonde -- kernel of the diagonal S4D SSM with zero-order
  * hold ([S4W] "S4D"; ZOH rule of [S4K] §3):
  *     Abar_n = exp(dt a_n),  Bbar_n = (exp(dt a_n) - 1)/a_n * B_n,

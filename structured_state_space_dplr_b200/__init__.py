@@ -20,7 +20,7 @@ from ._lib import (S4_FLAG_NONFINITE, S4_FLAG_UNSTABLE, S4_STEP_DENSE, S4_STEP_D
                    S4Error)
 
 __all__ = [
-    "kernel_dplr", "kernel_dplr_prepare", "forward_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
+    "kernel_dplr", "kernel_dplr_prepare", "layernorm_channels", "glu_projection_workspace_size", "glu_projection_prepare", "glu_projection_residual", "block_forward", "forward_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
     "fft_conv_static",
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
@@ -186,6 +186,82 @@ def fft_conv_apply(u, workspace, *, out=None):
     _lib.call("s4_fft_conv_apply", _ptr(u), _ptr(workspace), Bt, H, L, _ptr(out), workspace.numel(),
               _stream())
     return out
+
+
+# ------------------------------------------------------------ S4Block ----
+def layernorm_channels(x, gamma, beta, eps=1e-5, *, out=None):
+    """Layer norm over the H channels at each (b, t) of x [Bt, H, L]
+    (s4_layernorm_channels); out may be x."""
+    x = _cuda(x, "x", torch.float32)
+    gamma = _cuda(gamma, "gamma", torch.float32)
+    beta = _cuda(beta, "beta", torch.float32)
+    Bt, H, L = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_layernorm_channels", _ptr(x), _ptr(gamma), _ptr(beta), float(eps), Bt, H, L, _ptr(out),
+              _stream())
+    return out
+
+
+def glu_projection_workspace_size(H) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.call("s4_glu_projection_workspace_size", int(H), ctypes.byref(n))
+    return n.value
+
+
+def glu_projection_prepare(W, *, workspace=None):
+    """Split W [2H, H] into the projection's tensor-core operand images
+    (s4_glu_projection_prepare); returns the workspace."""
+    W = _cuda(W, "W", torch.float32)
+    H = W.shape[1]
+    if tuple(W.shape) != (2 * H, H):
+        raise ValueError("W must be [2H, H]")
+    need = glu_projection_workspace_size(H)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    _cuda(workspace, "workspace", torch.uint8)
+    _lib.call("s4_glu_projection_prepare", _ptr(W), H, _ptr(workspace), workspace.numel(), _stream())
+    return workspace
+
+
+def glu_projection_residual(y, x, bias, workspace, *, out=None, flags=None):
+    """out = x + p[:H] * sigmoid(p[H:]), p = W y + bias at each (b, t)
+    (s4_glu_projection_residual); out may be x."""
+    y = _cuda(y, "y", torch.float32)
+    x = _cuda(x, "x", torch.float32)
+    bias = _cuda(bias, "bias", torch.float32)
+    _cuda(workspace, "workspace", torch.uint8)
+    Bt, H, L = y.shape
+    if tuple(x.shape) != (Bt, H, L) or tuple(bias.shape) != (2 * H,):
+        raise ValueError("shapes: y, x [Bt, H, L], bias [2H]")
+    if out is None:
+        out = torch.empty_like(x)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_glu_projection_residual", _ptr(y), _ptr(x), _ptr(bias), _ptr(workspace), workspace.numel(),
+              Bt, H, L, _ptr(out), _flags_ptr(flags), _stream())
+    return out
+
+
+def block_forward(x, gamma, beta, eps, conv_workspace, bias, glu_workspace, *, z=None, y=None, out=None,
+                  flags=None):
+    """The S4Block: out = x + GLU(W S4(LN(x)) + bias) (s4_block_forward).
+    conv_workspace holds the layer's prepared spectrum (fft_conv_prepare or
+    kernel_dplr_prepare); glu_workspace comes from glu_projection_prepare.
+    Returns (out, z, y): z = LN(x) and y = S4(z) are kept for a backward pass."""
+    x = _cuda(x, "x", torch.float32)
+    for t, n in ((gamma, "gamma"), (beta, "beta"), (bias, "bias")):
+        _cuda(t, n, torch.float32)
+    _cuda(conv_workspace, "conv_workspace", torch.uint8)
+    _cuda(glu_workspace, "glu_workspace", torch.uint8)
+    Bt, H, L = x.shape
+    z = torch.empty_like(x) if z is None else _cuda(z, "z", torch.float32)
+    y = torch.empty_like(x) if y is None else _cuda(y, "y", torch.float32)
+    out = torch.empty_like(x) if out is None else _cuda(out, "out", torch.float32)
+    _lib.call("s4_block_forward", _ptr(x), _ptr(gamma), _ptr(beta), float(eps), _ptr(conv_workspace),
+              conv_workspace.numel(), _ptr(bias), _ptr(glu_workspace), glu_workspace.numel(), Bt, H, L,
+              _ptr(z), _ptr(y), _ptr(out), _flags_ptr(flags), _stream())
+    return out, z, y
 
 
 def fft_conv_apply_adjoint(dy, workspace, *, out=None):

@@ -30,6 +30,11 @@ SIGNATURES = {
     "s4_dplr_spectrum": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p, _p]),
     "s4_irfft_packed": (_i, [_p, _i, _i, _p]),
     "s4_fft_conv_workspace_size": (_i, [_i, _i, ctypes.POINTER(_sz)]),
+    "s4_layernorm_channels": (_i, [_p, _p, _p, ctypes.c_float, _i, _i, _i, _p, _p]),
+    "s4_glu_projection_workspace_size": (_i, [_i, ctypes.POINTER(_sz)]),
+    "s4_glu_projection_prepare": (_i, [_p, _i, _p, _sz, _p]),
+    "s4_glu_projection_residual": (_i, [_p, _p, _p, _p, _sz, _i, _i, _i, _p, _p, _p]),
+    "s4_block_forward": (_i, [_p, _p, _p, ctypes.c_float, _p, _sz, _p, _p, _sz, _i, _i, _i, _p, _p, _p, _p, _p]),
     "s4_fft_conv": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _sz, _p]),
     "s4_fft_conv_prepare": (_i, [_p, _p, _i, _i, _p, _sz, _p]),
     "s4_fft_conv_apply": (_i, [_p, _p, _i, _i, _i, _p, _sz, _p]),

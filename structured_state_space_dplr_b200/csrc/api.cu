@@ -116,6 +116,41 @@ s4_status host_buffer_checks(const float *u_host, const float *y_host, const flo
     return S4_OK;
 }
 
+// [Bt, H, L] activations of the S4Block entry points
+s4_status block_shape_checks(int Bt, int H, int L) {
+    if (Bt < 1 || H < 1 || H > S4_MAX_BLOCK_H) return S4_ERR_INVALID_ARG;
+    if (!pow2_L(L)) return S4_ERR_UNSUPPORTED;
+    if ((double)Bt * (double)H * (double)L >= 1099511627776.0) return S4_ERR_INVALID_ARG;   // 2^40
+    return S4_OK;
+}
+
+s4_status layernorm_checks(const float *x, const float *gamma, const float *beta, float eps, int Bt, int H, int L,
+                           const float *z) {
+    if (any_null(x, gamma, beta, z)) return S4_ERR_INVALID_ARG;
+    s4_status s = block_shape_checks(Bt, H, L);
+    if (s != S4_OK) return s;
+    if (!(eps > 0.0f) || !(eps < 3.0e38f)) return S4_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(z, 16) || !aligned(gamma, 4) || !aligned(beta, 4)) return S4_ERR_INVALID_ARG;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float);
+    if (z != x && overlap(x, nb, z, nb)) return S4_ERR_INVALID_ARG;
+    if (overlap(z, nb, gamma, (size_t)H * 4) || overlap(z, nb, beta, (size_t)H * 4)) return S4_ERR_INVALID_ARG;
+    return S4_OK;
+}
+
+s4_status glu_checks(const float *y, const float *x, const float *bias, const void *ws, size_t ws_bytes, int Bt,
+                     int H, int L, const float *out) {
+    if (any_null(y, x, bias, out) || ws == nullptr) return S4_ERR_INVALID_ARG;
+    s4_status s = block_shape_checks(Bt, H, L);
+    if (s != S4_OK) return s;
+    if (!aligned(y, 16) || !aligned(x, 16) || !aligned(out, 16) || !aligned(bias, 4)) return S4_ERR_INVALID_ARG;
+    if (!aligned(ws, 256) || ws_bytes < s4::glu_workspace_bytes(H)) return S4_ERR_WORKSPACE;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float);
+    if (overlap(out, nb, y, nb) || overlap(out, nb, ws, ws_bytes) || overlap(out, nb, bias, (size_t)2 * H * 4))
+        return S4_ERR_INVALID_ARG;
+    if (out != x && overlap(out, nb, x, nb)) return S4_ERR_INVALID_ARG;
+    return S4_OK;
+}
+
 // an event marking the work queued on st so far
 cudaError_t mark(cudaStream_t st, cudaEvent_t *ev) {
     cudaError_t e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
@@ -471,6 +506,57 @@ s4_status s4_recurrent_scan(s4_step_mode mode, const s4_c32 *Abar, const s4_c32 
     if (s != S4_OK) return s;
     return cuda_status(s4::launch_step((int)mode, (const float2 *)Abar, (const float2 *)Bbar, (const float2 *)C,
                                        D, Bt, H, Ns, T, (float2 *)x, u, y, stream));
+}
+
+// ---------------------------------------------------------------- S4Block
+s4_status s4_layernorm_channels(const float *x, const float *gamma, const float *beta, float eps, int Bt, int H,
+                                int L, float *z, cudaStream_t stream) {
+    s4_status s = layernorm_checks(x, gamma, beta, eps, Bt, H, L, z);
+    if (s != S4_OK) return s;
+    return cuda_status(s4::launch_layernorm_channels(x, gamma, beta, eps, Bt, H, L, z, stream));
+}
+
+s4_status s4_glu_projection_workspace_size(int H, size_t *bytes) {
+    if (bytes == nullptr || H < 1 || H > S4_MAX_BLOCK_H) return S4_ERR_INVALID_ARG;
+    *bytes = s4::glu_workspace_bytes(H);
+    return S4_OK;
+}
+
+s4_status s4_glu_projection_prepare(const float *W, int H, void *workspace, size_t workspace_bytes,
+                                    cudaStream_t stream) {
+    if (W == nullptr || workspace == nullptr || H < 1 || H > S4_MAX_BLOCK_H) return S4_ERR_INVALID_ARG;
+    if (!aligned(W, 4)) return S4_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || workspace_bytes < s4::glu_workspace_bytes(H)) return S4_ERR_WORKSPACE;
+    if (overlap(W, (size_t)2 * H * H * sizeof(float), workspace, workspace_bytes)) return S4_ERR_INVALID_ARG;
+    return cuda_status(s4::launch_glu_prepare(W, H, workspace, stream));
+}
+
+s4_status s4_glu_projection_residual(const float *y, const float *x, const float *bias, const void *workspace,
+                                     size_t workspace_bytes, int Bt, int H, int L, float *out, unsigned *d_flags,
+                                     cudaStream_t stream) {
+    s4_status s = glu_checks(y, x, bias, workspace, workspace_bytes, Bt, H, L, out);
+    if (s != S4_OK) return s;
+    return cuda_status(s4::launch_glu_projection(y, x, bias, workspace, Bt, H, L, out, d_flags, stream));
+}
+
+s4_status s4_block_forward(const float *x, const float *gamma, const float *beta, float eps,
+                           const void *conv_workspace, size_t conv_workspace_bytes, const float *bias,
+                           const void *glu_workspace, size_t glu_workspace_bytes, int Bt, int H, int L, float *z,
+                           float *y, float *out, unsigned *d_flags, cudaStream_t stream) {
+    s4_status s = layernorm_checks(x, gamma, beta, eps, Bt, H, L, z);
+    if (s == S4_OK && z == x) s = S4_ERR_INVALID_ARG;   // x is still needed for the residual
+    if (s == S4_OK) s = conv_checks(z, Bt, H, L, y, conv_workspace, conv_workspace_bytes);
+    if (s == S4_OK) s = glu_checks(y, x, bias, glu_workspace, glu_workspace_bytes, Bt, H, L, out);
+    if (s != S4_OK) return s;
+    const size_t nb = (size_t)Bt * H * L * sizeof(float);
+    if (overlap(x, nb, y, nb) || overlap(z, nb, out, nb) || overlap(z, nb, glu_workspace, glu_workspace_bytes) ||
+        overlap(y, nb, glu_workspace, glu_workspace_bytes) || overlap(z, nb, conv_workspace, conv_workspace_bytes) ||
+        overlap(out, nb, conv_workspace, conv_workspace_bytes))
+        return S4_ERR_INVALID_ARG;
+    cudaError_t e = s4::launch_layernorm_channels(x, gamma, beta, eps, Bt, H, L, z, stream);
+    if (e == cudaSuccess) e = s4::launch_fftconv(z, conv_workspace, Bt, H, L, y, stream);
+    if (e == cudaSuccess) e = s4::launch_glu_projection(y, x, bias, glu_workspace, Bt, H, L, out, d_flags, stream);
+    return cuda_status(e);
 }
 
 }  // extern "C"

@@ -49,6 +49,14 @@ cudaError_t launch_vandermonde(const float2 *A, const float2 *B, const float2 *C
 cudaError_t launch_s4d_zoh(const float2 *A, const float2 *B, const float *log_dt, int H, int Nh,
                            float2 *Abar, float2 *Bbar, cudaStream_t st);
 
+// ---- block.cu: the S4Block around the layer (norm, GLU projection, residual) ----
+size_t glu_workspace_bytes(int H);
+cudaError_t launch_layernorm_channels(const float *x, const float *gamma, const float *beta, float eps, int Bt,
+                                      int H, int L, float *z, cudaStream_t st);
+cudaError_t launch_glu_prepare(const float *W, int H, void *ws, cudaStream_t st);
+cudaError_t launch_glu_projection(const float *y, const float *x, const float *bias, const void *ws, int Bt, int H,
+                                  int L, float *out, unsigned *flags, cudaStream_t st);
+
 // ---- decode.cu ----
 cudaError_t launch_dplr_discretize(const float2 *Lambda, const float2 *P, const float2 *Q,
                                    const float2 *B, const float2 *C, const float *log_dt, int H, int Nh,

@@ -145,6 +145,41 @@ def test_backward_entries_reject_bad_arguments(lib):
     assert lib.s4_fft_conv_apply_adjoint(p(0), ws, 2, 4, 4096, dK, wsb, p(0)) == _lib.S4_ERR_INVALID_ARG
 
 
+def test_block_entries_reject_bad_arguments(lib):
+    n = ctypes.c_size_t()
+    assert lib.s4_glu_projection_workspace_size(0, ctypes.byref(n)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_glu_projection_workspace_size(8193, ctypes.byref(n)) == _lib.S4_ERR_INVALID_ARG
+    assert lib.s4_glu_projection_workspace_size(256, ctypes.byref(n)) == _lib.S4_OK
+    assert n.value == 4 * 8 * 2 * 8192          # (H/64 row blocks) x (H/32 chunks) x hi/lo x 8 KB
+    assert lib.s4_glu_projection_workspace_size(100, ctypes.byref(n)) == _lib.S4_OK
+    assert n.value == 2 * 4 * 2 * 8192          # ragged H rounds both counts up
+    x, z, g, b = p(FAKE), p(FAKE + 0x10000000), p(FAKE2), p(FAKE2 + 0x1000)
+    ln = lib.s4_layernorm_channels
+    assert ln(p(0), g, b, 1e-5, 2, 4, 64, z, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert ln(x, g, b, 0.0, 2, 4, 64, z, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert ln(x, g, b, float("nan"), 2, 4, 64, z, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert ln(x, g, b, 1e-5, 2, 4, 48, z, p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert ln(x, g, b, 1e-5, 0, 4, 64, z, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert ln(x, g, b, 1e-5, 2, 4, 64, p(FAKE + 64), p(0)) == _lib.S4_ERR_INVALID_ARG   # partial overlap
+    assert ln(x, g, b, 1e-5, 2, 4, 64, p(FAKE + 0x10000004), p(0)) == _lib.S4_ERR_INVALID_ARG   # misaligned
+    ws, wsb = p(FAKE2 + 0x100000), 4 * 8 * 2 * 8192
+    assert lib.s4_glu_projection_prepare(p(FAKE), 256, ws, wsb - 1, p(0)) == _lib.S4_ERR_WORKSPACE
+    assert lib.s4_glu_projection_prepare(p(FAKE), 256, p(FAKE2 + 0x100010), wsb, p(0)) == _lib.S4_ERR_WORKSPACE
+    assert lib.s4_glu_projection_prepare(p(0), 256, ws, wsb, p(0)) == _lib.S4_ERR_INVALID_ARG
+    y, out, bias = p(FAKE + 0x20000000), p(FAKE + 0x30000000), p(FAKE2 + 0x2000)
+    gl = lib.s4_glu_projection_residual
+    assert gl(y, x, bias, ws, wsb, 2, 256, 4096, y, p(0), p(0)) == _lib.S4_ERR_INVALID_ARG       # out = y
+    assert gl(y, x, bias, ws, wsb - 1, 2, 256, 4096, out, p(0), p(0)) == _lib.S4_ERR_WORKSPACE
+    assert gl(y, x, bias, ws, wsb, 2, 256, 1000, out, p(0), p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert gl(y, x, p(0), ws, wsb, 2, 256, 4096, out, p(0), p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert gl(y, x, bias, ws, wsb, 2, 256, 4096, p(FAKE + 4096), p(0), p(0)) == _lib.S4_ERR_INVALID_ARG
+    cws = p(FAKE2 + 0x40000000)
+    bf = lib.s4_block_forward
+    assert bf(x, g, b, 1e-5, cws, 1 << 30, bias, ws, wsb, 2, 256, 4096, x, y, out, p(0), p(0)) == \
+        _lib.S4_ERR_INVALID_ARG                                                                  # z = x
+    assert bf(x, g, b, 1e-5, cws, 16, bias, ws, wsb, 2, 256, 4096, z, y, out, p(0), p(0)) == _lib.S4_ERR_WORKSPACE
+
+
 def test_binding_refuses_cpu_tensors():
     torch = pytest.importorskip("torch")
     import structured_state_space_dplr_b200 as s4
