@@ -50,6 +50,11 @@ NOMINAL_SM_MHZ = 1965.0
 CAUCHY_FLOP_PER_TERM = 40
 VANDERMONDE_FLOP_PER_TERM = 4
 E2E_CHUNKS = 8   # row-pair chunks of the host-buffer pipeline
+# S4Block projection per (b, t) element of the output: 2 dot products of
+# length H (value and gate rows of W) = 4 H flop per output element; HBM
+# bytes: read y and x, write out
+BLOCK_FLOP_PER_ELEM = lambda H: 4 * H   # noqa: E731
+BLOCK_PROJ_BYTES_PER_ELEM = 12
 KERNEL_SOURCES = ["common.cuh", "fft.cuh", "pairs.cuh", "spectral.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fftconv_h256_l4096_b16_traffic.txt")
 
@@ -390,6 +395,53 @@ def run_gpu(args, rank, world, local_rank):
                     "calls": "s4_fft_conv_apply_adjoint + s4_fft_conv_kernel_grad"
                              + ("" if s4d else " + s4_kernel_dplr_backward") + ", one launch each"}
 
+    # the S4Block around the same layer: channel layer norm -> the layer's
+    # convolution (the prepared spectrum) -> GLU projection + residual, over
+    # the rotating input sets (x = the set's u)
+    bp = s4inputs.block_params(shard["seed"], H)
+    bdev = {k: torch.from_numpy(bp[k]).to(dev) for k in ("gamma", "beta", "W", "bias")}
+    glu_ws = s4.glu_projection_prepare(bdev["W"])
+    bz = [torch.empty_like(s["u"]) for s in sets]
+    bo = [torch.empty_like(s["u"]) for s in sets]
+
+    def blk(i, ev=None):
+        s, j = sets[i % nsets], i % nsets
+        if ev is not None:
+            ev[0].record()
+        s4.layernorm_channels(s["u"], bdev["gamma"], bdev["beta"], bp["eps"], out=bz[j])
+        if ev is not None:
+            ev[1].record()
+        s4.fft_conv_apply(bz[j], s["ws"], out=s["y"])
+        if ev is not None:
+            ev[2].record()
+        s4.glu_projection_residual(s["y"], s["u"], bdev["bias"], glu_ws, out=bo[j], flags=flags)
+        if ev is not None:
+            ev[3].record()
+
+    for i in range(args.warmup):
+        blk(i)
+    torch.cuda.synchronize()
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        blk(i, bev[i])
+    torch.cuda.synchronize()
+    if int(flags.item()) != 0:
+        raise RuntimeError(f"kernel flags set in the block: {int(flags.item())}")
+    kst = [sum(e[j].elapsed_time(e[j + 1]) for e in bev) / args.steps for j in range(3)]
+    del bz, bo
+    ktot = sum(kst)
+    proj_s = kst[2] * 1e-3
+    block = {"metric": "S4Block forward (batch*H*L) elems/s", "value": alg["elements"] / (ktot * 1e-3),
+             "ms_per_step": ktot,
+             "stages_us": {"layernorm": kst[0] * 1e3, "conv": kst[1] * 1e3, "glu_projection_residual": kst[2] * 1e3},
+             "glu_projection": {
+                 "tflops": BLOCK_FLOP_PER_ELEM(H) * alg["elements"] / proj_s / 1e12,
+                 "tensor_tflops_issued": 3 * BLOCK_FLOP_PER_ELEM(H) * alg["elements"] / proj_s / 1e12,
+                 "gbs": BLOCK_PROJ_BYTES_PER_ELEM * alg["elements"] / proj_s / 1e9,
+                 "operands": "fp32 split into bf16 hi/lo, 3 products (tcgen05 kind::f16), fp32 accumulate"},
+             "layernorm_gbs": 8 * alg["elements"] / (kst[0] * 1e-3) / 1e9,
+             "calls": "s4_layernorm_channels + s4_fft_conv_apply + s4_glu_projection_residual, one launch each"}
+
     # recurrent view (decode) of the same layer: up to 1024 tokens from a zero
     # state, as one s4_recurrent_scan and as single-token steps from a graph
     d = sets[0]
@@ -488,6 +540,7 @@ def run_gpu(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "decode": decode,
         "backward": backward,
+        "block": block,
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:

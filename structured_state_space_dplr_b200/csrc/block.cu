@@ -8,17 +8,34 @@
 //   out = x + p[:H] * sigmoid(p[H:])
 //
 // The projection is a dense contraction over channels and runs on the tensor
-// cores. Per CTA: one batch row b, 64 output channels and N (<= 128) time
-// steps; the 64 value rows and the 64 gate rows of W are interleaved into the
-// 128 rows of the MMA's A operand (row 2i = value of channel i, row 2i + 1 =
-// its gate), so the epilogue pairs them with one lane exchange. Operands are
-// fp32 split into bf16 high and low parts, and the three products
-// A_hi B_hi + A_hi B_lo + A_lo B_hi are accumulated in fp32 in tensor memory
-// (the dropped A_lo B_lo and the split residues are ~2^-17 relative). W is
-// split once into the MMA's shared-memory image by s4_glu_projection_prepare;
-// y is split on the way into shared memory, 32 channels per stage, two
-// stages in flight.
+// cores: D[t, n] = sum_h y[b, h, t0 + t] W'[n, h], one tile = 128 time steps
+// (the MMA's M, tensor-memory lanes) x 256 rows of W' (the MMA's N), where W'
+// interleaves the value and gate rows of 128 output channels (row 2i = value
+// of channel i, row 2i + 1 = its gate), so one thread holds both halves of a
+// GLU. Operands are fp32 split into bf16 high and low parts, and the three
+// products y_hi W_hi + y_hi W_lo + y_lo W_hi are accumulated in fp32 in
+// tensor memory (the dropped y_lo W_lo and the split residues are ~2^-17
+// relative). W is split once into the MMA's shared-memory image by
+// s4_glu_projection_prepare.
+//
+// The kernel is persistent (one CTA per SM) and warp-specialized:
+//   warp 0      loader: TMA of raw fp32 y chunks [32 channels x 128 steps]
+//               and bulk copies of the W image chunks, into rings;
+//   warps 1-4   split each raw y chunk into the bf16 image of the operand;
+//   warp 5      one thread issues the MMAs (6 per chunk) and the commits;
+//   warp 6      x loader: TMA of the residual x in [32 channels x 128 steps]
+//               chunks, into a ring;
+//   warps 7-14  epilogue: tensor memory -> GLU + bias + residual -> out; two
+//               warps per tensor-memory lane quadrant, each half the columns.
+// The accumulator is double-buffered (2 x 256 of the 512 tensor-memory
+// columns), so the epilogue of one tile overlaps the MMAs of the next. Every
+// wait is bounded: on expiry the CTA sets S4_FLAG_TIMEOUT, every role stops,
+// copies in flight are waited for (bounded) and tensor memory is freed.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "launch.h"
 #include "s4dplr.h"
@@ -27,25 +44,33 @@
 namespace s4 {
 
 namespace glu {
-constexpr int kRows = 128;                   // MMA M: 64 output channels x (value, gate)
-constexpr int kOut = kRows / 2;
-constexpr int kKc = 32;                      // channels per stage (two K = 16 MMA steps)
-constexpr int kNmax = 128;                   // time steps per tile (MMA N)
-constexpr int kThreads = 256;
-constexpr int kAImg = kRows * kKc * 2;       // bytes of one bf16 operand image of W (8 KB)
-constexpr int kBImg = kNmax * kKc * 2;       // bytes of one bf16 operand image of y (8 KB)
-constexpr int kStage = 2 * kAImg + 2 * kBImg;   // A hi, A lo, B hi, B lo
-constexpr int kStages = 2;
-constexpr int kTmemCols = 128;
-constexpr size_t kSmem = (size_t)kStages * kStage + 64;
-constexpr uint32_t kSpinLimit = 1u << 24;
-static_assert(kOut * (kNmax + 1) * 4 <= kStages * kStage, "epilogue tile must fit in the stage buffers");
+constexpr int kTm = 128;                      // MMA M: time steps per tile
+constexpr int kNr = 256;                      // MMA N: rows of W' per tile
+constexpr int kCh = kNr / 2;                  // output channels per tile
+constexpr int kKc = 32;                       // contraction channels per chunk (two K = 16 steps)
+constexpr int kYImg = kTm * kKc * 2;          // 8 KB: one bf16 image of a y chunk
+constexpr int kWImg = kNr * kKc * 2;          // 16 KB: one bf16 image of a W' chunk
+constexpr int kStage = 2 * kYImg + 2 * kWImg; // 48 KB: y hi, y lo, W hi, W lo
+constexpr int kRawBytes = kKc * kTm * 4;      // 16 KB: a raw fp32 chunk [32][<= 128]
+constexpr int kXc = 32;                       // output channels per x chunk of the epilogue
+constexpr int kS = 3, kR = 3, kX = 2;         // operand stages, raw y ring, x ring
+constexpr int kOffRaw = kS * kStage;
+constexpr int kOffX = kOffRaw + kR * kRawBytes;
+constexpr int kOffBar = kOffX + kX * kRawBytes;
+constexpr int kNumBars = 2 * kR + 3 * kS + 2 + 2 + 2 * kX;
+constexpr size_t kSmem = (size_t)kOffBar + kNumBars * 8 + 16;
+// warps: 0 y/W loader, 1-4 converters, 5 MMA, 6 x loader, 7-14 epilogue
+constexpr int kThreads = 15 * 32;
+constexpr int kEpiWarp0 = 7, kEpiThreads = 256;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kSpinLimit = 1u << 22;
+static_assert(kSmem <= 232448, "shared memory per CTA");
 }  // namespace glu
 
-__host__ __device__ inline int glu_nob(int H) { return (H + glu::kOut - 1) / glu::kOut; }
+__host__ __device__ inline int glu_nnb(int H) { return (H + glu::kCh - 1) / glu::kCh; }
 __host__ __device__ inline int glu_nkc(int H) { return (H + glu::kKc - 1) / glu::kKc; }
 
-size_t glu_workspace_bytes(int H) { return (size_t)glu_nob(H) * glu_nkc(H) * 2 * glu::kAImg; }
+size_t glu_workspace_bytes(int H) { return (size_t)glu_nkc(H) * glu_nnb(H) * 2 * glu::kWImg; }
 
 namespace {
 
@@ -69,75 +94,190 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4 &hi, uint4 &lo
     lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
-__device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + __expf(-g)); }
+// logistic function; __expf and __fdividef keep it to a few instructions
+// (relative error ~1e-7, far below the projection's)
+__device__ __forceinline__ float sigmoidf_(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+
+// ---- asynchronous copies and barrier arrivals (inline PTX)
+__device__ __forceinline__ void arrive(uint64_t *m) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(umma::saddr(m)) : "memory");
+}
+__device__ __forceinline__ void arrive_expect_tx(uint64_t *m, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(umma::saddr(m)), "r"(bytes)
+                 : "memory");
+}
+// 3-D tiled TMA load (no multicast) of the box at (x, y, z) into dst
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *m) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(umma::saddr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(umma::saddr(m))
+        : "memory");
+}
+// contiguous bulk copy global -> shared (no multicast); 16-byte aligned, size % 16 == 0
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *m) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     umma::saddr(dst)),
+                 "l"(src), "r"(bytes), "r"(umma::saddr(m))
+                 : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// AND of p over the `threads` threads of named barrier `id` (all of them get it)
+__device__ __forceinline__ bool named_and(int id, int threads, bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, o;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.and.pred o, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, o;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)p), "r"(id), "r"(threads)
+        : "memory");
+    return r != 0;
+}
+
+// the per-CTA tile sequence: tile i = ((b * ntt + tt) * nnb + nb), channel
+// block fastest (the tiles that read the same y chunks run side by side)
+struct Tile {
+    int b, t0, nb;
+};
+__device__ __forceinline__ Tile tile_of(long long i, int nnb, int ntt, int N) {
+    Tile t;
+    t.nb = (int)(i % nnb);
+    const long long r = i / nnb;
+    t.t0 = (int)(r % ntt) * N;
+    t.b = (int)(r / ntt);
+    return t;
+}
+// x chunks of a tile: 32 output channels each, up to H
+__device__ __forceinline__ int x_chunks(int H, int nb) {
+    const int left = H - nb * glu::kCh;
+    const int n = (left + glu::kXc - 1) / glu::kXc;
+    return n < glu::kCh / glu::kXc ? n : glu::kCh / glu::kXc;
+}
+
+// Shared state of the CTA's roles: a bounded wait that gives up when any
+// role has given up.
+struct Ctl {
+    volatile int *abort;
+    unsigned *flags;
+    __device__ __forceinline__ bool wait(uint64_t *m, uint32_t parity) {
+        uint32_t done = 0;
+        for (uint32_t it = 0; it < glu::kSpinLimit && !done; ++it) {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}\n"
+                : "=r"(done)
+                : "r"(umma::saddr(m)), "r"(parity)
+                : "memory");
+            if (!done && (it & 63) == 63 && *abort) return false;
+        }
+        if (!done) {
+            *abort = 1;
+            if (flags != nullptr) atomicOr(flags, S4_FLAG_TIMEOUT);
+        }
+        return done != 0;
+    }
+};
+
+// a ring position: slot and the parity of its current use
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++slot == n) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
 
 }  // namespace
 
 // ---------------------------------------------------------------- layer norm
-// One CTA: 32 consecutive time steps of one batch row; warp w sums channels
-// w, w + 8, ... (a warp reads 128 contiguous bytes per channel). The sums are
-// taken about x[b, 0, t] (shifted data: no cancellation for large means).
+// One CTA: 128 consecutive time steps of one batch row, 4 per thread (16-byte
+// accesses); warp w sums channels w, w + 8, ... with 8 loads in flight. The
+// sums are taken about x[b, 0, t] (shifted data: no cancellation for large
+// means). The second pass re-reads the CTA's slab, which is still in L2.
 // z may be x (in place): every element is read and then written by one thread.
+__device__ __forceinline__ float4 f4sub(float4 a, float4 b) { return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w); }
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+__device__ __forceinline__ float4 f4fma(float4 a, float4 b, float4 c) {
+    return make_float4(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y), fmaf(a.z, b.z, c.z), fmaf(a.w, b.w, c.w));
+}
+
 __global__ void __launch_bounds__(256) k_layernorm_channels(const float *x, const float *__restrict__ gamma,
                                                             const float *__restrict__ beta, float eps, int H,
                                                             int L, float *z) {
-    __shared__ float s1[8][33], s2[8][33], mu_s[32], rs_s[32];
+    __shared__ float4 s1[8][32], s2[8][32], mu_s[32], rs_s[32];
     const int tl = threadIdx.x & 31, hs = threadIdx.x >> 5;
-    const int t = blockIdx.x * 32 + tl;
-    const bool in = t < L;
+    const int t = blockIdx.x * 128 + 4 * tl;
+    const bool in = t < L;   // L is a multiple of 16: t < L implies t + 3 < L
     const size_t base = (size_t)blockIdx.y * H * L + t;
-    const float c = in ? x[base] : 0.0f;
-    float a1 = 0.0f, a2 = 0.0f;
+    const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const float4 c = in ? *reinterpret_cast<const float4 *>(x + base) : zero;
+    float4 a1 = zero, a2 = zero;
     if (in) {
-#pragma unroll 4
+#pragma unroll 8
         for (int h = hs; h < H; h += 8) {
-            const float d = x[base + (size_t)h * L] - c;
-            a1 += d;
-            a2 = fmaf(d, d, a2);
+            const float4 d = f4sub(*reinterpret_cast<const float4 *>(x + base + (size_t)h * L), c);
+            a1 = f4add(a1, d);
+            a2 = f4fma(d, d, a2);
         }
     }
     s1[hs][tl] = a1;
     s2[hs][tl] = a2;
     __syncthreads();
     if (hs == 0) {
-        float S1 = 0.0f, S2 = 0.0f;
+        float4 S1 = zero, S2 = zero;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            S1 += s1[i][tl];
-            S2 += s2[i][tl];
+            S1 = f4add(S1, s1[i][tl]);
+            S2 = f4add(S2, s2[i][tl]);
         }
-        const float m1 = S1 / (float)H;
-        const float var = fmaxf(S2 / (float)H - m1 * m1, 0.0f);
-        mu_s[tl] = c + m1;
-        rs_s[tl] = rsqrtf(var + eps);
+        const float inv = 1.0f / (float)H;
+        const float m[4] = {S1.x * inv, S1.y * inv, S1.z * inv, S1.w * inv};
+        const float q[4] = {S2.x * inv, S2.y * inv, S2.z * inv, S2.w * inv};
+        float r[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = rsqrtf(fmaxf(q[i] - m[i] * m[i], 0.0f) + eps);
+        mu_s[tl] = make_float4(c.x + m[0], c.y + m[1], c.z + m[2], c.w + m[3]);
+        rs_s[tl] = make_float4(r[0], r[1], r[2], r[3]);
     }
     __syncthreads();
     if (!in) return;
-    const float mu = mu_s[tl], rs = rs_s[tl];
-#pragma unroll 4
+    const float4 mu = mu_s[tl], rs = rs_s[tl];
+#pragma unroll 8
     for (int h = hs; h < H; h += 8) {
         const size_t o = base + (size_t)h * L;
-        z[o] = (x[o] - mu) * rs * __ldg(gamma + h) + __ldg(beta + h);
+        const float4 v = *reinterpret_cast<const float4 *>(x + o);
+        const float g = __ldg(gamma + h), bb = __ldg(beta + h);
+        *reinterpret_cast<float4 *>(z + o) = make_float4((v.x - mu.x) * rs.x * g + bb, (v.y - mu.y) * rs.y * g + bb,
+                                                          (v.z - mu.z) * rs.z * g + bb, (v.w - mu.w) * rs.w * g + bb);
     }
 }
 
 // ------------------------------------------------------- W -> operand images
-// Image (ob, c) holds rows 2i / 2i + 1 = W[64 ob + i] / W[H + 64 ob + i],
-// columns h = 32 c .. 32 c + 31, as bf16 high part (first kAImg bytes) and
-// low part (next kAImg bytes); rows and columns past H are zero. One thread
+// Image (c, nb): rows n of W' = W[128 nb + n/2] (n even) / W[H + 128 nb + n/2]
+// (n odd), columns h = 32 c .. 32 c + 31, K-major, bf16 high part (first
+// kWImg bytes) then low part; rows and columns past H are zero. Images are
+// stored chunk-major, (c, nb) at ((c * nnb) + nb) * 2 kWImg. One thread
 // writes 8 columns of one row.
 __global__ void k_glu_prepare(const float *__restrict__ W, int H, unsigned char *__restrict__ img) {
     using namespace glu;
-    const int nkc = glu_nkc(H);
-    const long long total = (long long)glu_nob(H) * nkc * kRows * (kKc / 8);
+    const int nnb = glu_nnb(H);
+    const long long total = (long long)glu_nkc(H) * nnb * kNr * (kKc / 8);
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= total) return;
     const int q = (int)(i % (kKc / 8));
-    const int r = (int)((i / (kKc / 8)) % kRows);
-    const long long oc = i / ((kKc / 8) * kRows);
-    const int c = (int)(oc % nkc), ob = (int)(oc / nkc);
-    const int o = ob * kOut + (r >> 1);
-    const size_t wrow = (size_t)((r & 1) ? H + o : o) * H;
+    const int n = (int)((i / (kKc / 8)) % kNr);
+    const long long cb = i / ((kKc / 8) * kNr);
+    const int nb = (int)(cb % nnb), c = (int)(cb / nnb);
+    const int o = nb * kCh + (n >> 1);
+    const size_t wrow = (size_t)((n & 1) ? H + o : o) * H;
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -146,180 +286,308 @@ __global__ void k_glu_prepare(const float *__restrict__ W, int H, unsigned char 
     }
     uint4 hi, lo;
     split8(v, hi, lo);
-    unsigned char *base = img + (size_t)oc * 2 * kAImg + kmajor_off(kRows, r, 8 * q);
+    unsigned char *base = img + (size_t)cb * 2 * kWImg + kmajor_off(kNr, n, 8 * q);
     *reinterpret_cast<uint4 *>(base) = hi;
-    *reinterpret_cast<uint4 *>(base + kAImg) = lo;
+    *reinterpret_cast<uint4 *>(base + kWImg) = lo;
 }
 
 // ------------------------------------------- projection + GLU + residual
 __global__ void __launch_bounds__(glu::kThreads, 1)
-k_glu_projection_tc(const float *__restrict__ y, const float *x, const float *__restrict__ bias,
-                    const unsigned char *__restrict__ img, int H, int L, int N, float *out,
-                    unsigned *__restrict__ flags) {
+k_glu_projection_ws(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_x,
+                    const float *__restrict__ bias, const unsigned char *__restrict__ wimg, int Bt, int H, int L,
+                    int N, float *__restrict__ out, unsigned *flags) {
     using namespace glu;
     extern __shared__ __align__(1024) unsigned char sm[];
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(sm + kStages * kStage);   // [2]
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 2);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBar);
+    uint64_t *rawfull = bars, *rawempty = rawfull + kR;
+    uint64_t *wfull = rawempty + kR, *yconv = wfull + kS, *opempty = yconv + kS;
+    uint64_t *accfull = opempty + kS, *accempty = accfull + 2, *xfull = accempty + 2, *xempty = xfull + kX;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(xempty + kX);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nob = glu_nob(H), nkc = glu_nkc(H), ntt = L / N;
-    int item = blockIdx.x;
-    const int ob = item % nob;
-    item /= nob;
-    const int tt = item % ntt, b = item / ntt;
-    const int t0 = tt * N;
+    const int nnb = glu_nnb(H), nkc = glu_nkc(H), ntt = L / N;
+    const long long ntiles = (long long)Bt * ntt * nnb;
+    Ctl ctl{abort_flag, flags};
 
     if (tid == 0) {
-        umma::mbar_init(&mbar[0], 1);
-        umma::mbar_init(&mbar[1], 1);
+        for (int i = 0; i < kR; ++i) {
+            umma::mbar_init(&rawfull[i], 1);
+            umma::mbar_init(&rawempty[i], 128);
+        }
+        for (int i = 0; i < kS; ++i) {
+            umma::mbar_init(&wfull[i], 1);
+            umma::mbar_init(&yconv[i], 128);
+            umma::mbar_init(&opempty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            umma::mbar_init(&accfull[i], 1);
+            umma::mbar_init(&accempty[i], kEpiThreads);
+        }
+        for (int i = 0; i < kX; ++i) {
+            umma::mbar_init(&xfull[i], 1);
+            umma::mbar_init(&xempty[i], kEpiThreads);
+        }
+        *abort_flag = 0;
         umma::fence_mbar_init();
     }
-    if (warp == 0) umma::tmem_alloc(tslot, kTmemCols);
+    if (warp == 5) umma::tmem_alloc(tslot, kTmemCols);
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = *tslot;
-    const uint32_t id = umma::idesc(1, kRows, N);
-    const uint32_t b_lbo = (uint32_t)(N / 8) * 128, a_lbo = (kRows / 8) * 128;
 
-    const float *yb = y + (size_t)b * H * L + t0;
-    const int tl = tid & (kNmax - 1), kg = tid >> 7;   // B-tile row (time step) and channel group
-    uint32_t ph = 0u;   // bit s: parity of the next completion of mbar[s]
-    bool ok = true;
-    for (int c = 0; c < nkc; ++c) {
-        const int s = c & 1;
-        unsigned char *stage = sm + s * kStage;
-        if (c >= 2) {   // the MMAs of chunk c - 2 read this stage: wait for them
-            const bool done = tid != 0 || umma::mbar_wait(&mbar[s], (ph >> s) & 1u, kSpinLimit);
-            ph ^= 1u << s;
-            ok = __syncthreads_and(done) != 0;
-            if (!ok) break;
-        }
-        // A: the prepared image of W for (ob, c), hi then lo, 16 bytes per copy
-        const unsigned char *src = img + ((size_t)ob * nkc + c) * 2 * kAImg;
-#pragma unroll
-        for (int i = 0; i < (2 * kAImg) / 16 / kThreads; ++i) {
-            const int j = tid + i * kThreads;
-            umma::cp_async16(stage + 16 * j, src + 16 * j);
-        }
-        umma::cp_async_commit();
-        // B: y[b, 32 c + 8 q + j, t0 + tl] for groups q = kg, kg + 2, split
-        if (tl < N) {
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const int q = kg + 2 * qq;
-                float v[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int h = c * kKc + 8 * q + j;
-                    v[j] = h < H ? __ldg(yb + (size_t)h * L + tl) : 0.0f;
+    if (warp == 0) {
+        // ---------------- loader: raw y chunks (TMA) and W' image chunks (bulk)
+        if (lane == 0) prefetch_tensormap(&tm_y);
+        Ring rr, ss;
+        int issued = 0;
+        bool ok = true;
+        for (long long i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
+            const Tile tl = tile_of(i, nnb, ntt, N);
+            for (int c = 0; c < nkc; ++c) {
+                if (!(ok = __all_sync(0xffffffffu, ctl.wait(&rawempty[rr.slot], rr.phase ^ 1u)))) break;
+                if (lane == 0) {
+                    arrive_expect_tx(&rawfull[rr.slot], (uint32_t)(N * kKc * 4));
+                    tma_load_3d(sm + kOffRaw + rr.slot * kRawBytes, &tm_y, tl.t0, c * kKc, tl.b, &rawfull[rr.slot]);
                 }
-                uint4 hi, lo;
-                split8(v, hi, lo);
-                unsigned char *bt = stage + 2 * kAImg + kmajor_off(N, tl, 8 * q);
-                *reinterpret_cast<uint4 *>(bt) = hi;
-                *reinterpret_cast<uint4 *>(bt + kBImg) = lo;
+                if (!(ok = __all_sync(0xffffffffu, ctl.wait(&opempty[ss.slot], ss.phase ^ 1u)))) break;
+                if (lane == 0) {
+                    arrive_expect_tx(&wfull[ss.slot], 2 * kWImg);
+                    bulk_load(sm + ss.slot * kStage + 2 * kYImg, wimg + ((size_t)c * nnb + tl.nb) * 2 * kWImg,
+                              2 * kWImg, &wfull[ss.slot]);
+                }
+                __syncwarp();
+                ++issued;
+                rr.next(kR);
+                ss.next(kS);
             }
         }
-        umma::cp_async_wait_all();
-        umma::fence_proxy_async();
-        umma::fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
+        if (!ok && lane == 0) {   // let the copies in flight land before the CTA exits
+            for (int k = 1; k <= kR && k <= issued; ++k) {
+                const int u = issued - k;
+                umma::mbar_wait(&rawfull[u % kR], (uint32_t)((u / kR) & 1), kSpinLimit);
+            }
+            for (int k = 1; k <= kS && k <= issued; ++k) {
+                const int u = issued - k;
+                umma::mbar_wait(&wfull[u % kS], (uint32_t)((u / kS) & 1), kSpinLimit);
+            }
+        }
+    } else if (warp <= 4) {
+        // ---------------- converters: raw fp32 y chunk -> bf16 hi / lo operand image
+        const int ct = tid - 32;   // time step within the tile (row of the operand)
+        Ring rr, ss;
+        bool ok = true;
+        for (long long i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
+            for (int c = 0; c < nkc; ++c) {
+                if (!(ok = __all_sync(0xffffffffu, ctl.wait(&rawfull[rr.slot], rr.phase)))) break;
+                if (!(ok = __all_sync(0xffffffffu, ctl.wait(&opempty[ss.slot], ss.phase ^ 1u)))) break;
+                if (ct < N) {
+                    const float *raw = reinterpret_cast<const float *>(sm + kOffRaw + rr.slot * kRawBytes);
+                    unsigned char *img = sm + ss.slot * kStage;
+#pragma unroll
+                    for (int q = 0; q < kKc / 8; ++q) {
+                        float v[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) v[j] = raw[(8 * q + j) * N + ct];
+                        uint4 hi, lo;
+                        split8(v, hi, lo);
+                        const int off = kmajor_off(kTm, ct, 8 * q);
+                        *reinterpret_cast<uint4 *>(img + off) = hi;
+                        *reinterpret_cast<uint4 *>(img + kYImg + off) = lo;
+                    }
+                }
+                umma::fence_proxy_async();   // the image, to the tensor cores
+                arrive(&rawempty[rr.slot]);
+                arrive(&yconv[ss.slot]);
+                rr.next(kR);
+                ss.next(kS);
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------- MMA issue (one thread), accumulator a of tile k = k % 2
+        const uint32_t id = umma::idesc(1, kTm, kNr);
+        constexpr uint32_t y_lbo = (kTm / 8) * 128, w_lbo = (kNr / 8) * 128;
+        Ring ss;
+        uint32_t tl = 0;
+        bool ok = true, any = false;
+        for (long long i = blockIdx.x; i < ntiles && ok; i += gridDim.x, ++tl) {
+            const int a = tl & 1;
+            if (!(ok = __all_sync(0xffffffffu, ctl.wait(&accempty[a], ((tl >> 1) & 1u) ^ 1u)))) break;
             umma::fence_after_sync();
-            const uint32_t Ah = umma::saddr(stage), Al = Ah + kAImg;
-            const uint32_t Bh = Ah + 2 * kAImg, Bl = Bh + kBImg;
-            const uint32_t As[3] = {Ah, Ah, Al}, Bs[3] = {Bh, Bl, Bh};
+            for (int c = 0; c < nkc; ++c) {
+                if (!(ok = __all_sync(0xffffffffu, ctl.wait(&wfull[ss.slot], ss.phase)))) break;
+                if (!(ok = __all_sync(0xffffffffu, ctl.wait(&yconv[ss.slot], ss.phase)))) break;
+                umma::fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t yh = umma::saddr(sm + ss.slot * kStage), yl = yh + kYImg;
+                    const uint32_t wh = yh + 2 * kYImg, wl = wh + kWImg;
+                    const uint32_t As[3] = {yh, yh, yl}, Bs[3] = {wh, wl, wh};
 #pragma unroll
-            for (int pr = 0; pr < 3; ++pr) {
+                    for (int kk = 0; kk < kKc / 16; ++kk)
 #pragma unroll
-                for (int kk = 0; kk < kKc / 16; ++kk) {
-                    const uint64_t da = umma::smem_desc(As[pr] + kk * 2 * a_lbo, a_lbo);
-                    const uint64_t db = umma::smem_desc(Bs[pr] + kk * 2 * b_lbo, b_lbo);
-                    umma::mma_bf16(tmem, da, db, id, c > 0 || pr > 0 || kk > 0);
+                        for (int pr = 0; pr < 3; ++pr)
+                            umma::mma_bf16(tmem + (uint32_t)(a * kNr),
+                                           umma::smem_desc(As[pr] + kk * 2 * y_lbo, y_lbo),
+                                           umma::smem_desc(Bs[pr] + kk * 2 * w_lbo, w_lbo), id,
+                                           c > 0 || kk > 0 || pr > 0);
+                    umma::commit(&opempty[ss.slot]);
                 }
+                __syncwarp();
+                any = true;
+                ss.next(kS);
             }
-            umma::commit(&mbar[s]);
+            if (!ok) break;
+            if (lane == 0) umma::commit(&accfull[a]);
+            __syncwarp();
         }
-    }
-    if (ok) {   // the last chunk's commit covers every MMA; also drain the other stage's
-        const int sl = (nkc - 1) & 1;
-        bool done = true;
-        if (tid == 0) {
-            done = umma::mbar_wait(&mbar[sl], (ph >> sl) & 1u, kSpinLimit);
-            if (done && nkc >= 2) done = umma::mbar_wait(&mbar[sl ^ 1], (ph >> (sl ^ 1)) & 1u, kSpinLimit);
+        if (!ok && any && lane == 0) {   // let the issued MMAs finish before tensor memory is freed
+            const int u = (ss.slot + kS - 1) % kS;
+            umma::mbar_wait(&opempty[u], ss.slot == 0 ? ss.phase ^ 1u : ss.phase, kSpinLimit);
         }
-        ok = __syncthreads_and(done) != 0;
-    }
-    if (!ok && tid == 0 && flags != nullptr) atomicOr(flags, S4_FLAG_TIMEOUT);
-    umma::fence_after_sync();
-
-    if (ok) {
-        // read back: warp w owns rows 32 (w % 4) + lane (row 2i value / 2i + 1
-        // gate of channel 64 ob + i) and the 16-column groups g = w / 4 (mod 2)
-        float *tile = reinterpret_cast<float *>(sm);   // [64][N + 1], over the stage buffers
-        const int q4 = warp & 3, row = 32 * q4 + lane, ol = row >> 1;
-        const bool gate_row = row & 1;
-        const int o = ob * kOut + ol;
-        const float bv = o < H ? __ldg(bias + o) : 0.0f, bg = o < H ? __ldg(bias + H + o) : 0.0f;
-        for (int g = warp >> 2; g < N / 16; g += 2) {
-            uint32_t v[16];
-            umma::ld_32x32b_x16(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(16 * g), v);
-            float r[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float mine = __uint_as_float(v[i]);
-                const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                const float val = gate_row ? other : mine, gt = gate_row ? mine : other;
-                r[i] = (val + bv) * sigmoidf_(gt + bg);
+    } else if (warp == 6) {
+        // ---------------- x loader: residual chunks (tile, e) in order, into the x ring
+        if (lane == 0) prefetch_tensormap(&tm_x);
+        float *xs = reinterpret_cast<float *>(sm + kOffX);
+        Ring xr;
+        int issued = 0;
+        bool ok = true;
+        for (long long i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
+            const Tile tc = tile_of(i, nnb, ntt, N);
+            const int nx = x_chunks(H, tc.nb);
+            for (int e = 0; e < nx; ++e) {
+                if (!(ok = __all_sync(0xffffffffu, ctl.wait(&xempty[xr.slot], xr.phase ^ 1u)))) break;
+                if (lane == 0) {
+                    arrive_expect_tx(&xfull[xr.slot], (uint32_t)(N * kXc * 4));
+                    tma_load_3d(xs + xr.slot * (kRawBytes / 4), &tm_x, tc.t0, tc.nb * kCh + e * kXc, tc.b,
+                                &xfull[xr.slot]);
+                }
+                __syncwarp();
+                ++issued;
+                xr.next(kX);
             }
-            // the value lane stores columns 0..7 of the group, the gate lane 8..15
-            const int i0 = gate_row ? 8 : 0;
+        }
+        if (!ok && lane == 0)   // let the copies in flight land before the CTA exits
+            for (int k = 1; k <= kX && k <= issued; ++k) {
+                const int u = issued - k;
+                umma::mbar_wait(&xfull[u % kX], (uint32_t)((u / kX) & 1), kSpinLimit);
+            }
+    } else {
+        // ---------------- epilogue: warps 7..14; warp w reads tensor-memory lanes
+        // 32 (w % 4) .. + 31 (time steps) and, of each 32-channel x chunk, the
+        // 8-channel groups gh, gh + 1 (gh = 0 for warps 7-10, 2 for 11-14)
+        const int q = warp & 3, t = 32 * q + lane;
+        const int gh = warp < kEpiWarp0 + 4 ? 0 : 2;
+        const float *xs = reinterpret_cast<const float *>(sm + kOffX);
+        Ring xr;
+        uint32_t tl = 0;
+        bool ok = true;
+        for (long long i = blockIdx.x; i < ntiles && ok; i += gridDim.x, ++tl) {
+            const Tile tc = tile_of(i, nnb, ntt, N);
+            const int a = tl & 1;
+            if (!(ok = named_and(1, kEpiThreads, ctl.wait(&accfull[a], (tl >> 1) & 1u)))) break;
+            umma::fence_after_sync();
+            const int nx = x_chunks(H, tc.nb);
+            const size_t row0 = ((size_t)tc.b * H) * L + tc.t0 + t;
+            for (int e = 0; e < nx; ++e) {
+                if (!(ok = named_and(1, kEpiThreads, ctl.wait(&xfull[xr.slot], xr.phase)))) break;
+                const float *xc = xs + xr.slot * (kRawBytes / 4);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) tile[ol * (N + 1) + 16 * g + i0 + i] = gate_row ? r[8 + i] : r[i];
+                for (int g = gh; g < gh + 2; ++g) {   // 16 columns = 8 channels
+                    uint32_t v[16];
+                    umma::ld_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * kNr + e * 2 * kXc + 16 * g),
+                                        v);
+                    const int o0 = tc.nb * kCh + e * kXc + 8 * g;
+                    float bv[8], bg[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        bv[j] = o0 + j < H ? __ldg(bias + o0 + j) : 0.0f;
+                        bg[j] = o0 + j < H ? __ldg(bias + H + o0 + j) : 0.0f;
+                    }
+                    if (t < N) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (o0 + j < H) {
+                                const float val = __uint_as_float(v[2 * j]) + bv[j];
+                                const float gt = __uint_as_float(v[2 * j + 1]) + bg[j];
+                                out[row0 + (size_t)(o0 + j) * L] = xc[(8 * g + j) * N + t] + val * sigmoidf_(gt);
+                            }
+                        }
+                    }
+                }
+                arrive(&xempty[xr.slot]);   // this thread is done with the x slot
+                xr.next(kX);
+            }
+            if (!ok) break;
+            umma::fence_before_sync();
+            arrive(&accempty[a]);
         }
     }
     umma::fence_before_sync();
     __syncthreads();
-    if (ok) {
-        const size_t ob_base = ((size_t)b * H + (size_t)ob * kOut) * L + t0;
-        const float *tile = reinterpret_cast<const float *>(sm);
-        for (int i = tid; i < kOut * N; i += kThreads) {
-            const int ol = i / N, t = i - ol * N;
-            if (ob * kOut + ol >= H) break;
-            const size_t gi = ob_base + (size_t)ol * L + t;
-            out[gi] = x[gi] + tile[ol * (N + 1) + t];   // out may be x: read, then written, by this thread
-        }
-    }
-    if (warp == 0) umma::tmem_dealloc(tmem, kTmemCols);
+    umma::fence_after_sync();
+    if (warp == 5) umma::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_layernorm_channels(const float *x, const float *gamma, const float *beta, float eps, int Bt,
                                       int H, int L, float *z, cudaStream_t st) {
-    dim3 grid((L + 31) / 32, Bt);
+    dim3 grid((L + 127) / 128, Bt);
     k_layernorm_channels<<<grid, 256, 0, st>>>(x, gamma, beta, eps, H, L, z);
     return cudaGetLastError();
 }
 
 cudaError_t launch_glu_prepare(const float *W, int H, void *ws, cudaStream_t st) {
-    const long long total = (long long)glu_nob(H) * glu_nkc(H) * glu::kRows * (glu::kKc / 8);
+    const long long total = (long long)glu_nkc(H) * glu_nnb(H) * glu::kNr * (glu::kKc / 8);
     k_glu_prepare<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(W, H, static_cast<unsigned char *>(ws));
     return cudaGetLastError();
 }
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+int g_glu_sms[64];
+
+// a [Bt, H, L] fp32 tensor as a 3-D TMA map with boxes [1][32][N]
+cudaError_t tensor_map_bhl(CUtensorMap *m, const float *p, int Bt, int H, int L, int N) {
+    std::call_once(g_encode_once, [] {
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", reinterpret_cast<void **>(&g_encode),
+                                    cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            g_encode = nullptr;
+    });
+    if (g_encode == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)Bt};
+    const cuuint64_t strides[2] = {(cuuint64_t)L * 4, (cuuint64_t)H * L * 4};
+    const cuuint32_t box[3] = {(cuuint32_t)N, (cuuint32_t)glu::kKc, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(p), dims, strides, box, es,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
+
 cudaError_t launch_glu_projection(const float *y, const float *x, const float *bias, const void *ws, int Bt, int H,
                                   int L, float *out, unsigned *flags, cudaStream_t st) {
-    static bool attr_set = false;   // per function; setting it twice is harmless
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_glu_projection_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)glu::kSmem);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int &sms = g_glu_sms[dev & 63];
+    if (sms == 0) {
+        e = cudaFuncSetAttribute(k_glu_projection_ws, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)glu::kSmem);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
-    const int N = L < glu::kNmax ? L : glu::kNmax;
-    const long long items = (long long)Bt * glu_nob(H) * (L / N);
-    k_glu_projection_tc<<<(unsigned)items, glu::kThreads, glu::kSmem, st>>>(
-        y, x, bias, static_cast<const unsigned char *>(ws), H, L, N, out, flags);
+    const int N = L < glu::kTm ? L : glu::kTm;
+    CUtensorMap my, mx;
+    e = tensor_map_bhl(&my, y, Bt, H, L, N);
+    if (e == cudaSuccess) e = tensor_map_bhl(&mx, x, Bt, H, L, N);
+    if (e != cudaSuccess) return e;
+    const long long tiles = (long long)Bt * (L / N) * glu_nnb(H);
+    const int grid = tiles < sms ? (int)tiles : sms;
+    k_glu_projection_ws<<<grid, glu::kThreads, glu::kSmem, st>>>(my, mx, bias, static_cast<const unsigned char *>(ws),
+                                                                  Bt, H, L, N, out, flags);
     return cudaGetLastError();
 }
 

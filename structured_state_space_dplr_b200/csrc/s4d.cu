@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "s4dplr.h"
+#include "umma.cuh"
 
 namespace s4 {
 
@@ -188,21 +189,11 @@ constexpr int kN = 64;    // kl columns (KB)
 constexpr int kK = 64;    // 2 x 32 modes per chunk
 constexpr int kThreads = 256;   // 8 warps: all build tables; warp w reads lanes 32 (w % 4).. back
 constexpr int kModes = kK / 2;
-constexpr uint32_t kIdesc = (1u << 4)                          // D: f32
-                          | (2u << 7) | (2u << 10)             // A, B: tf32
-                          | ((uint32_t)(kN >> 3) << 17)        // N
-                          | ((uint32_t)(kM >> 4) << 24);       // M (A and B K-major)
+constexpr uint32_t kIdesc = umma::idesc(2, kM, kN);   // tf32 operands, f32 accumulator
 constexpr uint32_t kSpinLimit = 1u << 24;
 
-__device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-// shared-memory matrix descriptor: K-major, no swizzle; element (row r, k)
-// of a tile with `rows` rows at byte (r%8)*16 + (r/8)*128 + (k/4)*lbo + (k%4)*4,
-// lbo = rows/8 * 128 (8-row core matrices of 16 bytes per row)
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo) {
-    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-           ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
-}
+// element (row r, k) of a K-major tf32 tile with `rows` rows (the layout of
+// umma.cuh: 8-row core matrices of 16 bytes per row), as a float index
 __device__ __forceinline__ int tile_index(int rows, int r, int k) {
     return ((r & 7) * 16 + (r >> 3) * 128 + (k >> 2) * (rows / 8) * 128 + (k & 3) * 4) >> 2;
 }
@@ -243,17 +234,13 @@ k_vandermonde_tc(const float2 *__restrict__ A, const float2 *__restrict__ B, con
     float *out = Ah;   // the finished tile leaves through the A_hi area (kM x kN floats)
     const int tid = threadIdx.x, warp = tid >> 5;
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(mbar)));
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        umma::mbar_init(mbar, 1);
+        umma::fence_mbar_init();
     }
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tslot)),
-                     "r"(kN));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    if (warp == 0) umma::tmem_alloc(tslot, kN);
+    umma::fence_before_sync();
     __syncthreads();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    umma::fence_after_sync();
     const uint32_t tmem = *tslot;
     uint32_t phase = 0;
     bool ok = true;
@@ -311,38 +298,26 @@ k_vandermonde_tc(const float2 *__restrict__ A, const float2 *__restrict__ B, con
                     g = zmul(g, a512);
                 }
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the tiles, to the tensor cores
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            umma::fence_proxy_async();   // the tiles, to the tensor cores
+            umma::fence_before_sync();
             __syncthreads();
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            umma::fence_after_sync();
             if (tid == 0) {
                 constexpr uint32_t a_lbo = (kM / 8) * 128, b_lbo = (kN / 8) * 128;
                 const float *As[3] = {Ah, Ah, Al}, *Bs[3] = {Bh, Bl, Bh};
+#pragma unroll
                 for (int pr = 0; pr < 3; ++pr) {
+#pragma unroll
                     for (int s = 0; s < kK / 8; ++s) {
-                        const uint64_t da = smem_desc(saddr(As[pr]) + s * 2 * a_lbo, a_lbo);
-                        const uint64_t db = smem_desc(saddr(Bs[pr]) + s * 2 * b_lbo, b_lbo);
-                        const uint32_t accumulate = (n0 > 0 || pr > 0 || s > 0) ? 1u : 0u;
-                        asm volatile(
-                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem),
-                            "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+                        const uint64_t da = umma::smem_desc(umma::saddr(As[pr]) + s * 2 * a_lbo, a_lbo);
+                        const uint64_t db = umma::smem_desc(umma::saddr(Bs[pr]) + s * 2 * b_lbo, b_lbo);
+                        umma::mma_tf32(tmem, da, db, kIdesc, n0 > 0 || pr > 0 || s > 0);
                     }
                 }
-                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                 saddr(mbar))
-                             : "memory");
+                umma::commit(mbar);
             }
             // the MMAs read the tiles: wait before the next chunk or the read-back
-            uint32_t done = 0;
-            for (uint32_t it = 0; it < kSpinLimit && !done; ++it) {
-                asm volatile(
-                    "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                    "selp.u32 %0, 1, 0, p;\n\t}\n"
-                    : "=r"(done)
-                    : "r"(saddr(mbar)), "r"(phase)
-                    : "memory");
-            }
+            const bool done = umma::mbar_wait(mbar, phase, kSpinLimit);
             phase ^= 1u;
             ok = __syncthreads_and(done) != 0;   // one decision for the whole CTA
             if (!ok) {   // never expected: report and stop, freeing tensor memory below
@@ -351,7 +326,7 @@ k_vandermonde_tc(const float2 *__restrict__ A, const float2 *__restrict__ B, con
             }
         }
         if (!ok) break;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        umma::fence_after_sync();
         // ---- read back: warp w holds rows 32 (w % 4) + lane, columns 32 (w / 4) .. + 31;
         // 2x; out through shared memory
         __syncthreads();   // every thread has passed the wait: the tiles may be overwritten
@@ -359,14 +334,7 @@ k_vandermonde_tc(const float2 *__restrict__ A, const float2 *__restrict__ B, con
         const int row = 32 * (warp & 3) + (tid & 31), col0 = 32 * (warp >> 2);
         for (int c0 = col0; c0 < col0 + 32; c0 += 16) {
             uint32_t v[16];
-            const uint32_t addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0;
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-                "[%16];"
-                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-                : "r"(addr));
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            umma::ld_32x32b_x16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0, v);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float k = 2.0f * __uint_as_float(v[i]);
@@ -374,15 +342,15 @@ k_vandermonde_tc(const float2 *__restrict__ A, const float2 *__restrict__ B, con
                 out[row * (kN + 1) + c0 + i] = k;   // padded rows: conflict-free columns
             }
         }
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        umma::fence_before_sync();
         __syncthreads();
         float *Kt = K + (size_t)h * L + (size_t)kh0 * kN;
         for (int i = tid; i < kM * kN; i += kThreads) Kt[i] = out[(i / kN) * (kN + 1) + i % kN];
         if (flags != nullptr && __any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(flags, S4_FLAG_NONFINITE);
     }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    umma::fence_before_sync();
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kN));
+    if (warp == 0) umma::tmem_dealloc(tmem, kN);
 }
 
 __global__ void k_s4d_zoh(const float2 *__restrict__ A, const float2 *__restrict__ B,

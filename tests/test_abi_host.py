@@ -150,9 +150,9 @@ def test_block_entries_reject_bad_arguments(lib):
     assert lib.s4_glu_projection_workspace_size(0, ctypes.byref(n)) == _lib.S4_ERR_INVALID_ARG
     assert lib.s4_glu_projection_workspace_size(8193, ctypes.byref(n)) == _lib.S4_ERR_INVALID_ARG
     assert lib.s4_glu_projection_workspace_size(256, ctypes.byref(n)) == _lib.S4_OK
-    assert n.value == 4 * 8 * 2 * 8192          # (H/64 row blocks) x (H/32 chunks) x hi/lo x 8 KB
+    assert n.value == 8 * 2 * 2 * 16384         # (H/32 chunks) x (H/128 row blocks) x hi/lo x 16 KB
     assert lib.s4_glu_projection_workspace_size(100, ctypes.byref(n)) == _lib.S4_OK
-    assert n.value == 2 * 4 * 2 * 8192          # ragged H rounds both counts up
+    assert n.value == 4 * 1 * 2 * 16384         # ragged H rounds both counts up
     x, z, g, b = p(FAKE), p(FAKE + 0x10000000), p(FAKE2), p(FAKE2 + 0x1000)
     ln = lib.s4_layernorm_channels
     assert ln(p(0), g, b, 1e-5, 2, 4, 64, z, p(0)) == _lib.S4_ERR_INVALID_ARG
