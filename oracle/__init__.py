@@ -8,7 +8,8 @@ and stored parameter data, no arithmetic of the method).
 
 Contents:
   hippo      HiPPO-LegS -> NPLR -> DPLR ("The S4 kernel, from scratch", §2)
-  ssm        discretisation, generating function, the pages' Cauchy/Woodbury
+  ssm        discretisation (bilinear; ZOH diagonal and dense), generating
+             function, the pages' Cauchy/Woodbury
              formula, aliased kernel by dense powers, direct causal
              convolution, recurrence, S4D kernel (§1, §3-§5; "S4" wiki, S4D)
   block      the S4Block around the layer: channel layer norm, GLU-gated

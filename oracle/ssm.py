@@ -22,6 +22,7 @@ Readings of points the pages leave open (listed in the design notes):
 from __future__ import annotations
 
 import numpy as np
+import scipy.linalg
 
 from . import _cloops
 
@@ -70,6 +71,22 @@ def zoh_diag(a, B, dt):
     big = ~small
     ratio[big] = (Ab[big] - 1.0) / a[big]
     return Ab, ratio * np.asarray(B, np.complex128)
+
+
+def zoh_dense(A, B, dt):
+    """Zero-order hold for a dense (non-diagonal) system, the rule of "The S4
+    kernel, from scratch", §3 applied to the full DPLR matrix:
+    Abar = exp(dt A), Bbar = (integral_0^dt exp(A s) ds) B. Both come from one
+    matrix exponential (scipy.linalg.expm) of the augmented matrix
+    [[dt A, dt B], [0, 0]]: its top-left block is Abar and its top-right column
+    is Bbar. No inverse of A is needed, so a singular A is fine."""
+    A = np.atleast_2d(np.asarray(A, np.complex128))
+    N = A.shape[0]
+    X = np.zeros((N + 1, N + 1), np.complex128)
+    X[:N, :N] = dt * A
+    X[:N, N] = dt * np.asarray(B, np.complex128).reshape(N)
+    E = scipy.linalg.expm(X)
+    return E[:N, :N], E[:N, N]
 
 
 # ------------------------------------------------------- generating function --

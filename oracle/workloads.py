@@ -30,6 +30,30 @@ def dplr_discretized(inp, h):
     return Ab, Bb, Cf
 
 
+def dplr_zoh_discretized(inp, h):
+    """Zero-order-hold (Abar, Bbar, Cbar = C_f) of channel h's full DPLR
+    system ("The S4 kernel, from scratch", §3, ZOH rule on the dense A)."""
+    A, Bf, Cf, dt = dplr_channel_system(inp, h)
+    Ab, Bb = ssm.zoh_dense(A, Bf, dt)
+    return Ab, Bb, Cf
+
+
+def dplr_zoh_kernel(inp, channels=None, imag_tol=1e-10):
+    """Truncated ZOH DPLR kernel K[h, k] = Re(C_f Abar^k Bbar), k < L, by dense
+    powers (no aliasing: the generating-function shortcut is bilinear only)."""
+    L = inp["L"]
+    channels = range(inp["H"]) if channels is None else channels
+    out = []
+    for h in channels:
+        Ab, Bb, Cf = dplr_zoh_discretized(inp, h)
+        K = ssm.truncated_kernel(Ab, Bb, Cf, L)
+        kmax = np.max(np.abs(K.real))
+        if np.max(np.abs(K.imag)) > imag_tol * max(kmax, 1e-300):
+            raise AssertionError(f"channel {h}: kernel not real (|Im K| = {np.max(np.abs(K.imag))})")
+        out.append(K.real)
+    return np.array(out)
+
+
 def dplr_kernel(inp, channels=None, method="closed", imag_tol=1e-10):
     """Aliased bilinear DPLR kernel K[h, 0..L-1] (fp64, real) for the given
     channels, by dense powers ("closed": one period from (I - Abar^L)^-1 Bbar;
