@@ -303,6 +303,38 @@ s4_status s4_fft_conv_static(const float *u, const float *K, const float *D,
                              int Bt, int H, int L, float *y, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Zero-order hold of the DPLR system ([S4K] §3: the ZOH rule, applied here to
+ * the dense matrix of the full conjugate-closed system A = diag(Lambda_f) -
+ * P_f Q_f^*, N = 2 Nh):
+ *     Abar = exp(dt A),  Bbar = (integral_0^dt exp(A s) ds) B_f,  Cbar = C_f.
+ * The generating-function shortcut of [S4K] §4 is specific to the bilinear
+ * rule, so under ZOH the kernel is formed from dense powers:
+ *     K[h, k] = Re(C_f Abar^k Bbar),  k = 0 .. L-1  (TRUNCATED: no aliasing).
+ * Computed per channel in fp64 (scaling and squaring of the augmented
+ * exponential, Taylor degree 16), results rounded to fp32.
+ *
+ * s4_dplr_discretize_zoh: Abar [H, N, N], Bbar [H, N], Cfull [H, N] out --
+ *   the layout of s4_dplr_discretize, so the dense recurrent step
+ *   (S4_STEP_DENSE) runs the ZOH system unchanged.
+ * s4_kernel_dplr_zoh: K [H, L] out (16-byte aligned); d_flags (nullable):
+ *   S4_FLAG_UNSTABLE if some Re(Lambda) >= 0, S4_FLAG_NONFINITE if a kernel
+ *   value is not finite. K then feeds s4_fft_conv_prepare like any kernel.
+ * Both: Lambda, P, Q, B, C [H, Nh] complex, log_dt [H]; 1 <= Nh <= 32
+ * (larger -> S4_ERR_UNSUPPORTED); L a power of two in [16, 65536]. Errors as
+ * s4_dplr_discretize / s4_kernel_dplr.
+ * ------------------------------------------------------------------------ */
+#define S4_MAX_ZOH_NH 32
+
+s4_status s4_dplr_discretize_zoh(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                                 const s4_c32 *B, const s4_c32 *C, const float *log_dt, int H,
+                                 int Nh, s4_c32 *Abar, s4_c32 *Bbar, s4_c32 *Cfull,
+                                 cudaStream_t stream);
+
+s4_status s4_kernel_dplr_zoh(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                             const s4_c32 *B, const s4_c32 *C, const float *log_dt, int H,
+                             int Nh, int L, float *K, unsigned *d_flags, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * The S4Block around the layer ([S4K] §6 "Trainable layer": a pre-norm, a
  * GLU-gated projection and a residual connection). All tensors [Bt, H, L]
  * float, device, 16-byte aligned, time (L) contiguous -- the layout of u and

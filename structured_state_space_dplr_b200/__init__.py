@@ -20,7 +20,7 @@ from ._lib import (S4_FLAG_NONFINITE, S4_FLAG_UNSTABLE, S4_STEP_DENSE, S4_STEP_D
                    S4Error)
 
 __all__ = [
-    "kernel_dplr", "kernel_dplr_prepare", "layernorm_channels", "glu_projection_workspace_size", "glu_projection_prepare", "glu_projection_residual", "block_forward", "forward_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
+    "kernel_dplr", "kernel_dplr_prepare", "kernel_dplr_zoh", "dplr_discretize_zoh", "layernorm_channels", "glu_projection_workspace_size", "glu_projection_prepare", "glu_projection_residual", "block_forward", "forward_dplr", "dplr_spectrum", "irfft_packed", "fft_conv", "fft_conv_workspace_size", "fft_conv_prepare", "fft_conv_apply",
     "fft_conv_static",
     "s4d_kernel_vandermonde", "dplr_discretize", "s4d_discretize_zoh", "recurrent_step",
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
@@ -444,6 +444,37 @@ def dplr_discretize(Lambda, P, Q, B, C, log_dt):
     _lib.call("s4_dplr_discretize", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
               H, Nh, _ptr(Ab), _ptr(Bb), _ptr(Cf), _stream())
     return Ab, Bb, Cf
+
+
+def dplr_discretize_zoh(Lambda, P, Q, B, C, log_dt):
+    """Zero-order hold of the full DPLR system (s4_dplr_discretize_zoh):
+    (Abar = exp(dt A) [H,N,N], Bbar [H,N], Cfull [H,N]) complex64, N = 2 Nh,
+    Nh <= 32; the dense recurrent step runs it unchanged."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    N = 2 * Nh
+    dev = Lambda.device
+    Ab = torch.empty(H, N, N, dtype=torch.complex64, device=dev)
+    Bb = torch.empty(H, N, dtype=torch.complex64, device=dev)
+    Cf = torch.empty(H, N, dtype=torch.complex64, device=dev)
+    _lib.call("s4_dplr_discretize_zoh", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              H, Nh, _ptr(Ab), _ptr(Bb), _ptr(Cf), _stream())
+    return Ab, Bb, Cf
+
+
+def kernel_dplr_zoh(Lambda, P, Q, B, C, log_dt, L, *, out=None, flags=None):
+    """Truncated kernel of the ZOH-discretised DPLR system K [H, L]
+    (s4_kernel_dplr_zoh), Nh <= 32."""
+    Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    H, Nh = Lambda.shape
+    if out is None:
+        out = torch.empty(H, L, device=Lambda.device, dtype=torch.float32)
+    _cuda(out, "out", torch.float32)
+    _lib.call("s4_kernel_dplr_zoh", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+              H, Nh, int(L), _ptr(out), _flags_ptr(flags), _stream())
+    return out
 
 
 def dplr_discretize_structured(Lambda, P, Q, B, log_dt):

@@ -559,4 +559,33 @@ s4_status s4_block_forward(const float *x, const float *gamma, const float *beta
     return cuda_status(e);
 }
 
+// ------------------------------------------------------- ZOH of the DPLR system
+s4_status s4_dplr_discretize_zoh(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B,
+                                 const s4_c32 *C, const float *log_dt, int H, int Nh, s4_c32 *Abar, s4_c32 *Bbar,
+                                 s4_c32 *Cfull, cudaStream_t stream) {
+    if (any_null(Lambda, P, Q, B, C) || any_null(Abar, Bbar, Cfull) || log_dt == nullptr)
+        return S4_ERR_INVALID_ARG;
+    s4_status s = check_modes(H, Nh, 0, false);
+    if (s != S4_OK) return s;
+    if (Nh > S4_MAX_ZOH_NH) return S4_ERR_UNSUPPORTED;
+    if (!params_aligned({Lambda, P, Q, B, C, Abar, Bbar, Cfull}) || !aligned(log_dt, 4)) return S4_ERR_INVALID_ARG;
+    const size_t N = 2 * (size_t)Nh, ab = (size_t)H * N * N * sizeof(s4_c32), vb = (size_t)H * N * sizeof(s4_c32);
+    if (overlap(Abar, ab, Bbar, vb) || overlap(Abar, ab, Cfull, vb) || overlap(Bbar, vb, Cfull, vb))
+        return S4_ERR_INVALID_ARG;
+    return cuda_status(s4::launch_dplr_zoh((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q,
+                                           (const float2 *)B, (const float2 *)C, log_dt, H, Nh, 0, (float2 *)Abar,
+                                           (float2 *)Bbar, (float2 *)Cfull, nullptr, nullptr, stream));
+}
+
+s4_status s4_kernel_dplr_zoh(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B,
+                             const s4_c32 *C, const float *log_dt, int H, int Nh, int L, float *K,
+                             unsigned *d_flags, cudaStream_t stream) {
+    s4_status s = dplr_checks(Lambda, P, Q, B, C, log_dt, H, Nh, L, K);
+    if (s != S4_OK) return s;
+    if (Nh > S4_MAX_ZOH_NH) return S4_ERR_UNSUPPORTED;
+    return cuda_status(s4::launch_dplr_zoh((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q,
+                                           (const float2 *)B, (const float2 *)C, log_dt, H, Nh, L, nullptr, nullptr,
+                                           nullptr, K, d_flags, stream));
+}
+
 }  // extern "C"

@@ -198,23 +198,28 @@ struct Ring {
 }  // namespace
 
 // ---------------------------------------------------------------- layer norm
-// One CTA: 128 consecutive time steps of one batch row, 4 per thread (16-byte
-// accesses); warp w sums channels w, w + 8, ... with 8 loads in flight. The
-// sums are taken about x[b, 0, t] (shifted data: no cancellation for large
-// means). The second pass re-reads the CTA's slab, which is still in L2.
-// z may be x (in place): every element is read and then written by one thread.
+// One CTA: 64 consecutive time steps of one batch row, 4 per thread (16-byte
+// accesses): thread (s, l) = (tid / 16, tid % 16) sums channels s, s + 16, ...
+// at steps 4 l .. 4 l + 3, with 8 loads in flight; a warp reads two 256-byte
+// channel rows per instruction. The sums are taken about x[b, 0, t] (shifted
+// data: no cancellation for large means). The second pass re-reads the CTA's
+// slab, which is still in L2. z may be x (in place): every element is read
+// and then written by one thread.
 __device__ __forceinline__ float4 f4sub(float4 a, float4 b) { return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w); }
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
 __device__ __forceinline__ float4 f4fma(float4 a, float4 b, float4 c) {
     return make_float4(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y), fmaf(a.z, b.z, c.z), fmaf(a.w, b.w, c.w));
 }
 
+constexpr int kLnSteps = 64, kLnSlices = 16;
+
 __global__ void __launch_bounds__(256) k_layernorm_channels(const float *x, const float *__restrict__ gamma,
                                                             const float *__restrict__ beta, float eps, int H,
                                                             int L, float *z) {
-    __shared__ float4 s1[8][32], s2[8][32], mu_s[32], rs_s[32];
-    const int tl = threadIdx.x & 31, hs = threadIdx.x >> 5;
-    const int t = blockIdx.x * 128 + 4 * tl;
+    __shared__ float4 s1[kLnSlices][kLnSteps / 4], s2[kLnSlices][kLnSteps / 4], mu_s[kLnSteps / 4],
+        rs_s[kLnSteps / 4];
+    const int tl = threadIdx.x % (kLnSteps / 4), hs = threadIdx.x / (kLnSteps / 4);
+    const int t = blockIdx.x * kLnSteps + 4 * tl;
     const bool in = t < L;   // L is a multiple of 16: t < L implies t + 3 < L
     const size_t base = (size_t)blockIdx.y * H * L + t;
     const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(256) k_layernorm_channels(const float *x, cons
     float4 a1 = zero, a2 = zero;
     if (in) {
 #pragma unroll 8
-        for (int h = hs; h < H; h += 8) {
+        for (int h = hs; h < H; h += kLnSlices) {
             const float4 d = f4sub(*reinterpret_cast<const float4 *>(x + base + (size_t)h * L), c);
             a1 = f4add(a1, d);
             a2 = f4fma(d, d, a2);
@@ -234,7 +239,7 @@ __global__ void __launch_bounds__(256) k_layernorm_channels(const float *x, cons
     if (hs == 0) {
         float4 S1 = zero, S2 = zero;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kLnSlices; ++i) {
             S1 = f4add(S1, s1[i][tl]);
             S2 = f4add(S2, s2[i][tl]);
         }
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(256) k_layernorm_channels(const float *x, cons
     if (!in) return;
     const float4 mu = mu_s[tl], rs = rs_s[tl];
 #pragma unroll 8
-    for (int h = hs; h < H; h += 8) {
+    for (int h = hs; h < H; h += kLnSlices) {
         const size_t o = base + (size_t)h * L;
         const float4 v = *reinterpret_cast<const float4 *>(x + o);
         const float g = __ldg(gamma + h), bb = __ldg(beta + h);
@@ -531,7 +536,7 @@ k_glu_projection_ws(const __grid_constant__ CUtensorMap tm_y, const __grid_const
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_layernorm_channels(const float *x, const float *gamma, const float *beta, float eps, int Bt,
                                       int H, int L, float *z, cudaStream_t st) {
-    dim3 grid((L + 127) / 128, Bt);
+    dim3 grid((L + kLnSteps - 1) / kLnSteps, Bt);
     k_layernorm_channels<<<grid, 256, 0, st>>>(x, gamma, beta, eps, H, L, z);
     return cudaGetLastError();
 }

@@ -57,6 +57,13 @@ cudaError_t launch_glu_prepare(const float *W, int H, void *ws, cudaStream_t st)
 cudaError_t launch_glu_projection(const float *y, const float *x, const float *bias, const void *ws, int Bt, int H,
                                   int L, float *out, unsigned *flags, cudaStream_t st);
 
+// ---- zoh_dplr.cu: zero-order hold of the full DPLR system (Nh <= 32) ----
+// K == nullptr: write Abar [H, N, N], Bbar [H, N], Cfull [H, N]; else the
+// truncated kernel K [H, L]
+cudaError_t launch_dplr_zoh(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
+                            const float2 *C, const float *log_dt, int H, int Nh, int L, float2 *Abar,
+                            float2 *Bbar, float2 *Cfull, float *K, unsigned *flags, cudaStream_t st);
+
 // ---- decode.cu ----
 cudaError_t launch_dplr_discretize(const float2 *Lambda, const float2 *P, const float2 *Q,
                                    const float2 *B, const float2 *C, const float *log_dt, int H, int Nh,

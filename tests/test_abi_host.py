@@ -180,6 +180,22 @@ def test_block_entries_reject_bad_arguments(lib):
     assert bf(x, g, b, 1e-5, cws, 16, bias, ws, wsb, 2, 256, 4096, z, y, out, p(0), p(0)) == _lib.S4_ERR_WORKSPACE
 
 
+def test_zoh_entries_reject_bad_arguments(lib):
+    five = [p(FAKE + 0x10000 * i) for i in range(5)]
+    ldt = p(FAKE + 0x60000)
+    out = [p(FAKE2), p(FAKE2 + 0x100000), p(FAKE2 + 0x200000)]
+    dz = lib.s4_dplr_discretize_zoh
+    assert dz(*five, ldt, 4, 33, *out, p(0)) == _lib.S4_ERR_UNSUPPORTED          # Nh > 32
+    assert dz(*five, ldt, 4, 0, *out, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert dz(p(0), *five[1:], ldt, 4, 32, *out, p(0)) == _lib.S4_ERR_INVALID_ARG
+    assert dz(*five, ldt, 4, 32, out[0], out[0], out[2], p(0)) == _lib.S4_ERR_INVALID_ARG   # Abar overlaps Bbar
+    kz = lib.s4_kernel_dplr_zoh
+    assert kz(*five, ldt, 4, 33, 1024, p(FAKE2), p(0), p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert kz(*five, ldt, 4, 32, 1000, p(FAKE2), p(0), p(0)) == _lib.S4_ERR_UNSUPPORTED
+    assert kz(*five, ldt, 4, 32, 1024, p(FAKE2 + 8), p(0), p(0)) == _lib.S4_ERR_INVALID_ARG   # K misaligned
+    assert kz(*five, ldt, 4, 32, 1024, p(0), p(0), p(0)) == _lib.S4_ERR_INVALID_ARG
+
+
 def test_binding_refuses_cpu_tensors():
     torch = pytest.importorskip("torch")
     import structured_state_space_dplr_b200 as s4
