@@ -166,13 +166,17 @@ s4_status s4_fft_conv_apply(const float *u, const void *workspace,
  *   Arguments and errors as s4_fft_conv_apply (dy in place of u, du of y).
  *
  * s4_fft_conv_kernel_grad: dK = dL/dK [H, L] and dD = dL/dD [H],
- *     dK[h,k] = sum_b sum_{t>=k} dy[b,h,t] u[b,h,t-k],   dD[h] = dK[h,0],
- *   for L <= 8192 (longer L -> S4_ERR_UNSUPPORTED). u, dy [Bt, H, L] device,
- *   16-byte aligned; dK [H, L] out, 16-byte aligned; dD [H] out, nullable.
- *   Workspace: s4_fft_conv_kernel_grad_workspace_size bytes (= 2 H 2L 8:
- *   a per-channel accumulator of the spectrum products and a per-channel
- *   scratch), 256-byte aligned, caller-owned, contents irrelevant on entry.
- *   Per channel the row pairs are summed in a fixed order (deterministic).
+ *     dK[h,k] = sum_b sum_{t>=k} dy[b,h,t] u[b,h,t-k],   dD[h] = dK[h,0].
+ *   u, dy [Bt, H, L] device, 16-byte aligned; dK [H, L] out, 16-byte
+ *   aligned; dD [H] out, nullable. Workspace:
+ *   s4_fft_conv_kernel_grad_workspace_size bytes, 256-byte aligned,
+ *   caller-owned, contents irrelevant on entry. L <= 8192: 2 H 2L 8 bytes (a
+ *   per-channel accumulator of the spectrum products and a per-channel
+ *   scratch; one launch). L > 8192: the convolution workspace of (H, L) plus
+ *   H L 4 bytes; per batch row b the spectrum of the zero-padded u[b] is
+ *   prepared as if it were the kernel and the adjoint convolution of dy[b]
+ *   gives that row's share of dK (2-3 launches per row). Either way the rows
+ *   are summed in a fixed order (deterministic).
  *   Errors: null pointers, Bt/H < 1, misalignment, overlapping buffers ->
  *   S4_ERR_INVALID_ARG; workspace too small or misaligned ->
  *   S4_ERR_WORKSPACE.
@@ -197,7 +201,7 @@ s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H
  * through DFT(dK) at the same roots of unity and the derivatives of the
  * four Cauchy sums, the Woodbury correction and the bilinear factor
  * (squared-denominator Cauchy sums for Lambda and dt), and the closed form at
- * the Nyquist bin. L <= 8192 (longer -> S4_ERR_UNSUPPORTED).
+ * the Nyquist bin. L <= 16384 (longer -> S4_ERR_UNSUPPORTED).
  *   Lambda, P, Q, B, C : [H, Nh] complex;  log_dt : [H];  dK : [H, L].
  *   dLambda, dP, dQ, dB, dC : [H, Nh] complex out;  dlog_dt : [H] out.
  * Errors: null pointers, misaligned complex arrays, outputs overlapping

@@ -105,7 +105,7 @@ def irfft_packed(K):
 
 
 def fft_conv_kernel_grad_workspace_size(H, L) -> int:
-    """Bytes of workspace fft_conv_kernel_grad needs (L <= 8192)."""
+    """Bytes of workspace fft_conv_kernel_grad needs."""
     n = ctypes.c_size_t()
     _lib.call("s4_fft_conv_kernel_grad_workspace_size", int(H), int(L), ctypes.byref(n))
     return n.value
@@ -280,7 +280,7 @@ def fft_conv_apply_adjoint(dy, workspace, *, out=None):
 
 def fft_conv_kernel_grad(u, dy, *, dK=None, dD=None, workspace=None):
     """Backward of the convolution in K and D (s4_fft_conv_kernel_grad):
-    (dK [H, L], dD [H]) for the batch u, dy [Bt, H, L]; L <= 8192."""
+    (dK [H, L], dD [H]) for the batch u, dy [Bt, H, L]."""
     u = _cuda(u, "u", torch.float32)
     dy = _cuda(dy, "dy", torch.float32)
     Bt, H, L = u.shape

@@ -253,7 +253,7 @@ s4_status s4_fft_conv_apply_adjoint(const float *dy, const void *workspace, int 
 
 s4_status s4_fft_conv_kernel_grad_workspace_size(int H, int L, size_t *bytes) {
     if (bytes == nullptr || H < 1) return S4_ERR_INVALID_ARG;
-    if (!pow2_L(L) || L > 8192) return S4_ERR_UNSUPPORTED;
+    if (!pow2_L(L)) return S4_ERR_UNSUPPORTED;
     *bytes = s4::corr_workspace_bytes(H, L);
     return S4_OK;
 }
@@ -262,7 +262,7 @@ s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H
                                   void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     if (any_null(u, dy, dK) || workspace == nullptr) return S4_ERR_INVALID_ARG;
     if (Bt < 1 || H < 1) return S4_ERR_INVALID_ARG;
-    if (!pow2_L(L) || L > 8192) return S4_ERR_UNSUPPORTED;
+    if (!pow2_L(L)) return S4_ERR_UNSUPPORTED;
     if ((double)Bt * (double)H * (double)L >= 1099511627776.0) return S4_ERR_INVALID_ARG;   // 2^40
     if (!aligned(u, 16) || !aligned(dy, 16) || !aligned(dK, 16) || (dD != nullptr && !aligned(dD, 4)))
         return S4_ERR_INVALID_ARG;
@@ -287,7 +287,7 @@ s4_status s4_kernel_dplr_backward(const s4_c32 *Lambda, const s4_c32 *P, const s
         return S4_ERR_INVALID_ARG;
     s4_status s = check_modes(H, Nh, L, true);
     if (s != S4_OK) return s;
-    if (L > 8192) return S4_ERR_UNSUPPORTED;
+    if (L > 16384) return S4_ERR_UNSUPPORTED;
     if (!params_aligned({Lambda, P, Q, B, C, dLambda, dP, dQ, dB, dC}) || !aligned(dK, 4)) return S4_ERR_INVALID_ARG;
     const size_t pb = (size_t)H * Nh * sizeof(s4_c32);
     const void *outs[] = {dLambda, dP, dQ, dB, dC};

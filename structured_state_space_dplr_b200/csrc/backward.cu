@@ -430,12 +430,61 @@ cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const fl
         case 2048: return S4_KBWD(11);
         case 4096: return S4_KBWD(12);
         case 8192: return S4_KBWD(13);
+        case 16384: return S4_KBWD(14);
         default: return cudaErrorInvalidValue;
     }
 #undef S4_KBWD
 }
 
+namespace {
+size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// dK += r (float4; n a multiple of 4)
+__global__ void k_accumulate(float *__restrict__ dK, const float *__restrict__ r, size_t n4) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        float4 a = reinterpret_cast<float4 *>(dK)[i];
+        const float4 b = reinterpret_cast<const float4 *>(r)[i];
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+        reinterpret_cast<float4 *>(dK)[i] = a;
+    }
+}
+// dD[h] = dK[h, 0]
+__global__ void k_lag0(const float *__restrict__ dK, int H, int L, float *__restrict__ dD) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h < H) dD[h] = dK[(size_t)h * L];
+}
+
+// L > 8192: per batch row b, the spectrum of the zero-padded u[b] rows is
+// prepared as if they were the kernel, and the adjoint convolution applied to
+// dy[b] gives sum_{t >= s} u[b, h, t - s] dy[b, h, t] = the row's share of
+// dK[h, s]; the shares are added in batch order.
+cudaError_t run_corr_long(const float *u, const float *dy, int Bt, int H, int L, float *dK, float *dD, void *ws,
+                          cudaStream_t st) {
+    void *spec = ws;
+    float *r = reinterpret_cast<float *>(static_cast<char *>(ws) + align256(conv_workspace_bytes(H, L)));
+    const size_t row = (size_t)H * L;
+    cudaError_t e = cudaSuccess;
+    for (int b = 0; b < Bt && e == cudaSuccess; ++b) {
+        e = launch_kspec(u + b * row, nullptr, H, L, spec, st);
+        if (e == cudaSuccess) e = launch_fftconv(dy + b * row, spec, 1, H, L, b == 0 ? dK : r, st, true);
+        if (e == cudaSuccess && b > 0) {
+            k_accumulate<<<1184, 256, 0, st>>>(dK, r, row / 4);
+            e = cudaGetLastError();
+        }
+    }
+    if (e == cudaSuccess && dD != nullptr) {
+        k_lag0<<<(H + 255) / 256, 256, 0, st>>>(dK, H, L, dD);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+}  // namespace
+
 size_t corr_workspace_bytes(int H, int L) {
+    if (L > 8192) return align256(conv_workspace_bytes(H, L)) + align256((size_t)H * L * sizeof(float));
     return 2 * (((size_t)H * 2 * L * sizeof(float2) + 255) & ~size_t(255));
 }
 
@@ -452,7 +501,7 @@ cudaError_t launch_corr(const float *u, const float *dy, int Bt, int H, int L, f
         case 2048: return run_corr<11>(u, dy, Bt, H, dK, dD, ws, st);
         case 4096: return run_corr<12>(u, dy, Bt, H, dK, dD, ws, st);
         case 8192: return run_corr<13>(u, dy, Bt, H, dK, dD, ws, st);
-        default: return cudaErrorInvalidValue;
+        default: return run_corr_long(u, dy, Bt, H, L, dK, dD, ws, st);
     }
 }
 

@@ -133,7 +133,9 @@ def test_vandermonde_and_discretize_reject_bad_arguments(lib):
 
 def test_backward_entries_reject_bad_arguments(lib):
     n = ctypes.c_size_t()
-    assert lib.s4_fft_conv_kernel_grad_workspace_size(4, 16384, ctypes.byref(n)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_fft_conv_kernel_grad_workspace_size(4, 1000, ctypes.byref(n)) == _lib.S4_ERR_UNSUPPORTED
+    assert lib.s4_fft_conv_kernel_grad_workspace_size(4, 16384, ctypes.byref(n)) == _lib.S4_OK
+    assert n.value >= 4 * 2 * 16384 * 8 + 4 * 16384 * 4   # spectrum of (H, L) + one row of shares
     assert lib.s4_fft_conv_kernel_grad_workspace_size(4, 4096, ctypes.byref(n)) == _lib.S4_OK
     assert n.value == 2 * 4 * 2 * 4096 * 8
     u, dy, dK, dD = p(FAKE), p(FAKE + 0x10000000), p(FAKE2), p(FAKE2 + 0x10000000)
