@@ -201,7 +201,12 @@ s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H
  * through DFT(dK) at the same roots of unity and the derivatives of the
  * four Cauchy sums, the Woodbury correction and the bilinear factor
  * (squared-denominator Cauchy sums for Lambda and dt), and the closed form at
- * the Nyquist bin. L <= 16384 (longer -> S4_ERR_UNSUPPORTED).
+ * the Nyquist bin. s4_kernel_dplr_backward: L <= 16384 (longer ->
+ * S4_ERR_UNSUPPORTED). s4_kernel_dplr_backward_ws: any L; for L > 16384
+ * DFT(dK) is formed by a four-step transform (L = 256 x L/256) in the
+ * workspace (s4_kernel_dplr_backward_workspace_size bytes: H L 8 + H (L/2+1) 8,
+ * each rounded up to 256; 0 for L <= 16384, where the workspace may be NULL),
+ * 256-byte aligned, caller-owned, not overlapping the outputs or dK.
  *   Lambda, P, Q, B, C : [H, Nh] complex;  log_dt : [H];  dK : [H, L].
  *   dLambda, dP, dQ, dB, dC : [H, Nh] complex out;  dlog_dt : [H] out.
  * Errors: null pointers, misaligned complex arrays, outputs overlapping
@@ -213,6 +218,15 @@ s4_status s4_kernel_dplr_backward(const s4_c32 *Lambda, const s4_c32 *P, const s
                                   const float *dK, int H, int Nh, int L, s4_c32 *dLambda,
                                   s4_c32 *dP, s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC,
                                   float *dlog_dt, cudaStream_t stream);
+
+s4_status s4_kernel_dplr_backward_workspace_size(int H, int L, size_t *bytes);
+
+s4_status s4_kernel_dplr_backward_ws(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q,
+                                     const s4_c32 *B, const s4_c32 *C, const float *log_dt,
+                                     const float *dK, int H, int Nh, int L, s4_c32 *dLambda,
+                                     s4_c32 *dP, s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC,
+                                     float *dlog_dt, void *workspace, size_t workspace_bytes,
+                                     cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * The whole forward pass of the layer's convolution view ([S4K] §4, §5).

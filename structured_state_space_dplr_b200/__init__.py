@@ -26,7 +26,7 @@ __all__ = [
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
     "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "dplr_ctilde", "forward_dplr_host",
     "fft_conv_host", "fft_conv_apply_adjoint", "fft_conv_kernel_grad", "fft_conv_kernel_grad_workspace_size",
-    "kernel_dplr_backward", "load",
+    "kernel_dplr_backward", "kernel_dplr_backward_workspace_size", "load",
 ]
 
 
@@ -298,10 +298,12 @@ def fft_conv_kernel_grad(u, dy, *, dK=None, dD=None, workspace=None):
     return dK, dD
 
 
-def kernel_dplr_backward(Lambda, P, Q, B, C, log_dt, dK):
-    """Gradient through the DPLR kernel (s4_kernel_dplr_backward): given
+def kernel_dplr_backward(Lambda, P, Q, B, C, log_dt, dK, *, workspace=None):
+    """Gradient through the DPLR kernel (s4_kernel_dplr_backward_ws): given
     dK = dLoss/dK [H, L], returns dict(Lambda, P, Q, B, C -> complex64
-    [H, Nh] as dLoss/dRe + i dLoss/dIm; log_dt -> float32 [H])."""
+    [H, Nh] as dLoss/dRe + i dLoss/dIm; log_dt -> float32 [H]). For
+    L > 16384 a workspace of kernel_dplr_backward_workspace_size(H, L) bytes
+    is used (allocated here when not given)."""
     Lambda, P, Q, B, C = (_cplx(x, n) for x, n in zip((Lambda, P, Q, B, C), "Lambda P Q B C".split()))
     log_dt = _cuda(log_dt, "log_dt", torch.float32)
     dK = _cuda(dK, "dK", torch.float32)
@@ -309,10 +311,24 @@ def kernel_dplr_backward(Lambda, P, Q, B, C, log_dt, dK):
     L = dK.shape[-1]
     out = {k: torch.empty_like(Lambda) for k in ("Lambda", "P", "Q", "B", "C")}
     out["log_dt"] = torch.empty_like(log_dt)
-    _lib.call("s4_kernel_dplr_backward", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
+    need = kernel_dplr_backward_workspace_size(H, L)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Lambda.device)
+    nbytes = 0
+    if workspace is not None:
+        _cuda(workspace, "workspace", torch.uint8)
+        nbytes = workspace.numel()
+    _lib.call("s4_kernel_dplr_backward_ws", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
               _ptr(dK), H, Nh, L, _ptr(out["Lambda"]), _ptr(out["P"]), _ptr(out["Q"]), _ptr(out["B"]),
-              _ptr(out["C"]), _ptr(out["log_dt"]), _stream())
+              _ptr(out["C"]), _ptr(out["log_dt"]), _ptr(workspace), nbytes, _stream())
     return out
+
+
+def kernel_dplr_backward_workspace_size(H, L) -> int:
+    """Bytes of workspace kernel_dplr_backward needs (0 for L <= 16384)."""
+    n = ctypes.c_size_t(0)
+    _lib.call("s4_kernel_dplr_backward_workspace_size", int(H), int(L), ctypes.byref(n))
+    return n.value
 
 
 def kernel_dplr_prepare(Lambda, P, Q, B, C, log_dt, D, L, *, K=None, workspace=None, flags=None):

@@ -44,6 +44,9 @@ SIGNATURES = {
     "s4_fft_conv_kernel_grad_workspace_size": (_i, [_i, _i, ctypes.POINTER(ctypes.c_size_t)]),
     "s4_fft_conv_kernel_grad": (_i, [_p, _p, _i, _i, _i, _p, _p, _p, _sz, _p]),
     "s4_kernel_dplr_backward": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
+    "s4_kernel_dplr_backward_workspace_size": (_i, [_i, _i, ctypes.POINTER(_sz)]),
+    "s4_kernel_dplr_backward_ws": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p,
+                                        _sz, _p]),
     "s4_fft_conv_static": (_i, [_p, _p, _p, _i, _i, _i, _p, _p]),
     "s4_kernel_dplr_prepare": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p, _sz, _p, _p]),
     "s4_forward_dplr": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _sz, _p, _p]),

@@ -279,15 +279,14 @@ s4_status s4_fft_conv_kernel_grad(const float *u, const float *dy, int Bt, int H
     return cuda_status(s4::launch_corr(u, dy, Bt, H, L, dK, dD, workspace, stream));
 }
 
-s4_status s4_kernel_dplr_backward(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B,
-                                  const s4_c32 *C, const float *log_dt, const float *dK, int H, int Nh, int L,
-                                  s4_c32 *dLambda, s4_c32 *dP, s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC,
-                                  float *dlog_dt, cudaStream_t stream) {
+namespace {
+s4_status kbwd_checks(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B, const s4_c32 *C,
+                      const float *log_dt, const float *dK, int H, int Nh, int L, s4_c32 *dLambda, s4_c32 *dP,
+                      s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC, float *dlog_dt) {
     if (any_null(Lambda, P, Q, B, C) || any_null(dLambda, dP, dQ, dB, dC) || any_null(log_dt, dK, dlog_dt))
         return S4_ERR_INVALID_ARG;
     s4_status s = check_modes(H, Nh, L, true);
     if (s != S4_OK) return s;
-    if (L > 16384) return S4_ERR_UNSUPPORTED;
     if (!params_aligned({Lambda, P, Q, B, C, dLambda, dP, dQ, dB, dC}) || !aligned(dK, 4)) return S4_ERR_INVALID_ARG;
     const size_t pb = (size_t)H * Nh * sizeof(s4_c32);
     const void *outs[] = {dLambda, dP, dQ, dB, dC};
@@ -301,10 +300,49 @@ s4_status s4_kernel_dplr_backward(const s4_c32 *Lambda, const s4_c32 *P, const s
             overlap(outs[i], pb, dlog_dt, (size_t)H * sizeof(float)))
             return S4_ERR_INVALID_ARG;
     }
+    return S4_OK;
+}
+}  // namespace
+
+s4_status s4_kernel_dplr_backward(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B,
+                                  const s4_c32 *C, const float *log_dt, const float *dK, int H, int Nh, int L,
+                                  s4_c32 *dLambda, s4_c32 *dP, s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC,
+                                  float *dlog_dt, cudaStream_t stream) {
+    s4_status s = kbwd_checks(Lambda, P, Q, B, C, log_dt, dK, H, Nh, L, dLambda, dP, dQ, dB, dC, dlog_dt);
+    if (s != S4_OK) return s;
+    if (L > 16384) return S4_ERR_UNSUPPORTED;   // needs the workspace form
     return cuda_status(s4::launch_kgen_backward((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q,
                                                 (const float2 *)B, (const float2 *)C, log_dt, dK, H, Nh, L,
                                                 (float2 *)dLambda, (float2 *)dP, (float2 *)dQ, (float2 *)dB,
-                                                (float2 *)dC, dlog_dt, stream));
+                                                (float2 *)dC, dlog_dt, nullptr, stream));
+}
+
+s4_status s4_kernel_dplr_backward_workspace_size(int H, int L, size_t *bytes) {
+    if (bytes == nullptr || H < 1) return S4_ERR_INVALID_ARG;
+    if (!pow2_L(L)) return S4_ERR_UNSUPPORTED;
+    *bytes = s4::kgen_backward_workspace_bytes(H, L);
+    return S4_OK;
+}
+
+s4_status s4_kernel_dplr_backward_ws(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32 *Q, const s4_c32 *B,
+                                     const s4_c32 *C, const float *log_dt, const float *dK, int H, int Nh, int L,
+                                     s4_c32 *dLambda, s4_c32 *dP, s4_c32 *dQ, s4_c32 *dB, s4_c32 *dC,
+                                     float *dlog_dt, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    s4_status s = kbwd_checks(Lambda, P, Q, B, C, log_dt, dK, H, Nh, L, dLambda, dP, dQ, dB, dC, dlog_dt);
+    if (s != S4_OK) return s;
+    const size_t need = s4::kgen_backward_workspace_bytes(H, L);
+    if (need > 0) {
+        if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need) return S4_ERR_WORKSPACE;
+        const size_t pb = (size_t)H * Nh * sizeof(s4_c32);
+        for (const void *o : {(const void *)dLambda, (const void *)dP, (const void *)dQ, (const void *)dB,
+                              (const void *)dC, (const void *)dlog_dt, (const void *)dK})
+            if (overlap(o, o == dK ? (size_t)H * L * sizeof(float) : pb, workspace, workspace_bytes))
+                return S4_ERR_INVALID_ARG;
+    }
+    return cuda_status(s4::launch_kgen_backward((const float2 *)Lambda, (const float2 *)P, (const float2 *)Q,
+                                                (const float2 *)B, (const float2 *)C, log_dt, dK, H, Nh, L,
+                                                (float2 *)dLambda, (float2 *)dP, (float2 *)dQ, (float2 *)dB,
+                                                (float2 *)dC, dlog_dt, need > 0 ? workspace : nullptr, stream));
 }
 
 s4_status s4_fft_conv(const float *u, const float *K, const float *D, int Bt, int H, int L, float *y,

@@ -155,9 +155,12 @@ k_corr_pair(const float *__restrict__ u, const float *__restrict__ dy, int Bt, i
 constexpr int kBwdThreads = 256;
 constexpr int kModeFloats = 20;   // lambda(2) C(2) B(2) P(2) Q(2) v00..v11(8) -(2)
 
-template <int LG>
+// GG: G_hat comes from global memory (computed by the four-step DFT below), no
+// transform in shared memory
+template <int LG, bool GG>
 __host__ __device__ constexpr size_t kbwd_smem_bytes(int Nh) {
-    return sizeof(float2) * ((size_t)padded(1 << LG) + plan_tw_size(LG) + ((1 << LG) >> plan_lr(LG, 0))) +
+    return (GG ? 0
+               : sizeof(float2) * ((size_t)padded(1 << LG) + plan_tw_size(LG) + ((1 << LG) >> plan_lr(LG, 0)))) +
            sizeof(float) * ((size_t)kModeFloats * Nh + 9 * kBwdThreads + 16 * kBwdThreads + 32);
 }
 
@@ -168,26 +171,28 @@ __device__ __forceinline__ float2 crcp(float2 d) {
     return make_float2(d.x * inv, -d.y * inv);
 }
 
-template <int LG>
+template <int LG, bool GG>
 __global__ void __launch_bounds__(kBwdThreads, 2)
 k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const float2 *__restrict__ Q,
                 const float2 *__restrict__ B, const float2 *__restrict__ Cc, const float *__restrict__ log_dt,
-                const float *__restrict__ dK, int H, int Nh, float2 *__restrict__ dLambda,
-                float2 *__restrict__ dP, float2 *__restrict__ dQ, float2 *__restrict__ dB,
-                float2 *__restrict__ dC, float *__restrict__ dlog_dt) {
+                const float *__restrict__ dK, const float2 *__restrict__ ghat, int H, int Nh,
+                float2 *__restrict__ dLambda, float2 *__restrict__ dP, float2 *__restrict__ dQ,
+                float2 *__restrict__ dB, float2 *__restrict__ dC, float *__restrict__ dlog_dt) {
     constexpr int m = 1 << LG, L = m, T = kBwdThreads;
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
     extern __shared__ float2 smb[];
-    float2 *buf = smb, *tws = buf + padded(m), *tb = tws + plan_tw_size(LG);
-    float *md = reinterpret_cast<float *>(tb + S0);         // [Nh][kModeFloats]
+    float2 *buf = smb, *tws = buf + (GG ? 0 : padded(m)), *tb = tws + (GG ? 0 : plan_tw_size(LG));
+    float *md = reinterpret_cast<float *>(tb + (GG ? 0 : S0));   // [Nh][kModeFloats]
     float *chA = md + kModeFloats * Nh;                      // [T][8]  a_v of the chunk
     float *chG = chA + 8 * T;                                // [T]     gamma of the chunk
     float *red = chG + T;                                    // [T][16] partial sums
     float *red32 = red + 16 * T;                             // [32]
     const int tid = threadIdx.x;
-    for (int j = tid; j < S0; j += T) tb[j] = unit_root(j, m);
-    build_middle_tables<LG>(tws, tid, T);
+    if constexpr (!GG) {
+        for (int j = tid; j < S0; j += T) tb[j] = unit_root(j, m);
+        build_middle_tables<LG>(tws, tid, T);
+    }
     const int nq = T / Nh;   // frequency slices per mode (Nh <= T)
     const int my_n = tid % Nh, my_q = tid / Nh;
 
@@ -205,6 +210,7 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
         }
         // ---- G_hat = DFT(dK): forward transform, digit-reversed result in buf
         const float *dKh = dK + (size_t)h * L;
+        if constexpr (!GG) {
         for (int j = tid; j < S0; j += T) {
             float2 x[R0];
             static_for<0, R0>([&](auto p) { x[p] = make_float2(__ldg(dKh + j + p * S0), 0.0f); });
@@ -227,7 +233,9 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
             dft<RL, -1>(x);
             store_contig<RL>(o, x);
         }
+        }   // !GG
         __syncthreads();
+        const float2 *gh = ghat + (size_t)h * (L / 2 + 1);
 
         float ld_acc = 0.0f;
         float2 S[4], S2[4];
@@ -267,7 +275,9 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
                 e[1] = cscale(cmul(c, cmul(k[2], iden)), -1.0f);
                 e[2] = cscale(cmul(c, cmul(k[1], iden)), -1.0f);
                 e[3] = cmul(c, cmul(cmul(k[1], k[2]), cmul(iden, iden)));
-                const float2 G = buf[pidx(digrev_inv<LG>(j))];
+                float2 G;
+                if constexpr (GG) G = gh[j];
+                else G = buf[pidx(digrev_inv<LG>(j))];
                 const float wj = (j == 0 ? 1.0f : 2.0f) / (float)L;
                 const float2 gj = make_float2(G.x * wj, G.y * wj);
                 float2 dw = make_float2(0.f, 0.f);
@@ -313,7 +323,9 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
             red[16 * tid + 8 + 2 * v] = S2[v].x;
             red[16 * tid + 8 + 2 * v + 1] = S2[v].y;
         }
-        const float gN = buf[pidx(digrev_inv<LG>(L / 2))].x / (float)L;
+        float gN;
+        if constexpr (GG) gN = gh[L / 2].x / (float)L;
+        else gN = buf[pidx(digrev_inv<LG>(L / 2))].x / (float)L;
         if (tid < Nh) {   // Nyquist share of dlog_dt: gN dt Re(C_n B_n), summed below
             const float *w = md + kModeFloats * tid;
             ld_acc = fmaf(gN * dt, w[10], ld_acc);
@@ -392,33 +404,139 @@ cudaError_t run_corr(const float *u, const float *dy, int Bt, int H, float *dK, 
 }  // namespace
 
 namespace {
-template <int LG>
+template <int LG, bool GG = false>
 cudaError_t run_kgen_backward(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
                               const float2 *C, const float *log_dt, const float *dK, int H, int Nh,
                               float2 *dLambda, float2 *dP, float2 *dQ, float2 *dB, float2 *dC, float *dlog_dt,
-                              cudaStream_t st) {
-    const size_t smem = kbwd_smem_bytes<LG>(Nh);
+                              cudaStream_t st, const float2 *ghat = nullptr) {
+    const size_t smem = kbwd_smem_bytes<LG, GG>(Nh);
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess && smem > 48 * 1024)
-        e = cudaFuncSetAttribute(k_kgen_backward<LG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(k_kgen_backward<LG, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_kgen_backward<LG>, kBwdThreads, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_kgen_backward<LG, GG>, kBwdThreads, smem);
     if (e != cudaSuccess) return e;
     const int slots = (per_sm > 0 ? per_sm : 1) * sms;
     const int grid = H < slots ? H : slots;
-    k_kgen_backward<LG><<<grid, kBwdThreads, smem, st>>>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ,
-                                                         dB, dC, dlog_dt);
+    k_kgen_backward<LG, GG><<<grid, kBwdThreads, smem, st>>>(Lambda, P, Q, B, C, log_dt, dK, ghat, H, Nh, dLambda,
+                                                             dP, dQ, dB, dC, dlog_dt);
     return cudaGetLastError();
 }
 }  // namespace
 
+// ---- DFT of dK for L >= 32768 by four steps, L = n1 n2, n1 = 256:
+//   G[h, j1 + n1 j2] = sum_{k2} w_n2^{j2 k2} ( w_L^{j1 k2} sum_{k1} w_n1^{j1 k1} dK[h, n2 k1 + k2] ),
+// w_n = exp(-2 pi i / n). Each kernel runs 32 sequences of one size
+// n = 16 R2 (R2 = 8 or 16) per CTA in shared memory (element k of sequence c
+// at k * 33 + c): with k = R2 a + b and j = p + 16 q, pass 1 takes the
+// length-16 DFT over a for each b and multiplies by w_n^{b p} (in place, at
+// R2 p + b), pass 2 the length-R2 DFT over b, leaving X[p + 16 q] at
+// R2 p + q.
+template <int R2>
+__device__ void dft32_smem(float2 *s) {
+    constexpr int n = 16 * R2, T = kBwdThreads;
+    for (int it = threadIdx.x; it < 32 * R2; it += T) {
+        const int c = it & 31, b = it >> 5;
+        float2 x[16];
+#pragma unroll
+        for (int a = 0; a < 16; ++a) x[a] = s[(R2 * a + b) * 33 + c];
+        dft<16, -1>(x);
+#pragma unroll
+        for (int p = 0; p < 16; ++p) s[(R2 * p + b) * 33 + c] = cmul(x[p], unit_root(b * p, n));
+    }
+    __syncthreads();
+    for (int it = threadIdx.x; it < 32 * 16; it += T) {
+        const int c = it & 31, p = it >> 5;
+        float2 z[R2];
+#pragma unroll
+        for (int b = 0; b < R2; ++b) z[b] = s[(R2 * p + b) * 33 + c];
+        dft<R2, -1>(z);
+#pragma unroll
+        for (int q = 0; q < R2; ++q) s[(R2 * p + q) * 33 + c] = z[q];
+    }
+    __syncthreads();
+}
+constexpr int kDftN1 = 256;
+
+// columns: CTA (x, h) takes k2 = 32 x .. 32 x + 31; Y[h, j1, k2] = w_L^{j1 k2} X
+__global__ void __launch_bounds__(kBwdThreads) k_dft_cols(const float *__restrict__ dK, int L,
+                                                          float2 *__restrict__ Y) {
+    extern __shared__ float2 s[];   // [kDftN1][33]
+    const int h = blockIdx.y, k20 = blockIdx.x * 32, n2 = L / kDftN1;
+    const float *src = dK + (size_t)h * L;
+    for (int i = threadIdx.x; i < kDftN1 * 32; i += kBwdThreads) {
+        const int k1 = i >> 5, c = i & 31;
+        s[k1 * 33 + c] = make_float2(src[(size_t)n2 * k1 + k20 + c], 0.0f);
+    }
+    __syncthreads();
+    dft32_smem<kDftN1 / 16>(s);
+    float2 *dst = Y + (size_t)h * L;
+    for (int i = threadIdx.x; i < kDftN1 * 32; i += kBwdThreads) {
+        const int c = i & 31, j1 = i >> 5, p = j1 & 15, q = j1 >> 4;
+        const int k2 = k20 + c;
+        dst[(size_t)j1 * n2 + k2] = cmul(s[(16 * p + q) * 33 + c], unit_root((j1 * k2) & (L - 1), L));
+    }
+}
+
+// rows: CTA (x, h) takes j1 = 32 x .. 32 x + 31; G[h, j1 + n1 j2] for j <= L / 2
+template <int R2>
+__global__ void __launch_bounds__(kBwdThreads) k_dft_rows(const float2 *__restrict__ Y, int L,
+                                                          float2 *__restrict__ G) {
+    constexpr int n2 = 16 * R2;
+    extern __shared__ float2 s[];   // [n2][33]
+    const int h = blockIdx.y, j10 = blockIdx.x * 32;
+    const float2 *src = Y + (size_t)h * L;
+    for (int i = threadIdx.x; i < n2 * 32; i += kBwdThreads) {
+        const int k2 = i % n2, c = i / n2;
+        s[k2 * 33 + c] = src[(size_t)(j10 + c) * n2 + k2];
+    }
+    __syncthreads();
+    dft32_smem<R2>(s);
+    float2 *dst = G + (size_t)h * (L / 2 + 1);
+    for (int i = threadIdx.x; i < n2 * 32; i += kBwdThreads) {
+        const int c = i & 31, j2 = i >> 5, p = j2 & 15, q = j2 >> 4;
+        const int j = j10 + c + kDftN1 * j2;
+        if (j <= L / 2) dst[j] = s[(R2 * p + q) * 33 + c];
+    }
+}
+
+size_t kgen_backward_workspace_bytes(int H, int L) {
+    if (L <= 16384) return 0;
+    return (((size_t)H * L * sizeof(float2) + 255) & ~size_t(255)) +
+           (((size_t)H * (L / 2 + 1) * sizeof(float2) + 255) & ~size_t(255));
+}
+
 cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
                                  const float2 *C, const float *log_dt, const float *dK, int H, int Nh, int L,
                                  float2 *dLambda, float2 *dP, float2 *dQ, float2 *dB, float2 *dC,
-                                 float *dlog_dt, cudaStream_t st) {
+                                 float *dlog_dt, void *ws, cudaStream_t st) {
 #define S4_KBWD(LG) run_kgen_backward<LG>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC, dlog_dt, st)
+    if (L > 16384) {   // G_hat by the four-step DFT into the workspace, then the gradients
+        float2 *Y = static_cast<float2 *>(ws);
+        float2 *G = reinterpret_cast<float2 *>(static_cast<char *>(ws) +
+                                               (((size_t)H * L * sizeof(float2) + 255) & ~size_t(255)));
+        const int n2 = L / kDftN1;
+        const size_t smc = (size_t)kDftN1 * 33 * sizeof(float2), smr = (size_t)n2 * 33 * sizeof(float2);
+        cudaError_t e = cudaFuncSetAttribute(k_dft_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smc);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(n2 == 128 ? k_dft_rows<8> : k_dft_rows<16>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+        if (e != cudaSuccess) return e;
+        k_dft_cols<<<dim3(n2 / 32, H), kBwdThreads, smc, st>>>(dK, L, Y);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        if (n2 == 128) k_dft_rows<8><<<dim3(kDftN1 / 32, H), kBwdThreads, smr, st>>>(Y, L, G);
+        else k_dft_rows<16><<<dim3(kDftN1 / 32, H), kBwdThreads, smr, st>>>(Y, L, G);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        if (L == 32768)
+            return run_kgen_backward<15, true>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC,
+                                               dlog_dt, st, G);
+        return run_kgen_backward<16, true>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC,
+                                           dlog_dt, st, G);
+    }
     switch (L) {
         case 16: return S4_KBWD(4);
         case 32: return S4_KBWD(5);

@@ -25,10 +25,12 @@ size_t corr_workspace_bytes(int H, int L);
 cudaError_t launch_corr(const float *u, const float *dy, int Bt, int H, int L, float *dK, float *dD, void *ws,
                         cudaStream_t st);
 
+// L > 16384 needs kgen_backward_workspace_bytes(H, L) of workspace (ws), else ws may be null
+size_t kgen_backward_workspace_bytes(int H, int L);
 cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
                                  const float2 *C, const float *log_dt, const float *dK, int H, int Nh, int L,
                                  float2 *dLambda, float2 *dP, float2 *dQ, float2 *dB, float2 *dC,
-                                 float *dlog_dt, cudaStream_t st);
+                                 float *dlog_dt, void *ws, cudaStream_t st);
 
 cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st);
 

@@ -182,6 +182,24 @@ def test_block_entries_reject_bad_arguments(lib):
     assert bf(x, g, b, 1e-5, cws, 16, bias, ws, wsb, 2, 256, 4096, z, y, out, p(0), p(0)) == _lib.S4_ERR_WORKSPACE
 
 
+def test_kernel_backward_workspace(lib):
+    n = ctypes.c_size_t()
+    assert lib.s4_kernel_dplr_backward_workspace_size(4, 16384, ctypes.byref(n)) == _lib.S4_OK and n.value == 0
+    assert lib.s4_kernel_dplr_backward_workspace_size(4, 65536, ctypes.byref(n)) == _lib.S4_OK
+    assert n.value == 4 * 65536 * 8 + 4 * 32769 * 8 + (256 - (4 * 32769 * 8) % 256) % 256
+    five = [p(FAKE + 0x10000 * i) for i in range(5)]
+    outs = [p(FAKE2 + 0x10000 * i) for i in range(5)]
+    ldt, dK, dl = p(FAKE + 0x60000), p(FAKE + 0x1000000), p(FAKE2 + 0x60000)
+    ws = p(FAKE2 + 0x10000000)
+    kb = lib.s4_kernel_dplr_backward
+    assert kb(*five, ldt, dK, 4, 5, 65536, *outs, dl, p(0)) == _lib.S4_ERR_UNSUPPORTED   # needs the _ws form
+    kw = lib.s4_kernel_dplr_backward_ws
+    assert kw(*five, ldt, dK, 4, 5, 65536, *outs, dl, p(0), 0, p(0)) == _lib.S4_ERR_WORKSPACE
+    assert kw(*five, ldt, dK, 4, 5, 65536, *outs, dl, ws, n.value - 1, p(0)) == _lib.S4_ERR_WORKSPACE
+    assert kw(*five, ldt, dK, 4, 5, 65536, *outs, dl, p(FAKE2 + 0x10000010), n.value, p(0)) == \
+        _lib.S4_ERR_WORKSPACE                                                              # misaligned
+
+
 def test_zoh_entries_reject_bad_arguments(lib):
     five = [p(FAKE + 0x10000 * i) for i in range(5)]
     ldt = p(FAKE + 0x60000)

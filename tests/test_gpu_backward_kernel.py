@@ -39,7 +39,7 @@ def _check(g, ref, channels, tol=P_TOL):
         assert err <= tol, (k, err)
 
 
-@pytest.mark.parametrize("L", [16, 64, 256, 1024, 4096, 8192, 16384])
+@pytest.mark.parametrize("L", [16, 64, 256, 1024, 4096, 8192, 16384, 32768, 65536])
 def test_random_dplr_parameter_gradients(L):
     inp = s4inputs.random_dplr(40 + L, H=2, Nh=5, L=L, Bt=1)
     dK = np.random.default_rng(L).standard_normal((2, L))
