@@ -354,46 +354,49 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
 
-    # backward pass of the same layer (L <= 8192): du by the adjoint
-    # convolution, dK and dD by the batch correlation, and (DPLR) the
-    # parameter gradients through the kernel; dy is another input set's u
+    # backward pass of the same layer: du by the adjoint convolution, dK and
+    # dD by the batch correlation (L > 8192: per batch row through the
+    # adjoint convolution), and (DPLR) the parameter gradients through the
+    # kernel (L > 16384: four-step DFT of dK); dy is another input set's u
     backward = None
-    if L <= 8192:
-        d, dy = sets[0], sets[1 % nsets]["u"]
-        du = torch.empty_like(dy)
-        gK = torch.empty(H, L, device=dev)
-        gD = torch.empty(H, device=dev)
-        gws = torch.empty(s4.fft_conv_kernel_grad_workspace_size(H, L), dtype=torch.uint8, device=dev)
+    d, dy = sets[0], sets[1 % nsets]["u"]
+    du = torch.empty_like(dy)
+    gK = torch.empty(H, L, device=dev)
+    gD = torch.empty(H, device=dev)
+    gws = torch.empty(s4.fft_conv_kernel_grad_workspace_size(H, L), dtype=torch.uint8, device=dev)
+    kneed = s4.kernel_dplr_backward_workspace_size(H, L)
+    kws = torch.empty(kneed, dtype=torch.uint8, device=dev) if kneed > 0 else None
 
-        def bwd(ev=None):
-            if ev is not None:
-                ev[0].record()
-            s4.fft_conv_apply_adjoint(dy, d["ws"], out=du)
-            if ev is not None:
-                ev[1].record()
-            s4.fft_conv_kernel_grad(d["u"], dy, dK=gK, dD=gD, workspace=gws)
-            if ev is not None:
-                ev[2].record()
-            if not s4d:
-                s4.kernel_dplr_backward(d["Lambda"], d["P"], d["Q"], d["B"], d["C"], d["log_dt"], gK)
-            if ev is not None:
-                ev[3].record()
+    def bwd(ev=None):
+        if ev is not None:
+            ev[0].record()
+        s4.fft_conv_apply_adjoint(dy, d["ws"], out=du)
+        if ev is not None:
+            ev[1].record()
+        s4.fft_conv_kernel_grad(d["u"], dy, dK=gK, dD=gD, workspace=gws)
+        if ev is not None:
+            ev[2].record()
+        if not s4d:
+            s4.kernel_dplr_backward(d["Lambda"], d["P"], d["Q"], d["B"], d["C"], d["log_dt"], gK,
+                                    workspace=kws)
+        if ev is not None:
+            ev[3].record()
 
-        for _ in range(max(1, args.warmup)):
-            bwd()
-        torch.cuda.synchronize()
-        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-        for i in range(args.steps):
-            bwd(bev[i])
-        torch.cuda.synchronize()
-        bst = [sum(e[j].elapsed_time(e[j + 1]) for e in bev) / args.steps for j in range(3)]
-        total = sum(bst)
-        backward = {"metric": "S4 layer backward (batch*H*L) elems/s", "value": alg["elements"] / (total * 1e-3),
-                    "ms_per_step": total,
-                    "stages_ms": {"du_adjoint_conv": bst[0], "dK_dD_batch_correlation": bst[1],
-                                  "kernel_param_grads": bst[2]},
-                    "calls": "s4_fft_conv_apply_adjoint + s4_fft_conv_kernel_grad"
-                             + ("" if s4d else " + s4_kernel_dplr_backward") + ", one launch each"}
+    for _ in range(max(1, args.warmup)):
+        bwd()
+    torch.cuda.synchronize()
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        bwd(bev[i])
+    torch.cuda.synchronize()
+    bst = [sum(e[j].elapsed_time(e[j + 1]) for e in bev) / args.steps for j in range(3)]
+    total = sum(bst)
+    backward = {"metric": "S4 layer backward (batch*H*L) elems/s", "value": alg["elements"] / (total * 1e-3),
+                "ms_per_step": total,
+                "stages_ms": {"du_adjoint_conv": bst[0], "dK_dD_batch_correlation": bst[1],
+                              "kernel_param_grads": bst[2]},
+                "calls": "s4_fft_conv_apply_adjoint + s4_fft_conv_kernel_grad"
+                         + ("" if s4d else " + s4_kernel_dplr_backward") + ", one launch each"}
 
     # the S4Block around the same layer: channel layer norm -> the layer's
     # convolution (the prepared spectrum) -> GLU projection + residual, over
