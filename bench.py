@@ -376,7 +376,9 @@ def run_gpu(args, rank, world, local_rank):
         s4.fft_conv_kernel_grad(d["u"], dy, dK=gK, dD=gD, workspace=gws)
         if ev is not None:
             ev[2].record()
-        if not s4d:
+        if s4d:
+            s4.s4d_kernel_vandermonde_backward(d["A"], d["B"], d["C"], d["log_dt"], gK)
+        else:
             s4.kernel_dplr_backward(d["Lambda"], d["P"], d["Q"], d["B"], d["C"], d["log_dt"], gK,
                                     workspace=kws)
         if ev is not None:
@@ -395,8 +397,12 @@ def run_gpu(args, rank, world, local_rank):
                 "ms_per_step": total,
                 "stages_ms": {"du_adjoint_conv": bst[0], "dK_dD_batch_correlation": bst[1],
                               "kernel_param_grads": bst[2]},
-                "calls": "s4_fft_conv_apply_adjoint + s4_fft_conv_kernel_grad"
-                         + ("" if s4d else " + s4_kernel_dplr_backward") + ", one launch each"}
+                "calls": "s4_fft_conv_apply_adjoint (1 launch) + s4_fft_conv_kernel_grad ("
+                         + ("1 launch" if L <= 8192
+                            else f"{3 * Bt} launches: per batch row spectrum, adjoint convolution, accumulate")
+                         + ")" + (" + s4d_kernel_vandermonde_backward (1 launch)" if s4d
+                                  else " + s4_kernel_dplr_backward_ws ("
+                                  + ("1 launch" if L <= 16384 else "3 launches: four-step DFT, gradients") + ")")}
 
     # the S4Block around the same layer: channel layer norm -> the layer's
     # convolution (the prepared spectrum) -> GLU projection + residual, over

@@ -429,6 +429,25 @@ s4_status s4d_kernel_vandermonde(const s4_c32 *A, const s4_c32 *B, const s4_c32 
                                  const float *log_dt, int H, int Nh, int L, float *K,
                                  unsigned *d_flags, cudaStream_t stream);
 
+/* s4d_kernel_vandermonde_backward: the gradient of a loss through the S4D
+ * kernel ([S4W] "S4D"; the layer is trained as in [S4K] §6) given
+ * dK = dLoss/dK [H, L]: dA, dB, dC [H, Nh] complex out as dLoss/dRe +
+ * i dLoss/dIm of each stored mode (its conjugate partner accounted for), and
+ * dlog_dt [H] out. With V_n = sum_k dK[k] Abar_n^k, W_n = sum_k k dK[k]
+ * Abar_n^k and r_n = (exp(dt a_n) - 1)/a_n:
+ *   dC = 2 conj(Bbar V), dB = 2 conj(C r V),
+ *   dA = 2 conj(C B dt^2 phi1'(dt a) V + C Bbar dt W), phi1(x) = (e^x - 1)/x,
+ *   dlog_dt = 2 dt Re sum_n (C B Abar V + C Bbar a W).
+ * V, W are summed over 64-step blocks whose first power is evaluated
+ * directly (fp64 phase reduction); fp64 accumulation across blocks.
+ * Any L (power of two in [16, 65536]), Nh <= 256. Errors: null pointers,
+ * misaligned complex arrays, outputs overlapping inputs or each other ->
+ * S4_ERR_INVALID_ARG; bad L, Nh -> S4_ERR_UNSUPPORTED. */
+s4_status s4d_kernel_vandermonde_backward(const s4_c32 *A, const s4_c32 *B, const s4_c32 *C,
+                                          const float *log_dt, const float *dK, int H, int Nh,
+                                          int L, s4_c32 *dA, s4_c32 *dB, s4_c32 *dC,
+                                          float *dlog_dt, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Decode set-up ([S4K] §3 and §5, recurrent view).
  *

@@ -158,3 +158,26 @@ def dplr_kernel_param_grad(inp, dK, channels=None, eps=1e-6):
         for k in keys:
             res[k].append(g[k][0])
     return {k: np.array(v) for k, v in res.items()}
+
+
+def s4d_kernel_param_grad(inp, dK, channels=None, eps=1e-6):
+    """Gradient of <K, dK> (K = the S4D ZOH kernel of the "S4" wiki page,
+    section "S4D": 2 Re sum_n C_n Bbar_n Abar_n^k) with respect to each
+    channel's A, B, C (complex: d/dRe + i d/dIm) and log_dt, by central
+    differences of ssm.s4d_kernel in fp64. dK: [len(channels), L]. Returns a
+    dict of arrays [len(channels), Nh] (log_dt: [len(channels)])."""
+    channels = list(range(inp["H"]) if channels is None else channels)
+    keys = ("A", "B", "C", "log_dt")
+    res = {k: [] for k in keys}
+    for i, h in enumerate(channels):
+        params = {k: _f64(inp[k])[h:h + 1] for k in keys}
+        dKh = np.asarray(dK[i], np.float64)
+
+        def fun(p):
+            K = ssm.s4d_kernel(p["A"], p["B"], p["C"], np.exp(p["log_dt"]), inp["L"])
+            return float(np.dot(K[0], dKh))
+
+        g = fd_gradient(fun, params, keys, eps)
+        for k in keys:
+            res[k].append(g[k][0])
+    return {k: np.array(v) for k, v in res.items()}

@@ -26,7 +26,7 @@ __all__ = [
     "recurrent_scan", "S4Error", "S4_FLAG_UNSTABLE", "S4_FLAG_NONFINITE", "S4_STEP_DENSE",
     "S4_STEP_DIAG", "S4_STEP_DPLR", "dplr_discretize_structured", "dplr_ctilde", "forward_dplr_host",
     "fft_conv_host", "fft_conv_apply_adjoint", "fft_conv_kernel_grad", "fft_conv_kernel_grad_workspace_size",
-    "kernel_dplr_backward", "kernel_dplr_backward_workspace_size", "load",
+    "kernel_dplr_backward", "kernel_dplr_backward_workspace_size", "s4d_kernel_vandermonde_backward", "load",
 ]
 
 
@@ -321,6 +321,22 @@ def kernel_dplr_backward(Lambda, P, Q, B, C, log_dt, dK, *, workspace=None):
     _lib.call("s4_kernel_dplr_backward_ws", _ptr(Lambda), _ptr(P), _ptr(Q), _ptr(B), _ptr(C), _ptr(log_dt),
               _ptr(dK), H, Nh, L, _ptr(out["Lambda"]), _ptr(out["P"]), _ptr(out["Q"]), _ptr(out["B"]),
               _ptr(out["C"]), _ptr(out["log_dt"]), _ptr(workspace), nbytes, _stream())
+    return out
+
+
+def s4d_kernel_vandermonde_backward(A, B, C, log_dt, dK):
+    """Gradient through the S4D kernel (s4d_kernel_vandermonde_backward): given
+    dK [H, L], returns dict(A, B, C -> complex64 [H, Nh] as dLoss/dRe +
+    i dLoss/dIm; log_dt -> float32 [H])."""
+    A, B, C = (_cplx(x, n) for x, n in zip((A, B, C), "A B C".split()))
+    log_dt = _cuda(log_dt, "log_dt", torch.float32)
+    dK = _cuda(dK, "dK", torch.float32)
+    H, Nh = A.shape
+    L = dK.shape[-1]
+    out = {k: torch.empty_like(A) for k in ("A", "B", "C")}
+    out["log_dt"] = torch.empty_like(log_dt)
+    _lib.call("s4d_kernel_vandermonde_backward", _ptr(A), _ptr(B), _ptr(C), _ptr(log_dt), _ptr(dK), H, Nh, L,
+              _ptr(out["A"]), _ptr(out["B"]), _ptr(out["C"]), _ptr(out["log_dt"]), _stream())
     return out
 
 

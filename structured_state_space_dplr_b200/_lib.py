@@ -32,6 +32,7 @@ SIGNATURES = {
     "s4_fft_conv_workspace_size": (_i, [_i, _i, ctypes.POINTER(_sz)]),
     "s4_dplr_discretize_zoh": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _p, _p, _p, _p]),
     "s4_kernel_dplr_zoh": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _p, _p, _p]),
+    "s4d_kernel_vandermonde_backward": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p, _p, _p, _p]),
     "s4_layernorm_channels": (_i, [_p, _p, _p, ctypes.c_float, _i, _i, _i, _p, _p]),
     "s4_glu_projection_workspace_size": (_i, [_i, ctypes.POINTER(_sz)]),
     "s4_glu_projection_prepare": (_i, [_p, _i, _p, _sz, _p]),

@@ -626,4 +626,30 @@ s4_status s4_kernel_dplr_zoh(const s4_c32 *Lambda, const s4_c32 *P, const s4_c32
                                            nullptr, K, d_flags, stream));
 }
 
+// ----------------------------------------------------------- S4D backward
+s4_status s4d_kernel_vandermonde_backward(const s4_c32 *A, const s4_c32 *B, const s4_c32 *C, const float *log_dt,
+                                          const float *dK, int H, int Nh, int L, s4_c32 *dA, s4_c32 *dB,
+                                          s4_c32 *dC, float *dlog_dt, cudaStream_t stream) {
+    if (any_null(A, B, C) || any_null(dA, dB, dC) || any_null(log_dt, dK, dlog_dt)) return S4_ERR_INVALID_ARG;
+    s4_status s = check_modes(H, Nh, L, true);
+    if (s != S4_OK) return s;
+    if (!params_aligned({A, B, C, dA, dB, dC}) || !aligned(dK, 4) || !aligned(log_dt, 4) || !aligned(dlog_dt, 4))
+        return S4_ERR_INVALID_ARG;
+    const size_t pb = (size_t)H * Nh * sizeof(s4_c32);
+    const void *outs[] = {dA, dB, dC};
+    const void *ins[] = {A, B, C};
+    for (int i = 0; i < 3; ++i) {
+        for (int k = 0; k < 3; ++k) {
+            if (overlap(outs[i], pb, ins[k], pb)) return S4_ERR_INVALID_ARG;
+            if (k > i && overlap(outs[i], pb, outs[k], pb)) return S4_ERR_INVALID_ARG;
+        }
+        if (overlap(outs[i], pb, dK, (size_t)H * L * sizeof(float)) ||
+            overlap(outs[i], pb, dlog_dt, (size_t)H * sizeof(float)))
+            return S4_ERR_INVALID_ARG;
+    }
+    return cuda_status(s4::launch_vandermonde_backward((const float2 *)A, (const float2 *)B, (const float2 *)C,
+                                                       log_dt, dK, H, Nh, L, (float2 *)dA, (float2 *)dB,
+                                                       (float2 *)dC, dlog_dt, stream));
+}
+
 }  // extern "C"

@@ -48,6 +48,9 @@ cudaError_t launch_cauchy(const float2 *Lambda, const float2 *P, const float2 *Q
 // ---- s4d.cu ----
 cudaError_t launch_vandermonde(const float2 *A, const float2 *B, const float2 *C, const float *log_dt,
                                int H, int Nh, int L, float *K, unsigned *flags, cudaStream_t st);
+cudaError_t launch_vandermonde_backward(const float2 *A, const float2 *B, const float2 *C, const float *log_dt,
+                                        const float *dK, int H, int Nh, int L, float2 *dA, float2 *dB, float2 *dC,
+                                        float *dlog_dt, cudaStream_t st);
 cudaError_t launch_s4d_zoh(const float2 *A, const float2 *B, const float *log_dt, int H, int Nh,
                            float2 *Abar, float2 *Bbar, cudaStream_t st);
 
