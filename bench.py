@@ -534,11 +534,15 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": {"kernel": "k_fftconv_pair" if L <= 8192 else "k_fftconv", "bound": "hbm", "achieved": conv_gbs, "peak": hbm,
                      "unit": "GB/s", "frac": conv_gbs / hbm, "traffic": traffic,
                      "peak_source": peak_src, "algorithmic_bytes": alg["conv_bytes"]},
-        "cauchy": {"kernel": "k_vandermonde" if s4d else "k_cauchy", "bound": "alu", "achieved": cauchy_tflops,
+        "cauchy": {"kernel": ("k_vandermonde_tc" if L % 8192 == 0 else "k_vandermonde") if s4d else "k_cauchy",
+                   "bound": "alu", "achieved": cauchy_tflops,
                    "peak": fp32_peak,
                    "unit": "TFLOP/s", "frac": cauchy_tflops / fp32_peak,
                    "peak_derivation": f"{SM_COUNT} SM x {FP32_LANES_PER_SM} FP32 lanes x 2 x {sm_max_mhz:.0f} MHz",
-                   "algorithmic_flop": alg["kernel_flop"]},
+                   "algorithmic_flop": alg["kernel_flop"],
+                   **({"note": "the Vandermonde product runs on the tensor cores (3 tf32 products); achieved is the "
+                               "algorithmic FP32-equivalent rate (2 FMAs per term) against the CUDA-core FP32 peak"}
+                      if s4d and L % 8192 == 0 else {})},
         "e2e": None if args.no_e2e else {"value": job_throughput(alg["elements"], world, args.steps, e2e_ms),
                                          "unit": UNIT,
                                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
