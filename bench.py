@@ -402,7 +402,7 @@ def run_gpu(args, rank, world, local_rank):
                             else f"{3 * Bt} launches: per batch row spectrum, adjoint convolution, accumulate")
                          + ")" + (" + s4d_kernel_vandermonde_backward (1 launch)" if s4d
                                   else " + s4_kernel_dplr_backward_ws ("
-                                  + ("1 launch" if L <= 16384 else "3 launches: four-step DFT, gradients") + ")")}
+                                  + ("1 launch" if L <= 16384 else "4 launches: four-step DFT, sliced gradients, assembly") + ")")}
 
     # the S4Block around the same layer: channel layer norm -> the layer's
     # convolution (the prepared spectrum) -> GLU projection + residual, over

@@ -175,9 +175,10 @@ template <int LG, bool GG>
 __global__ void __launch_bounds__(kBwdThreads, 2)
 k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, const float2 *__restrict__ Q,
                 const float2 *__restrict__ B, const float2 *__restrict__ Cc, const float *__restrict__ log_dt,
-                const float *__restrict__ dK, const float2 *__restrict__ ghat, int H, int Nh,
-                float2 *__restrict__ dLambda, float2 *__restrict__ dP, float2 *__restrict__ dQ,
-                float2 *__restrict__ dB, float2 *__restrict__ dC, float *__restrict__ dlog_dt) {
+                const float *__restrict__ dK, const float2 *__restrict__ ghat, int H, int Nh, int FS,
+                float *__restrict__ part, float2 *__restrict__ dLambda, float2 *__restrict__ dP,
+                float2 *__restrict__ dQ, float2 *__restrict__ dB, float2 *__restrict__ dC,
+                float *__restrict__ dlog_dt) {
     constexpr int m = 1 << LG, L = m, T = kBwdThreads;
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
@@ -196,7 +197,13 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
     const int nq = T / Nh;   // frequency slices per mode (Nh <= T)
     const int my_n = tid % Nh, my_q = tid / Nh;
 
-    for (int h = blockIdx.x; h < H; h += gridDim.x) {
+    // GG: item = (channel, frequency slice f of FS); the slice's per-mode
+    // sums go to part[item] and k_kgen_backward_assemble adds the slices
+    const int nitems = GG ? H * FS : H;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        const int h = GG ? item / FS : item;
+        const int jb = GG ? (int)((long long)(L / 2) * (item % FS) / FS) : 0;
+        const int je = GG ? (int)((long long)(L / 2) * (item % FS + 1) / FS) : L / 2;
         const size_t po = (size_t)h * Nh;
         const float dt = expf(__ldg(log_dt + h));
         for (int n = tid; n < Nh; n += T) {
@@ -242,13 +249,13 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
 #pragma unroll
         for (int v = 0; v < 4; ++v) S[v] = S2[v] = make_float2(0.f, 0.f);
         const float2 lam_n = make_float2(md[kModeFloats * my_n], md[kModeFloats * my_n + 1]);
-        for (int j0 = 0; j0 < L / 2; j0 += T) {
+        for (int j0 = jb; j0 < je; j0 += T) {
             // ---- per frequency: k_v, e_v, a_v
             const int j = j0 + tid;
             float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                            make_float2(0.f, 0.f)};
             float gam = 0.0f;
-            if (j < L / 2) {
+            if (j < je) {
                 float sn, cs;
                 sincospif((float)j / (float)L, &sn, &cs);
                 const float t = sn / cs;
@@ -299,7 +306,7 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
             __syncthreads();
             // ---- per mode: S_v, S2_v over this chunk
             if (my_q < nq) {
-                const int jn = (L / 2 - j0) < T ? (L / 2 - j0) : T;
+                const int jn = (je - j0) < T ? (je - j0) : T;
                 for (int jj = my_q; jj < jn; jj += nq) {
                     const float g = chG[jj];
                     const float2 r1 = crcp(make_float2(-lam_n.x, g - lam_n.y));
@@ -322,6 +329,31 @@ k_kgen_backward(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
             red[16 * tid + 2 * v + 1] = S[v].y;
             red[16 * tid + 8 + 2 * v] = S2[v].x;
             red[16 * tid + 8 + 2 * v + 1] = S2[v].y;
+        }
+        if constexpr (GG) {   // the slice's per-mode sums and its dlog_dt share (no Nyquist term)
+            for (int off = 16; off > 0; off >>= 1) ld_acc += __shfl_xor_sync(0xffffffffu, ld_acc, off);
+            if ((tid & 31) == 0) red32[tid >> 5] = ld_acc;
+            __syncthreads();
+            float *pi = part + (size_t)item * (16 * Nh + 1);
+            if (tid == 0) {
+                float sum = 0.0f;
+                for (int i = 0; i < T / 32; ++i) sum += red32[i];
+                pi[16 * Nh] = sum;
+            }
+            for (int n = tid; n < Nh; n += T) {
+                float acc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+                for (int qq = 0; qq < nq; ++qq) {
+                    const float *r = red + 16 * (qq * Nh + n);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[i] += r[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pi[16 * n + i] = acc[i];
+            }
+            __syncthreads();   // shared memory is reused by the next item
+            continue;
         }
         float gN;
         if constexpr (GG) gN = gh[L / 2].x / (float)L;
@@ -408,7 +440,7 @@ template <int LG, bool GG = false>
 cudaError_t run_kgen_backward(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
                               const float2 *C, const float *log_dt, const float *dK, int H, int Nh,
                               float2 *dLambda, float2 *dP, float2 *dQ, float2 *dB, float2 *dC, float *dlog_dt,
-                              cudaStream_t st, const float2 *ghat = nullptr) {
+                              cudaStream_t st, const float2 *ghat = nullptr, int FS = 1, float *part = nullptr) {
     const size_t smem = kbwd_smem_bytes<LG, GG>(Nh);
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -419,12 +451,82 @@ cudaError_t run_kgen_backward(const float2 *Lambda, const float2 *P, const float
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_kgen_backward<LG, GG>, kBwdThreads, smem);
     if (e != cudaSuccess) return e;
     const int slots = (per_sm > 0 ? per_sm : 1) * sms;
-    const int grid = H < slots ? H : slots;
-    k_kgen_backward<LG, GG><<<grid, kBwdThreads, smem, st>>>(Lambda, P, Q, B, C, log_dt, dK, ghat, H, Nh, dLambda,
-                                                             dP, dQ, dB, dC, dlog_dt);
+    const long long items = (long long)H * (GG ? FS : 1);
+    const int grid = items < slots ? (int)items : slots;
+    k_kgen_backward<LG, GG><<<grid, kBwdThreads, smem, st>>>(Lambda, P, Q, B, C, log_dt, dK, ghat, H, Nh, FS, part,
+                                                             dLambda, dP, dQ, dB, dC, dlog_dt);
     return cudaGetLastError();
 }
 }  // namespace
+
+// frequency slices per channel for L > 16384: enough items for ~2 CTAs per
+// SM of a 148-SM device, a power of two, at most 64 (fixed by H alone, so the
+// workspace size does not depend on the device)
+int kbwd_slices(int H) {
+    int fs = 1;
+    while (fs < 64 && (long long)H * fs < 296) fs *= 2;
+    return fs;
+}
+
+// L > 16384: adds the FS slices of every mode in slice order, then the
+// Nyquist bin, and forms the gradients (the formulas of k_kgen_backward)
+__global__ void __launch_bounds__(kBwdThreads)
+k_kgen_backward_assemble(const float2 *__restrict__ Lambda, const float2 *__restrict__ P,
+                         const float2 *__restrict__ Q, const float2 *__restrict__ B, const float2 *__restrict__ Cc,
+                         const float *__restrict__ log_dt, const float2 *__restrict__ ghat, int Nh, int L, int FS,
+                         const float *__restrict__ part, float2 *__restrict__ dLambda, float2 *__restrict__ dP,
+                         float2 *__restrict__ dQ, float2 *__restrict__ dB, float2 *__restrict__ dC,
+                         float *__restrict__ dlog_dt) {
+    __shared__ float red32[kBwdThreads / 32];
+    const int h = blockIdx.x, tid = threadIdx.x;
+    const float dt = expf(__ldg(log_dt + h));
+    const float gN = ghat[(size_t)h * (L / 2 + 1) + L / 2].x / (float)L;
+    const size_t stride = 16 * (size_t)Nh + 1;
+    const float *ph = part + (size_t)h * FS * stride;
+    float ld = 0.0f;
+    if (tid == 0)
+        for (int f = 0; f < FS; ++f) ld += ph[f * stride + 16 * Nh];
+    for (int n = tid; n < Nh; n += kBwdThreads) {
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+        for (int f = 0; f < FS; ++f)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] += ph[f * stride + 16 * n + i];
+        float2 Sv[4], S2v[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            Sv[v] = make_float2(acc[2 * v], acc[2 * v + 1]);
+            S2v[v] = make_float2(acc[8 + 2 * v], acc[9 + 2 * v]);
+        }
+        const size_t o = (size_t)h * Nh + n;
+        const float2 c = Cc[o], b = B[o], p = P[o], q = Q[o];
+        const float2 vv[4] = {cmul(c, b), cmul(c, p), cmulc(b, q), cmulc(p, q)};
+        float2 gC = cadd(cmulc(Sv[0], b), cmulc(Sv[1], p));      // conj(B) S00 + conj(P) S01
+        float2 gB = cadd(cmulc(Sv[0], c), cmul(q, Sv[2]));       // conj(C) S00 + Q S10
+        const float2 gP = cadd(cmulc(Sv[1], c), cmul(q, Sv[3]));  // conj(C) S01 + Q S11
+        const float2 gQ = cadd(cmulc(b, Sv[2]), cmulc(p, Sv[3]));  // B conj(S10) + P conj(S11)
+        float2 gL = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) gL = cadd(gL, cmulc(S2v[v], vv[v]));
+        gC = cadd(gC, cscale(cconj(b), gN * dt));
+        gB = cadd(gB, cscale(cconj(c), gN * dt));
+        dLambda[o] = gL;
+        dP[o] = gP;
+        dQ[o] = gQ;
+        dB[o] = gB;
+        dC[o] = gC;
+        ld = fmaf(gN * dt, vv[0].x, ld);   // Nyquist share: gN dt Re(C_n B_n)
+    }
+    for (int off = 16; off > 0; off >>= 1) ld += __shfl_xor_sync(0xffffffffu, ld, off);
+    if ((tid & 31) == 0) red32[tid >> 5] = ld;
+    __syncthreads();
+    if (tid == 0) {
+        float sum = 0.0f;
+        for (int i = 0; i < kBwdThreads / 32; ++i) sum += red32[i];
+        dlog_dt[h] = sum;
+    }
+}
 
 // ---- DFT of dK for L >= 32768 by four steps, L = n1 n2, n1 = 256:
 //   G[h, j1 + n1 j2] = sum_{k2} w_n2^{j2 k2} ( w_L^{j1 k2} sum_{k1} w_n1^{j1 k1} dK[h, n2 k1 + k2] ),
@@ -502,10 +604,13 @@ __global__ void __launch_bounds__(kBwdThreads) k_dft_rows(const float2 *__restri
     }
 }
 
+// Y (four-step intermediate), G_hat, and the slices' partial sums (bounded
+// with Nh = S4_MAX_NH)
 size_t kgen_backward_workspace_bytes(int H, int L) {
     if (L <= 16384) return 0;
     return (((size_t)H * L * sizeof(float2) + 255) & ~size_t(255)) +
-           (((size_t)H * (L / 2 + 1) * sizeof(float2) + 255) & ~size_t(255));
+           (((size_t)H * (L / 2 + 1) * sizeof(float2) + 255) & ~size_t(255)) +
+           (((size_t)H * kbwd_slices(H) * (16 * (size_t)S4_MAX_NH + 1) * sizeof(float) + 255) & ~size_t(255));
 }
 
 cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
@@ -531,11 +636,17 @@ cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const fl
         else k_dft_rows<16><<<dim3(kDftN1 / 32, H), kBwdThreads, smr, st>>>(Y, L, G);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        if (L == 32768)
-            return run_kgen_backward<15, true>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC,
-                                               dlog_dt, st, G);
-        return run_kgen_backward<16, true>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC,
-                                           dlog_dt, st, G);
+        float *part = reinterpret_cast<float *>(reinterpret_cast<char *>(G) +
+                                                (((size_t)H * (L / 2 + 1) * sizeof(float2) + 255) & ~size_t(255)));
+        const int FS = kbwd_slices(H);
+        e = L == 32768 ? run_kgen_backward<15, true>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC,
+                                                     dlog_dt, st, G, FS, part)
+                       : run_kgen_backward<16, true>(Lambda, P, Q, B, C, log_dt, dK, H, Nh, dLambda, dP, dQ, dB, dC,
+                                                     dlog_dt, st, G, FS, part);
+        if (e != cudaSuccess) return e;
+        k_kgen_backward_assemble<<<H, kBwdThreads, 0, st>>>(Lambda, P, Q, B, C, log_dt, G, Nh, L, FS, part, dLambda,
+                                                              dP, dQ, dB, dC, dlog_dt);
+        return cudaGetLastError();
     }
     switch (L) {
         case 16: return S4_KBWD(4);

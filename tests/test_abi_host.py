@@ -186,7 +186,9 @@ def test_kernel_backward_workspace(lib):
     n = ctypes.c_size_t()
     assert lib.s4_kernel_dplr_backward_workspace_size(4, 16384, ctypes.byref(n)) == _lib.S4_OK and n.value == 0
     assert lib.s4_kernel_dplr_backward_workspace_size(4, 65536, ctypes.byref(n)) == _lib.S4_OK
-    assert n.value == 4 * 65536 * 8 + 4 * 32769 * 8 + (256 - (4 * 32769 * 8) % 256) % 256
+    # four-step intermediate, G_hat (rounded to 256 bytes), and the partial sums of
+    # 64 frequency slices per channel (16 floats per mode + 1, for up to 256 modes)
+    assert n.value == 4 * 65536 * 8 + 1048832 + 4 * 64 * (16 * 256 + 1) * 4
     five = [p(FAKE + 0x10000 * i) for i in range(5)]
     outs = [p(FAKE2 + 0x10000 * i) for i in range(5)]
     ldt, dK, dl = p(FAKE + 0x60000), p(FAKE + 0x1000000), p(FAKE2 + 0x60000)
