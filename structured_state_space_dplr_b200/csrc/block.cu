@@ -265,6 +265,72 @@ __global__ void __launch_bounds__(256) k_layernorm_channels(const float *x, cons
     }
 }
 
+// H <= 16 NV: one pass. Thread (s, l) keeps channels s, s + 16, ... of its 4
+// time steps in registers (all loads in flight at once); the mean and then
+// the variance about it are two reductions over those registers, and z is
+// written from them: x is read once.
+template <int NV>
+__global__ void __launch_bounds__(256, 2) k_layernorm_channels_reg(const float *x, const float *__restrict__ gamma,
+                                                                const float *__restrict__ beta, float eps, int H,
+                                                                int L, float *z) {
+    __shared__ float4 sred[kLnSlices][kLnSteps / 4], sstat[kLnSteps / 4];
+    const int tl = threadIdx.x % (kLnSteps / 4), hs = threadIdx.x / (kLnSteps / 4);
+    const int t = blockIdx.x * kLnSteps + 4 * tl;
+    const bool in = t < L;   // L is a multiple of 16: t < L implies t + 3 < L
+    const size_t base = (size_t)blockIdx.y * H * L + t;
+    const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float4 v[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int h = hs + kLnSlices * i;
+        v[i] = (in && h < H) ? *reinterpret_cast<const float4 *>(x + base + (size_t)h * L) : zero;
+    }
+    const float inv = 1.0f / (float)H;
+    float4 a = zero;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) a = f4add(a, v[i]);
+    sred[hs][tl] = a;
+    __syncthreads();
+    if (hs == 0) {
+        float4 S = zero;
+#pragma unroll
+        for (int i = 0; i < kLnSlices; ++i) S = f4add(S, sred[i][tl]);
+        sstat[tl] = make_float4(S.x * inv, S.y * inv, S.z * inv, S.w * inv);
+    }
+    __syncthreads();
+    const float4 mu = sstat[tl];
+    a = zero;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+        if (hs + kLnSlices * i < H) {
+            const float4 d = f4sub(v[i], mu);
+            a = f4fma(d, d, a);
+        }
+    __syncthreads();   // every thread has read sstat
+    sred[hs][tl] = a;
+    __syncthreads();
+    if (hs == 0) {
+        float4 S = zero;
+#pragma unroll
+        for (int i = 0; i < kLnSlices; ++i) S = f4add(S, sred[i][tl]);
+        sstat[tl] = make_float4(rsqrtf(S.x * inv + eps), rsqrtf(S.y * inv + eps), rsqrtf(S.z * inv + eps),
+                                rsqrtf(S.w * inv + eps));
+    }
+    __syncthreads();
+    if (!in) return;
+    const float4 rs = sstat[tl];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int h = hs + kLnSlices * i;
+        if (h < H) {
+            const float g = __ldg(gamma + h), bb = __ldg(beta + h);
+            *reinterpret_cast<float4 *>(z + base + (size_t)h * L) =
+                make_float4((v[i].x - mu.x) * rs.x * g + bb, (v[i].y - mu.y) * rs.y * g + bb,
+                            (v[i].z - mu.z) * rs.z * g + bb, (v[i].w - mu.w) * rs.w * g + bb);
+        }
+    }
+}
+
 // ------------------------------------------------------- W -> operand images
 // Image (c, nb): rows n of W' = W[128 nb + n/2] (n even) / W[H + 128 nb + n/2]
 // (n odd), columns h = 32 c .. 32 c + 31, K-major, bf16 high part (first
@@ -537,7 +603,12 @@ k_glu_projection_ws(const __grid_constant__ CUtensorMap tm_y, const __grid_const
 cudaError_t launch_layernorm_channels(const float *x, const float *gamma, const float *beta, float eps, int Bt,
                                       int H, int L, float *z, cudaStream_t st) {
     dim3 grid((L + kLnSteps - 1) / kLnSteps, Bt);
-    k_layernorm_channels<<<grid, 256, 0, st>>>(x, gamma, beta, eps, H, L, z);
+    if (H <= 4 * kLnSlices)
+        k_layernorm_channels_reg<4><<<grid, 256, 0, st>>>(x, gamma, beta, eps, H, L, z);
+    else if (H <= 16 * kLnSlices)
+        k_layernorm_channels_reg<16><<<grid, 256, 0, st>>>(x, gamma, beta, eps, H, L, z);
+    else
+        k_layernorm_channels<<<grid, 256, 0, st>>>(x, gamma, beta, eps, H, L, z);
     return cudaGetLastError();
 }
 
