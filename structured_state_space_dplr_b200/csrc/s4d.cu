@@ -505,11 +505,14 @@ cudaError_t launch_vandermonde(const float2 *A, const float2 *B, const float2 *C
     dim3 grid((nkh + kVdmKH - 1) / kVdmKH, H);
     constexpr size_t smem = 2 * kVdmModes * sizeof(double) +
                             (size_t)kVdmModes * (kVdmKH + kVdmKB + 1) * sizeof(float2);
-    static bool attr_set = false;   // the attribute is per function; setting it twice is harmless
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_vandermonde, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static bool attr_set[64];   // per device; setting the attribute twice is harmless
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!attr_set[dev & 63]) {
+        e = cudaFuncSetAttribute(k_vandermonde, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set[dev & 63] = true;
     }
     k_vandermonde<<<grid, kVdmThreads, smem, st>>>(A, B, C, log_dt, Nh, L, K, flags);
     return cudaGetLastError();

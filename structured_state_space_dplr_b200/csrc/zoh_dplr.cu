@@ -287,13 +287,16 @@ k_dplr_zoh(const float2 *__restrict__ Lambda, const float2 *__restrict__ P, cons
 cudaError_t launch_dplr_zoh(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B,
                             const float2 *C, const float *log_dt, int H, int Nh, int L, float2 *Abar,
                             float2 *Bbar, float2 *Cfull, float *K, unsigned *flags, cudaStream_t st) {
-    static bool attr_set[2] = {false, false};   // per function; setting it twice is harmless
+    static bool attr_set[64][2];   // per device and mode; setting the attribute twice is harmless
     const int mode = K != nullptr ? 1 : 0;
-    if (!attr_set[mode]) {
-        cudaError_t e = cudaFuncSetAttribute(mode ? k_dplr_zoh<1> : k_dplr_zoh<0>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)zoh::kSmem);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!attr_set[dev & 63][mode]) {
+        e = cudaFuncSetAttribute(mode ? k_dplr_zoh<1> : k_dplr_zoh<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)zoh::kSmem);
         if (e != cudaSuccess) return e;
-        attr_set[mode] = true;
+        attr_set[dev & 63][mode] = true;
     }
     if (mode)
         k_dplr_zoh<1><<<H, zoh::kThreads, zoh::kSmem, st>>>(Lambda, P, Q, B, C, log_dt, Nh, L, nullptr, nullptr,
