@@ -399,7 +399,8 @@ def run_gpu(args, rank, world, local_rank):
                               "kernel_param_grads": bst[2]},
                 "calls": "s4_fft_conv_apply_adjoint (1 launch) + s4_fft_conv_kernel_grad ("
                          + ("1 launch" if L <= 8192
-                            else f"{3 * Bt} launches: per batch row spectrum, adjoint convolution, accumulate")
+                            else f"{3 * ((Bt + 1) // 2) + 1} launches: per batch row pair spectrum, adjoint "
+                             "convolution, accumulate")
                          + ")" + (" + s4d_kernel_vandermonde_backward (1 launch)" if s4d
                                   else " + s4_kernel_dplr_backward_ws ("
                                   + ("1 launch" if L <= 16384 else "4 launches: four-step DFT, sliced gradients, assembly") + ")")}

@@ -173,10 +173,11 @@ s4_status s4_fft_conv_apply(const float *u, const void *workspace,
  *   caller-owned, contents irrelevant on entry. L <= 8192: 2 H 2L 8 bytes (a
  *   per-channel accumulator of the spectrum products and a per-channel
  *   scratch; one launch). L > 8192: the convolution workspace of (H, L) plus
- *   H L 4 bytes; per batch row b the spectrum of the zero-padded u[b] is
- *   prepared as if it were the kernel and the adjoint convolution of dy[b]
- *   gives that row's share of dK (2-3 launches per row). Either way the rows
- *   are summed in a fixed order (deterministic).
+ *   2 H L 4 bytes; per pair of batch rows the spectrum of the zero-padded
+ *   complex signal u[b] + i u[b+1] is prepared as if it were a kernel
+ *   spectrum, and the real part of the adjoint convolution of dy[b], dy[b+1]
+ *   with it is the two rows' share of dK (3 launches per row pair). Either
+ *   way the rows are summed in a fixed order (deterministic).
  *   Errors: null pointers, Bt/H < 1, misalignment, overlapping buffers ->
  *   S4_ERR_INVALID_ARG; workspace too small or misaligned ->
  *   S4_ERR_WORKSPACE.

@@ -668,16 +668,20 @@ cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const fl
 namespace {
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// dK += r (float4; n a multiple of 4)
-__global__ void k_accumulate(float *__restrict__ dK, const float *__restrict__ r, size_t n4) {
+// dK = r (first) or dK += r (float4; n a multiple of 4)
+__global__ void k_accumulate(float *__restrict__ dK, const float *__restrict__ r, size_t n4, bool first) {
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
-        float4 a = reinterpret_cast<float4 *>(dK)[i];
         const float4 b = reinterpret_cast<const float4 *>(r)[i];
-        a.x += b.x;
-        a.y += b.y;
-        a.z += b.z;
-        a.w += b.w;
-        reinterpret_cast<float4 *>(dK)[i] = a;
+        if (first) {
+            reinterpret_cast<float4 *>(dK)[i] = b;
+        } else {
+            float4 a = reinterpret_cast<float4 *>(dK)[i];
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+            reinterpret_cast<float4 *>(dK)[i] = a;
+        }
     }
 }
 // dD[h] = dK[h, 0]
@@ -686,21 +690,26 @@ __global__ void k_lag0(const float *__restrict__ dK, int H, int L, float *__rest
     if (h < H) dD[h] = dK[(size_t)h * L];
 }
 
-// L > 8192: per batch row b, the spectrum of the zero-padded u[b] rows is
-// prepared as if they were the kernel, and the adjoint convolution applied to
-// dy[b] gives sum_{t >= s} u[b, h, t - s] dy[b, h, t] = the row's share of
-// dK[h, s]; the shares are added in batch order.
+// L > 8192, per pair of batch rows (b, b + 1): the spectrum Z_u of the
+// zero-padded complex signal u[b] + i u[b + 1] is prepared as if it were a
+// kernel spectrum, and the adjoint convolution of the row pair dy[b], dy[b+1]
+// (packed dy[b] + i dy[b + 1], multiplied by conj(Z_u)) has as its real part
+//   sum_t dy[b,h,t] u[b,h,t-s] + sum_t dy[b+1,h,t] u[b+1,h,t-s],
+// the two rows' shares of dK[h, s] (the imaginary part holds cross terms and
+// goes to scratch). An odd last row uses the real spectrum of u[b] alone.
+// The shares are added in batch order.
 cudaError_t run_corr_long(const float *u, const float *dy, int Bt, int H, int L, float *dK, float *dD, void *ws,
                           cudaStream_t st) {
     void *spec = ws;
     float *r = reinterpret_cast<float *>(static_cast<char *>(ws) + align256(conv_workspace_bytes(H, L)));
     const size_t row = (size_t)H * L;
     cudaError_t e = cudaSuccess;
-    for (int b = 0; b < Bt && e == cudaSuccess; ++b) {
-        e = launch_kspec(u + b * row, nullptr, H, L, spec, st);
-        if (e == cudaSuccess) e = launch_fftconv(dy + b * row, spec, 1, H, L, b == 0 ? dK : r, st, true);
-        if (e == cudaSuccess && b > 0) {
-            k_accumulate<<<1184, 256, 0, st>>>(dK, r, row / 4);
+    for (int b = 0; b < Bt && e == cudaSuccess; b += 2) {
+        const int nb = (b + 1 < Bt) ? 2 : 1;
+        e = launch_kspec(u + b * row, nullptr, H, L, spec, st, nb == 2 ? u + (b + 1) * row : nullptr);
+        if (e == cudaSuccess) e = launch_fftconv(dy + b * row, spec, nb, H, L, r, st, true);
+        if (e == cudaSuccess) {
+            k_accumulate<<<1184, 256, 0, st>>>(dK, r, row / 4, b == 0);
             e = cudaGetLastError();
         }
     }
@@ -713,7 +722,7 @@ cudaError_t run_corr_long(const float *u, const float *dy, int Bt, int H, int L,
 }  // namespace
 
 size_t corr_workspace_bytes(int H, int L) {
-    if (L > 8192) return align256(conv_workspace_bytes(H, L)) + align256((size_t)H * L * sizeof(float));
+    if (L > 8192) return align256(conv_workspace_bytes(H, L)) + align256((size_t)2 * H * L * sizeof(float));
     return 2 * (((size_t)H * 2 * L * sizeof(float2) + 255) & ~size_t(255));
 }
 

@@ -14,8 +14,10 @@ struct ConvGeom { int C; int lg; bool tw0_global; };
 ConvGeom conv_geom(int L);
 size_t conv_workspace_bytes(int H, int L);
 
-// spectrum of K + D delta_0 (D may be null: no feed-through) into ws
-cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st);
+// spectrum of K + D delta_0 (D may be null: no feed-through) into ws; with Ki
+// (L > 8192 only) the spectrum of the complex signal K + i Ki instead
+cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st,
+                         const float *Ki = nullptr);
 // adjoint: the correlation with the same spectrum (conjugated), y[s] = sum_{t>=s} K[t-s] u[t] + D u[s]
 cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L, float *y, cudaStream_t st,
                            bool adjoint = false);

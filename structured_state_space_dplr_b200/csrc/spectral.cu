@@ -83,10 +83,12 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // spec[h][c][pos] = (FFT_2L(K_h zero-padded)[f] + D_h) / 2L for the frequency
 // f = C f' + c held at pos: the spectrum of K + D delta_0, so the convolution
 // adds the D u term with no extra pass over u.
-template <int LG, int C, bool TW0G>
+// CPLX: the input is the complex signal K + i Ki (Ki [H, L]); its spectrum
+// then has no conjugate symmetry, which the convolution does not assume.
+template <int LG, int C, bool TW0G, bool CPLX = false>
 __global__ void __launch_bounds__(threads_for<LG>())
-k_kspec(const float *__restrict__ K, const float *__restrict__ D, int H, int L, float2 *__restrict__ spec,
-        const float2 *__restrict__ tw0g) {
+k_kspec(const float *__restrict__ K, const float *__restrict__ Ki, const float *__restrict__ D, int H, int L,
+        float2 *__restrict__ spec, const float2 *__restrict__ tw0g) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
     extern __shared__ float2 sm[];
     const Smem s = carve<LG, TW0G>(sm);
@@ -99,14 +101,19 @@ k_kspec(const float *__restrict__ K, const float *__restrict__ D, int H, int L, 
     const float scale = 1.0f / (float)(C * m);
     for (int h = slot; h < H; h += nslots) {
         const float *Kh = K + (size_t)h * L;
+        const float *Kih = CPLX ? Ki + (size_t)h * L : nullptr;
         const float Dh = D != nullptr ? __ldg(D + h) : 0.0f;
         forward_first<LG, T>(s.buf, t0, s.pre, [&](int k) {
-            float2 v = make_float2(__ldg(Kh + k), 0.0f);
+            float2 v = make_float2(__ldg(Kh + k), CPLX ? __ldg(Kih + k) : 0.0f);
             static_for<1, C / 2>([&](auto r) {
                 const float kr = __ldg(Kh + k + r * m);
                 const float2 w = s.wcr[r];
-                v.x = fmaf(kr, w.x, v.x);
-                v.y = fmaf(kr, w.y, v.y);
+                if constexpr (CPLX) {
+                    v = cadd(v, cmul(make_float2(kr, __ldg(Kih + k + r * m)), w));
+                } else {
+                    v.x = fmaf(kr, w.x, v.x);
+                    v.y = fmaf(kr, w.y, v.y);
+                }
             });
             return v;
         });
@@ -430,8 +437,10 @@ k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int
 // spec4_index order, rank c holding (FFT_N(K + D delta_0))[4f + c] / N. One
 // CTA per (channel, rank pair), persistent; K's two chunks enter as the
 // convolution's input rows do.
+template <bool CPLX>
 __global__ void __launch_bounds__(pair_threads<kQuadLG>(), 1)
-k_kspec_quad(const float *__restrict__ K, const float *__restrict__ D, int H, float2 *__restrict__ spec) {
+k_kspec_quad(const float *__restrict__ K, const float *__restrict__ Ki, const float *__restrict__ D, int H,
+             float2 *__restrict__ spec) {
     constexpr int LG = kQuadLG, m = 1 << LG, L = 2 * m;
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     extern __shared__ float2 sm[];
@@ -444,11 +453,13 @@ k_kspec_quad(const float *__restrict__ K, const float *__restrict__ D, int H, fl
     for (int it = blockIdx.x; it < 2 * H; it += gridDim.x) {
         const int h = it >> 1, cr = it & 1;
         const float *Kh = K + (size_t)h * L;
+        const float *Kih = CPLX ? Ki + (size_t)h * L : nullptr;
         float2 v0[R0], v1[R0];
         static_for<0, R0>([&](auto p) {
             const int k = j + p * S0;
-            quad_inputs<decltype(p)::value>(cr, make_float2(__ldg(Kh + k), 0.0f),
-                                           make_float2(__ldg(Kh + k + m), 0.0f), v0[p], v1[p]);
+            quad_inputs<decltype(p)::value>(cr, make_float2(__ldg(Kh + k), CPLX ? __ldg(Kih + k) : 0.0f),
+                                           make_float2(__ldg(Kh + k + m), CPLX ? __ldg(Kih + k + m) : 0.0f),
+                                           v0[p], v1[p]);
         });
         if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
         else first_pass_halves2<LG, true>(s, v0, v1, j, tc[j]);
@@ -598,13 +609,16 @@ struct ConvKernels {
     static constexpr int T = threads_for<LG>();
     static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>(TW0G);
     static constexpr size_t smem_conv = smem + (STAGE ? 2 * sizeof(float) * (size_t)(C * (1 << LG) / 2) : 0);
-    static LaunchInfo info_conv, info_kspec;
+    static LaunchInfo info_conv, info_kspec, info_kspec_c;
 
     static LaunchInfo info_kspec_pair;
 
-    static cudaError_t kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st) {
+    // Ki non-null: the spectrum of K + i Ki (cluster paths only)
+    static cudaError_t kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st,
+                             const float *Ki = nullptr) {
         float2 *spec = (float2 *)ws;
         if constexpr (C == 2 && !TW0G && LG <= 13) {
+            if (Ki != nullptr) return cudaErrorInvalidValue;
             // the one-CTA convolution's spectrum: persistent, one channel per CTA at a time
             auto kern = k_kspec_pair<LG>;
             constexpr size_t psmem = pair_smem_bytes<LG>(0);
@@ -621,15 +635,15 @@ struct ConvKernels {
             cudaError_t e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
-        auto kern = k_kspec<LG, C, TW0G>;
+        auto kern = Ki != nullptr ? k_kspec<LG, C, TW0G, true> : k_kspec<LG, C, TW0G, false>;
         int res = 0;
-        cudaError_t e = resident_units(kern, info_kspec, 1, T, smem, &res);
+        cudaError_t e = resident_units(kern, Ki != nullptr ? info_kspec_c : info_kspec, 1, T, smem, &res);
         if (e != cudaSuccess) return e;
         // whole rank groups: nslots CTAs per rank
         int nslots = res / C;
         if (nslots < 1) nslots = 1;
         if (nslots > H) nslots = H;
-        kern<<<nslots * C, T, smem, st>>>(K, D, H, L, spec, (const float2 *)tw0g);
+        kern<<<nslots * C, T, smem, st>>>(K, Ki, D, H, L, spec, (const float2 *)tw0g);
         return cudaGetLastError();
     }
 
@@ -668,6 +682,7 @@ struct ConvKernels {
 };
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_conv;
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec;
+template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec_c;
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_pair[2];
 template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec_pair;
 
@@ -745,14 +760,17 @@ size_t conv_workspace_bytes(int H, int L) {
     X(65536, 14, 8, true, false)
 
 namespace {
-LaunchInfo g_quad_conv[2], g_quad_kspec;
+LaunchInfo g_quad_conv[2], g_quad_kspec[2];
 
-cudaError_t quad_kspec(const float *K, const float *D, int H, void *ws, cudaStream_t st) {
+// Ki non-null: the spectrum of K + i Ki
+cudaError_t quad_kspec(const float *K, const float *D, int H, void *ws, cudaStream_t st, const float *Ki) {
     constexpr size_t smem = pair_smem_bytes<kQuadLG>(0);
+    const bool cplx = Ki != nullptr;
+    auto kern = cplx ? k_kspec_quad<true> : k_kspec_quad<false>;
     int res = 0;
-    cudaError_t e = resident_units(k_kspec_quad, g_quad_kspec, 1, pair_threads<kQuadLG>(), smem, &res);
+    cudaError_t e = resident_units(kern, g_quad_kspec[cplx], 1, pair_threads<kQuadLG>(), smem, &res);
     if (e != cudaSuccess) return e;
-    k_kspec_quad<<<res < 2 * H ? res : 2 * H, pair_threads<kQuadLG>(), smem, st>>>(K, D, H, (float2 *)ws);
+    kern<<<res < 2 * H ? res : 2 * H, pair_threads<kQuadLG>(), smem, st>>>(K, Ki, D, H, (float2 *)ws);
     return cudaGetLastError();
 }
 
@@ -771,10 +789,10 @@ cudaError_t quad_conv(const float *u, const void *ws, int Bt, int H, float *y, b
 }
 }  // namespace
 
-cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st) {
-    if (L == 2 << kQuadLG) return quad_kspec(K, D, H, ws, st);
+cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st, const float *Ki) {
+    if (L == 2 << kQuadLG) return quad_kspec(K, D, H, ws, st, Ki);
     switch (L) {
-#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::kspec(K, D, H, L, ws, st);
+#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::kspec(K, D, H, L, ws, st, Ki);
         S4_CONV_CASES(X)
 #undef X
         default: return cudaErrorInvalidValue;
