@@ -135,10 +135,17 @@ k_kspec(const float *__restrict__ K, const float *__restrict__ Ki, const float *
 // STAGE: the input rows of the next row pair are copied to shared memory with
 // cp.async while the current pair is transformed (used when the whole pair,
 // 8 L bytes, fits next to the transform).
+// Without STAGE (L >= 32768) the first-pass inputs of all C ranks are formed
+// cooperatively: for each row pair, CTA c combines the chunks of the
+// positions k in its slice [c m/C, (c+1) m/C) for every rank r,
+//   v_r[k] = sum_{q < C/2} W_C^{q r} (u0[k + q m] + i u1[k + q m]),
+// into the cluster's slot of the scratch xs [C][m]; after a cluster barrier
+// each CTA reads its own rank's m inputs contiguously (each input value is
+// read from L2 once per cluster instead of once per CTA).
 template <int LG, int C, bool TW0G, bool STAGE>
 __global__ void __launch_bounds__(threads_for<LG>())
 k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
-          float *__restrict__ y, const float2 *__restrict__ tw0g, float conj_sign) {
+          float *__restrict__ y, const float2 *__restrict__ tw0g, float conj_sign, float2 *__restrict__ xs) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
     constexpr int SL = m / C;                     // combine slice per rank
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
@@ -183,39 +190,47 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
         const float *u0, *u1; bool has1; int h, b0;
         rows(pr, u0, u1, has1, h, b0);
         // ---- forward pass 0: x = u0 + i u1 (zero-padded to 2L), rank c's share
+        float2 *xsc = nullptr;
         if constexpr (STAGE) {
             cp_async_wait_all();
             __syncthreads();
+        } else {   // the cooperative combination of the chunks (see above)
+            if (!first) cluster_wait();   // the partners are done reading this CTA's buffer
+            xsc = xs + (size_t)cl * C * m;
+            constexpr int SLC = m / C;
+            for (int i = threadIdx.x; i < SLC; i += T) {
+                const int k = c * SLC + i;
+                float2 x[C];
+                static_for<0, C / 2>([&](auto q) {
+                    x[q] = make_float2(__ldg(u0 + k + q * m), has1 ? __ldg(u1 + k + q * m) : 0.0f);
+                });
+                static_for<C / 2, C>([&](auto q) { x[q] = make_float2(0.0f, 0.0f); });
+                dft<C, -1>(x);   // x[r] = sum_q W_C^{q r} x_q
+                static_for<0, C>([&](auto r) { xsc[(size_t)r * m + k] = x[r]; });
+            }
+            cluster_arrive_release();
+            cluster_wait();
         }
         auto fetch = [&](int k) {
-            float2 v;
             if constexpr (STAGE) {
-                v = make_float2(stage[k], stage[L + k]);
+                float2 v = make_float2(stage[k], stage[L + k]);
+                static_for<1, C / 2>([&](auto r) {
+                    v = cadd(v, cmul(make_float2(stage[k + r * m], stage[L + k + r * m]), s.wcr[r]));
+                });
+                return v;
             } else {
-                v = make_float2(__ldg(u0 + k), has1 ? __ldg(u1 + k) : 0.0f);
+                return __ldcg(xsc + (size_t)c * m + k);
             }
-            static_for<1, C / 2>([&](auto r) {
-                float a, b;
-                if constexpr (STAGE) {
-                    a = stage[k + r * m];
-                    b = stage[L + k + r * m];
-                } else {
-                    a = __ldg(u0 + k + r * m);
-                    b = has1 ? __ldg(u1 + k + r * m) : 0.0f;
-                }
-                v = cadd(v, cmul(make_float2(a, b), s.wcr[r]));
-            });
-            return v;
         };
         if constexpr (S0 == T) {
-            // one group per thread: compute it, then wait until the partner
-            // ranks have finished reading this CTA's buffer (previous combine)
+            // one group per thread: compute it, then (staged path) wait until
+            // the partner ranks have finished reading this CTA's buffer
             float2 x[R0];
             first_group<LG>(x, threadIdx.x, t0, s.pre, fetch);
-            if (!first) cluster_wait();
+            if (STAGE && !first) cluster_wait();
             store_first_group<LG>(s.buf, x, threadIdx.x);
         } else {
-            if (!first) cluster_wait();
+            if (STAGE && !first) cluster_wait();
             forward_first<LG, T>(s.buf, t0, s.pre, fetch);
         }
         first = false;
@@ -604,6 +619,10 @@ cudaError_t launch_clustered(Kern kern, int C, int nclusters, int T, size_t smem
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 // ---- convolution / kspec instantiation for one L ----
+// clusters of the L >= 32768 convolution launched at most (each owns a 2L
+// complex slot of scratch in the workspace for its cooperative first pass)
+constexpr int kMaxConvClusters = 24;
+
 template <int LG, int C, bool TW0G, bool STAGE>
 struct ConvKernels {
     static constexpr int T = threads_for<LG>();
@@ -668,6 +687,9 @@ struct ConvKernels {
         const float2 *tw0g = TW0G
             ? (const float2 *)((const char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)))
             : nullptr;
+        float2 *xs = STAGE ? nullptr
+                           : (float2 *)((char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)) +
+                                        (TW0G ? align256((size_t)C * (1 << LG) * sizeof(float2)) : 0));
         auto kern = k_fftconv<LG, C, TW0G, STAGE>;
         int res = 0;
         cudaError_t e = resident_units(kern, info_conv, C, T, smem_conv, &res);
@@ -675,7 +697,9 @@ struct ConvKernels {
         const long long npairs = (long long)H * ((Bt + 1) / 2);
         int ncl = res;
         if ((long long)ncl > npairs) ncl = (int)npairs;
-        e = launch_clustered(kern, C, ncl, T, smem_conv, st, u, spec, Bt, H, L, y, tw0g, adjoint ? -1.0f : 1.0f);
+        if (ncl > kMaxConvClusters) ncl = kMaxConvClusters;   // scratch slots in the workspace
+        e = launch_clustered(kern, C, ncl, T, smem_conv, st, u, spec, Bt, H, L, y, tw0g, adjoint ? -1.0f : 1.0f,
+                             xs);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
@@ -734,6 +758,7 @@ size_t conv_workspace_bytes(int H, int L) {
     ConvGeom g = conv_geom(L);
     size_t b = align256((size_t)H * 2 * L * sizeof(float2));
     if (g.tw0_global) b += align256((size_t)2 * L * sizeof(float2));
+    if (L >= 32768) b += align256((size_t)kMaxConvClusters * 2 * L * sizeof(float2));   // cluster scratch
     return b;
 }
 
