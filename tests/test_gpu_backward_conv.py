@@ -38,7 +38,7 @@ def test_adjoint_convolution(L, Bt, H):
 
 
 @pytest.mark.parametrize("L,Bt,H", [(16, 3, 2), (128, 2, 3), (1024, 5, 2), (4096, 4, 2), (8192, 3, 1),
-                                    (16384, 3, 2), (32768, 2, 1), (65536, 2, 1)])
+                                    (16384, 3, 2), (32768, 2, 1), (65536, 2, 1), (16384, 1, 3)])
 def test_kernel_and_skip_gradients(L, Bt, H):
     """L <= 8192: the batch correlation kernel; longer L: per batch row, the
     adjoint convolution with u's spectrum (the cluster transforms)."""

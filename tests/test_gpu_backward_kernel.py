@@ -48,6 +48,15 @@ def test_random_dplr_parameter_gradients(L):
     _check(g, ref, slice(None))
 
 
+def test_four_step_gradients_single_channel():
+    """L = 32768 with H = 1: 64 frequency slices for the one channel."""
+    inp = s4inputs.random_dplr(91, H=1, Nh=3, L=32768, Bt=1)
+    dK = np.random.default_rng(5).standard_normal((1, 32768))
+    g = _gpu_grad(inp, dK)
+    ref = workloads.dplr_kernel_param_grad(inp, dK)
+    _check(g, ref, slice(None))
+
+
 def test_hippo_parameter_gradients_one_channel():
     """HiPPO-LegS modes (Nh = 32, |Im Lambda| up to ~1300), L = 1024."""
     inp = s4inputs.make_inputs(1, with_u=False)
@@ -80,7 +89,7 @@ def test_layer_backward_composes_to_finite_differences():
 S4D_KEYS = ("A", "B", "C", "log_dt")
 
 
-@pytest.mark.parametrize("L,Nh", [(16, 4), (64, 32), (1024, 32), (8192, 32), (16384, 7), (65536, 3)])
+@pytest.mark.parametrize("L,Nh", [(16, 4), (64, 32), (1024, 32), (8192, 32), (16384, 7), (65536, 3), (256, 1)])
 def test_s4d_parameter_gradients(L, Nh):
     """The S4D kernel's backward against central differences of the oracle's
     fp64 Vandermonde sum (S4D-Lin modes: a_n = -1/2 + i pi n)."""

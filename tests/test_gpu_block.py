@@ -102,7 +102,7 @@ def test_glu_projection_full_size_sampled():
         assert (np.abs(o[b:b + 1][:, :, ts] - ref) <= _glu_bound(ys, p["W"], p["bias"])).all()
 
 
-@pytest.mark.parametrize("H,L,Bt", [(4, 1024, 2), (64, 256, 3)])
+@pytest.mark.parametrize("H,L,Bt", [(4, 1024, 2), (64, 256, 3), (100, 16, 1)])
 def test_block_forward_dplr(H, L, Bt):
     """The composed block with the DPLR layer: norm -> convolution with the
     aliased kernel (and D) -> projection, GLU, residual."""

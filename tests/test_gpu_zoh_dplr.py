@@ -17,12 +17,14 @@ KEYS = ["Lambda", "P", "Q", "B", "C", "log_dt"]
 def _inputs(kind, L):
     if kind == "hippo":          # HiPPO-LegS, H = 4, Nh = 32 (the full 64-state system)
         return s4inputs.make_inputs(1, L=L)
+    if kind == "one":            # a single stored mode (N = 2)
+        return s4inputs.random_dplr(23, H=2, Nh=1, L=L, Bt=1)
     if kind == "small":          # Nh = 5: the state is padded inside the kernel
         return s4inputs.random_dplr(21, H=3, Nh=5, L=L, Bt=2)
     return s4inputs.random_dplr(22, H=3, Nh=32, L=L, Bt=2, re_min=-0.5, re_max=-0.02)
 
 
-@pytest.mark.parametrize("kind", ["hippo", "small", "random"])
+@pytest.mark.parametrize("kind", ["hippo", "small", "random", "one"])
 def test_discretize_zoh_matches_oracle(kind):
     import structured_state_space_dplr_b200 as s4
     inp = _inputs(kind, 64)
@@ -38,7 +40,7 @@ def test_discretize_zoh_matches_oracle(kind):
 
 
 @pytest.mark.parametrize("kind,L", [("hippo", 1024), ("small", 16), ("small", 64), ("random", 256),
-                                    ("random", 4096)])
+                                    ("random", 4096), ("one", 128)])
 def test_kernel_zoh_matches_oracle(kind, L):
     """L = 16 (shorter than one 64-step block), whole blocks, long L with
     slowly decaying modes (many r <- r Abar^64 steps)."""
