@@ -357,3 +357,39 @@ def test_fd_gradient_matches_s4d_closed_form_derivative():
              for n in range(Nh))
     ref_dt = float(np.dot(dK, G))
     assert abs(g1 - ref_dt) <= 1e-7 * abs(ref_dt)
+
+
+def test_s4d_gradient_closed_forms_match_finite_differences():
+    """The closed forms of the S4D kernel's gradient (with V_n = sum_k G[k]
+    Abar_n^k, W_n = sum_k k G[k] Abar_n^k, r_n = (e^{dt a_n} - 1)/a_n:
+    dC = 2 conj(Bbar V), dB = 2 conj(C r V), dA = 2 conj(C B dt^2 phi1'(dt a) V
+    + C Bbar dt W), dlog_dt = 2 dt Re sum (C B Abar V + C Bbar a W)) against
+    central differences of the oracle's Vandermonde sum; one mode sits in the
+    small-|dt a| range where phi1' is taken from its series."""
+    rng = np.random.default_rng(12)
+    Nh, L, dt = 4, 40, 0.05
+    a = -rng.uniform(0.05, 1.0, Nh) + 1j * rng.uniform(-20, 20, Nh)
+    a[1] = -2e-3 + 1e-3j          # |dt a| = 1.1e-4: the series branch of phi1'
+    B = rng.standard_normal(Nh) + 1j * rng.standard_normal(Nh)
+    C = rng.standard_normal(Nh) + 1j * rng.standard_normal(Nh)
+    G = rng.standard_normal(L)
+    inp = dict(H=1, L=L, A=a[None].astype(np.complex64), B=B[None].astype(np.complex64),
+               C=C[None].astype(np.complex64), log_dt=np.array([np.log(dt)], np.float32))
+    ref = workloads.s4d_kernel_param_grad(inp, G[None])
+    a, B, C = (inp[k][0].astype(np.complex128) for k in ("A", "B", "C"))
+    dt = float(np.exp(np.float64(inp["log_dt"][0])))
+    Ab, Bb = ssm.zoh_diag(a, B, dt)
+    k = np.arange(L)
+    V = np.array([np.sum(G * Ab[n] ** k) for n in range(Nh)])
+    W = np.array([np.sum(k * G * Ab[n] ** k) for n in range(Nh)])
+    r = Bb / B
+    x = dt * a
+    phi1p = np.where(np.abs(x) < 1e-3, 0.5 + x / 3 + x ** 2 / 8 + x ** 3 / 30 + x ** 4 / 144,
+                     (x * np.exp(x) - (np.exp(x) - 1)) / np.where(x == 0, 1, x) ** 2)
+    dC = 2 * np.conj(Bb * V)
+    dB = 2 * np.conj(C * r * V)
+    dA = 2 * np.conj(C * B * dt ** 2 * phi1p * V + C * Bb * dt * W)
+    dld = 2 * dt * np.real(np.sum(C * B * Ab * V + C * Bb * a * W))
+    for name, mine in (("C", dC), ("B", dB), ("A", dA)):
+        assert np.abs(mine - ref[name][0]).max() <= 1e-6 * np.abs(ref[name][0]).max(), name
+    assert abs(dld - ref["log_dt"][0]) <= 1e-6 * abs(ref["log_dt"][0])
