@@ -393,3 +393,51 @@ def test_s4d_gradient_closed_forms_match_finite_differences():
     for name, mine in (("C", dC), ("B", dB), ("A", dA)):
         assert np.abs(mine - ref[name][0]).max() <= 1e-6 * np.abs(ref[name][0]).max(), name
     assert abs(dld - ref["log_dt"][0]) <= 1e-6 * abs(ref["log_dt"][0])
+
+
+def test_dplr_gradient_closed_forms_match_finite_differences():
+    """The closed forms of the gradient through the DPLR kernel (the
+    generating function of "The S4 kernel, from scratch" §4 differentiated:
+    g_j = (2/L) DFT(dK)_j, the Woodbury partials e_v, a_v = conj(g_j) e_v,
+    per stored mode S_v = sum_j a_v r' + conj(a_v r), S2_v likewise with the
+    squares, the Nyquist closed form) against central differences of the
+    oracle's dense aliased kernel."""
+    inp = s4inputs.random_dplr(31, H=1, Nh=3, L=32, Bt=1)
+    L = inp["L"]
+    dK = np.random.default_rng(2).standard_normal(L)
+    ref = workloads.dplr_kernel_param_grad(inp, dK[None])
+    lam, P, Q, B, C = (inp[k][0].astype(np.complex128) for k in ("Lambda", "P", "Q", "B", "C"))
+    dt = float(np.exp(np.float64(inp["log_dt"][0])))
+    full = lambda x: np.concatenate([x, np.conj(x)])
+    lf = full(lam)
+    vs = [C * B, C * P, np.conj(Q) * B, np.conj(Q) * P]    # v00, v01, v10, v11 of the stored modes
+    vf = [full(v) for v in vs]
+    G = np.fft.fft(dK)
+    S = [np.zeros(3, complex) for _ in range(4)]
+    S2 = [np.zeros(3, complex) for _ in range(4)]
+    dld = 0.0
+    for j in range(L // 2):
+        g = (1.0 if j == 0 else 2.0) / L * G[j]
+        t = np.tan(np.pi * j / L)
+        s = 1j * 2.0 * t / dt
+        c = 1.0 + 1j * t
+        ri = 1.0 / (s - lf)
+        k = [np.sum(v * ri) for v in vf]
+        den = 1.0 + k[3]
+        e = [c, -c * k[2] / den, -c * k[1] / den, c * k[1] * k[2] / den ** 2]
+        rn, rc = 1.0 / (s - lam), 1.0 / (s - np.conj(lam))
+        for v in range(4):
+            a = np.conj(g) * e[v]
+            S[v] += a * rc + np.conj(a * rn)
+            S2[v] += a * rc ** 2 + np.conj(a * rn ** 2)
+        dld += np.real(np.conj(g) * s * sum(e[v] * np.sum(vf[v] * ri ** 2) for v in range(4)))
+    gN = np.real(G[L // 2]) / L
+    dC = np.conj(B) * S[0] + np.conj(P) * S[1] + gN * dt * np.conj(B)
+    dB = np.conj(C) * S[0] + Q * S[2] + gN * dt * np.conj(C)
+    dP = np.conj(C) * S[1] + Q * S[3]
+    dQ = B * np.conj(S[2]) + P * np.conj(S[3])
+    dL = sum(np.conj(vs[v]) * S2[v] for v in range(4))
+    dld += gN * dt * np.real(np.sum(C * B))
+    for name, mine in (("C", dC), ("B", dB), ("P", dP), ("Q", dQ), ("Lambda", dL)):
+        assert np.abs(mine - ref[name][0]).max() <= 1e-6 * np.abs(ref[name][0]).max(), name
+    assert abs(dld - ref["log_dt"][0]) <= 1e-6 * abs(ref["log_dt"][0])
