@@ -452,41 +452,6 @@ def run_gpu(args, rank, world, local_rank):
              "layernorm_gbs": 8 * alg["elements"] / (kst[0] * 1e-3) / 1e9,
              "calls": "s4_layernorm_channels + s4_fft_conv_apply + s4_glu_projection_residual, one launch each"}
 
-    # the set-up variants of the DPLR layer (timed once per call, not per
-    # batch): the ZOH discretisation and its truncated kernel (fp64 matrix
-    # exponential per channel, Nh <= 32), and C~ = C (I - Abar^L) with the
-    # truncated kernel from the Cauchy path. A failure here is reported in the
-    # line, never fatal to it.
-    variants = None
-    if not s4d and c["N"] // 2 <= 32:
-        try:
-            d = sets[0]
-            pk = [d[k] for k in ("Lambda", "P", "Q", "B", "C", "log_dt")]
-            Kz = torch.empty(H, L, device=dev)
-
-            def timed(fn, reps=3):
-                fn()
-                torch.cuda.synchronize()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                for _ in range(reps):
-                    fn()
-                e1.record()
-                torch.cuda.synchronize()
-                return e0.elapsed_time(e1) * 1e3 / reps
-
-            def ct_kernel():
-                Ct = s4.dplr_ctilde(d["Lambda"], d["P"], d["Q"], d["C"], d["log_dt"], L)
-                s4.kernel_dplr(d["Lambda"], d["P"], d["Q"], d["B"], Ct, d["log_dt"], L, out=Kz)
-
-            variants = {
-                "zoh_kernel_us": timed(lambda: s4.kernel_dplr_zoh(*pk, L, out=Kz)),
-                "zoh_discretize_us": timed(lambda: s4.dplr_discretize_zoh(*pk)),
-                "ctilde_truncated_kernel_us": timed(ct_kernel),
-                "calls": "s4_kernel_dplr_zoh; s4_dplr_discretize_zoh; s4_dplr_ctilde + s4_kernel_dplr"}
-        except Exception as exc:   # noqa: BLE001 - reported, the main line stands
-            variants = {"error": f"{type(exc).__name__}: {exc}"}
-
     # recurrent view (decode) of the same layer: up to 1024 tokens from a zero
     # state, as one s4_recurrent_scan and as single-token steps from a graph
     d = sets[0]
@@ -526,6 +491,41 @@ def run_gpu(args, rank, world, local_rank):
               "step_us_per_token": e[2].elapsed_time(e[3]) * 1e3 / T,
               "step_launch": f"{T} s4_recurrent_step launches replayed from one CUDA graph"}
     del g_steps
+
+    # the set-up variants of the DPLR layer (timed once per call, not per
+    # batch): the ZOH discretisation and its truncated kernel (fp64 matrix
+    # exponential per channel, Nh <= 32), and C~ = C (I - Abar^L) with the
+    # truncated kernel from the Cauchy path. A failure here is reported in the
+    # line, never fatal to it.
+    variants = None
+    if not s4d and c["N"] // 2 <= 32:
+        try:
+            d = sets[0]
+            pk = [d[k] for k in ("Lambda", "P", "Q", "B", "C", "log_dt")]
+            Kz = torch.empty(H, L, device=dev)
+
+            def timed(fn, reps=3):
+                fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(reps):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                return e0.elapsed_time(e1) * 1e3 / reps
+
+            def ct_kernel():
+                Ct = s4.dplr_ctilde(d["Lambda"], d["P"], d["Q"], d["C"], d["log_dt"], L)
+                s4.kernel_dplr(d["Lambda"], d["P"], d["Q"], d["B"], Ct, d["log_dt"], L, out=Kz)
+
+            variants = {
+                "zoh_kernel_us": timed(lambda: s4.kernel_dplr_zoh(*pk, L, out=Kz)),
+                "zoh_discretize_us": timed(lambda: s4.dplr_discretize_zoh(*pk)),
+                "ctilde_truncated_kernel_us": timed(ct_kernel),
+                "calls": "s4_kernel_dplr_zoh; s4_dplr_discretize_zoh; s4_dplr_ctilde + s4_kernel_dplr"}
+        except Exception as exc:   # noqa: BLE001 - reported, the main line stands
+            variants = {"error": f"{type(exc).__name__}: {exc}"}
 
     times = max_over_ranks([ms, e2e_ms] + stage, dist, dev)
     if dist is not None:
