@@ -53,3 +53,33 @@ def test_job_throughput_is_total_over_slowest():
     # 2 ranks x 3 steps x 1000 elements in 2 ms (the slower rank) -> 3e6 elements/s
     assert bench.job_throughput(1000, 2, 3, 2.0) == pytest.approx(3.0e6)
     assert bench.max_over_ranks([1, 2]) == [1.0, 2.0]
+
+
+def test_recorded_traffic_follows_the_convolution_sources(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic is reported only while the hash of the
+    convolution's sources matches the one the counters were taken with."""
+    import bench
+    good = tmp_path / "traffic.txt"
+    good.write_text(f"kernel_source_sha256_16: {bench.kernel_source_hash()}\n"
+                    "dram_bytes_per_launch_full_size: 123456\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(good))
+    assert bench.recorded_traffic() == 123456.0
+    stale = tmp_path / "stale.txt"
+    stale.write_text("kernel_source_sha256_16: 0000000000000000\ndram_bytes_per_launch_full_size: 1\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(stale))
+    assert bench.recorded_traffic() is None
+
+
+def test_algorithmic_units_of_the_workloads():
+    """Per-step units behind the roofline: 8 B per element of u and y plus
+    16 B per (h, t) of spectrum for the convolution; 40 FLOP per (channel,
+    frequency < L/2, mode pair) for the Cauchy sums; 4 per (channel, k, mode)
+    for the Vandermonde product."""
+    import bench
+    import s4inputs
+    a = bench.algorithmic(s4inputs.CONFIGS[2])
+    assert a["elements"] == 16 * 256 * 4096
+    assert a["conv_bytes"] == 8 * 16 * 256 * 4096 + 16 * 256 * 4096
+    assert a["kernel_flop"] == 40 * 256 * 2048 * 32
+    a5 = bench.algorithmic(s4inputs.CONFIGS[5])
+    assert a5["kernel_flop"] == 4 * 1024 * 8192 * 32
