@@ -106,7 +106,7 @@ __device__ __forceinline__ void arrive_expect_tx(uint64_t *m, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(umma::saddr(m)), "r"(bytes)
                  : "memory");
 }
-// 3-D tiled TMA load (no multicast) of the box at (x, y, z) into dst
+// 3-D tiled TMA load of the box at (x, y, z) into this CTA's shared memory only
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *m) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
@@ -114,7 +114,7 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(umma::saddr(m))
         : "memory");
 }
-// contiguous bulk copy global -> shared (no multicast); 16-byte aligned, size % 16 == 0
+// contiguous bulk copy global -> this CTA's shared memory; 16-byte aligned, size % 16 == 0
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *m) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                      umma::saddr(dst)),
