@@ -314,7 +314,10 @@ s4_status s4_forward_dplr_host(const float *u_host, const s4_c32 *Lambda, const 
  *
  * Arguments, layouts and errors are those of s4_fft_conv; in addition the
  * call returns S4_ERR_UNSUPPORTED when s4_fft_conv_workspace_size(H, L)
- * exceeds S4_STATIC_SCRATCH_BYTES (about H * L <= 2 M elements).
+ * exceeds S4_STATIC_SCRATCH_BYTES (about H * L <= 2 M elements), and
+ * S4_ERR_INVALID_ARG when u, K, D or y is not memory the current device can
+ * address as its own (a device buffer of another GPU, or unregistered host
+ * memory): the scratch used is the current device's.
  * ------------------------------------------------------------------------ */
 #define S4_STATIC_SCRATCH_BYTES (32u << 20)
 

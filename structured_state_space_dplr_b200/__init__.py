@@ -46,6 +46,13 @@ def _ptr(t):
 def _cuda(t, name, dtype=None):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
+    # the library launches on the current device's current stream (and the
+    # static-scratch entry point uses that device's scratch), so every
+    # operand must live there: a pointer of another device would be an
+    # illegal address on this one
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()} (use torch.cuda.device({t.device}))")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():

@@ -411,7 +411,10 @@ k_glu_projection_ws(const __grid_constant__ CUtensorMap tm_y, const __grid_const
         // ---------------- loader: raw y chunks (TMA) and W' image chunks (bulk)
         if (lane == 0) prefetch_tensormap(&tm_y);
         Ring rr, ss;
-        int issued = 0;
+        // copies issued so far, counted per ring right after each issue: an
+        // abort between the y copy and the W copy of one chunk leaves one
+        // more y copy than W copies in flight, and the drain must see it
+        int raw_issued = 0, w_issued = 0;
         bool ok = true;
         for (long long i = blockIdx.x; i < ntiles && ok; i += gridDim.x) {
             const Tile tl = tile_of(i, nnb, ntt, N);
@@ -421,6 +424,8 @@ k_glu_projection_ws(const __grid_constant__ CUtensorMap tm_y, const __grid_const
                     arrive_expect_tx(&rawfull[rr.slot], (uint32_t)(N * kKc * 4));
                     tma_load_3d(sm + kOffRaw + rr.slot * kRawBytes, &tm_y, tl.t0, c * kKc, tl.b, &rawfull[rr.slot]);
                 }
+                ++raw_issued;
+                rr.next(kR);
                 if (!(ok = __all_sync(0xffffffffu, ctl.wait(&opempty[ss.slot], ss.phase ^ 1u)))) break;
                 if (lane == 0) {
                     arrive_expect_tx(&wfull[ss.slot], 2 * kWImg);
@@ -428,18 +433,17 @@ k_glu_projection_ws(const __grid_constant__ CUtensorMap tm_y, const __grid_const
                               2 * kWImg, &wfull[ss.slot]);
                 }
                 __syncwarp();
-                ++issued;
-                rr.next(kR);
+                ++w_issued;
                 ss.next(kS);
             }
         }
         if (!ok && lane == 0) {   // let the copies in flight land before the CTA exits
-            for (int k = 1; k <= kR && k <= issued; ++k) {
-                const int u = issued - k;
+            for (int k = 1; k <= kR && k <= raw_issued; ++k) {
+                const int u = raw_issued - k;
                 umma::mbar_wait(&rawfull[u % kR], (uint32_t)((u / kR) & 1), kSpinLimit);
             }
-            for (int k = 1; k <= kS && k <= issued; ++k) {
-                const int u = issued - k;
+            for (int k = 1; k <= kS && k <= w_issued; ++k) {
+                const int u = w_issued - k;
                 umma::mbar_wait(&wfull[u % kS], (uint32_t)((u / kS) & 1), kSpinLimit);
             }
         }

@@ -41,6 +41,18 @@ cudaError_t scratch_of_current_device(void **out) {
 
 bool is_aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
+// Buffers of another device, or unregistered host memory, would be illegal
+// addresses for the kernels on the current device (whose scratch is used).
+bool on_current_device(const void *p, int dev) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();   // a failed query leaves its error behind: clear it
+        return false;
+    }
+    if (a.type == cudaMemoryTypeUnregistered) return false;
+    return a.type != cudaMemoryTypeDevice || a.device == dev;
+}
+
 bool ranges_overlap(const void *a, size_t an, const void *b, size_t bn) {
     const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
     return x < y + bn && y < x + an;
@@ -61,8 +73,17 @@ extern "C" s4_status s4_fft_conv_static(const float *u, const float *K, const fl
         ranges_overlap(y, nb, D, (size_t)H * sizeof(float)))
         return S4_ERR_INVALID_ARG;
     if (s4::conv_workspace_bytes(H, L) > (size_t)S4_STATIC_SCRATCH_BYTES) return S4_ERR_UNSUPPORTED;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        s4::record_cuda_error(e);
+        return S4_ERR_CUDA;
+    }
+    if (!on_current_device(u, dev) || !on_current_device(K, dev) || !on_current_device(D, dev) ||
+        !on_current_device(y, dev))
+        return S4_ERR_INVALID_ARG;
     void *ws = nullptr;
-    cudaError_t e = scratch_of_current_device(&ws);
+    e = scratch_of_current_device(&ws);
     if (e == cudaSuccess) e = s4::launch_kspec(K, D, H, L, ws, stream);
     if (e == cudaSuccess) e = s4::launch_fftconv(u, ws, Bt, H, L, y, stream);
     if (e != cudaSuccess) {

@@ -62,12 +62,23 @@ def test_recorded_traffic_follows_the_convolution_sources(tmp_path, monkeypatch)
     good = tmp_path / "traffic.txt"
     good.write_text(f"kernel_source_sha256_16: {bench.kernel_source_hash()}\n"
                     "dram_bytes_per_launch_full_size: 123456\n")
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(good))
-    assert bench.recorded_traffic() == 123456.0
+    monkeypatch.setitem(bench.TRAFFIC_FILES, 3, str(good))
+    assert bench.recorded_traffic(3) == 123456.0
     stale = tmp_path / "stale.txt"
     stale.write_text("kernel_source_sha256_16: 0000000000000000\ndram_bytes_per_launch_full_size: 1\n")
-    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(stale))
-    assert bench.recorded_traffic() is None
+    monkeypatch.setitem(bench.TRAFFIC_FILES, 3, str(stale))
+    assert bench.recorded_traffic(3) is None
+    assert bench.recorded_traffic(1) is None     # no capture recorded for that workload
+
+
+def test_launch_counts_and_reference_sample_sizes():
+    """Launches per forward step as the library issues them, and the
+    reference arm's per-step sample (about 1e9 multiply-adds of direct sum)."""
+    import bench
+    import s4inputs
+    C = s4inputs.CONFIGS
+    assert [bench.launches_per_step(C[k]) for k in (1, 2, 3, 4, 5)] == [2, 2, 4, 5, 3]
+    assert [bench.reference_chunk(C[k]) for k in (1, 2, 3, 4, 5)] == [4, 7, 1, 1, 1]
 
 
 def test_algorithmic_units_of_the_workloads():
