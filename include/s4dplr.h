@@ -279,7 +279,9 @@ s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P,
  *   nchunks        : >= 1 (clamped to the number of row pairs).
  *   h2d_stream, d2h_stream : caller-owned streams (may be `stream` itself,
  *                    which serialises the pipeline).
- * The call creates and releases a few CUDA events; it allocates no memory.
+ * The first call on each (host thread, device) creates the few CUDA events
+ * the pipeline orders itself with, and later calls from that thread reuse
+ * them (they live until the process exits); no call allocates memory.
  * Errors: as the device-buffer forms; null host pointers, overlapping host
  * buffers or nchunks < 1 -> S4_ERR_INVALID_ARG.
  * ------------------------------------------------------------------------ */

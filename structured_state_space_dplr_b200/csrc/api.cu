@@ -66,6 +66,26 @@ s4_status prepare_checks(const float *K, const float *D, int H, int L, const voi
     return S4_OK;
 }
 
+// Ordering events of the host-buffer pipeline, created once per (host
+// thread, device) and reused by every later call: an event may be recorded
+// again as soon as the waits on its previous record are enqueued, which the
+// pipeline does in order. They live until the process exits.
+cudaError_t pipeline_events(size_t n, cudaEvent_t **out) {
+    thread_local std::vector<cudaEvent_t> pools[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::vector<cudaEvent_t> &pool = pools[dev & 63];
+    while (pool.size() < n) {
+        cudaEvent_t ev = nullptr;
+        e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        pool.push_back(ev);
+    }
+    *out = pool.data();
+    return cudaSuccess;
+}
+
 // The convolution of a batch held in host memory. Chunk c (whole row pairs)
 // is uploaded on h2d, convolved on st once it has arrived and downloaded on
 // d2h once convolved, so uploads, convolutions and downloads of consecutive
@@ -81,10 +101,8 @@ cudaError_t conv_host_pipeline(const float *u_host, const void *ws, int Bt, int 
     const int pairs_per_chunk = (npairs + nchunks - 1) / nchunks;
     nchunks = (npairs + pairs_per_chunk - 1) / pairs_per_chunk;
     const size_t row = (size_t)H * L;
-    std::vector<cudaEvent_t> ev(2 * (size_t)nchunks + 1, nullptr);
-    cudaError_t e = cudaSuccess;
-    for (auto &x : ev)
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+    cudaEvent_t *ev = nullptr;   // [2 nchunks + 1]: upload c done, convolution c done, last download done
+    cudaError_t e = pipeline_events(2 * (size_t)nchunks + 1, &ev);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(h2d, start, 0);
     for (int c = 0; c < nchunks && e == cudaSuccess; ++c) {
         const int b0 = 2 * c * pairs_per_chunk;
@@ -98,10 +116,8 @@ cudaError_t conv_host_pipeline(const float *u_host, const void *ws, int Bt, int 
         if (e == cudaSuccess) e = cudaStreamWaitEvent(d2h, ev[2 * c + 1], 0);
         if (e == cudaSuccess) e = cudaMemcpyAsync(y_host + off, y_dev + off, bytes, cudaMemcpyDeviceToHost, d2h);
     }
-    if (e == cudaSuccess) e = cudaEventRecord(ev.back(), d2h);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev.back(), 0);
-    for (auto &x : ev)   // released by the runtime once their work completes
-        if (x != nullptr) cudaEventDestroy(x);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2 * nchunks], d2h);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev[2 * nchunks], 0);
     return e;
 }
 
@@ -151,10 +167,17 @@ s4_status glu_checks(const float *y, const float *x, const float *bias, const vo
     return S4_OK;
 }
 
-// an event marking the work queued on st so far
+// an event marking the work queued on st so far (the pipeline's own events
+// follow it in the pool, so it is recorded before they are)
 cudaError_t mark(cudaStream_t st, cudaEvent_t *ev) {
-    cudaError_t e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventRecord(*ev, st);
+    thread_local cudaEvent_t marks[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    cudaEvent_t &m = marks[dev & 63];
+    if (m == nullptr) e = cudaEventCreateWithFlags(&m, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(m, st);
+    *ev = m;
     return e;
 }
 
@@ -413,7 +436,6 @@ s4_status s4_fft_conv_host(const float *u_host, const float *K, const float *D, 
     if (e == cudaSuccess)
         e = conv_host_pipeline(u_host, workspace, Bt, H, L, y_host, u_dev, y_dev, nchunks, stream, h2d_stream,
                                d2h_stream, start);
-    if (start != nullptr) cudaEventDestroy(start);
     return cuda_status(e);
 }
 
@@ -444,7 +466,6 @@ s4_status s4_forward_dplr_host(const float *u_host, const s4_c32 *Lambda, const 
     if (e == cudaSuccess)
         e = conv_host_pipeline(u_host, workspace, Bt, H, L, y_host, u_dev, y_dev, nchunks, stream, h2d_stream,
                                d2h_stream, start);
-    if (start != nullptr) cudaEventDestroy(start);
     return cuda_status(e);
 }
 

@@ -34,11 +34,14 @@ namespace s4 {
 // ------------------------------------------------------------------ plan --
 // log2 of the radix of pass s for a 2^lg-point transform. The first and the
 // last pass are radix 16 (from lg = 8 on); the bits left over go to the
-// middle passes, split as evenly as they allow. Every strided pass then has a
-// stride of at least 16 points and the last pass works on 16 consecutive
-// points (moved as 16-byte pairs), which keeps all of them free of
-// shared-memory bank conflicts with the padding below.
-__host__ __device__ constexpr int plan_P(int lg) { return lg <= 8 ? 2 : (lg + 3) / 4; }
+// fewest middle passes of radix at most 32, split as evenly as they allow
+// (lg = 13: 16 x 32 x 16, three passes; every pass is one round trip through
+// shared memory, which bounds these transforms as much as the arithmetic
+// does). Every strided pass then has a stride of at least 16 points and the
+// last pass works on 16 consecutive points (moved as 16-byte pairs), which
+// keeps all of them free of shared-memory bank conflicts with the padding
+// below.
+__host__ __device__ constexpr int plan_P(int lg) { return lg <= 8 ? 2 : 2 + (lg - 8 + 4) / 5; }
 __host__ __device__ constexpr int plan_lr(int lg, int s) {
     if (lg == 4) return 2;
     if (lg <= 8) return s == 0 ? lg - 4 : 4;
@@ -421,6 +424,23 @@ __device__ __forceinline__ void pass_x2(float2 *b0, float2 *b1, const float2 *tw
     constexpr int B = plan_B(LG, s), S = B / R, G = (1 << LG) / R;
     constexpr int lS = ilog2(S);
     const float2 *tw = tws + plan_tw_off(LG, s);
+    if constexpr (R >= 32) {
+        // a group of both buffers would hold 2R points in registers: each
+        // thread takes one group of one buffer instead (2G groups in all)
+        for (int i = threadIdx.x; i < 2 * G; i += T) {
+            float2 *b = i < G ? b0 : b1;
+            const int g = i < G ? i : i - G;
+            const int j = g & (S - 1);
+            float2 *p = b + pidx(((g >> lS) << (lS + lr)) + j);
+            float2 x[R];
+            static_for<0, R>([&](auto q) { x[q] = p[poff<decltype(q)::value * S>()]; });
+            if constexpr (TW_FIRST) apply_powers<DIR, R>(x, tw[j]);
+            dft<R, DIR>(x);
+            if constexpr (!TW_FIRST) apply_powers<DIR, R>(x, tw[j]);
+            static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
+        }
+        return;
+    }
     for (int g = threadIdx.x; g < G; g += T) {
         const int j = g & (S - 1);
         const int o = pidx(((g >> lS) << (lS + lr)) + j);

@@ -9,7 +9,8 @@
 //      zero-padded K (both halves of the transform, as in k_fftconv_pair);
 //      its spectrum, plus D and times 1/2L, goes to the convolution workspace
 //      in the layout k_fftconv_pair reads.
-// Longer kernels take the three-kernel path (k_cauchy, k_irfft, k_kspec).
+// Longer kernels take k_cauchy, then (L = 16384) the inverse transform fused
+// with the spectrum in k_kspec_quad_half, or (L >= 32768) k_irfft + k_kspec.
 #include "launch.h"
 #include "pairs.cuh"
 
@@ -65,8 +66,7 @@ cudaError_t launch_kgen(const float2 *Lambda, const float2 *P, const float2 *Q, 
         case 8192: return run_kgen<13>(Lambda, P, Q, B, C, log_dt, D, H, Nh, K, ws, flags, st);
         default: {
             cudaError_t e = launch_cauchy(Lambda, P, Q, B, C, log_dt, H, Nh, L, K, flags, st);
-            if (e == cudaSuccess) e = launch_irfft_packed(K, H, L, st);
-            if (e == cudaSuccess) e = launch_kspec(K, D, H, L, ws, st);
+            if (e == cudaSuccess) e = launch_kspec_from_half(K, D, H, L, ws, st);
             return e;
         }
     }

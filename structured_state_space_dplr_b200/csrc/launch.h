@@ -35,9 +35,13 @@ cudaError_t launch_kgen_backward(const float2 *Lambda, const float2 *P, const fl
                                  float *dlog_dt, void *ws, cudaStream_t st);
 
 cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st);
+// K holds the packed half spectrum (k_cauchy's output) on entry and the kernel
+// on exit; ws receives the spectrum of K + D delta_0 as launch_kspec leaves it
+// (L = 16384: one fused launch; other L: launch_irfft_packed + launch_kspec)
+cudaError_t launch_kspec_from_half(float *K, const float *D, int H, int L, void *ws, cudaStream_t st);
 
 // ---- kgen.cu: K and the convolution spectrum of K + D delta_0 in one launch
-// (L <= 4096; longer L runs k_cauchy, k_irfft and k_kspec) ----
+// (L <= 8192; longer L runs k_cauchy, then launch_kspec_from_half) ----
 cudaError_t launch_kgen(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B, const float2 *C,
                         const float *log_dt, const float *D, int H, int Nh, int L, float *K, void *ws,
                         unsigned *flags, cudaStream_t st);

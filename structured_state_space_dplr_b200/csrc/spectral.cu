@@ -343,8 +343,13 @@ k_kspec_pair(const float *__restrict__ K, const float *__restrict__ D, int H, fl
 // at every k, and
 //   x[k] = S_0 + W_N^-k S_1,   x[k + m] = M_0 + i W_N^-k M_1.
 // So CTA 0 keeps S_0 and hands M_0 over, CTA 1 keeps i W_N^-k M_1 and hands
-// W_N^-k S_1 over, through distributed shared memory; CTA 0 writes x[k], CTA 1
-// x[k + m]. The spectrum holds 4 ranks x m points per channel (k_kspec_quad).
+// W_N^-k S_1 over; CTA 0 writes x[k], CTA 1 x[k + m]. The kept values stay in
+// the CTA's own buffer and the hand-over goes into the partner's receive
+// buffer with distributed-shared-memory stores (which do not wait on a round
+// trip), under a split cluster barrier: release after the stores, acquire
+// before reading the own buffer, and a relaxed arrive once it is read, which
+// the partner waits on before its next stores. The spectrum holds 4 ranks x
+// m points per channel (k_kspec_quad).
 constexpr int kQuadLG = 13;
 
 // the two ranks' inputs of point k = j + p S0 from the chunks a = x0[k], b = x1[k]
@@ -368,32 +373,44 @@ k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int
     static_assert(S0 == T, "one first-pass group per thread");
     extern __shared__ float2 sm[];
     const PairSmem s = pair_carve<LG>(sm);
-    float2 *tc = reinterpret_cast<float2 *>(s.stage);   // W_N^j (the stage area is free here)
+    // the partner's hand-over lands in this CTA's stage area (m points, one
+    // per (thread, p): index t = j + p S0), written there by the partner with
+    // remote stores, so the exchange never waits on a remote load
+    float2 *recv = reinterpret_cast<float2 *>(s.stage);
     cg::cluster_group cluster = cg::this_cluster();
     const int cr = (int)cluster.block_rank();
-    const float2 *rb0 = cluster.map_shared_rank(s.b0, cr ^ 1);
+    float2 *precv = cluster.map_shared_rank(recv, cr ^ 1);
     pair_tables<LG>(s);
     const int j = threadIdx.x;
-    tc[j] = unit_root(j, 2 * L);
+    const float2 tcj = unit_root(j, 2 * L);   // W_N^j
+    const float2 cj = cconj(tcj);             // W_N^-j
     __syncthreads();
     const long long npairs = (long long)H * ((Bt + 1) / 2);
     const long long cl = blockIdx.x / 2, ncl = gridDim.x / 2;
-    bool first = true;
-    for (long long pr = cl; pr < npairs; pr += ncl) {
+    // a[p], b[p]: the two input chunks (row 0 + i row 1) at k = j + p S0
+    // (holding them a pair ahead, across the exchange, costs more in
+    // registers than it hides in latency)
+    float2 a[R0], b[R0];
+    auto load_inputs = [&](long long pr) {
         const RowPair r = row_pair(pr, Bt);
         const float *u0 = u + ((size_t)r.b0 * H + r.h) * L;
         const float *u1 = u0 + (size_t)H * L;
-        float2 v0[R0], v1[R0];
         static_for<0, R0>([&](auto p) {
             const int k = j + p * S0;
-            const float2 a = make_float2(__ldg(u0 + k), r.has1 ? __ldg(u1 + k) : 0.0f);
-            const float2 b = make_float2(__ldg(u0 + k + m), r.has1 ? __ldg(u1 + k + m) : 0.0f);
-            quad_inputs<decltype(p)::value>(cr, a, b, v0[p], v1[p]);
+            a[p] = make_float2(__ldg(u0 + k), r.has1 ? __ldg(u1 + k) : 0.0f);
+            b[p] = make_float2(__ldg(u0 + k + m), r.has1 ? __ldg(u1 + k + m) : 0.0f);
         });
-        if (!first) cluster_wait();   // the partner has read this CTA's previous hand-over
-        first = false;
-        if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
-        else first_pass_halves2<LG, true>(s, v0, v1, j, tc[j]);
+    };
+    bool first = true;
+    for (long long pr = cl; pr < npairs; pr += ncl) {
+        const RowPair r = row_pair(pr, Bt);
+        load_inputs(pr);
+        {
+            float2 v0[R0], v1[R0];
+            static_for<0, R0>([&](auto p) { quad_inputs<decltype(p)::value>(cr, a[p], b[p], v0[p], v1[p]); });
+            if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
+            else first_pass_halves2<LG, true>(s, v0, v1, j, tcj);
+        }
         __syncthreads();
         forward_middle_x2<LG, T>(s.b0, s.b1, s.tws);
         const float2 *sh = spec + (size_t)r.h * 2 * L;
@@ -420,17 +437,20 @@ k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int
         });
         __syncthreads();
         inverse_middle_x2<LG, T>(s.b0, s.b1, s.tws);
-        // ---- keep one of (S, M) in b1, hand the other over in b0 (each thread
-        // writes only the positions of its own group, which it has just read)
-        const float2 cj = cconj(tc[j]);   // W_N^-j
+        // ---- last pass: keep one of (S, M) in registers, store the other
+        // into the partner's receive buffer (once the partner has read the
+        // previous pair's hand-over from it)
+        if (!first) cluster_wait();
+        float2 *keep = s.b1;   // position pidx(t) of this thread's own group
         last_pass_halves_sum<LG>(s, [&](auto pc, int t, float2 S, float2 M) {
             constexpr int p = decltype(pc)::value;
+            const int kp = pidx(t);
             if (cr == 0) {
-                s.b1[pidx(t)] = S;
-                s.b0[pidx(t)] = M;
+                keep[kp] = S;
+                precv[t] = M;
             } else {   // W_N^-t = W_N^-j W_64^-p
-                s.b1[pidx(t)] = mul_i<+1>(rot<p, 64, +1>(cmul(M, cj)));
-                s.b0[pidx(t)] = rot<p, 64, +1>(cmul(S, cj));
+                keep[kp] = mul_i<+1>(rot<p, 64, +1>(cmul(M, cj)));
+                precv[t] = rot<p, 64, +1>(cmul(S, cj));
             }
         });
         cluster_arrive_release();
@@ -439,13 +459,14 @@ k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int
         float *y1 = y0 + (size_t)H * L;
         static_for<0, R0>([&](auto p) {
             const int t = j + p * S0;
-            const float2 o = cadd(s.b1[pidx(t)], rb0[pidx(t)]);
+            const float2 o = cadd(keep[pidx(t)], recv[t]);
             y0[t] = o.x;
             if (r.has1) y1[t] = o.y;
         });
-        cluster_arrive_relaxed();
+        cluster_arrive_relaxed();   // done reading the receive buffer
+        first = false;
     }
-    if (!first) cluster_wait();   // the partner may still read this CTA's buffer
+    if (!first) cluster_wait();   // pairs the last arrive
 }
 
 // The spectrum k_fftconv_quad reads: per channel 4 ranks x m points in
@@ -460,10 +481,9 @@ k_kspec_quad(const float *__restrict__ K, const float *__restrict__ Ki, const fl
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     extern __shared__ float2 sm[];
     const PairSmem s = pair_carve<LG>(sm);
-    float2 *tc = reinterpret_cast<float2 *>(s.stage);
     pair_tables<LG>(s);
     const int j = threadIdx.x;
-    tc[j] = unit_root(j, 2 * L);
+    const float2 tcj = unit_root(j, 2 * L);   // W_N^j
     __syncthreads();
     for (int it = blockIdx.x; it < 2 * H; it += gridDim.x) {
         const int h = it >> 1, cr = it & 1;
@@ -477,7 +497,99 @@ k_kspec_quad(const float *__restrict__ K, const float *__restrict__ Ki, const fl
                                            v0[p], v1[p]);
         });
         if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
-        else first_pass_halves2<LG, true>(s, v0, v1, j, tc[j]);
+        else first_pass_halves2<LG, true>(s, v0, v1, j, tcj);
+        __syncthreads();
+        float4 *sh = reinterpret_cast<float4 *>(spec + (size_t)h * 2 * L);
+        spectrum_tail2<LG>(s, D != nullptr ? __ldg(D + h) : 0.0f, 1.0f / (float)(2 * L), sh + (size_t)cr * (m / 2),
+                           sh + (size_t)(cr + 2) * (m / 2));
+        __syncthreads();
+    }
+}
+
+// The same spectrum straight from the packed half spectrum that k_cauchy
+// leaves in K (K[0] = K_hat_0, K[1] = K_hat_{L/2}, K[2f], K[2f+1] = K_hat_f,
+// all times 1/L), with the inverse real transform folded in, so K does not
+// round-trip through memory between the two: one cluster of two CTAs per
+// channel, CTA cr holding ranks cr and cr + 2 as in k_kspec_quad. Each CTA
+// turns the half spectrum into the length-M = L/2 complex sequence
+//   Z[k] = (X[k] + conj X[M-k]) + i w^k (X[k] - conj X[M-k]),  w = e^{2 pi i/L},
+// whose unnormalised inverse transform is z[n] = K[2n] + i K[2n+1]; CTA 0
+// also stores K (in place, after a cluster barrier that orders its stores
+// after the partner's last read of the half spectrum). The chunks
+// x0 = K[0, m), x1 = K[m, 2m) of the zero-padded length-2L transform are
+// then read back from the natural-order z in shared memory.
+__global__ void __launch_bounds__(pair_threads<kQuadLG>(), 1)
+k_kspec_quad_half(float *__restrict__ K, const float *__restrict__ D, int H, float2 *__restrict__ spec) {
+    constexpr int LG = kQuadLG, m = 1 << LG, L = 2 * m, M = L / 2, T = pair_threads<LG>();
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0, NP = plan_P(LG);
+    static_assert(M == m && S0 == T, "z holds m points, one first-pass group per thread");
+    extern __shared__ float2 sm[];
+    const PairSmem s = pair_carve<LG>(sm);
+    cg::cluster_group cluster = cg::this_cluster();
+    const int cr = (int)cluster.block_rank();
+    pair_tables<LG>(s);
+    const int j = threadIdx.x;
+    const float2 tcj = unit_root(j, 2 * L);   // W_N^j
+    __syncthreads();
+    float2 *X = s.b0;   // the length-M inverse transform
+    for (int h = blockIdx.x / 2; h < H; h += gridDim.x / 2) {
+        float *Kh = K + (size_t)h * L;
+        // ---- Z at its digit-reversed position (k and M - k from one pair of loads)
+        for (int k = j; k <= M / 2; k += T) {
+            float2 A, Bc;
+            if (k == 0) {
+                A = make_float2(__ldcg(Kh), 0.0f);
+                Bc = make_float2(__ldcg(Kh + 1), 0.0f);
+            } else {
+                A = __ldcg(reinterpret_cast<const float2 *>(Kh) + k);
+                Bc = cconj(__ldcg(reinterpret_cast<const float2 *>(Kh) + (M - k)));
+            }
+            float sn, cs;
+            sincospif(2.0f * (float)k / (float)L, &sn, &cs);   // w^k = cs + i sn
+            const float2 wk = make_float2(cs, sn);
+            X[pidx(digrev_inv<LG>(k))] = cadd(cadd(A, Bc), mul_i<+1>(cmul(wk, csub(A, Bc))));
+            if (k != 0 && k != M / 2) {   // Z[M - k]: A' = conj Bc, Bc' = conj A, w^{M-k} = -conj w^k
+                const float2 A2 = cconj(Bc), B2 = cconj(A);
+                X[pidx(digrev_inv<LG>(M - k))] =
+                    csub(cadd(A2, B2), mul_i<+1>(cmul(cconj(wk), csub(A2, B2))));
+            }
+        }
+        cluster_arrive_relaxed();   // this CTA's reads of the half spectrum are done
+        __syncthreads();
+        // ---- inverse transform, passes P-1 .. 1, then the last pass in registers
+        dit_pass<LG, NP - 1, +1, T>(X, s.tws);
+        __syncthreads();
+        inverse_middle<LG, T>(X, s.tws);
+        float2 z[R0];
+        {
+            const int o = pidx(j);
+            const float2 b = s.tb[j];
+            float2 w = b;
+            z[0] = X[o];
+            static_for<1, R0>([&](auto q) {
+                z[q] = cmulc(X[o + poff<decltype(q)::value * S0>()], w);
+                w = cmul(w, b);
+            });
+            dft<R0, +1>(z);   // z[p] = K[2n] + i K[2n+1], n = j + p S0
+        }
+        cluster_wait();   // the partner has read the half spectrum: K may be overwritten
+        if (cr == 0)
+            static_for<0, R0>([&](auto p) { reinterpret_cast<float2 *>(Kh)[j + p * S0] = z[p]; });
+        __syncthreads();   // every thread has read its group of X
+        static_for<0, R0>([&](auto p) { X[pidx(j + p * S0)] = z[p]; });
+        __syncthreads();
+        // ---- chunks x0[k] = K[k], x1[k] = K[k + m] at k = j + p S0: K[k] is a
+        // component of z[k / 2]
+        float2 v0[R0], v1[R0];
+        static_for<0, R0>([&](auto p) {
+            const int k = j + p * S0;
+            const float2 za = X[pidx(k >> 1)], zb = X[pidx((k + m) >> 1)];
+            const float ka = (k & 1) ? za.y : za.x, kb = (k & 1) ? zb.y : zb.x;
+            quad_inputs<decltype(p)::value>(cr, make_float2(ka, 0.0f), make_float2(kb, 0.0f), v0[p], v1[p]);
+        });
+        __syncthreads();   // X (= b0) is read: the first pass may overwrite it
+        if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
+        else first_pass_halves2<LG, true>(s, v0, v1, j, tcj);
         __syncthreads();
         float4 *sh = reinterpret_cast<float4 *>(spec + (size_t)h * 2 * L);
         spectrum_tail2<LG>(s, D != nullptr ? __ldg(D + h) : 0.0f, 1.0f / (float)(2 * L), sh + (size_t)cr * (m / 2),
@@ -799,6 +911,21 @@ cudaError_t quad_kspec(const float *K, const float *D, int H, void *ws, cudaStre
     return cudaGetLastError();
 }
 
+LaunchInfo g_quad_half;
+
+// K holds the packed half spectrum on entry and the kernel on exit
+cudaError_t quad_kspec_half(float *K, const float *D, int H, void *ws, cudaStream_t st) {
+    constexpr size_t smem = pair_smem_bytes<kQuadLG>(0);
+    constexpr int T = pair_threads<kQuadLG>();
+    int res = 0;
+    cudaError_t e = resident_units(k_kspec_quad_half, g_quad_half, 2, T, smem, &res);
+    if (e != cudaSuccess) return e;
+    const int ncl = res < H ? res : H;
+    e = launch_clustered(k_kspec_quad_half, 2, ncl, T, smem, st, K, D, H, (float2 *)ws);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 cudaError_t quad_conv(const float *u, const void *ws, int Bt, int H, float *y, bool adjoint, cudaStream_t st) {
     constexpr size_t smem = pair_smem_bytes<kQuadLG>(0);
     constexpr int T = pair_threads<kQuadLG>();
@@ -833,6 +960,13 @@ cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L,
 #undef X
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_kspec_from_half(float *K, const float *D, int H, int L, void *ws, cudaStream_t st) {
+    if (L == 2 << kQuadLG) return quad_kspec_half(K, D, H, ws, st);
+    cudaError_t e = launch_irfft_packed(K, H, L, st);
+    if (e == cudaSuccess) e = launch_kspec(K, D, H, L, ws, st);
+    return e;
 }
 
 cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st) {

@@ -1,5 +1,6 @@
 """GPU parity of the fused entry points: s4_kernel_dplr_prepare (K and the
-convolution spectrum of K + D delta_0 in one launch for L <= 8192) and
+convolution spectrum of K + D delta_0 in one launch for L <= 8192, two for
+L = 16384) and
 s4_forward_dplr (the whole convolution-view forward), against the fp64 oracle
 and against the modular calls."""
 import numpy as np
@@ -28,8 +29,11 @@ def _fused(inp):
     return K.cpu().numpy(), y.cpu().numpy(), K3.cpu().numpy(), y3.cpu().numpy()
 
 
-@pytest.mark.parametrize("L", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192])
+@pytest.mark.parametrize("L", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536])
 def test_random_dplr_all_outputs(L):
+    """Every output, odd H and batch; L = 16384 takes the inverse transform
+    fused into the spectrum kernel (one cluster per channel, K stored in
+    place of the half spectrum), longer L the separate inverse transform."""
     inp = s4inputs.random_dplr(500 + L, H=3, Nh=6, L=L, Bt=3)
     K, y, K3, y3 = _fused(inp)
     Kr = workloads.dplr_kernel(inp)
