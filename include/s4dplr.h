@@ -260,7 +260,9 @@ s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P,
 /* ------------------------------------------------------------------------
  * Host-buffer forms: s4_fft_conv and s4_forward_dplr with u and y in HOST
  * memory, the copies pipelined with the convolution. The batch is cut into
- * nchunks chunks of whole row pairs; chunk c is uploaded on h2d_stream,
+ * nchunks chunks of whole row pairs (when it has fewer row pairs than
+ * nchunks and L <= 16384, into row pairs cut into channel slices, so that a
+ * small batch still pipelines); chunk c is uploaded on h2d_stream,
  * convolved on `stream` once it has arrived, and downloaded on d2h_stream
  * once convolved, so the upload of one chunk, the convolution of the next
  * earlier one and the download of the one before overlap (the two copy
@@ -275,7 +277,9 @@ s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P,
  *                    asynchronously and overlap, pageable memory still works.
  *   u_dev, y_dev   : [Bt, H, L] device staging buffers owned by the caller
  *                    (16-byte aligned, not overlapping each other, K, D,
- *                    the workspace or the parameters).
+ *                    the workspace or the parameters); what they hold on
+ *                    return is staging data in the chunks' own order, not a
+ *                    copy of u or y.
  *   nchunks        : >= 1 (clamped to the number of row pairs).
  *   h2d_stream, d2h_stream : caller-owned streams (may be `stream` itself,
  *                    which serialises the pipeline).

@@ -86,6 +86,49 @@ cudaError_t pipeline_events(size_t n, cudaEvent_t **out) {
     return cudaSuccess;
 }
 
+// The same pipeline when the batch has fewer row pairs than chunks asked for
+// (L <= 16384, where the workspace is only the per-channel spectrum, so the
+// spectrum of channels [h0, h1) starts at h0 * 2L complex values): each row
+// pair is also cut into channel slices. Chunk (pair, slice) is staged in
+// u_dev / y_dev as a contiguous [rows][h1 - h0][L] block at
+// b0 H L + rows h0 L (one copy per row each way) and convolved as a batch of
+// its own; the blocks tile the buffers without overlap.
+cudaError_t conv_host_pipeline_sliced(const float *u_host, const void *ws, int Bt, int H, int L, float *y_host,
+                                      float *u_dev, float *y_dev, int nchunks, cudaStream_t st, cudaStream_t h2d,
+                                      cudaStream_t d2h, cudaEvent_t start) {
+    const int npairs = (Bt + 1) / 2;
+    int slices = (nchunks + npairs - 1) / npairs;
+    if (slices > H) slices = H;
+    const int hc = (H + slices - 1) / slices;
+    slices = (H + hc - 1) / hc;
+    const int total = npairs * slices;
+    cudaEvent_t *ev = nullptr;   // [2 total + 1]: upload c done, convolution c done, last download done
+    cudaError_t e = pipeline_events(2 * (size_t)total + 1, &ev);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h2d, start, 0);
+    for (int c = 0; c < total && e == cudaSuccess; ++c) {
+        const int pr = c / slices, q = c % slices;
+        const int b0 = 2 * pr, nb = b0 + 1 < Bt ? 2 : 1;
+        const int h0 = q * hc, nh = h0 + hc < H ? hc : H - h0;
+        const size_t blk = (size_t)b0 * H * L + (size_t)nb * h0 * L, rowb = (size_t)nh * L;
+        for (int r = 0; r < nb && e == cudaSuccess; ++r)
+            e = cudaMemcpyAsync(u_dev + blk + r * rowb, u_host + ((size_t)(b0 + r) * H + h0) * L,
+                                rowb * sizeof(float), cudaMemcpyHostToDevice, h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[2 * c], h2d);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev[2 * c], 0);
+        if (e == cudaSuccess)
+            e = s4::launch_fftconv(u_dev + blk, (const char *)ws + (size_t)h0 * 2 * L * 2 * sizeof(float), nb, nh, L,
+                                   y_dev + blk, st);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[2 * c + 1], st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(d2h, ev[2 * c + 1], 0);
+        for (int r = 0; r < nb && e == cudaSuccess; ++r)
+            e = cudaMemcpyAsync(y_host + ((size_t)(b0 + r) * H + h0) * L, y_dev + blk + r * rowb,
+                                rowb * sizeof(float), cudaMemcpyDeviceToHost, d2h);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2 * total], d2h);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev[2 * total], 0);
+    return e;
+}
+
 // The convolution of a batch held in host memory. Chunk c (whole row pairs)
 // is uploaded on h2d, convolved on st once it has arrived and downloaded on
 // d2h once convolved, so uploads, convolutions and downloads of consecutive
@@ -97,6 +140,8 @@ cudaError_t conv_host_pipeline(const float *u_host, const void *ws, int Bt, int 
                                float *u_dev, float *y_dev, int nchunks, cudaStream_t st, cudaStream_t h2d,
                                cudaStream_t d2h, cudaEvent_t start) {
     const int npairs = (Bt + 1) / 2;
+    if (nchunks > npairs && H > 1 && L <= 16384)
+        return conv_host_pipeline_sliced(u_host, ws, Bt, H, L, y_host, u_dev, y_dev, nchunks, st, h2d, d2h, start);
     if (nchunks > npairs) nchunks = npairs;
     const int pairs_per_chunk = (npairs + nchunks - 1) / nchunks;
     nchunks = (npairs + pairs_per_chunk - 1) / pairs_per_chunk;

@@ -7,7 +7,10 @@
 
 namespace s4 {
 
-constexpr int kCauchyThreads = 256;
+// 128 threads x 2 frequencies per CTA: small CTAs keep the last wave full
+// (at H = 256, L = 4096: 2048 CTAs over 7 x 148 resident, 1.98 waves, where
+// 256-thread CTAs made 1024 over 3 x 148, 2.3 waves with the last 30 % full)
+constexpr int kCauchyThreads = 128;
 constexpr int kCauchyFreqs = 2;   // frequencies per thread
 
 template <int T, int F>

@@ -510,32 +510,47 @@ k_kspec_quad(const float *__restrict__ K, const float *__restrict__ Ki, const fl
 // leaves in K (K[0] = K_hat_0, K[1] = K_hat_{L/2}, K[2f], K[2f+1] = K_hat_f,
 // all times 1/L), with the inverse real transform folded in, so K does not
 // round-trip through memory between the two: one cluster of two CTAs per
-// channel, CTA cr holding ranks cr and cr + 2 as in k_kspec_quad. Each CTA
-// turns the half spectrum into the length-M = L/2 complex sequence
-//   Z[k] = (X[k] + conj X[M-k]) + i w^k (X[k] - conj X[M-k]),  w = e^{2 pi i/L},
-// whose unnormalised inverse transform is z[n] = K[2n] + i K[2n+1]; CTA 0
-// also stores K (in place, after a cluster barrier that orders its stores
-// after the partner's last read of the half spectrum). The chunks
-// x0 = K[0, m), x1 = K[m, 2m) of the zero-padded length-2L transform are
-// then read back from the natural-order z in shared memory.
+// channel, CTA cr holding ranks cr and cr + 2 as in k_kspec_quad. With
+// M = L/2 and w = e^{2 pi i/L}, the length-M sequence
+//   Z[k] = (X[k] + conj X[M-k]) + i w^k (X[k] - conj X[M-k])
+// has the unnormalised inverse transform z[n] = K[2n] + i K[2n+1]. CTA cr
+// inverts the frequencies k = 2k' + cr (a length-M/2 transform z_cr; Z[k]
+// and Z[M-k] share a parity, so each pair of loads stays in one CTA), and
+//   z[n] = z_0[n'] + e^{2 pi i n/M} z_1[n'],  n' = n mod M/2.
+// The CTAs exchange z_cr through each other's stage area (distributed
+// shared-memory stores, split cluster barrier as in k_fftconv_quad); then
+// both read the chunks x0 = K[0, m), x1 = K[m, 2m) of the zero-padded
+// transform: for k < m, K[k] and K[k + m] are components of
+// z_0[k/2] +- e^{2 pi i (k/2)/M} z_1[k/2]. CTA 0 stores K[0, m) and CTA 1
+// K[m, 2m) in place of the half spectrum; the barrier of the exchange orders
+// those stores after both CTAs' reads of it.
 __global__ void __launch_bounds__(pair_threads<kQuadLG>(), 1)
 k_kspec_quad_half(float *__restrict__ K, const float *__restrict__ D, int H, float2 *__restrict__ spec) {
     constexpr int LG = kQuadLG, m = 1 << LG, L = 2 * m, M = L / 2, T = pair_threads<LG>();
-    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0, NP = plan_P(LG);
-    static_assert(M == m && S0 == T, "z holds m points, one first-pass group per thread");
+    constexpr int LGH = LG - 1, MH = M / 2;                        // the half-length inverse: 2^12 points
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    constexpr int RH = 1 << plan_lr(LGH, 0), SH = MH / RH, NPH = plan_P(LGH);
+    static_assert(M == m && S0 == T && SH <= T, "one first-pass group per thread");
     extern __shared__ float2 sm[];
     const PairSmem s = pair_carve<LG>(sm);
     cg::cluster_group cluster = cg::this_cluster();
     const int cr = (int)cluster.block_rank();
+    float2 *recv = reinterpret_cast<float2 *>(s.stage);            // [MH]: the partner's z
+    float2 *twh = recv + MH;                                       // middle-pass twiddles of the half-length inverse
+    float2 *precv = cluster.map_shared_rank(recv, cr ^ 1);
     pair_tables<LG>(s);
+    build_middle_tables<LGH>(twh, threadIdx.x, T);
     const int j = threadIdx.x;
     const float2 tcj = unit_root(j, 2 * L);   // W_N^j
     __syncthreads();
-    float2 *X = s.b0;   // the length-M inverse transform
+    float2 *X = s.b0;   // the length-MH inverse transform of this CTA's parity
+    bool first = true;
     for (int h = blockIdx.x / 2; h < H; h += gridDim.x / 2) {
         float *Kh = K + (size_t)h * L;
-        // ---- Z at its digit-reversed position (k and M - k from one pair of loads)
-        for (int k = j; k <= M / 2; k += T) {
+        // ---- Z[2k' + cr] at the digit-reversed position of k' (k and M - k from one pair of loads)
+        for (int i = j; i <= MH / 2; i += T) {
+            const int k = 2 * i + cr;
+            if (k > M / 2) break;
             float2 A, Bc;
             if (k == 0) {
                 A = make_float2(__ldcg(Kh), 0.0f);
@@ -547,55 +562,63 @@ k_kspec_quad_half(float *__restrict__ K, const float *__restrict__ D, int H, flo
             float sn, cs;
             sincospif(2.0f * (float)k / (float)L, &sn, &cs);   // w^k = cs + i sn
             const float2 wk = make_float2(cs, sn);
-            X[pidx(digrev_inv<LG>(k))] = cadd(cadd(A, Bc), mul_i<+1>(cmul(wk, csub(A, Bc))));
+            X[pidx(digrev_inv<LGH>(k >> 1))] = cadd(cadd(A, Bc), mul_i<+1>(cmul(wk, csub(A, Bc))));
             if (k != 0 && k != M / 2) {   // Z[M - k]: A' = conj Bc, Bc' = conj A, w^{M-k} = -conj w^k
                 const float2 A2 = cconj(Bc), B2 = cconj(A);
-                X[pidx(digrev_inv<LG>(M - k))] =
+                X[pidx(digrev_inv<LGH>((M - k) >> 1))] =
                     csub(cadd(A2, B2), mul_i<+1>(cmul(cconj(wk), csub(A2, B2))));
             }
         }
-        cluster_arrive_relaxed();   // this CTA's reads of the half spectrum are done
         __syncthreads();
-        // ---- inverse transform, passes P-1 .. 1, then the last pass in registers
-        dit_pass<LG, NP - 1, +1, T>(X, s.tws);
+        // ---- half-length inverse transform, passes P-1 .. 1, then the last pass in registers
+        dit_pass<LGH, NPH - 1, +1, T>(X, twh);
         __syncthreads();
-        inverse_middle<LG, T>(X, s.tws);
-        float2 z[R0];
-        {
+        inverse_middle<LGH, T>(X, twh);
+        if (!first) cluster_wait();   // the partner has read the previous channel's hand-over
+        if (j < SH) {
             const int o = pidx(j);
-            const float2 b = s.tb[j];
+            const float2 b = unit_root(j, MH);
+            float2 z[RH];
             float2 w = b;
             z[0] = X[o];
-            static_for<1, R0>([&](auto q) {
-                z[q] = cmulc(X[o + poff<decltype(q)::value * S0>()], w);
+            static_for<1, RH>([&](auto q) {
+                z[q] = cmulc(X[o + poff<decltype(q)::value * SH>()], w);
                 w = cmul(w, b);
             });
-            dft<R0, +1>(z);   // z[p] = K[2n] + i K[2n+1], n = j + p S0
+            dft<RH, +1>(z);   // z[p] = z_cr[j + p SH]
+            static_for<0, RH>([&](auto p) {
+                X[o + poff<decltype(p)::value * SH>()] = z[p];   // natural order, own group positions
+                precv[j + p * SH] = z[p];
+            });
         }
-        cluster_wait();   // the partner has read the half spectrum: K may be overwritten
-        if (cr == 0)
-            static_for<0, R0>([&](auto p) { reinterpret_cast<float2 *>(Kh)[j + p * S0] = z[p]; });
-        __syncthreads();   // every thread has read its group of X
-        static_for<0, R0>([&](auto p) { X[pidx(j + p * S0)] = z[p]; });
-        __syncthreads();
-        // ---- chunks x0[k] = K[k], x1[k] = K[k + m] at k = j + p S0: K[k] is a
-        // component of z[k / 2]
+        cluster_arrive_release();
+        cluster_wait();   // both halves are in place; both CTAs are done reading the half spectrum
+        // ---- chunks x0[k] = K[k], x1[k] = K[k + m] at k = j + p S0
         float2 v0[R0], v1[R0];
         static_for<0, R0>([&](auto p) {
-            const int k = j + p * S0;
-            const float2 za = X[pidx(k >> 1)], zb = X[pidx((k + m) >> 1)];
+            const int k = j + p * S0, n = k >> 1;
+            const float2 zo = X[pidx(n)], zr = recv[n];
+            const float2 z0 = cr == 0 ? zo : zr, z1 = cr == 0 ? zr : zo;
+            float sn, cs;
+            sincospif(2.0f * (float)n / (float)M, &sn, &cs);
+            const float2 wz = cmul(make_float2(cs, sn), z1);
+            const float2 za = cadd(z0, wz), zb = csub(z0, wz);
             const float ka = (k & 1) ? za.y : za.x, kb = (k & 1) ? zb.y : zb.x;
+            Kh[k + cr * m] = cr == 0 ? ka : kb;
             quad_inputs<decltype(p)::value>(cr, make_float2(ka, 0.0f), make_float2(kb, 0.0f), v0[p], v1[p]);
         });
-        __syncthreads();   // X (= b0) is read: the first pass may overwrite it
+        __syncthreads();   // X (in b0) is read: the first pass may overwrite it
         if (cr == 0) first_pass_halves2<LG, false>(s, v0, v1, j, make_float2(1.0f, 0.0f));
         else first_pass_halves2<LG, true>(s, v0, v1, j, tcj);
+        cluster_arrive_relaxed();   // the values read from recv went into the stores above
+        first = false;
         __syncthreads();
         float4 *sh = reinterpret_cast<float4 *>(spec + (size_t)h * 2 * L);
         spectrum_tail2<LG>(s, D != nullptr ? __ldg(D + h) : 0.0f, 1.0f / (float)(2 * L), sh + (size_t)cr * (m / 2),
                            sh + (size_t)(cr + 2) * (m / 2));
         __syncthreads();
     }
+    if (!first) cluster_wait();   // pairs the last arrive
 }
 
 // ------------------------------------------------------------------ irfft --
