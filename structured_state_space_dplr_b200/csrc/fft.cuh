@@ -1,8 +1,9 @@
 // fft.cuh -- shared-memory mixed-radix FFT building blocks for sm_100a.
 //
 // A CTA holds m = 2^LG complex points in shared memory and transforms them
-// in place with radix-16 passes (plus one radix-8/4 pass when LG is not a
-// multiple of 4), each thread keeping a whole radix group in registers:
+// in place with radix-16 first and last passes and the bits left over in
+// the fewest middle passes of radix at most 32, each thread keeping a whole
+// radix group in registers:
 //
 //   forward  = decimation in frequency: natural input -> digit-reversed
 //              output (no reorder pass);
@@ -14,15 +15,15 @@
 // consecutive points, so they are fused with the pointwise product and the
 // data stays in registers across them.
 //
-// A length-N transform is split over a cluster of C CTAs (N = C m): CTA c
-// owns the frequencies C f + c. Forward, each CTA forms its own input
-//     v_c[k] = W_N^{k c} sum_r x[k + r m] W_C^{r c}
-// straight from global memory and runs an m-point transform; inverse, each
-// CTA runs an m-point transform and the C partial results are combined over
-// distributed shared memory:
+// A length-N transform is split over C ranks (N = C m): rank c owns the
+// frequencies C f + c and transforms its own input
+//     v_c[k] = W_N^{k c} sum_r x[k + r m] W_C^{r c};
+// inverse, each rank runs an m-point transform and the C partial results are
+// combined:
 //     x[k + r m] = sum_c W_C^{-c r} W_N^{-c k} Z_c[k].
 // The twist W_N^{k c} is folded into the first pass: a per-rank constant on
-// each input of a group plus a per-rank first-pass twiddle table.
+// each input of a group (pre) and, with the pass twiddles, ta[j] tb[j]^q
+// formed by recurrence from two tables of m/16 entries (build_rank_tables).
 //
 // Shared memory is padded by two points after every 16 (pidx below): with
 // the pass plan, every pass is free of bank conflicts.
@@ -172,17 +173,6 @@ __device__ __forceinline__ void dft(float2 (&x)[R]) {
 }
 
 // ---------------------------------------------------------------- tables --
-// First-pass table of rank c of a C-way split of an N = C m transform:
-//   tw0[q S0 + j] = W_N^{j (C q + c)}     (S0 = m / R0)
-template <int LG>
-__device__ __forceinline__ float2 tw0_entry(int i, int C, int c) {
-    constexpr int m = 1 << LG;
-    constexpr int lS0 = LG - plan_lr(LG, 0);
-    int q = i >> lS0, j = i & ((1 << lS0) - 1);
-    int N = C * m;
-    return unit_root((j * (C * q + c)) & (N - 1), N);
-}
-
 // Base twiddles of the middle passes: tws[off_s + j] = W_{B_s}^j, j < S_s.
 template <int LG>
 __device__ void build_middle_tables(float2 *tws, int tid, int nthreads) {
@@ -193,19 +183,6 @@ __device__ void build_middle_tables(float2 *tws, int tid, int nthreads) {
         float2 *t = tws + plan_tw_off(LG, s);
         for (int j = tid; j < S; j += nthreads) t[j] = unit_root(j, B);
     });
-}
-
-// Fill (with nthreads threads, index tid) the per-CTA tables:
-//   tw0 (pass 0, rank c; skipped when null), tws (passes 1..P-2), pre[p] = W_{C R0}^{p c}.
-template <int LG>
-__device__ void build_tables(float2 *tw0, float2 *tws, float2 *pre, int C, int c, int tid, int nthreads) {
-    constexpr int m = 1 << LG;
-    constexpr int P = plan_P(LG);
-    constexpr int R0 = 1 << plan_lr(LG, 0);
-    if (tw0 != nullptr)
-        for (int i = tid; i < m; i += nthreads) tw0[i] = tw0_entry<LG>(i, C, c);
-    build_middle_tables<LG>(tws, tid, nthreads);
-    for (int p = tid; p < R0; p += nthreads) pre[p] = unit_root((p * c) % (C * R0), C * R0);
 }
 
 // ---------------------------------------------------------------- passes --
@@ -308,11 +285,28 @@ __device__ __forceinline__ void inverse_middle(float2 *buf, const float2 *tws, i
     });
 }
 
-// First forward pass of group j, in registers: x_p = fetch(j + p S0) * pre[p],
-// DFT, times tw0[q S0 + j].
+// Per-CTA tables of rank c of a C-way split of an N = C m transform, small
+// enough to sit in shared memory at every length: the first-pass twiddle
+// W_N^{j (C q + c)} = W_N^{j c} W_m^{j q} is ta[j] tb[j]^q (j < S0, formed by
+// recurrence over q), and pre[p] = W_{C R0}^{p c} is the in-group share of the
+// rank's twist.
+template <int LG>
+__device__ void build_rank_tables(float2 *ta, float2 *tb, float2 *pre, int C, int c, int tid, int nthreads) {
+    constexpr int m = 1 << LG;
+    constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
+    const int N = C * m;
+    for (int j = tid; j < S0; j += nthreads) {
+        ta[j] = unit_root((j * c) & (N - 1), N);
+        tb[j] = unit_root(j, m);
+    }
+    for (int p = tid; p < R0; p += nthreads) pre[p] = unit_root((p * c) % (C * R0), C * R0);
+}
+
+// First forward pass of group j with the rank tables: x_p = fetch(j + p S0)
+// pre[p], DFT, times ta[j] tb[j]^q.
 template <int LG, class Fetch>
-__device__ __forceinline__ void first_group(float2 (&x)[1 << plan_lr(LG, 0)], int j, const float2 *tw0,
-                                            const float2 *pre, Fetch &&fetch) {
+__device__ __forceinline__ void first_group_rec(float2 (&x)[1 << plan_lr(LG, 0)], int j, const float2 *ta,
+                                                const float2 *tb, const float2 *pre, Fetch &&fetch) {
     constexpr int R = 1 << plan_lr(LG, 0);
     constexpr int S = (1 << LG) / R;
     static_for<0, R>([&](auto p) {
@@ -320,43 +314,43 @@ __device__ __forceinline__ void first_group(float2 (&x)[1 << plan_lr(LG, 0)], in
         if constexpr (decltype(p)::value == 0) x[p] = v; else x[p] = cmul(v, pre[p]);
     });
     dft<R, -1>(x);
-    static_for<0, R>([&](auto q) { x[q] = cmul(x[q], tw0[q * S + j]); });
-}
-template <int LG>
-__device__ __forceinline__ void store_first_group(float2 *buf, const float2 (&x)[1 << plan_lr(LG, 0)], int j) {
-    constexpr int R = 1 << plan_lr(LG, 0);
-    constexpr int S = (1 << LG) / R;
-    float2 *p = buf + pidx(j);
-    static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
+    const float2 b = tb[j];
+    float2 w = ta[j];
+    static_for<0, R>([&](auto q) {
+        x[q] = cmul(x[q], w);
+        if constexpr (decltype(q)::value + 1 < R) w = cmul(w, b);
+    });
 }
 
-// First forward pass over all groups (input through fetch(k), k in [0, m)).
-template <int LG, int T, class Fetch>
-__device__ __forceinline__ void forward_first(float2 *buf, const float2 *tw0, const float2 *pre, Fetch &&fetch) {
-    constexpr int S = (1 << LG) >> plan_lr(LG, 0);
-    for (int j = threadIdx.x; j < S; j += T) {
-        float2 x[1 << plan_lr(LG, 0)];
-        first_group<LG>(x, j, tw0, pre, fetch);
-        store_first_group<LG>(buf, x, j);
-    }
-}
-
-// Last inverse pass: conjugate tw0, inverse DFT, conjugate pre; natural order
-// result W_N^{-c k} Z_c[k] stored at pidx(k).
+// Last inverse pass with the rank tables (the conjugate of the above):
+// W_N^{-c k} Z_c[k] stored at pidx(k), natural order.
 template <int LG, int T>
-__device__ __forceinline__ void inverse_last(float2 *buf, const float2 *tw0, const float2 *pre) {
-    constexpr int lr = plan_lr(LG, 0), R = 1 << lr;
+__device__ __forceinline__ void inverse_last_rec(float2 *buf, const float2 *ta, const float2 *tb, const float2 *pre) {
+    constexpr int R = 1 << plan_lr(LG, 0);
     constexpr int S = (1 << LG) / R;
     for (int j = threadIdx.x; j < S; j += T) {
         float2 *p = buf + pidx(j);
+        const float2 b = tb[j];
+        float2 w = ta[j];
         float2 x[R];
-        static_for<0, R>([&](auto q) { x[q] = cmulc(p[poff<decltype(q)::value * S>()], tw0[q * S + j]); });
+        static_for<0, R>([&](auto q) {
+            x[q] = cmulc(p[poff<decltype(q)::value * S>()], w);
+            if constexpr (decltype(q)::value + 1 < R) w = cmul(w, b);
+        });
         dft<R, +1>(x);
         static_for<0, R>([&](auto q) {
             if constexpr (decltype(q)::value == 0) p[0] = x[q];
             else p[poff<decltype(q)::value * S>()] = cmulc(x[q], pre[q]);
         });
     }
+}
+
+template <int LG>
+__device__ __forceinline__ void store_first_group(float2 *buf, const float2 (&x)[1 << plan_lr(LG, 0)], int j) {
+    constexpr int R = 1 << plan_lr(LG, 0);
+    constexpr int S = (1 << LG) / R;
+    float2 *p = buf + pidx(j);
+    static_for<0, R>([&](auto q) { p[poff<decltype(q)::value * S>()] = x[q]; });
 }
 
 // Fused last forward pass + pointwise product + first inverse pass. The group

@@ -10,7 +10,7 @@ void record_cuda_error(cudaError_t e);
 
 // ---- spectral.cu: FFT convolution and inverse real FFT ----
 // Cluster split used for the length-2L convolution transforms.
-struct ConvGeom { int C; int lg; bool tw0_global; };
+struct ConvGeom { int C; int lg; };
 ConvGeom conv_geom(int L);
 size_t conv_workspace_bytes(int H, int L);
 

@@ -36,35 +36,27 @@ __host__ __device__ constexpr int threads_for() {
     return (1 << LG) / 16 < 32 ? 32 : ((1 << LG) / 16 > 512 ? 512 : (1 << LG) / 16);
 }
 
-// dynamic shared memory, in float2: buf | tw0 (unless in global) | tws | pre[16] | wcr[8]
-// (| stage[2][L] floats for the staged convolution, 16-byte aligned)
+// dynamic shared memory of the C-way split kernels, in float2:
+// buf | tws | ta[S0] | tb[S0] | pre[16] | wcr[8]
 template <int LG>
-__host__ __device__ constexpr int smem_f2(bool tw0_global) {
-    return (padded(1 << LG) + (tw0_global ? 0 : (1 << LG)) + plan_tw_size(LG) + 16 + 8 + 1) / 2 * 2;
+__host__ __device__ constexpr int smem_f2() {
+    return (padded(1 << LG) + plan_tw_size(LG) + 2 * ((1 << LG) >> plan_lr(LG, 0)) + 16 + 8 + 1) / 2 * 2;
 }
 
 struct Smem {
-    float2 *buf, *tw0, *tws, *pre, *wcr;
+    float2 *buf, *tws, *ta, *tb, *pre, *wcr;
 };
-template <int LG, bool TW0G>
+template <int LG>
 __device__ __forceinline__ Smem carve(float2 *sm) {
+    constexpr int S0 = (1 << LG) >> plan_lr(LG, 0);
     Smem s;
     s.buf = sm;
-    s.tw0 = TW0G ? nullptr : sm + padded(1 << LG);
-    s.tws = sm + padded(1 << LG) + (TW0G ? 0 : (1 << LG));
-    s.pre = s.tws + plan_tw_size(LG);
+    s.tws = sm + padded(1 << LG);
+    s.ta = s.tws + plan_tw_size(LG);
+    s.tb = s.ta + S0;
+    s.pre = s.tb + S0;
     s.wcr = s.pre + 16;
     return s;
-}
-
-// ------------------------------------------------------------ tables (global)
-// First-pass tables of all C ranks, for transforms too long to keep them in
-// shared memory next to the data: tw0g[c m + i] = tw0_entry(i, C, c).
-template <int LG>
-__global__ void k_tw0_init(float2 *__restrict__ tw0g, int C) {
-    constexpr int m = 1 << LG;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < C * m; i += gridDim.x * blockDim.x)
-        tw0g[i] = tw0_entry<LG>(i % m, C, i / m);
 }
 
 // ------------------------------------------------------ async copy, cluster --
@@ -82,41 +74,47 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // ------------------------------------------------------------------ kspec --
 // spec[h][c][pos] = (FFT_2L(K_h zero-padded)[f] + D_h) / 2L for the frequency
 // f = C f' + c held at pos: the spectrum of K + D delta_0, so the convolution
-// adds the D u term with no extra pass over u.
+// adds the D u term with no extra pass over u. One CTA per (channel, rank);
+// the rank's twist comes from the per-CTA rank tables.
 // CPLX: the input is the complex signal K + i Ki (Ki [H, L]); its spectrum
 // then has no conjugate symmetry, which the convolution does not assume.
-template <int LG, int C, bool TW0G, bool CPLX = false>
+template <int LG, int C, bool CPLX = false>
 __global__ void __launch_bounds__(threads_for<LG>())
 k_kspec(const float *__restrict__ K, const float *__restrict__ Ki, const float *__restrict__ D, int H, int L,
-        float2 *__restrict__ spec, const float2 *__restrict__ tw0g) {
+        float2 *__restrict__ spec) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
     extern __shared__ float2 sm[];
-    const Smem s = carve<LG, TW0G>(sm);
+    const Smem s = carve<LG>(sm);
     const int c = blockIdx.x % C;
     const int slot = blockIdx.x / C, nslots = gridDim.x / C;
-    build_tables<LG>(s.tw0, s.tws, s.pre, C, c, threadIdx.x, T);
+    build_rank_tables<LG>(s.ta, s.tb, s.pre, C, c, threadIdx.x, T);
+    build_middle_tables<LG>(s.tws, threadIdx.x, T);
     if (threadIdx.x < C / 2) s.wcr[threadIdx.x] = unit_root((threadIdx.x * c) % C, C);
-    const float2 *t0 = TW0G ? tw0g + (size_t)c * m : s.tw0;
     __syncthreads();
+    constexpr int S0 = m >> plan_lr(LG, 0);
     const float scale = 1.0f / (float)(C * m);
     for (int h = slot; h < H; h += nslots) {
         const float *Kh = K + (size_t)h * L;
         const float *Kih = CPLX ? Ki + (size_t)h * L : nullptr;
         const float Dh = D != nullptr ? __ldg(D + h) : 0.0f;
-        forward_first<LG, T>(s.buf, t0, s.pre, [&](int k) {
-            float2 v = make_float2(__ldg(Kh + k), CPLX ? __ldg(Kih + k) : 0.0f);
-            static_for<1, C / 2>([&](auto r) {
-                const float kr = __ldg(Kh + k + r * m);
-                const float2 w = s.wcr[r];
-                if constexpr (CPLX) {
-                    v = cadd(v, cmul(make_float2(kr, __ldg(Kih + k + r * m)), w));
-                } else {
-                    v.x = fmaf(kr, w.x, v.x);
-                    v.y = fmaf(kr, w.y, v.y);
-                }
+        for (int j = threadIdx.x; j < S0; j += T) {
+            float2 x[1 << plan_lr(LG, 0)];
+            first_group_rec<LG>(x, j, s.ta, s.tb, s.pre, [&](int k) {
+                float2 v = make_float2(__ldg(Kh + k), CPLX ? __ldg(Kih + k) : 0.0f);
+                static_for<1, C / 2>([&](auto r) {
+                    const float kr = __ldg(Kh + k + r * m);
+                    const float2 w = s.wcr[r];
+                    if constexpr (CPLX) {
+                        v = cadd(v, cmul(make_float2(kr, __ldg(Kih + k + r * m)), w));
+                    } else {
+                        v.x = fmaf(kr, w.x, v.x);
+                        v.y = fmaf(kr, w.y, v.y);
+                    }
+                });
+                return v;
             });
-            return v;
-        });
+            store_first_group<LG>(s.buf, x, j);
+        }
         __syncthreads();
         forward_middle<LG, T>(s.buf, s.tws);
         float4 *out = reinterpret_cast<float4 *>(spec + ((size_t)h * C + c) * m);
@@ -132,125 +130,88 @@ k_kspec(const float *__restrict__ K, const float *__restrict__ Ki, const float *
 }
 
 // ---------------------------------------------------------------- fftconv --
-// STAGE: the input rows of the next row pair are copied to shared memory with
-// cp.async while the current pair is transformed (used when the whole pair,
-// 8 L bytes, fits next to the transform).
-// Without STAGE (L >= 32768) the first-pass inputs of all C ranks are formed
-// cooperatively: for each row pair, CTA c combines the chunks of the
-// positions k in its slice [c m/C, (c+1) m/C) for every rank r,
-//   v_r[k] = sum_{q < C/2} W_C^{q r} (u0[k + q m] + i u1[k + q m]),
-// into the cluster's slot of the scratch xs [C][m]; after a cluster barrier
-// each CTA reads its own rank's m inputs contiguously (each input value is
-// read from L2 once per cluster instead of once per CTA).
-template <int LG, int C, bool TW0G, bool STAGE>
+// L >= 32768: a cluster of C CTAs per row pair, CTA c holding rank c (the
+// frequencies C f + c, m = 2L / C points), persistent over row pairs. Rank c's
+// input is v_c[k] = W_N^{kc} sum_{q < C/2} W_C^{qc} x_q[k] from the C/2
+// nonzero input chunks x_q[k] = (u0 + i u1)[k + q m]. The C CTAs form these
+// cooperatively: CTA c takes the positions k of its slice [c m/C, (c+1) m/C),
+// loads the chunks of both rows once, runs the length-C DFT of
+// [x_0 .. x_{C/2-1}, 0 ..] and stores each rank r's value straight into CTA
+// r's buffer at k (distributed shared memory). After a cluster barrier every
+// CTA runs its first pass in place (the twist W_N^{kc} from its rank tables),
+// the transform, the product with its spectrum rank, the inverse; the C
+// partial results are then combined over distributed shared memory, rank c
+// writing the outputs t' = c SL + i + r m (r < C/2) of its slice:
+//   x[t' + r m] = sum_c W_C^{-c r} (W_N^{-c t'} Z_c[t']).
+// Barriers: the buffers are overwritten by the next pair's stores only after
+// every CTA's relaxed arrive that follows its combine's output stores (which
+// consume every remote value read).
+template <int LG, int C, bool CONJ>
 __global__ void __launch_bounds__(threads_for<LG>())
-k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L,
-          float *__restrict__ y, const float2 *__restrict__ tw0g, float conj_sign, float2 *__restrict__ xs) {
+k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L, float *__restrict__ y) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
-    constexpr int SL = m / C;                     // combine slice per rank
+    constexpr int SL = m / C;                     // slice of positions per rank
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     static_assert(C >= 2, "the convolution uses at least two ranks");
     extern __shared__ float2 sm[];
-    const Smem s = carve<LG, TW0G>(sm);
-    float *stage = reinterpret_cast<float *>(sm + smem_f2<LG>(TW0G));   // [2][L] when STAGE
+    const Smem s = carve<LG>(sm);
     cg::cluster_group cluster = cg::this_cluster();
     const int c = (int)cluster.block_rank();
     const int cl = blockIdx.x / C, ncl = gridDim.x / C;
     float2 *rbuf[C];
     static_for<0, C>([&](auto cc) { rbuf[cc] = cluster.map_shared_rank(s.buf, (int)cc); });
-    build_tables<LG>(s.tw0, s.tws, s.pre, C, c, threadIdx.x, T);
-    if (threadIdx.x < C / 2) s.wcr[threadIdx.x] = unit_root((threadIdx.x * c) % C, C);
-    const float2 *t0 = TW0G ? tw0g + (size_t)c * m : s.tw0;
+    build_rank_tables<LG>(s.ta, s.tb, s.pre, C, c, threadIdx.x, T);
+    build_middle_tables<LG>(s.tws, threadIdx.x, T);
+    cluster.sync();   // every CTA of the cluster runs before any reaches into its memory
 
     const int nbp = (Bt + 1) / 2;
     const long long npairs = (long long)H * nbp;
-    auto rows = [&](long long pr, const float *&u0, const float *&u1, bool &has1, int &h, int &b0) {
-        h = (int)(pr / nbp);
-        b0 = 2 * (int)(pr % nbp);
-        has1 = (b0 + 1) < Bt;
-        u0 = u + ((size_t)b0 * H + h) * L;
-        u1 = has1 ? u0 + (size_t)H * L : u0;
-    };
-    auto stage_rows = [&](long long pr) {   // both rows of pair pr -> stage (cp.async)
-        const float *u0, *u1; bool has1; int h, b0;
-        rows(pr, u0, u1, has1, h, b0);
-        for (int i = threadIdx.x; i < L / 2; i += T) {     // 16-byte chunks, L/4 per row
-            const int row = i >= L / 4, k = (i - row * (L / 4)) * 4;
-            cp_async16(stage + row * L + k, (row ? u1 : u0) + k, !row || has1);
-        }
-        cp_async_commit();
-    };
-    if constexpr (STAGE) {
-        if (cl < npairs) stage_rows(cl);
-    }
-    __syncthreads();
-
     bool first = true;
     for (long long pr = cl; pr < npairs; pr += ncl) {
-        const float *u0, *u1; bool has1; int h, b0;
-        rows(pr, u0, u1, has1, h, b0);
-        // ---- forward pass 0: x = u0 + i u1 (zero-padded to 2L), rank c's share
-        float2 *xsc = nullptr;
-        if constexpr (STAGE) {
-            cp_async_wait_all();
-            __syncthreads();
-        } else {   // the cooperative combination of the chunks (see above)
-            if (!first) cluster_wait();   // the partners are done reading this CTA's buffer
-            xsc = xs + (size_t)cl * C * m;
-            constexpr int SLC = m / C;
-            for (int i = threadIdx.x; i < SLC; i += T) {
-                const int k = c * SLC + i;
-                float2 x[C];
-                static_for<0, C / 2>([&](auto q) {
-                    x[q] = make_float2(__ldg(u0 + k + q * m), has1 ? __ldg(u1 + k + q * m) : 0.0f);
-                });
-                static_for<C / 2, C>([&](auto q) { x[q] = make_float2(0.0f, 0.0f); });
-                dft<C, -1>(x);   // x[r] = sum_q W_C^{q r} x_q
-                static_for<0, C>([&](auto r) { xsc[(size_t)r * m + k] = x[r]; });
-            }
-            cluster_arrive_release();
-            cluster_wait();
-        }
-        auto fetch = [&](int k) {
-            if constexpr (STAGE) {
-                float2 v = make_float2(stage[k], stage[L + k]);
-                static_for<1, C / 2>([&](auto r) {
-                    v = cadd(v, cmul(make_float2(stage[k + r * m], stage[L + k + r * m]), s.wcr[r]));
-                });
-                return v;
-            } else {
-                return __ldcg(xsc + (size_t)c * m + k);
-            }
-        };
-        if constexpr (S0 == T) {
-            // one group per thread: compute it, then (staged path) wait until
-            // the partner ranks have finished reading this CTA's buffer
-            float2 x[R0];
-            first_group<LG>(x, threadIdx.x, t0, s.pre, fetch);
-            if (STAGE && !first) cluster_wait();
-            store_first_group<LG>(s.buf, x, threadIdx.x);
-        } else {
-            if (STAGE && !first) cluster_wait();
-            forward_first<LG, T>(s.buf, t0, s.pre, fetch);
-        }
+        const int h = (int)(pr / nbp), b0 = 2 * (int)(pr % nbp);
+        const bool has1 = (b0 + 1) < Bt;
+        const float *u0 = u + ((size_t)b0 * H + h) * L;
+        const float *u1 = has1 ? u0 + (size_t)H * L : u0;
+        // ---- every rank's first-pass input, from this CTA's slice of positions
+        if (!first) cluster_wait();   // all buffers are read (previous combine)
         first = false;
-        __syncthreads();
-        if constexpr (STAGE) {   // the stage is free again: fetch the next pair
-            if (pr + ncl < npairs) stage_rows(pr + ncl);
+        for (int i = threadIdx.x; i < SL; i += T) {
+            const int k = c * SL + i;
+            float2 x[C];
+            static_for<0, C / 2>([&](auto q) {
+                x[q] = make_float2(__ldg(u0 + k + q * m), has1 ? __ldg(u1 + k + q * m) : 0.0f);
+            });
+            static_for<C / 2, C>([&](auto q) { x[q] = make_float2(0.0f, 0.0f); });
+            dft<C, -1>(x);   // x[r] = sum_q W_C^{q r} x_q
+            static_for<0, C>([&](auto r) { rbuf[r][pidx(k)] = x[r]; });
         }
+        cluster_arrive_release();
+        cluster_wait();
+        // ---- first pass in place, then the transform
+        for (int j = threadIdx.x; j < S0; j += T) {
+            float2 x[R0];
+            first_group_rec<LG>(x, j, s.ta, s.tb, s.pre, [&](int k) { return s.buf[pidx(k)]; });
+            store_first_group<LG>(s.buf, x, j);
+        }
+        __syncthreads();
         forward_middle<LG, T>(s.buf, s.tws);
         const float4 *sp = reinterpret_cast<const float4 *>(spec + ((size_t)h * C + c) * m);
         fused_middle<LG, T>(s.buf, [&](int base, auto &x) {
             constexpr int R = sizeof(x) / sizeof(float2);
             static_for<0, R / 2>([&](auto i) {
                 const float4 k2 = __ldg(sp + spec4_index<LG>(base, i));
-                x[2 * i] = cmul(x[2 * i], make_float2(k2.x, conj_sign * k2.y));
-                x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k2.z, conj_sign * k2.w));
+                if constexpr (CONJ) {
+                    x[2 * i] = cmulc(x[2 * i], make_float2(k2.x, k2.y));
+                    x[2 * i + 1] = cmulc(x[2 * i + 1], make_float2(k2.z, k2.w));
+                } else {
+                    x[2 * i] = cmul(x[2 * i], make_float2(k2.x, k2.y));
+                    x[2 * i + 1] = cmul(x[2 * i + 1], make_float2(k2.z, k2.w));
+                }
             });
         });
         __syncthreads();
         inverse_middle<LG, T>(s.buf, s.tws);
-        inverse_last<LG, T>(s.buf, t0, s.pre);
+        inverse_last_rec<LG, T>(s.buf, s.ta, s.tb, s.pre);
         cluster_arrive_release();
         cluster_wait();
         // ---- combine the C partial transforms; rank c writes t' in [c SL, (c+1) SL)
@@ -280,7 +241,7 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
                 }
             });
         }
-        cluster_arrive_relaxed();
+        cluster_arrive_relaxed();   // after the stores that consume every remote value read
     }
     // the partners may still read this CTA's buffer: wait before exiting
     if (!first) cluster_wait();
@@ -384,7 +345,7 @@ k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int
     const int j = threadIdx.x;
     const float2 tcj = unit_root(j, 2 * L);   // W_N^j
     const float2 cj = cconj(tcj);             // W_N^-j
-    __syncthreads();
+    cluster.sync();   // both CTAs run before either reaches into the other's memory
     const long long npairs = (long long)H * ((Bt + 1) / 2);
     const long long cl = blockIdx.x / 2, ncl = gridDim.x / 2;
     // a[p], b[p]: the two input chunks (row 0 + i row 1) at k = j + p S0
@@ -542,7 +503,7 @@ k_kspec_quad_half(float *__restrict__ K, const float *__restrict__ D, int H, flo
     build_middle_tables<LGH>(twh, threadIdx.x, T);
     const int j = threadIdx.x;
     const float2 tcj = unit_root(j, 2 * L);   // W_N^j
-    __syncthreads();
+    cluster.sync();   // both CTAs run before either reaches into the other's memory
     float2 *X = s.b0;   // the length-MH inverse transform of this CTA's parity
     bool first = true;
     for (int h = blockIdx.x / 2; h < H; h += gridDim.x / 2) {
@@ -636,14 +597,15 @@ k_irfft(float *K, int H, int L) {
     constexpr int m = 1 << LG, T = threads_for<LG>(), P = plan_P(LG);
     constexpr int SL = m / C;
     extern __shared__ float2 sm[];
-    const Smem s = carve<LG, false>(sm);
+    const Smem s = carve<LG>(sm);
     int c = 0, cl = blockIdx.x, ncl = gridDim.x;
     if constexpr (C > 1) {
         c = (int)cg::this_cluster().block_rank();
         cl = blockIdx.x / C;
         ncl = gridDim.x / C;
     }
-    build_tables<LG>(s.tw0, s.tws, s.pre, C, c, threadIdx.x, T);
+    build_rank_tables<LG>(s.ta, s.tb, s.pre, C, c, threadIdx.x, T);
+    build_middle_tables<LG>(s.tws, threadIdx.x, T);
     __syncthreads();
     const int npairs = (H + 1) / 2;
     for (int pr = cl; pr < npairs; pr += ncl) {
@@ -660,7 +622,7 @@ k_irfft(float *K, int H, int L) {
         dit_pass<LG, P - 1, +1, T>(s.buf, s.tws);
         __syncthreads();
         inverse_middle<LG, T>(s.buf, s.tws);
-        inverse_last<LG, T>(s.buf, s.tw0, s.pre);
+        inverse_last_rec<LG, T>(s.buf, s.ta, s.tb, s.pre);
         if constexpr (C > 1) cg::this_cluster().sync(); else __syncthreads();
         for (int i = threadIdx.x; i < SL; i += T) {
             const int tp = c * SL + i;
@@ -754,24 +716,20 @@ cudaError_t launch_clustered(Kern kern, int C, int nclusters, int T, size_t smem
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 // ---- convolution / kspec instantiation for one L ----
-// clusters of the L >= 32768 convolution launched at most (each owns a 2L
-// complex slot of scratch in the workspace for its cooperative first pass)
-constexpr int kMaxConvClusters = 24;
-
-template <int LG, int C, bool TW0G, bool STAGE>
+// C == 2 with LG <= 13: the one-CTA pair kernels (L <= 8192); otherwise the
+// C-way cluster kernels (L >= 32768; L = 16384 has its own below).
+template <int LG, int C>
 struct ConvKernels {
     static constexpr int T = threads_for<LG>();
-    static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>(TW0G);
-    static constexpr size_t smem_conv = smem + (STAGE ? 2 * sizeof(float) * (size_t)(C * (1 << LG) / 2) : 0);
-    static LaunchInfo info_conv, info_kspec, info_kspec_c;
-
-    static LaunchInfo info_kspec_pair;
+    static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>();
+    static constexpr bool kPair = C == 2 && LG <= 13;
+    static LaunchInfo info_conv[2], info_kspec, info_kspec_c, info_kspec_pair, info_pair[2];
 
     // Ki non-null: the spectrum of K + i Ki (cluster paths only)
     static cudaError_t kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st,
                              const float *Ki = nullptr) {
         float2 *spec = (float2 *)ws;
-        if constexpr (C == 2 && !TW0G && LG <= 13) {
+        if constexpr (kPair) {
             if (Ki != nullptr) return cudaErrorInvalidValue;
             // the one-CTA convolution's spectrum: persistent, one channel per CTA at a time
             auto kern = k_kspec_pair<LG>;
@@ -781,32 +739,25 @@ struct ConvKernels {
             if (e != cudaSuccess) return e;
             kern<<<res < H ? res : H, pair_threads<LG>(), psmem, st>>>(K, D, H, spec);
             return cudaGetLastError();
-        }
-        float2 *tw0g = nullptr;
-        if (TW0G) {
-            tw0g = (float2 *)((char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)));
-            k_tw0_init<LG><<<(C * (1 << LG) + 255) / 256, 256, 0, st>>>(tw0g, C);
-            cudaError_t e = cudaGetLastError();
+        } else {
+            auto kern = Ki != nullptr ? k_kspec<LG, C, true> : k_kspec<LG, C, false>;
+            int res = 0;
+            cudaError_t e = resident_units(kern, Ki != nullptr ? info_kspec_c : info_kspec, 1, T, smem, &res);
             if (e != cudaSuccess) return e;
+            // whole rank groups: nslots CTAs per rank
+            int nslots = res / C;
+            if (nslots < 1) nslots = 1;
+            if (nslots > H) nslots = H;
+            kern<<<nslots * C, T, smem, st>>>(K, Ki, D, H, L, spec);
+            return cudaGetLastError();
         }
-        auto kern = Ki != nullptr ? k_kspec<LG, C, TW0G, true> : k_kspec<LG, C, TW0G, false>;
-        int res = 0;
-        cudaError_t e = resident_units(kern, Ki != nullptr ? info_kspec_c : info_kspec, 1, T, smem, &res);
-        if (e != cudaSuccess) return e;
-        // whole rank groups: nslots CTAs per rank
-        int nslots = res / C;
-        if (nslots < 1) nslots = 1;
-        if (nslots > H) nslots = H;
-        kern<<<nslots * C, T, smem, st>>>(K, Ki, D, H, L, spec, (const float2 *)tw0g);
-        return cudaGetLastError();
     }
-
-    static LaunchInfo info_pair[2];
 
     static cudaError_t conv(const float *u, const void *ws, int Bt, int H, int L, float *y, bool adjoint,
                             cudaStream_t st) {
         const float2 *spec = (const float2 *)ws;
-        if constexpr (C == 2 && !TW0G && LG <= 13) {
+        const long long npairs = (long long)H * ((Bt + 1) / 2);
+        if constexpr (kPair) {
             // one CTA per row pair, both halves in one CTA; persistent grid
             auto kern = adjoint ? k_fftconv_pair<LG, true> : k_fftconv_pair<LG, false>;
             constexpr int TT = pair_threads<LG>();
@@ -814,42 +765,32 @@ struct ConvKernels {
             int res = 0;
             cudaError_t e = resident_units(kern, info_pair[adjoint], 1, TT, psmem, &res);
             if (e != cudaSuccess) return e;
-            const long long npairs = (long long)H * ((Bt + 1) / 2);
             const int grid = (long long)res < npairs ? res : (int)npairs;
             kern<<<grid, TT, psmem, st>>>(u, spec, Bt, H, L, y);
             return cudaGetLastError();
+        } else {
+            auto kern = adjoint ? k_fftconv<LG, C, true> : k_fftconv<LG, C, false>;
+            int res = 0;
+            cudaError_t e = resident_units(kern, info_conv[adjoint], C, T, smem, &res);
+            if (e != cudaSuccess) return e;
+            const int ncl = (long long)res < npairs ? res : (int)npairs;
+            e = launch_clustered(kern, C, ncl, T, smem, st, u, spec, Bt, H, L, y);
+            if (e != cudaSuccess) return e;
+            return cudaGetLastError();
         }
-        const float2 *tw0g = TW0G
-            ? (const float2 *)((const char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)))
-            : nullptr;
-        float2 *xs = STAGE ? nullptr
-                           : (float2 *)((char *)ws + align256((size_t)H * C * (1 << LG) * sizeof(float2)) +
-                                        (TW0G ? align256((size_t)C * (1 << LG) * sizeof(float2)) : 0));
-        auto kern = k_fftconv<LG, C, TW0G, STAGE>;
-        int res = 0;
-        cudaError_t e = resident_units(kern, info_conv, C, T, smem_conv, &res);
-        if (e != cudaSuccess) return e;
-        const long long npairs = (long long)H * ((Bt + 1) / 2);
-        int ncl = res;
-        if ((long long)ncl > npairs) ncl = (int)npairs;
-        if (ncl > kMaxConvClusters) ncl = kMaxConvClusters;   // scratch slots in the workspace
-        e = launch_clustered(kern, C, ncl, T, smem_conv, st, u, spec, Bt, H, L, y, tw0g, adjoint ? -1.0f : 1.0f,
-                             xs);
-        if (e != cudaSuccess) return e;
-        return cudaGetLastError();
     }
 };
-template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_conv;
-template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec;
-template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec_c;
-template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_pair[2];
-template <int LG, int C, bool TW0G, bool STAGE> LaunchInfo ConvKernels<LG, C, TW0G, STAGE>::info_kspec_pair;
+template <int LG, int C> LaunchInfo ConvKernels<LG, C>::info_conv[2];
+template <int LG, int C> LaunchInfo ConvKernels<LG, C>::info_kspec;
+template <int LG, int C> LaunchInfo ConvKernels<LG, C>::info_kspec_c;
+template <int LG, int C> LaunchInfo ConvKernels<LG, C>::info_kspec_pair;
+template <int LG, int C> LaunchInfo ConvKernels<LG, C>::info_pair[2];
 
 // ---- irfft instantiation ----
 template <int LG, int C>
 struct IrfftKernels {
     static constexpr int T = threads_for<LG>();
-    static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>(false);
+    static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>();
     static LaunchInfo info;
     static cudaError_t run(float *K, int H, int L, cudaStream_t st) {
         auto kern = k_irfft<LG, C>;
@@ -867,57 +808,44 @@ template <int LG, int C> LaunchInfo IrfftKernels<LG, C>::info;
 
 }  // namespace
 
-// Cluster split of the length-2L convolution transform: C CTAs of m = 2L/C
-// points, m <= 4096 up to L = 16384 (three CTAs fit one SM), longer
-// transforms use m = 8192 / 16384.
+// Cluster split of the length-2L convolution transform: C ranks of m = 2L/C
+// points (C = 2 up to L = 8192 is the one-CTA pair kernel's two halves).
 ConvGeom conv_geom(int L) {
     switch (L) {
-        case 16: return {2, 4, false};
-        case 32: return {2, 5, false};
-        case 64: return {2, 6, false};
-        case 128: return {2, 7, false};
-        case 256: return {2, 8, false};
-        case 512: return {2, 9, false};
-        case 1024: return {2, 10, false};
-        case 2048: return {2, 11, false};
-        case 4096: return {2, 12, false};
-        case 8192: return {2, 13, false};
-        case 16384: return {8, 12, false};
-        case 32768: return {8, 13, false};
-        case 65536: return {8, 14, true};
-        default: return {0, 0, false};
+        case 16: return {2, 4};
+        case 32: return {2, 5};
+        case 64: return {2, 6};
+        case 128: return {2, 7};
+        case 256: return {2, 8};
+        case 512: return {2, 9};
+        case 1024: return {2, 10};
+        case 2048: return {2, 11};
+        case 4096: return {2, 12};
+        case 8192: return {2, 13};
+        case 16384: return {4, 13};
+        case 32768: return {8, 13};
+        case 65536: return {8, 14};
+        default: return {0, 0};
     }
 }
 
-size_t conv_workspace_bytes(int H, int L) {
-    ConvGeom g = conv_geom(L);
-    size_t b = align256((size_t)H * 2 * L * sizeof(float2));
-    if (g.tw0_global) b += align256((size_t)2 * L * sizeof(float2));
-    if (L >= 32768) b += align256((size_t)kMaxConvClusters * 2 * L * sizeof(float2));   // cluster scratch
-    return b;
-}
+// the workspace holds only the spectrum of K + D delta_0: H x 2L complex values
+size_t conv_workspace_bytes(int H, int L) { return align256((size_t)H * 2 * L * sizeof(float2)); }
 
-// Longest L whose convolution stages the next row pair in shared memory
-// (cp.async prefetch; costs 8 L bytes of shared memory per CTA).
-#ifndef S4_CONV_STAGE_MAX_L
-#define S4_CONV_STAGE_MAX_L 4096
-#endif
-#define S4_STG(LL) ((LL) <= S4_CONV_STAGE_MAX_L)
-// (L, log2 m, C, first-pass table in global memory, staged input)
-#define S4_CONV_CASES(X)            \
-    X(16, 4, 2, false, S4_STG(16))        \
-    X(32, 5, 2, false, S4_STG(32))        \
-    X(64, 6, 2, false, S4_STG(64))        \
-    X(128, 7, 2, false, S4_STG(128))      \
-    X(256, 8, 2, false, S4_STG(256))      \
-    X(512, 9, 2, false, S4_STG(512))      \
-    X(1024, 10, 2, false, S4_STG(1024))   \
-    X(2048, 11, 2, false, S4_STG(2048))   \
-    X(4096, 12, 2, false, S4_STG(4096))   \
-    X(8192, 13, 2, false, false)    \
-    X(16384, 12, 8, false, false)   \
-    X(32768, 13, 8, false, false)   \
-    X(65536, 14, 8, true, false)
+// (L, log2 m, C)
+#define S4_CONV_CASES(X) \
+    X(16, 4, 2)          \
+    X(32, 5, 2)          \
+    X(64, 6, 2)          \
+    X(128, 7, 2)         \
+    X(256, 8, 2)         \
+    X(512, 9, 2)         \
+    X(1024, 10, 2)       \
+    X(2048, 11, 2)       \
+    X(4096, 12, 2)       \
+    X(8192, 13, 2)       \
+    X(32768, 13, 8)      \
+    X(65536, 14, 8)
 
 namespace {
 LaunchInfo g_quad_conv[2], g_quad_kspec[2];
@@ -967,7 +895,7 @@ cudaError_t quad_conv(const float *u, const void *ws, int Bt, int H, float *y, b
 cudaError_t launch_kspec(const float *K, const float *D, int H, int L, void *ws, cudaStream_t st, const float *Ki) {
     if (L == 2 << kQuadLG) return quad_kspec(K, D, H, ws, st, Ki);
     switch (L) {
-#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::kspec(K, D, H, L, ws, st, Ki);
+#define X(LL, LG, C) case LL: return ConvKernels<LG, C>::kspec(K, D, H, L, ws, st, Ki);
         S4_CONV_CASES(X)
 #undef X
         default: return cudaErrorInvalidValue;
@@ -978,7 +906,7 @@ cudaError_t launch_fftconv(const float *u, const void *ws, int Bt, int H, int L,
                            bool adjoint) {
     if (L == 2 << kQuadLG) return quad_conv(u, ws, Bt, H, y, adjoint, st);
     switch (L) {
-#define X(LL, LG, C, G, S) case LL: return ConvKernels<LG, C, G, S>::conv(u, ws, Bt, H, L, y, adjoint, st);
+#define X(LL, LG, C) case LL: return ConvKernels<LG, C>::conv(u, ws, Bt, H, L, y, adjoint, st);
         S4_CONV_CASES(X)
 #undef X
         default: return cudaErrorInvalidValue;
