@@ -33,21 +33,25 @@
 namespace s4 {
 
 // ------------------------------------------------------------------ plan --
-// log2 of the radix of pass s for a 2^lg-point transform. The first and the
-// last pass are radix 16 (from lg = 8 on); the bits left over go to the
-// fewest middle passes of radix at most 32, split as evenly as they allow
-// (lg = 13: 16 x 32 x 16, three passes; every pass is one round trip through
-// shared memory, which bounds these transforms as much as the arithmetic
-// does). Every strided pass then has a stride of at least 16 points and the
+// log2 of the radix of pass s for a 2^lg-point transform. The last pass is
+// radix 16 and so is the first (radix 32 from lg = 14 on); the bits left
+// over go to the fewest middle passes of radix at most 32, split as evenly
+// as they allow (lg = 13: 16 x 32 x 16, lg = 14: 32 x 32 x 16, three passes;
+// every pass is one round trip through shared memory, which bounds these
+// transforms as much as the arithmetic does). Every strided pass then has a stride of at least 16 points and the
 // last pass works on 16 consecutive points (moved as 16-byte pairs), which
 // keeps all of them free of shared-memory bank conflicts with the padding
 // below.
-__host__ __device__ constexpr int plan_P(int lg) { return lg <= 8 ? 2 : 2 + (lg - 8 + 4) / 5; }
+// radix bits of the first pass: 16, or 32 from 2^14 points on (one middle
+// pass of radix 32 then still covers the rest)
+__host__ __device__ constexpr int plan_first(int lg) { return lg >= 14 ? 5 : 4; }
+__host__ __device__ constexpr int plan_P(int lg) { return lg <= 8 ? 2 : 2 + (lg - plan_first(lg) - 4 + 4) / 5; }
 __host__ __device__ constexpr int plan_lr(int lg, int s) {
     if (lg == 4) return 2;
     if (lg <= 8) return s == 0 ? lg - 4 : 4;
-    if (s == 0 || s == plan_P(lg) - 1) return 4;
-    const int k = plan_P(lg) - 2, mid = lg - 8;
+    if (s == 0) return plan_first(lg);
+    if (s == plan_P(lg) - 1) return 4;
+    const int k = plan_P(lg) - 2, mid = lg - plan_first(lg) - 4;
     return mid / k + (s - 1 < mid % k ? 1 : 0);
 }
 // block size of pass s (the sub-transform length it starts)

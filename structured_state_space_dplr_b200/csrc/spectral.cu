@@ -37,10 +37,10 @@ __host__ __device__ constexpr int threads_for() {
 }
 
 // dynamic shared memory of the C-way split kernels, in float2:
-// buf | tws | ta[S0] | tb[S0] | pre[16] | wcr[8]
+// buf | tws | ta[S0] | tb[S0] | pre[32] | wcr[8]
 template <int LG>
 __host__ __device__ constexpr int smem_f2() {
-    return (padded(1 << LG) + plan_tw_size(LG) + 2 * ((1 << LG) >> plan_lr(LG, 0)) + 16 + 8 + 1) / 2 * 2;
+    return (padded(1 << LG) + plan_tw_size(LG) + 2 * ((1 << LG) >> plan_lr(LG, 0)) + 32 + 8 + 1) / 2 * 2;
 }
 
 struct Smem {
@@ -55,7 +55,7 @@ __device__ __forceinline__ Smem carve(float2 *sm) {
     s.ta = s.tws + plan_tw_size(LG);
     s.tb = s.ta + S0;
     s.pre = s.tb + S0;
-    s.wcr = s.pre + 16;
+    s.wcr = s.pre + 32;
     return s;
 }
 
@@ -74,45 +74,57 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // ------------------------------------------------------------------ kspec --
 // spec[h][c][pos] = (FFT_2L(K_h zero-padded)[f] + D_h) / 2L for the frequency
 // f = C f' + c held at pos: the spectrum of K + D delta_0, so the convolution
-// adds the D u term with no extra pass over u. One CTA per (channel, rank);
-// the rank's twist comes from the per-CTA rank tables.
-// CPLX: the input is the complex signal K + i Ki (Ki [H, L]); its spectrum
-// then has no conjugate symmetry, which the convolution does not assume.
-template <int LG, int C, bool CPLX = false>
+// adds the D u term with no extra pass over u. CPLX: the input is the
+// complex signal K + i Ki (Ki [H, L]); its spectrum then has no conjugate
+// symmetry, which the convolution does not assume.
+// The same spectrum for the cluster convolution (L >= 32768), one cluster of
+// C CTAs per channel (persistent over channels), CTA c producing rank c.
+// Rank c's input v_c[k] = W_N^{kc} sum_{q < C/2} W_C^{qc} K[k + q m] is formed
+// cooperatively as in k_fftconv: CTA c reads K (and Ki) once for its slice of
+// positions, runs the length-C DFT of the chunks and stores each rank's value
+// into that rank's buffer (distributed shared memory). Barriers: release /
+// acquire around those stores; a relaxed arrive after the rank's spectrum is
+// stored (its buffer is no longer read), waited on before the next channel's
+// stores.
+template <int LG, int C, bool CPLX>
 __global__ void __launch_bounds__(threads_for<LG>())
-k_kspec(const float *__restrict__ K, const float *__restrict__ Ki, const float *__restrict__ D, int H, int L,
-        float2 *__restrict__ spec) {
+k_kspec_cl(const float *__restrict__ K, const float *__restrict__ Ki, const float *__restrict__ D, int H, int L,
+           float2 *__restrict__ spec) {
     constexpr int m = 1 << LG, T = threads_for<LG>();
+    constexpr int SL = m / C, S0 = m >> plan_lr(LG, 0);
     extern __shared__ float2 sm[];
     const Smem s = carve<LG>(sm);
-    const int c = blockIdx.x % C;
-    const int slot = blockIdx.x / C, nslots = gridDim.x / C;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int c = (int)cluster.block_rank();
+    const int cl = blockIdx.x / C, ncl = gridDim.x / C;
+    float2 *rbuf[C];
+    static_for<0, C>([&](auto cc) { rbuf[cc] = cluster.map_shared_rank(s.buf, (int)cc); });
     build_rank_tables<LG>(s.ta, s.tb, s.pre, C, c, threadIdx.x, T);
     build_middle_tables<LG>(s.tws, threadIdx.x, T);
-    if (threadIdx.x < C / 2) s.wcr[threadIdx.x] = unit_root((threadIdx.x * c) % C, C);
-    __syncthreads();
-    constexpr int S0 = m >> plan_lr(LG, 0);
+    cluster.sync();   // every CTA of the cluster runs before any reaches into its memory
     const float scale = 1.0f / (float)(C * m);
-    for (int h = slot; h < H; h += nslots) {
+    bool first = true;
+    for (int h = cl; h < H; h += ncl) {
         const float *Kh = K + (size_t)h * L;
         const float *Kih = CPLX ? Ki + (size_t)h * L : nullptr;
         const float Dh = D != nullptr ? __ldg(D + h) : 0.0f;
+        if (!first) cluster_wait();   // every rank's buffer is free (previous channel done)
+        first = false;
+        for (int i = threadIdx.x; i < SL; i += T) {
+            const int k = c * SL + i;
+            float2 x[C];
+            static_for<0, C / 2>([&](auto q) {
+                x[q] = make_float2(__ldg(Kh + k + q * m), CPLX ? __ldg(Kih + k + q * m) : 0.0f);
+            });
+            static_for<C / 2, C>([&](auto q) { x[q] = make_float2(0.0f, 0.0f); });
+            dft<C, -1>(x);
+            static_for<0, C>([&](auto r) { rbuf[r][pidx(k)] = x[r]; });
+        }
+        cluster_arrive_release();
+        cluster_wait();
         for (int j = threadIdx.x; j < S0; j += T) {
             float2 x[1 << plan_lr(LG, 0)];
-            first_group_rec<LG>(x, j, s.ta, s.tb, s.pre, [&](int k) {
-                float2 v = make_float2(__ldg(Kh + k), CPLX ? __ldg(Kih + k) : 0.0f);
-                static_for<1, C / 2>([&](auto r) {
-                    const float kr = __ldg(Kh + k + r * m);
-                    const float2 w = s.wcr[r];
-                    if constexpr (CPLX) {
-                        v = cadd(v, cmul(make_float2(kr, __ldg(Kih + k + r * m)), w));
-                    } else {
-                        v.x = fmaf(kr, w.x, v.x);
-                        v.y = fmaf(kr, w.y, v.y);
-                    }
-                });
-                return v;
-            });
+            first_group_rec<LG>(x, j, s.ta, s.tb, s.pre, [&](int k) { return s.buf[pidx(k)]; });
             store_first_group<LG>(s.buf, x, j);
         }
         __syncthreads();
@@ -125,8 +137,10 @@ k_kspec(const float *__restrict__ K, const float *__restrict__ Ki, const float *
                                                 (x[2 * i + 1].x + Dh) * scale, x[2 * i + 1].y * scale);
             });
         });
-        __syncthreads();
+        // the buffer was read into the stores above: partners may write it again
+        cluster_arrive_relaxed();
     }
+    if (!first) cluster_wait();   // pairs the last arrive
 }
 
 // ---------------------------------------------------------------- fftconv --
@@ -740,15 +754,13 @@ struct ConvKernels {
             kern<<<res < H ? res : H, pair_threads<LG>(), psmem, st>>>(K, D, H, spec);
             return cudaGetLastError();
         } else {
-            auto kern = Ki != nullptr ? k_kspec<LG, C, true> : k_kspec<LG, C, false>;
+            auto kern = Ki != nullptr ? k_kspec_cl<LG, C, true> : k_kspec_cl<LG, C, false>;
             int res = 0;
-            cudaError_t e = resident_units(kern, Ki != nullptr ? info_kspec_c : info_kspec, 1, T, smem, &res);
+            cudaError_t e = resident_units(kern, Ki != nullptr ? info_kspec_c : info_kspec, C, T, smem, &res);
             if (e != cudaSuccess) return e;
-            // whole rank groups: nslots CTAs per rank
-            int nslots = res / C;
-            if (nslots < 1) nslots = 1;
-            if (nslots > H) nslots = H;
-            kern<<<nslots * C, T, smem, st>>>(K, Ki, D, H, L, spec);
+            const int ncl = res < H ? res : H;
+            e = launch_clustered(kern, C, ncl, T, smem, st, K, Ki, D, H, L, spec);
+            if (e != cudaSuccess) return e;
             return cudaGetLastError();
         }
     }
