@@ -7,11 +7,13 @@
 
 namespace s4 {
 
-// 128 threads x 2 frequencies per CTA: small CTAs keep the last wave full
-// (at H = 256, L = 4096: 2048 CTAs over 7 x 148 resident, 1.98 waves, where
-// 256-thread CTAs made 1024 over 3 x 148, 2.3 waves with the last 30 % full)
+// 128 threads x 4 frequencies per CTA (126 registers, four independent
+// frequencies in flight per thread), the fastest of the shapes measured
+// (CUDA events, H = 256: 21.0 us at L = 4096 and 66.7 us at L = 16384,
+// against 21.3 / 70.6 us for 256 x 2, 21.6 / 70.7 for 128 x 2 and
+// 21.3 / 68.5 for 64 x 4)
 constexpr int kCauchyThreads = 128;
-constexpr int kCauchyFreqs = 2;   // frequencies per thread
+constexpr int kCauchyFreqs = 4;   // frequencies per thread
 
 template <int T, int F>
 __global__ void __launch_bounds__(T)
