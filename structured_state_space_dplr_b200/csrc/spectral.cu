@@ -35,6 +35,12 @@ template <int LG>
 __host__ __device__ constexpr int threads_for() {
     return (1 << LG) / 16 < 32 ? 32 : ((1 << LG) / 16 > 512 ? 512 : (1 << LG) / 16);
 }
+// threads and CTAs per SM of the C-way cluster kernels: a split 16 ways keeps
+// two 256-thread CTAs on an SM (registers and shared memory for both)
+template <int LG, int C>
+__host__ __device__ constexpr int cl_threads() { return C >= 16 ? 256 : threads_for<LG>(); }
+template <int C>
+__host__ __device__ constexpr int cl_min_blocks() { return C >= 16 ? 2 : 1; }
 
 // dynamic shared memory of the C-way split kernels, in float2:
 // buf | tws | ta[S0] | tb[S0] | pre[32] | wcr[8]
@@ -87,10 +93,10 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // stored (its buffer is no longer read), waited on before the next channel's
 // stores.
 template <int LG, int C, bool CPLX>
-__global__ void __launch_bounds__(threads_for<LG>())
+__global__ void __launch_bounds__(cl_threads<LG, C>(), cl_min_blocks<C>())
 k_kspec_cl(const float *__restrict__ K, const float *__restrict__ Ki, const float *__restrict__ D, int H, int L,
            float2 *__restrict__ spec) {
-    constexpr int m = 1 << LG, T = threads_for<LG>();
+    constexpr int m = 1 << LG, T = cl_threads<LG, C>();
     constexpr int SL = m / C, S0 = m >> plan_lr(LG, 0);
     extern __shared__ float2 sm[];
     const Smem s = carve<LG>(sm);
@@ -161,9 +167,9 @@ k_kspec_cl(const float *__restrict__ K, const float *__restrict__ Ki, const floa
 // every CTA's relaxed arrive that follows its combine's output stores (which
 // consume every remote value read).
 template <int LG, int C, bool CONJ>
-__global__ void __launch_bounds__(threads_for<LG>())
+__global__ void __launch_bounds__(cl_threads<LG, C>(), cl_min_blocks<C>())
 k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, int H, int L, float *__restrict__ y) {
-    constexpr int m = 1 << LG, T = threads_for<LG>();
+    constexpr int m = 1 << LG, T = cl_threads<LG, C>();
     constexpr int SL = m / C;                     // slice of positions per rank
     constexpr int R0 = 1 << plan_lr(LG, 0), S0 = m / R0;
     static_assert(C >= 2, "the convolution uses at least two ranks");
@@ -702,6 +708,10 @@ cudaError_t resident_units(Kern kern, LaunchInfo &info, int C, int T, size_t sme
     if (v == 0) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
+        if (C > 8) {   // clusters beyond the portable size of 8 are opted into per kernel
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+        }
         if (C > 1) {
             cudaLaunchConfig_t cfg = {};
             cudaLaunchAttribute at[1];
@@ -749,7 +759,7 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 // C-way cluster kernels (L >= 32768; L = 16384 has its own below).
 template <int LG, int C>
 struct ConvKernels {
-    static constexpr int T = threads_for<LG>();
+    static constexpr int T = cl_threads<LG, C>();
     static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>();
     static constexpr bool kPair = C == 2 && LG <= 13;
     static LaunchInfo info_conv[2], info_kspec, info_kspec_c, info_kspec_pair, info_pair[2];
@@ -836,7 +846,11 @@ template <int LG, int C> LaunchInfo IrfftKernels<LG, C>::info;
 }  // namespace
 
 // Cluster split of the length-2L convolution transform: C ranks of m = 2L/C
-// points (C = 2 up to L = 8192 is the one-CTA pair kernel's two halves).
+// points (C = 2 up to L = 8192 is the one-CTA pair kernel's two halves). At
+// L = 65536 the split is 16 ways (a cluster of 16, beyond the portable size,
+// two 256-thread CTAs per SM): 219 us against 231 us for 8 ranks of 2^14
+// points at H = 64, batch 4, where one 156 KB CTA per SM left 28 SMs idle
+// (15 clusters of 8 fit).
 ConvGeom conv_geom(int L) {
     switch (L) {
         case 16: return {2, 4};
@@ -851,7 +865,7 @@ ConvGeom conv_geom(int L) {
         case 8192: return {2, 13};
         case 16384: return {4, 13};
         case 32768: return {8, 13};
-        case 65536: return {8, 14};
+        case 65536: return {16, 13};
         default: return {0, 0};
     }
 }
@@ -872,7 +886,7 @@ size_t conv_workspace_bytes(int H, int L) { return align256((size_t)H * 2 * L * 
     X(4096, 12, 2)       \
     X(8192, 13, 2)       \
     X(32768, 13, 8)      \
-    X(65536, 14, 8)
+    X(65536, 13, 16)
 
 namespace {
 LaunchInfo g_quad_conv[2], g_quad_kspec[2];
