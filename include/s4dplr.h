@@ -132,8 +132,9 @@ s4_status s4_irfft_packed(float *K, int H, int L, cudaStream_t stream);
  *   device, 16-byte aligned, must not overlap u, K, D or the workspace.
  *   Bt, H >= 1; L a power of two in [16, 65536]; Bt*H*L < 2^40.
  *   workspace : device, 256-byte aligned, at least
- *               s4_fft_conv_workspace_size(H, L) bytes; holds the spectrum
- *               of the zero-padded K + D delta_0 after the call.
+ *               s4_fft_conv_workspace_size(H, L) bytes (H * 2L complex
+ *               floats, rounded up to 256 bytes); holds the spectrum of the
+ *               zero-padded K + D delta_0 after the call.
  * Errors: S4_ERR_INVALID_ARG, S4_ERR_UNSUPPORTED, S4_ERR_WORKSPACE, S4_ERR_CUDA.
  * ------------------------------------------------------------------------ */
 s4_status s4_fft_conv_workspace_size(int H, int L, size_t *bytes);
@@ -234,11 +235,14 @@ s4_status s4_kernel_dplr_backward_ws(const s4_c32 *Lambda, const s4_c32 *P, cons
  *
  * s4_kernel_dplr_prepare = s4_kernel_dplr(...) followed by
  * s4_fft_conv_prepare(K, D, ...): it writes K[H, L] and the convolution
- * spectrum of K + D delta_0 into the workspace. For L <= 4096 both come out
+ * spectrum of K + D delta_0 into the workspace. For L <= 8192 both come out
  * of a single kernel per channel (the generating function is written
  * straight into the inverse transform's input order, and the inverse
- * transform's output starts the zero-padded forward transform). D may be
- * NULL (no feed-through term).
+ * transform's output starts the zero-padded forward transform); for
+ * L = 16384 the Cauchy stage is one launch and the inverse transform, K and
+ * the spectrum a second (K is stored, never read back); longer L run the
+ * Cauchy stage, the inverse transform and the spectrum as three launches.
+ * D may be NULL (no feed-through term).
  *
  * s4_forward_dplr = s4_kernel_dplr_prepare followed by s4_fft_conv_apply:
  * y[Bt, H, L] from the DPLR parameters and u in one call; K and the

@@ -77,6 +77,12 @@ def test_workspace_size(lib):
     assert lib.s4_fft_conv_workspace_size(256, 1000, ctypes.byref(n)) == _lib.S4_ERR_UNSUPPORTED
     assert lib.s4_fft_conv_workspace_size(0, 1024, ctypes.byref(n)) == _lib.S4_ERR_INVALID_ARG
     assert lib.s4_fft_conv_workspace_size(4, 1024, None) == _lib.S4_ERR_INVALID_ARG
+    # the workspace is the spectrum alone at every length: H x 2L complex floats
+    for H in (1, 3, 256):
+        for lg in range(4, 17):
+            L = 1 << lg
+            assert lib.s4_fft_conv_workspace_size(H, L, ctypes.byref(n)) == 0
+            assert n.value == (H * 2 * L * 8 + 255) // 256 * 256
 
 
 def conv(lib, u=FAKE, K=FAKE + 0x10000000, D=FAKE + 0x20000000, Bt=2, H=4, L=1024, y=FAKE2,

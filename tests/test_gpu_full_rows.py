@@ -28,7 +28,8 @@ def _check_rows(inp, yg_rows, Kref, rows):
         assert rel_l2(ys[i], yr[i]) <= 4 * Y_TOL, rows[i]
 
 
-@pytest.mark.parametrize("cfg,rows", [(3, [(0, 3), (7, 254)]), (4, [(0, 1), (3, 62)])])
+@pytest.mark.parametrize("cfg,rows", [(2, [(0, 0), (15, 255), (8, 128)]), (3, [(0, 3), (7, 254)]),
+                                      (4, [(0, 1), (3, 62)])])
 def test_dplr_full_size_full_rows(cfg, rows):
     import structured_state_space_dplr_b200 as s4
     torch = torch_cuda()
