@@ -60,12 +60,19 @@ E2E_CHUNKS = 16   # row-pair chunks of the host-buffer pipeline
 # bytes: read y and x, write out
 BLOCK_FLOP_PER_ELEM = lambda H: 4 * H   # noqa: E731
 BLOCK_PROJ_BYTES_PER_ELEM = 12
-KERNEL_SOURCES = ["common.cuh", "fft.cuh", "pairs.cuh", "spectral.cu"]
+# the sources each workload's convolution kernel is built from (L <= 8192:
+# the one-CTA pair kernel; L = 16384: the cluster of two; longer: the
+# cluster split), hashed to tell whether a recorded ncu figure still holds
+_CONV_COMMON = ["common.cuh", "fft.cuh", "pairs.cuh", "cluster.cuh"]
+KERNEL_SOURCES = {1: _CONV_COMMON + ["spectral.cu"], 2: _CONV_COMMON + ["spectral.cu"],
+                  3: _CONV_COMMON + ["quad.cu"], 4: _CONV_COMMON + ["spectral.cu"],
+                  5: _CONV_COMMON + ["spectral.cu"]}
 # DRAM traffic of one convolution launch per workload, from committed ncu
 # summaries (reported only while the convolution's sources are unchanged)
 TRAFFIC_FILES = {
     2: os.path.join(ROOT, "profiles", "fftconv_h256_l4096_b16_traffic.txt"),
     3: os.path.join(ROOT, "profiles", "fftconv_h256_l16384_b8_traffic.txt"),
+    4: os.path.join(ROOT, "profiles", "fftconv_h64_l65536_b4_traffic.txt"),
 }
 # channels of each workload the CPU leg runs the oracle on (every row, every
 # output), sized to a few seconds of fp64 work on the host
@@ -86,9 +93,9 @@ def peaks():
     return FALLBACK_HBM_GBS, NOMINAL_SM_MHZ, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(cfg):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[cfg]:
         with open(os.path.join(ROOT, "structured_state_space_dplr_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -107,7 +114,7 @@ def recorded_traffic(cfg):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash(cfg):
         return None
     try:
         return float(vals["dram_bytes_per_launch_full_size"])

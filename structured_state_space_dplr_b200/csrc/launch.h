@@ -40,6 +40,12 @@ cudaError_t launch_irfft_packed(float *K, int H, int L, cudaStream_t st);
 // (L = 16384: one fused launch; other L: launch_irfft_packed + launch_kspec)
 cudaError_t launch_kspec_from_half(float *K, const float *D, int H, int L, void *ws, cudaStream_t st);
 
+// ---- quad.cu: L = 16384 (a cluster of two CTAs holding four ranks) ----
+cudaError_t launch_kspec_l16k(const float *K, const float *D, int H, void *ws, cudaStream_t st, const float *Ki);
+cudaError_t launch_fftconv_l16k(const float *u, const void *ws, int Bt, int H, float *y, bool adjoint,
+                                cudaStream_t st);
+cudaError_t launch_kspec_from_half_l16k(float *K, const float *D, int H, void *ws, cudaStream_t st);
+
 // ---- kgen.cu: K and the convolution spectrum of K + D delta_0 in one launch
 // (L <= 8192; longer L runs k_cauchy, then launch_kspec_from_half) ----
 cudaError_t launch_kgen(const float2 *Lambda, const float2 *P, const float2 *Q, const float2 *B, const float2 *C,

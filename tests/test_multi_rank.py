@@ -60,7 +60,7 @@ def test_recorded_traffic_follows_the_convolution_sources(tmp_path, monkeypatch)
     convolution's sources matches the one the counters were taken with."""
     import bench
     good = tmp_path / "traffic.txt"
-    good.write_text(f"kernel_source_sha256_16: {bench.kernel_source_hash()}\n"
+    good.write_text(f"kernel_source_sha256_16: {bench.kernel_source_hash(3)}\n"
                     "dram_bytes_per_launch_full_size: 123456\n")
     monkeypatch.setitem(bench.TRAFFIC_FILES, 3, str(good))
     assert bench.recorded_traffic(3) == 123456.0
@@ -69,6 +69,9 @@ def test_recorded_traffic_follows_the_convolution_sources(tmp_path, monkeypatch)
     monkeypatch.setitem(bench.TRAFFIC_FILES, 3, str(stale))
     assert bench.recorded_traffic(3) is None
     assert bench.recorded_traffic(1) is None     # no capture recorded for that workload
+    # each workload's hash covers the sources of its own convolution kernel
+    assert bench.kernel_source_hash(3) != bench.kernel_source_hash(2)
+    assert bench.kernel_source_hash(2) == bench.kernel_source_hash(5)
 
 
 def test_launch_counts_and_reference_sample_sizes():
