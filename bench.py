@@ -223,16 +223,40 @@ def conv_kernel_name(L):
         return "k_fftconv_pair"
     if L == 16384:
         return "k_fftconv_quad"
-    return "k_fftconv (cluster of 8)"
+    return "k_fftconv (cluster of 16)"
+
+
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured torch CUDA graph (kept with keep_graph=True):
+    the launches one replay issues."""
+    from cuda.bindings import runtime as rt
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, _, n = rt.cudaGraphGetNodes(graph, 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    count = 0
+    for nd in nodes[:n]:
+        err, kind = rt.cudaGraphNodeGetType(nd)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaGraphNodeGetType: {err}")
+        count += kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    return count
 
 
 def launches_per_step(c):
     """Kernel launches of one forward step (generation + convolution)."""
     L = c["L"]
     if c["kind"] == "s4d":
-        gen = 2 + (1 if L == 65536 else 0)   # Vandermonde, spectrum (+ first-pass table)
+        gen = 2                               # Vandermonde, spectrum
+    elif L <= 8192:
+        gen = 1                               # k_kgen (Cauchy, inverse, spectrum)
+    elif L == 16384:
+        gen = 2                               # k_cauchy, k_kspec_quad_half
     else:
-        gen = 1 if L <= 8192 else (3 + (1 if L == 65536 else 0))
+        gen = 3                               # k_cauchy, k_irfft, k_kspec_cl
     return gen + 1
 
 
@@ -293,7 +317,7 @@ def forward_case(s4, torch, dev, cfg, seed, steps, warmup, flags, dist=None, clo
     cap.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap):
         for s in sets:
-            g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            g1, g2 = torch.cuda.CUDAGraph(keep_graph=True), torch.cuda.CUDAGraph(keep_graph=True)
             with torch.cuda.graph(g1, stream=cap):
                 gen_stage(s)
             with torch.cuda.graph(g2, stream=cap):
@@ -301,6 +325,9 @@ def forward_case(s4, torch, dev, cfg, seed, steps, warmup, flags, dist=None, clo
             gen_graphs.append(g1)
             conv_graphs.append(g2)
     torch.cuda.current_stream().wait_stream(cap)
+    launches = graph_kernel_nodes(gen_graphs[0]) + graph_kernel_nodes(conv_graphs[0])
+    for g in gen_graphs + conv_graphs:
+        g.instantiate()
     for i in range(warmup):
         gen_graphs[i % nsets].replay()
         conv_graphs[i % nsets].replay()
@@ -355,7 +382,7 @@ def forward_case(s4, torch, dev, cfg, seed, steps, warmup, flags, dist=None, clo
     stage.append(cev[0].elapsed_time(cev[1]) / steps)
 
     rec = {"c": c, "alg": alg, "ms": ms, "stage": stage, "clocks": clk, "nsets": nsets, "set_bytes": set_bytes,
-           "inp": inp if keep else None, "sets": sets if keep else None, "names": names}
+           "launches": launches, "inp": inp if keep else None, "sets": sets if keep else None, "names": names}
     if not keep:
         del sets
         torch.cuda.empty_cache()
@@ -403,7 +430,7 @@ def forward_record(rec, steps, world, hbm, fp32_peak, sm_max_mhz, peak_src, with
                      "algorithmic_bytes": alg["conv_bytes"],
                      "algorithmic_bytes_formula": "8*Bt*H*L (u read, y written) + 16*H*L (spectrum read)"},
         "cauchy": cauchy,
-        "gpu_launches_per_step": launches_per_step(c),
+        "gpu_launches_per_step": rec["launches"],
     }
 
 
@@ -700,7 +727,8 @@ def run_gpu(args, rank, world, local_rank):
                                                   else "s4_forward_dplr_host")
                                          + f", pinned host u/y, {E2E_CHUNKS} row-pair chunks; the layer's "
                                            "parameters resident on the device"},
-        "gpu_launches": launches_per_step(c) * args.steps,
+        "gpu_launches": rec["launches"] * args.steps,
+        "gpu_launches_source": "kernel nodes of the captured generation and convolution graphs, x steps",
         "decode": decode,
         "variants": variants,
         "backward": backward,

@@ -80,7 +80,7 @@ def test_launch_counts_and_reference_sample_sizes():
     import bench
     import s4inputs
     C = s4inputs.CONFIGS
-    assert [bench.launches_per_step(C[k]) for k in (1, 2, 3, 4, 5)] == [2, 2, 4, 5, 3]
+    assert [bench.launches_per_step(C[k]) for k in (1, 2, 3, 4, 5)] == [2, 2, 3, 4, 3]
     assert [bench.reference_chunk(C[k]) for k in (1, 2, 3, 4, 5)] == [4, 7, 1, 1, 1]
 
 
