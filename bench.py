@@ -54,7 +54,8 @@ NOMINAL_SM_MHZ = 1965.0
 # two products by 1/|q|^2) and four complex Cauchy sums as 16 FMAs (32 flop)
 CAUCHY_FLOP_PER_TERM = 40
 VANDERMONDE_FLOP_PER_TERM = 4
-E2E_CHUNKS = 16   # row-pair chunks of the host-buffer pipeline
+E2E_CHUNKS = 2     # row-pair chunks of the host-buffer pipeline
+E2E_INFLIGHT = 2   # consecutive end-to-end steps in flight
 # S4Block projection per (b, t) element of the output: 2 dot products of
 # length H (value and gate rows of W) = 4 H flop per output element; HBM
 # bytes: read y and x, write out
@@ -518,36 +519,50 @@ def run_gpu(args, rank, world, local_rank):
     # every step uploads that step's batch u and downloads its output y; the
     # layer's parameters are resident on the device (uploaded once, as a
     # model's weights are)
+    # E2E_INFLIGHT consecutive steps overlap (one step's downloads with the
+    # next one's uploads), each on its own stream with its own device buffers
+    # and host output, as a serving loop over a stream of batches runs
     host = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory() for k in names}
-    y_host = torch.empty(Bt, H, L, dtype=torch.float32).pin_memory()
-    dsets = sets[0]
-    for k in names:
-        if k != "u":
-            dsets[k].copy_(host[k])
+    esets = [sets[i % nsets] for i in range(E2E_INFLIGHT)]
+    y_hosts = [torch.empty(Bt, H, L, dtype=torch.float32).pin_memory() for _ in esets]
+    e2e_streams = [torch.cuda.Stream() for _ in esets]
+    for ds in esets:
+        for k in names:
+            if k != "u":
+                ds[k].copy_(host[k])
     h2d = host["u"].numel() * 4
-    d2h = y_host.numel() * 4
+    d2h = y_hosts[0].numel() * 4
 
-    def e2e_step():
-        if s4d:
-            K = s4.s4d_kernel_vandermonde(dsets["A"], dsets["B"], dsets["C"], dsets["log_dt"], L, out=dsets["K"])
-            s4.fft_conv_host(host["u"], K, dsets["D"], y_host=y_host, u_dev=dsets["u"], y_dev=dsets["y"],
-                             workspace=dsets["ws"], chunks=E2E_CHUNKS)
-        else:
-            s4.forward_dplr_host(host["u"], dsets["Lambda"], dsets["P"], dsets["Q"], dsets["B"], dsets["C"],
-                                 dsets["log_dt"], dsets["D"], y_host=y_host, K=dsets["K"], u_dev=dsets["u"],
-                                 y_dev=dsets["y"], workspace=dsets["ws"], chunks=E2E_CHUNKS)
+    def e2e_step(i):
+        ds, y_host = esets[i % E2E_INFLIGHT], y_hosts[i % E2E_INFLIGHT]
+        with torch.cuda.stream(e2e_streams[i % E2E_INFLIGHT]):
+            if s4d:
+                K = s4.s4d_kernel_vandermonde(ds["A"], ds["B"], ds["C"], ds["log_dt"], L, out=ds["K"])
+                s4.fft_conv_host(host["u"], K, ds["D"], y_host=y_host, u_dev=ds["u"], y_dev=ds["y"],
+                                 workspace=ds["ws"], chunks=E2E_CHUNKS)
+            else:
+                s4.forward_dplr_host(host["u"], ds["Lambda"], ds["P"], ds["Q"], ds["B"], ds["C"],
+                                     ds["log_dt"], ds["D"], y_host=y_host, K=ds["K"], u_dev=ds["u"],
+                                     y_dev=ds["y"], workspace=ds["ws"], chunks=E2E_CHUNKS)
+
+    def e2e_steps(n):
+        cur = torch.cuda.current_stream()
+        for st in e2e_streams:
+            st.wait_stream(cur)
+        for i in range(n):
+            e2e_step(i)
+        for st in e2e_streams:
+            cur.wait_stream(st)
 
     e2e_ms = float("nan")
     if not args.no_e2e:
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+        e2e_steps(max(E2E_INFLIGHT, args.warmup))
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if dist is not None:
             dist.barrier()
         e0.record()
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_steps(args.steps)
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
@@ -689,7 +704,7 @@ def run_gpu(args, rank, world, local_rank):
         dist.destroy_process_group()
     ms, e2e_ms = times[0], times[1]
     rec["ms"], rec["stage"] = ms, times[2:]
-    del sets, dsets, d, rec["sets"]
+    del sets, esets, d, rec["sets"]
     torch.cuda.empty_cache()
     if rank != 0:
         return None
@@ -725,8 +740,9 @@ def run_gpu(args, rank, world, local_rank):
                                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                                          "call": ("s4d_kernel_vandermonde + s4_fft_conv_host" if s4d
                                                   else "s4_forward_dplr_host")
-                                         + f", pinned host u/y, {E2E_CHUNKS} row-pair chunks; the layer's "
-                                           "parameters resident on the device"},
+                                         + f", pinned host u/y, {E2E_CHUNKS} row-pair chunks, "
+                                           f"{E2E_INFLIGHT} steps in flight (own stream, device buffers and host "
+                                           "output each); the layer's parameters resident on the device"},
         "gpu_launches": rec["launches"] * args.steps,
         "gpu_launches_source": "kernel nodes of the captured generation and convolution graphs, x steps",
         "decode": decode,

@@ -284,9 +284,17 @@ s4_status s4_forward_dplr(const float *u, const s4_c32 *Lambda, const s4_c32 *P,
  *                    the workspace or the parameters); what they hold on
  *                    return is staging data in the chunks' own order, not a
  *                    copy of u or y.
- *   nchunks        : >= 1 (clamped to the number of row pairs).
+ *   nchunks        : >= 1 (clamped to the number of row pairs). Every
+ *                    copy has a fixed cost on the PCIe link, so a few large
+ *                    chunks beat many small ones: on a B200 at
+ *                    Bt*H*L = 2^25 floats, 2 to 4 chunks ran fastest and 32
+ *                    or more cost 20 to 45 % more per call.
  *   h2d_stream, d2h_stream : caller-owned streams (may be `stream` itself,
  *                    which serialises the pipeline).
+ * Calls on different `stream`s, each with its own staging buffers,
+ * workspace and K, may be in flight together: with shared copy streams one
+ * call's downloads then overlap the next call's uploads, which removes the
+ * pipeline's fill and drain from all but the first and last call.
  * The first call on each (host thread, device) creates the few CUDA events
  * the pipeline orders itself with, and later calls from that thread reuse
  * them (they live until the process exits); no call allocates memory.

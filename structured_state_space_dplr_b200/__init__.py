@@ -422,7 +422,7 @@ def _host_call_buffers(u_host, y_host, u_dev, y_dev, dev):
 
 
 def forward_dplr_host(u_host, Lambda, P, Q, B, C, log_dt, D, *, y_host=None, K=None, u_dev=None, y_dev=None,
-                      workspace=None, flags=None, chunks=8):
+                      workspace=None, flags=None, chunks=4):
     """forward_dplr with u and y in host memory (s4_forward_dplr_host): the
     uploads, convolutions and downloads of `chunks` row-pair chunks overlap.
     u_host: float32 CPU tensor [Bt, H, L] (pinned memory for overlap).
@@ -443,7 +443,7 @@ def forward_dplr_host(u_host, Lambda, P, Q, B, C, log_dt, D, *, y_host=None, K=N
     return y_host
 
 
-def fft_conv_host(u_host, K, D, *, y_host=None, u_dev=None, y_dev=None, workspace=None, chunks=8):
+def fft_conv_host(u_host, K, D, *, y_host=None, u_dev=None, y_dev=None, workspace=None, chunks=4):
     """fft_conv with u and y in host memory (s4_fft_conv_host); K, D on the
     device. Returns y_host, complete once torch's current stream is
     synchronised."""

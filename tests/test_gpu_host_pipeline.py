@@ -57,3 +57,41 @@ def test_channel_sliced_chunks_equal_device_path(Bt, H, L, chunks):
     y_host = s4.fft_conv_host(torch.from_numpy(u).pin_memory(), K, D, chunks=chunks)
     torch.cuda.current_stream().synchronize()
     assert torch.equal(y_host, y_dev.cpu())
+
+
+def test_calls_in_flight_on_separate_streams_keep_their_results():
+    """Three host-buffer calls with different parameters and inputs, each on
+    its own stream with its own staging buffers, workspace, K and host
+    output, queued back to back so that they overlap on the shared copy
+    streams; the six steps rotate through the three buffer sets (a set is
+    reused once its stream has finished the previous call). Every host
+    output equals its own device-path result."""
+    import structured_state_space_dplr_b200 as s4
+    torch = torch_cuda()
+    H, L, Bt = 8, 4096, 6
+    cases = []
+    for seed in range(3):
+        inp = s4inputs.make_inputs(2, seed=seed, H=H, Bt=Bt, L=L)
+        t = to_dev(inp)
+        y_ref = s4.forward_dplr(t["u"], t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], t["D"]).cpu()
+        cases.append({"t": t, "u_host": torch.from_numpy(inp["u"].copy()).pin_memory(), "y_ref": y_ref,
+                      "y_host": torch.empty(Bt, H, L).pin_memory(), "u_dev": torch.empty(Bt, H, L, device="cuda"),
+                      "y_dev": torch.empty(Bt, H, L, device="cuda"), "K": torch.empty(H, L, device="cuda"),
+                      "ws": torch.empty(s4.fft_conv_workspace_size(H, L), dtype=torch.uint8, device="cuda"),
+                      "stream": torch.cuda.Stream()})
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    for c in cases:
+        c["stream"].wait_stream(cur)
+    for step in range(6):
+        c = cases[step % 3]
+        t = c["t"]
+        with torch.cuda.stream(c["stream"]):
+            s4.forward_dplr_host(c["u_host"], t["Lambda"], t["P"], t["Q"], t["B"], t["C"], t["log_dt"], t["D"],
+                                 y_host=c["y_host"], K=c["K"], u_dev=c["u_dev"], y_dev=c["y_dev"],
+                                 workspace=c["ws"], chunks=2)
+    for c in cases:
+        cur.wait_stream(c["stream"])
+    torch.cuda.synchronize()
+    for c in cases:
+        assert torch.equal(c["y_host"], c["y_ref"])
