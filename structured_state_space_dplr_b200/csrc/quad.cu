@@ -19,6 +19,11 @@ namespace cg = cooperative_groups;
 
 namespace s4 {
 
+// a hint that brings the line holding p into L2 (no registers, no completion)
+__device__ __forceinline__ void l2_prefetch(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(p)));
+}
+
 // ------------------------------------------------ fftconv, cluster of two --
 // L = 16384: the zero-padded length-N = 2L transform split four ways, rank c
 // holding the frequencies 4f + c (m = N/4 = 8192 points each). With the
@@ -97,6 +102,15 @@ k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int
     bool first = true;
     for (long long pr = cl; pr < npairs; pr += ncl) {
         const RowPair r = row_pair(pr, Bt);
+        // the cluster's next row pair into L2 (CTA cr takes row cr, a 128-byte
+        // line per thread), so its loads a pair from now hit L2 rather than
+        // HBM: 251.8 -> 239.6 us at H = 256, batch 8. Two or three pairs ahead
+        // was slower (247.9, 259.0 us), and so was also prefetching the next
+        // channel's spectrum (245.7 us).
+        if (pr + ncl < npairs) {
+            const RowPair rn = row_pair(pr + ncl, Bt);
+            if (cr == 0 || rn.has1) l2_prefetch(u + ((size_t)(rn.b0 + cr) * H + rn.h) * L + (size_t)j * 32);
+        }
         load_inputs(pr);
         {
             float2 v0[R0], v1[R0];
