@@ -66,7 +66,7 @@ BLOCK_PROJ_BYTES_PER_ELEM = 12
 # cluster split), hashed to tell whether a recorded ncu figure still holds
 _CONV_COMMON = ["common.cuh", "fft.cuh", "pairs.cuh", "cluster.cuh"]
 KERNEL_SOURCES = {1: _CONV_COMMON + ["spectral.cu"], 2: _CONV_COMMON + ["spectral.cu"],
-                  3: _CONV_COMMON + ["quad.cu"], 4: _CONV_COMMON + ["spectral.cu"],
+                  3: _CONV_COMMON + ["quad.cuh", "quad.cu"], 4: _CONV_COMMON + ["spectral.cu"],
                   5: _CONV_COMMON + ["spectral.cu"]}
 # DRAM traffic of one convolution launch per workload, from committed ncu
 # summaries (reported only while the convolution's sources are unchanged)
@@ -255,7 +255,7 @@ def launches_per_step(c):
     elif L <= 8192:
         gen = 1                               # k_kgen (Cauchy, inverse, spectrum)
     elif L == 16384:
-        gen = 2                               # k_cauchy, k_kspec_quad_half
+        gen = 2                               # k_cauchy, k_kspec_quad_pair
     else:
         gen = 3                               # k_cauchy, k_irfft, k_kspec_cl
     return gen + 1

@@ -20,8 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libs4dplr.so")
-SOURCES = ["api.cu", "cauchy.cu", "kgen.cu", "spectral.cu", "quad.cu", "s4d.cu", "decode.cu", "noalloc.cu", "backward.cu", "block.cu", "zoh_dplr.cu"]
-HEADERS = ["common.cuh", "fft.cuh", "cauchy.cuh", "pairs.cuh", "cluster.cuh", "launch.h", "umma.cuh"]
+SOURCES = ["api.cu", "cauchy.cu", "kgen.cu", "spectral.cu", "quad.cu", "quad_spec.cu", "s4d.cu", "decode.cu", "noalloc.cu", "backward.cu", "block.cu", "zoh_dplr.cu"]
+HEADERS = ["common.cuh", "fft.cuh", "cauchy.cuh", "pairs.cuh", "cluster.cuh", "quad.cuh", "launch.h", "umma.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

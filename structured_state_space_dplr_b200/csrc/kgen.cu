@@ -10,7 +10,7 @@
 //      its spectrum, plus D and times 1/2L, goes to the convolution workspace
 //      in the layout k_fftconv_pair reads.
 // Longer kernels take k_cauchy, then (L = 16384) the inverse transform fused
-// with the spectrum in k_kspec_quad_half, or (L >= 32768) k_irfft + k_kspec.
+// with the spectrum in k_kspec_quad_pair, or (L >= 32768) k_irfft + k_kspec.
 #include "launch.h"
 #include "pairs.cuh"
 
