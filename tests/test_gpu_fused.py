@@ -32,14 +32,33 @@ def _fused(inp):
 @pytest.mark.parametrize("L", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536])
 def test_random_dplr_all_outputs(L):
     """Every output, odd H and batch; L = 16384 takes the inverse transform
-    fused into the spectrum kernel (one cluster per channel, K stored in
-    place of the half spectrum), longer L the separate inverse transform."""
+    fused into the spectrum kernel (one cluster per channel pair, K stored in
+    place of the half spectra; with H = 3 the last cluster has one channel),
+    longer L the separate inverse transform."""
     inp = s4inputs.random_dplr(500 + L, H=3, Nh=6, L=L, Bt=3)
     K, y, K3, y3 = _fused(inp)
     Kr = workloads.dplr_kernel(inp)
     yr = workloads.conv_full(inp, Kr)
     assert kernel_err(K, Kr) <= K_TOL
     assert rel_l2(y, yr) <= Y_TOL
+    assert kernel_err(K, K3) <= K_TOL
+    assert rel_l2(y, y3) <= Y_TOL
+
+
+@pytest.mark.parametrize("H", [1, 2, 5])
+def test_l16384_channel_pairs_all_outputs(H):
+    """L = 16384 inverts and transforms two channels at once and separates
+    their spectra by conjugate symmetry: one channel alone (H = 1), one full
+    pair, and two pairs plus a lone channel, each with its own D; every
+    output of K and y against the oracle."""
+    inp = s4inputs.random_dplr(900 + H, H=H, Nh=8, L=16384, Bt=2)
+    K, y, K3, y3 = _fused(inp)
+    Kr = workloads.dplr_kernel(inp)
+    yr = workloads.conv_full(inp, Kr)
+    assert kernel_err(K, Kr) <= K_TOL
+    assert rel_l2(y, yr) <= Y_TOL
+    for h in range(H):
+        assert rel_l2(y[:, h], yr[:, h]) <= 4 * Y_TOL
     assert kernel_err(K, K3) <= K_TOL
     assert rel_l2(y, y3) <= Y_TOL
 
