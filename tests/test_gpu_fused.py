@@ -45,13 +45,16 @@ def test_random_dplr_all_outputs(L):
     assert rel_l2(y, y3) <= Y_TOL
 
 
-@pytest.mark.parametrize("H", [1, 2, 5])
-def test_l16384_channel_pairs_all_outputs(H):
-    """L = 16384 inverts and transforms two channels at once and separates
-    their spectra by conjugate symmetry: one channel alone (H = 1), one full
-    pair, and two pairs plus a lone channel, each with its own D; every
-    output of K and y against the oracle."""
-    inp = s4inputs.random_dplr(900 + H, H=H, Nh=8, L=16384, Bt=2)
+@pytest.mark.parametrize("L,H", [(16384, 1), (16384, 2), (16384, 5), (32768, 1), (32768, 4), (65536, 2)])
+def test_channel_pairs_all_outputs(L, H):
+    """Channel counts around the pairing of the generation kernels: at
+    L = 16384 two channels are inverted and transformed at once and their
+    spectra come apart by conjugate symmetry; at L >= 32768 the inverse
+    transform packs channel pairs and the spectrum takes one channel per
+    cluster. One channel alone, full pairs, and pairs plus a lone channel,
+    each channel with its own D; every output of K and y against the
+    oracle."""
+    inp = s4inputs.random_dplr(900 + H + L, H=H, Nh=8, L=L, Bt=2)
     K, y, K3, y3 = _fused(inp)
     Kr = workloads.dplr_kernel(inp)
     yr = workloads.conv_full(inp, Kr)
