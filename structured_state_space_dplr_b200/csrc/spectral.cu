@@ -305,10 +305,17 @@ __device__ __forceinline__ float2 half_spec(const float *Kh, int f, int L) {
     return cconj(reinterpret_cast<const float2 *>(Kh)[L - f]);
 }
 
+// Split 8 ways or more, two 256-thread CTAs share an SM, so twice the
+// clusters are resident: at L = 65536 (H = 64) all 32 channel pairs run at
+// once on 37 clusters of 8 instead of two rounds on 18, 65 -> 47 us.
 template <int LG, int C>
-__global__ void __launch_bounds__(threads_for<LG>())
+__host__ __device__ constexpr int irfft_threads() { return C >= 8 ? 256 : threads_for<LG>(); }
+template <int C>
+__host__ __device__ constexpr int irfft_min_blocks() { return C >= 8 ? 2 : 1; }
+template <int LG, int C>
+__global__ void __launch_bounds__(irfft_threads<LG, C>(), irfft_min_blocks<C>())
 k_irfft(float *K, int H, int L) {
-    constexpr int m = 1 << LG, T = threads_for<LG>(), P = plan_P(LG);
+    constexpr int m = 1 << LG, T = irfft_threads<LG, C>(), P = plan_P(LG);
     constexpr int SL = m / C;
     extern __shared__ float2 sm[];
     const Smem s = carve<LG>(sm);
@@ -452,7 +459,7 @@ template <int LG, int C> LaunchInfo ConvKernels<LG, C>::info_pair[2];
 // ---- irfft instantiation ----
 template <int LG, int C>
 struct IrfftKernels {
-    static constexpr int T = threads_for<LG>();
+    static constexpr int T = irfft_threads<LG, C>();
     static constexpr size_t smem = sizeof(float2) * (size_t)smem_f2<LG>();
     static LaunchInfo info;
     static cudaError_t run(float *K, int H, int L, cudaStream_t st) {
