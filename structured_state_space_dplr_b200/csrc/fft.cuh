@@ -505,4 +505,62 @@ __device__ __forceinline__ void fused_middle_x2(float2 *b0, float2 *b1, Fetch &&
     }
 }
 
+// ------------------------------------------- warp-level middle barriers --
+// With a single middle pass of radix R1, that pass hands each block of
+// B1 = m / R0 points to S1 = B1 / R1 consecutive threads. When the fused pass
+// (last forward pass, product, first inverse pass) takes a block's groups
+// with the same threads, nothing written in one of these three passes is read
+// by another warp in the next, and the barriers between them are __syncwarp.
+// Two layouts qualify (R0 = RL = 16, one middle-pass item per thread):
+//   16 x 16 x 16, two buffers, T = m / 16: thread g runs group g of both
+//     buffers in every pass (fused_middle_x2 already does), S1 = 16;
+//   16 x 32 x 16, T = m / 16 on two buffers (thread i: buffer i / (m/32)) or
+//     T = m / 32 on one: the radix-32 pass gives thread t the block
+//     (t % (m/32)) / 16 of its buffer, and fused_blocks(_x2) give it that
+//     block's 16-point groups (t % 16) and (t % 16) + 16.
+template <int LG, int T, int NBUF>
+__host__ __device__ constexpr bool warp_local_middle() {
+    return plan_P(LG) == 3 && plan_lr(LG, 0) == 4 && plan_lr(LG, 2) == 4 &&
+           ((plan_lr(LG, 1) == 4 && NBUF == 2 && T == (1 << LG) / 16) ||
+            (plan_lr(LG, 1) == 5 && T == NBUF * ((1 << LG) / 32)));
+}
+
+// the fused pass of the 16 x 32 x 16 plan, one buffer or two, spectrum words
+// in spec4_index order from kp (buffer b0 / the single buffer) and kq (b1)
+template <int LG, int NBUF, bool CONJ>
+__device__ __forceinline__ void fused_blocks(float2 *b0, float2 *b1, const float4 *__restrict__ kp,
+                                             const float4 *__restrict__ kq) {
+    constexpr int R = 16, GM = (1 << LG) / 32;   // radix-32 groups per buffer
+    static_assert(plan_lr(LG, 1) == 5 && plan_lr(LG, 2) == 4, "the 16 x 32 x 16 plan");
+    const int i = threadIdx.x;
+    const bool second = NBUF == 2 && i >= GM;
+    float2 *b = second ? b1 : b0;
+    const float4 *k = second ? kq : kp;
+    const int t = i % GM;
+    const int g0 = (t >> 4) * 32 + (t & 15), g1 = g0 + 16;
+    float4 w0[R / 2], w1[R / 2];
+    static_for<0, R / 2>([&](auto ii) {
+        w0[ii] = __ldg(k + spec4_index<LG>(g0 * R, ii));
+        w1[ii] = __ldg(k + spec4_index<LG>(g1 * R, ii));
+    });
+    float2 x[R], z[R];
+    load_contig<R>(b + pidx(g0 * R), x);
+    load_contig<R>(b + pidx(g1 * R), z);
+    dft<R, -1>(x);
+    dft<R, -1>(z);
+    auto mul = [](float2 a, float x0, float x1) {
+        if constexpr (CONJ) return cmulc(a, make_float2(x0, x1)); else return cmul(a, make_float2(x0, x1));
+    };
+    static_for<0, R / 2>([&](auto ii) {
+        x[2 * ii] = mul(x[2 * ii], w0[ii].x, w0[ii].y);
+        x[2 * ii + 1] = mul(x[2 * ii + 1], w0[ii].z, w0[ii].w);
+        z[2 * ii] = mul(z[2 * ii], w1[ii].x, w1[ii].y);
+        z[2 * ii + 1] = mul(z[2 * ii + 1], w1[ii].z, w1[ii].w);
+    });
+    dft<R, +1>(x);
+    dft<R, +1>(z);
+    store_contig<R>(b + pidx(g0 * R), x);
+    store_contig<R>(b + pidx(g1 * R), z);
+}
+
 }  // namespace s4

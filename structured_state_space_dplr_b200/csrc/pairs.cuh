@@ -263,19 +263,19 @@ __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__res
     }
     __syncthreads();
     after_first();
-    forward_middle_x2<LG, T>(b0, b1, s.tws);
     const float4 *s0 = reinterpret_cast<const float4 *>(spec_h);
     const float4 *s1 = s0 + m / 2;
     constexpr int RL = 1 << plan_lr(LG, plan_P(LG) - 1);
     struct SpecWords { float4 k0[RL / 2], k1[RL / 2]; };
-    fused_middle_x2<LG, T>(b0, b1, [&](int base) {
+    auto fetch = [&](int base) {
         SpecWords w;
         static_for<0, RL / 2>([&](auto i) {
             w.k0[i] = __ldg(s0 + spec4_index<LG>(base, i));
             w.k1[i] = __ldg(s1 + spec4_index<LG>(base, i));
         });
         return w;
-    }, [&](const SpecWords &w, auto &x, auto &z) {
+    };
+    auto product = [&](const SpecWords &w, auto &x, auto &z) {
         auto mul = [](float2 a, float x0, float x1) {
             if constexpr (CONJ) return cmulc(a, make_float2(x0, x1)); else return cmul(a, make_float2(x0, x1));
         };
@@ -285,9 +285,21 @@ __device__ __forceinline__ void conv_pair(const PairSmem &s, const float2 *__res
             z[2 * i] = mul(z[2 * i], w.k1[i].x, w.k1[i].y);
             z[2 * i + 1] = mul(z[2 * i + 1], w.k1[i].z, w.k1[i].w);
         });
-    });
-    __syncthreads();
-    inverse_middle_x2<LG, T>(b0, b1, s.tws);
+    };
+    if constexpr (warp_local_middle<LG, T, 2>()) {   // barriers between the middle passes per warp
+        pass_x2<LG, 1, -1, false, T>(b0, b1, s.tws);
+        __syncwarp();
+        if constexpr (plan_lr(LG, 1) == 5) fused_blocks<LG, 2, CONJ>(b0, b1, s0, s1);
+        else fused_middle_x2<LG, T>(b0, b1, fetch, product);
+        __syncwarp();
+        pass_x2<LG, 1, +1, true, T>(b0, b1, s.tws);
+        __syncthreads();
+    } else {
+        forward_middle_x2<LG, T>(b0, b1, s.tws);
+        fused_middle_x2<LG, T>(b0, b1, fetch, product);
+        __syncthreads();
+        inverse_middle_x2<LG, T>(b0, b1, s.tws);
+    }
     // ---- last inverse pass of both halves + their sum, straight to y
     last_pass_halves_sum<LG>(s, [&](auto, int t, float2 r, float2) {
         y0[t] = r.x;

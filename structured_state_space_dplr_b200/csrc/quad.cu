@@ -73,31 +73,16 @@ k_fftconv_quad(const float *__restrict__ u, const float2 *__restrict__ spec, int
             else first_pass_halves2<LG, true>(s, v0, v1, j, tcj);
         }
         __syncthreads();
-        forward_middle_x2<LG, T>(s.b0, s.b1, s.tws);
+        // the middle passes with warp-level barriers (warp_local_middle, fft.cuh)
+        static_assert(warp_local_middle<LG, T, 2>(), "the 16 x 32 x 16 plan on 512 threads");
         const float2 *sh = spec + (size_t)r.h * 2 * L;
-        const float4 *k0p = reinterpret_cast<const float4 *>(sh + (size_t)cr * m);
-        const float4 *k1p = reinterpret_cast<const float4 *>(sh + (size_t)(cr + 2) * m);
-        struct SpecWords { float4 k0[RL / 2], k1[RL / 2]; };
-        fused_middle_x2<LG, T>(s.b0, s.b1, [&](int base) {
-            SpecWords w;
-            static_for<0, RL / 2>([&](auto i) {
-                w.k0[i] = __ldg(k0p + spec4_index<LG>(base, i));
-                w.k1[i] = __ldg(k1p + spec4_index<LG>(base, i));
-            });
-            return w;
-        }, [&](const SpecWords &w, auto &x, auto &z) {
-            auto mul = [](float2 a, float x0, float x1) {
-                if constexpr (CONJ) return cmulc(a, make_float2(x0, x1)); else return cmul(a, make_float2(x0, x1));
-            };
-            static_for<0, RL / 2>([&](auto i) {
-                x[2 * i] = mul(x[2 * i], w.k0[i].x, w.k0[i].y);
-                x[2 * i + 1] = mul(x[2 * i + 1], w.k0[i].z, w.k0[i].w);
-                z[2 * i] = mul(z[2 * i], w.k1[i].x, w.k1[i].y);
-                z[2 * i + 1] = mul(z[2 * i + 1], w.k1[i].z, w.k1[i].w);
-            });
-        });
+        pass_x2<LG, 1, -1, false, T>(s.b0, s.b1, s.tws);
+        __syncwarp();
+        fused_blocks<LG, 2, CONJ>(s.b0, s.b1, reinterpret_cast<const float4 *>(sh + (size_t)cr * m),
+                                  reinterpret_cast<const float4 *>(sh + (size_t)(cr + 2) * m));
+        __syncwarp();
+        pass_x2<LG, 1, +1, true, T>(s.b0, s.b1, s.tws);
         __syncthreads();
-        inverse_middle_x2<LG, T>(s.b0, s.b1, s.tws);
         // ---- last pass: keep one of (S, M) in registers, store the other
         // into the partner's receive buffer (once the partner has read the
         // previous pair's hand-over from it)

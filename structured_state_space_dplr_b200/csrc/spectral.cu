@@ -204,8 +204,16 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
             store_first_group<LG>(s.buf, x, j);
         }
         __syncthreads();
-        forward_middle<LG, T>(s.buf, s.tws);
         const float4 *sp = reinterpret_cast<const float4 *>(spec + ((size_t)h * C + c) * m);
+        if constexpr (warp_local_middle<LG, T, 1>()) {   // barriers between the middle passes per warp
+            dif_pass<LG, 1, -1, T>(s.buf, s.tws);
+            __syncwarp();
+            fused_blocks<LG, 1, CONJ>(s.buf, nullptr, sp, nullptr);
+            __syncwarp();
+            dit_pass<LG, 1, +1, T>(s.buf, s.tws);
+            __syncthreads();
+        } else {
+        forward_middle<LG, T>(s.buf, s.tws);
         fused_middle<LG, T>(s.buf, [&](int base, auto &x) {
             constexpr int R = sizeof(x) / sizeof(float2);
             static_for<0, R / 2>([&](auto i) {
@@ -221,6 +229,7 @@ k_fftconv(const float *__restrict__ u, const float2 *__restrict__ spec, int Bt, 
         });
         __syncthreads();
         inverse_middle<LG, T>(s.buf, s.tws);
+        }
         inverse_last_rec<LG, T>(s.buf, s.ta, s.tb, s.pre);
         cluster_arrive_release();
         cluster_wait();
