@@ -72,12 +72,6 @@ k_kspec_quad(const float *__restrict__ K, const float *__restrict__ Ki, const fl
 // the same CTA (0 and 2 in CTA 0, 1 and 3 in CTA 1), and the position of
 // m - 1 - f' is m - 1 - p (the digit reversal permutes bits), so only rank 0
 // looks its partners up by frequency.
-__device__ __forceinline__ float2 half_spec_l2(const float *Kh, int f, int L) {
-    if (f == 0) return make_float2(__ldcg(Kh), 0.0f);
-    if (f == L / 2) return make_float2(__ldcg(Kh + 1), 0.0f);
-    if (f < L / 2) return __ldcg(reinterpret_cast<const float2 *>(Kh) + f);
-    return cconj(__ldcg(reinterpret_cast<const float2 *>(Kh) + (L - f)));
-}
 
 __global__ void __launch_bounds__(pair_threads<kQuadLG>(), 1)
 k_kspec_quad_pair(float *__restrict__ K, const float *__restrict__ D, int H, float2 *__restrict__ spec) {
@@ -104,12 +98,38 @@ k_kspec_quad_pair(float *__restrict__ K, const float *__restrict__ D, int H, flo
         const bool hasb = ha + 1 < H;
         float *Ka = K + (size_t)ha * L;
         float *Kb = hasb ? Ka + L : Ka;   // channel ha + 1 (read and written only if hasb)
-        // ---- Y[2k' + cr] at the digit-reversed position of k'
-        for (int kk = j; kk < m; kk += T) {
-            const int f = 2 * kk + cr;
-            const float2 a = half_spec_l2(Ka, f, L);
-            const float2 b = hasb ? half_spec_l2(Kb, f, L) : make_float2(0.0f, 0.0f);
-            s.b0[pidx(digrev_inv<LG>(kk))] = make_float2(a.x - b.y, a.y + b.x);
+        // ---- Y[2k' + cr] at the digit-reversed position of k', k' = j + q T:
+        // all loads first (one L2 latency instead of one per k'), without
+        // branches: f < L/2 for q < NQ/2 (X[f]; f = 0 holds X_0 and X_{L/2}
+        // as the word (K[0], K[1])), f > L/2 beyond (conj X[L - f]; f = L/2
+        // reads that first word too)
+        {
+            constexpr int NQ = m / T;
+            const float2 *Xa = reinterpret_cast<const float2 *>(Ka);
+            const float2 *Xb = reinterpret_cast<const float2 *>(Kb);
+            float2 va[NQ], vb[NQ];
+            static_for<0, NQ>([&](auto qc) {
+                constexpr int q = decltype(qc)::value;
+                const int f = 2 * (j + q * T) + cr;
+                const int w = q < NQ / 2 ? f : (f == L / 2 ? 0 : L - f);
+                va[q] = __ldcg(Xa + w);
+                vb[q] = hasb ? __ldcg(Xb + w) : make_float2(0.0f, 0.0f);
+            });
+            static_for<0, NQ>([&](auto qc) {
+                constexpr int q = decltype(qc)::value;
+                const int kk = j + q * T, f = 2 * kk + cr;
+                float2 a = va[q], b = vb[q];
+                if constexpr (q < NQ / 2) {
+                    if (f == 0) { a.y = 0.0f; b.y = 0.0f; }
+                } else if (f == L / 2) {
+                    a = make_float2(a.y, 0.0f);
+                    b = make_float2(b.y, 0.0f);
+                } else {
+                    a = cconj(a);
+                    b = cconj(b);
+                }
+                s.b0[pidx(digrev_inv<LG>(kk))] = make_float2(a.x - b.y, a.y + b.x);
+            });
         }
         __syncthreads();
         // ---- the length-m inverse: passes P-1 .. 1, then the first pass in registers

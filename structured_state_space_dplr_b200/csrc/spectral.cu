@@ -354,11 +354,40 @@ k_irfft(float *K, int H, int L) {
             // (a strided gather of every C-th frequency fetches each 32-byte
             // sector once per CTA: 56.0 against 66.5 us at C = 8; at C = 2
             // the strided form is the faster, 29.6 against 35.5 us)
+            // Loads go out NB at a time before their stores (one L2 latency per
+            // batch), without branches: f < L/2 reads X[f] (f = 0: the word
+            // (K[0], K[1]) holding X_0 and X_{L/2}), f > L/2 conj X[L - f],
+            // f = L/2 that first word again.
             cg::cluster_group cluster = cg::this_cluster();
-            for (int i = threadIdx.x; i < m; i += T) {
-                const int f = c * m + i;
-                const int r = f % C, fr = f / C;
-                cluster.map_shared_rank(s.buf, r)[pidx(digrev_inv<LG>(fr))] = value(f);
+            constexpr int NB = 8;
+            static_assert(m % (T * NB) == 0, "whole batches");
+            const float2 *X1 = reinterpret_cast<const float2 *>(K1);
+            const float2 *X2 = reinterpret_cast<const float2 *>(K2);
+            for (int i0 = threadIdx.x; i0 < m; i0 += T * NB) {
+                float2 va[NB], vb[NB];
+                static_for<0, NB>([&](auto e) {
+                    const int f = c * m + i0 + decltype(e)::value * T;
+                    const int w = f < L / 2 ? f : (f == L / 2 ? 0 : L - f);
+                    va[e] = __ldcg(X1 + w);
+                    vb[e] = has2 ? __ldcg(X2 + w) : make_float2(0.0f, 0.0f);
+                });
+                static_for<0, NB>([&](auto e) {
+                    const int f = c * m + i0 + decltype(e)::value * T;
+                    float2 a = va[e], b = vb[e];
+                    if (f == 0) {
+                        a.y = 0.0f;
+                        b.y = 0.0f;
+                    } else if (f == L / 2) {
+                        a = make_float2(a.y, 0.0f);
+                        b = make_float2(b.y, 0.0f);
+                    } else if (f > L / 2) {
+                        a = cconj(a);
+                        b = cconj(b);
+                    }
+                    const int r = f % C, fr = f / C;
+                    cluster.map_shared_rank(s.buf, r)[pidx(digrev_inv<LG>(fr))] =
+                        make_float2(a.x - b.y, a.y + b.x);
+                });
             }
             cluster.sync();
         } else {
