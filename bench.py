@@ -435,6 +435,53 @@ def forward_record(rec, steps, world, hbm, fp32_peak, sm_max_mhz, peak_src, with
     }
 
 
+def torch_fft_context(s4, torch, sets, nsets, c, steps, warmup, flags, lib_conv_us):
+    """Context beside the library's convolution (feeds no value of this line):
+    the same convolution as the pages write it, with torch.fft (cuFFT) on the
+    same device and rotating inputs, y = irfft(rfft(u, 2L) rfft(K, 2L))[:L] + D u,
+    timed with CUDA events -- once with rfft(K) precomputed (the library's
+    apply stage also starts from a stored spectrum) and once per call as the
+    pages' fft_conv does -- and its largest difference from the library's y."""
+    L, n = c["L"], 2 * c["L"]
+    s4d = c["kind"] == "s4d"
+    for s in sets:   # K as the forward produced it (the kernel-only timing left its own data there)
+        if s4d:
+            s4.s4d_kernel_vandermonde(s["A"], s["B"], s["C"], s["log_dt"], L, out=s["K"])
+        else:
+            s4.kernel_dplr_prepare(s["Lambda"], s["P"], s["Q"], s["B"], s["C"], s["log_dt"], s["D"], L,
+                                   K=s["K"], workspace=s["ws"], flags=flags)
+    kf = [torch.fft.rfft(s["K"], n=n) for s in sets]
+
+    def conv(i, with_kernel_fft):
+        s = sets[i % nsets]
+        k = torch.fft.rfft(s["K"], n=n) if with_kernel_fft else kf[i % nsets]
+        y = torch.fft.irfft(torch.fft.rfft(s["u"], n=n) * k, n=n)[..., :L]
+        return y + s["D"][:, None] * s["u"]
+
+    out = {}
+    for key, wk in (("torch_fft_conv_us", False), ("torch_fft_conv_with_kernel_fft_us", True)):
+        for i in range(warmup):
+            conv(i, wk)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            conv(i, wk)
+        e1.record()
+        torch.cuda.synchronize()
+        out[key] = e0.elapsed_time(e1) * 1e3 / steps
+    ref = conv(0, False)
+    s4.fft_conv_apply(sets[0]["u"], sets[0]["ws"], out=sets[0]["y"])
+    torch.cuda.synchronize()
+    out["max_abs_diff_over_max_abs_y"] = float((ref - sets[0]["y"]).abs().max() / sets[0]["y"].abs().max())
+    out["library_fft_conv_us"] = lib_conv_us
+    out["note"] = ("torch.fft (cuFFT) in fp32 on the same inputs; the library's convolution is "
+                   "s4_fft_conv_apply from the spectrum its generation stage stored")
+    del kf
+    torch.cuda.empty_cache()
+    return out
+
+
 def block_case(s4, torch, dev, sets, nsets, H, seed, steps, warmup, flags):
     """The S4Block around the layer: channel layer norm -> the layer's
     convolution (the prepared spectrum) -> GLU projection + residual, over the
@@ -621,6 +668,15 @@ def run_gpu(args, rank, world, local_rank):
     block = block_record(block_case(s4, torch, dev, sets, nsets, H, shard["seed"], args.steps, args.warmup, flags),
                          alg, H)
 
+    # ---- context: the same convolution through torch.fft (cuFFT)
+    torch_fft = None
+    if not args.headline_only:
+        try:
+            torch_fft = torch_fft_context(s4, torch, sets, nsets, c, args.steps, args.warmup, flags,
+                                          rec["stage"][1] * 1e3)
+        except Exception as exc:   # noqa: BLE001 - reported, the main line stands
+            torch_fft = {"error": f"{type(exc).__name__}: {exc}"}
+
     # ---- recurrent view (decode): up to 1024 tokens from a zero state, as
     # one s4_recurrent_scan and as single-token steps replayed from a graph
     d = sets[0]
@@ -749,6 +805,7 @@ def run_gpu(args, rank, world, local_rank):
         "variants": variants,
         "backward": backward,
         "block": block,
+        "torch_fft_context": torch_fft,
         "clocks": rec["clocks"],
     }
 
