@@ -86,11 +86,28 @@ CPU_BUDGET_S = 10.0
 
 # ----------------------------------------------------------------- helpers --
 def peaks():
+    """(HBM GB/s, SM MHz for the derived FP32 peak, source): the measured copy
+    bandwidth from MEASURED_PEAKS.json when the file has a usable one, else
+    the fallback figure, labelled as such."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+
+    def number(v):
+        if isinstance(v, dict):   # {"value": ...} style entries
+            v = v.get("value")
+        try:
+            v = float(v)
+        except (TypeError, ValueError):
+            return None
+        return v if v > 0 else None
+
+    try:
         with open(p) as f:
             d = json.load(f)
-        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), float(d.get("sm_max_mhz", NOMINAL_SM_MHZ)), "measured"
+    except (OSError, ValueError):
+        d = None
+    if isinstance(d, dict) and number(d.get("hbm_gbs")) is not None:
+        mhz = number(d.get("sm_max_mhz")) or NOMINAL_SM_MHZ
+        return number(d["hbm_gbs"]), mhz, "measured"
     return FALLBACK_HBM_GBS, NOMINAL_SM_MHZ, "fallback"
 
 

@@ -97,3 +97,21 @@ def test_algorithmic_units_of_the_workloads():
     assert a["kernel_flop"] == 40 * 256 * 2048 * 32
     a5 = bench.algorithmic(s4inputs.CONFIGS[5])
     assert a5["kernel_flop"] == 4 * 1024 * 8192 * 32
+
+
+def test_peak_file_is_read_or_falls_back(tmp_path, monkeypatch):
+    """The HBM peak comes from MEASURED_PEAKS.json when it holds a usable
+    copy bandwidth (plain or {"value": ...}), and falls back, labelled as
+    such, when the file is missing, malformed or lacks the figure."""
+    import json
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f = tmp_path / "MEASURED_PEAKS.json"
+    assert bench.peaks() == (bench.FALLBACK_HBM_GBS, bench.NOMINAL_SM_MHZ, "fallback")
+    f.write_text(json.dumps({"hbm_gbs": 6541.8, "bf16_tflops": 1643.0}))
+    assert bench.peaks() == (6541.8, bench.NOMINAL_SM_MHZ, "measured")
+    f.write_text(json.dumps({"hbm_gbs": {"value": 6000.0}, "sm_max_mhz": 1900}))
+    assert bench.peaks() == (6000.0, 1900.0, "measured")
+    for bad in ("not json", json.dumps({"bf16_tflops": 1643.0}), json.dumps({"hbm_gbs": "n/a"}), json.dumps([1, 2])):
+        f.write_text(bad)
+        assert bench.peaks()[2] == "fallback"
