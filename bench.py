@@ -499,52 +499,54 @@ def torch_fft_context(s4, torch, sets, nsets, c, steps, warmup, flags, lib_conv_
     return out
 
 
+def torch_dplr_kernel(torch, d, L, chunk=32):
+    """The DPLR kernel as the pages write it, with torch complex64 tensors (on
+    whatever device d's tensors are): at the roots of unity z_j (j < L/2),
+    g_j = (2/dt)(1 - z_j)/(1 + z_j); the four Cauchy sums over all N = 2 Nh
+    modes (the stored ones and their conjugates) of v / (g - lambda) for
+    v = C B, C P, conj(Q) B, conj(Q) P; K_hat = 2/(1 + z) (k00 - k01 k10 /
+    (1 + k11)); the Nyquist bin from its limit dt sum Re(C B); K =
+    irfft(K_hat, L). Channels in chunks of `chunk` to bound the
+    (chunk, L/2, N) intermediates."""
+    import math
+    lam, C, B, P, Q = (d[k] for k in ("Lambda", "C", "B", "P", "Q"))
+    H = lam.shape[0]
+    jj = torch.arange(L // 2, device=lam.device, dtype=torch.float32)
+    z = torch.polar(torch.ones_like(jj), -2.0 * math.pi * jj / L)
+    dt = torch.exp(d["log_dt"])
+    Ks = []
+    for h0 in range(0, H, chunk):
+        hs = slice(h0, min(H, h0 + chunk))
+        lm = torch.cat([lam[hs], lam[hs].conj()], dim=1)                       # [hc, N]
+        V = torch.stack([C[hs] * B[hs], C[hs] * P[hs], Q[hs].conj() * B[hs], Q[hs].conj() * P[hs]], 1)
+        V = torch.cat([V, V.conj()], dim=2)                                      # [hc, 4, N]
+        g = (2.0 / dt[hs])[:, None] * ((1 - z) / (1 + z))[None, :]              # [hc, L/2]
+        r = 1.0 / (g[:, :, None] - lm[:, None, :])                              # [hc, L/2, N]
+        k = torch.einsum("hjn,hvn->hvj", r, V)                                  # [hc, 4, L/2]
+        kh = (2.0 / (1 + z))[None, :] * (k[:, 0] - k[:, 1] * k[:, 2] / (1 + k[:, 3]))
+        nyq = dt[hs] * (C[hs] * B[hs]).real.sum(1)
+        kh = torch.cat([kh, nyq.to(kh.dtype)[:, None]], dim=1)                   # [hc, L/2 + 1]
+        Ks.append(torch.fft.irfft(kh, n=L))
+    return torch.cat(Ks, 0)
+
+
 def torch_generation_context(torch, d, c, steps, warmup, lib_gen_us, chunk=32):
     """Context beside the library's kernel generation (feeds no value of this
-    line): the DPLR kernel as the pages write it, with torch complex64
-    tensors on the same device. At the roots of unity z_j (j < L/2), g_j =
-    (2/dt)(1 - z_j)/(1 + z_j); the four Cauchy sums over all N = 2 Nh modes
-    (the stored ones and their conjugates) of v / (g - lambda) for v = C B,
-    C P, conj(Q) B, conj(Q) P; K_hat = 2/(1 + z) (k00 - k01 k10 / (1 + k11));
-    the Nyquist bin from its limit dt sum Re(C B); K = irfft(K_hat, L).
-    Channels in chunks of `chunk` to bound the (chunk, L/2, N) intermediates.
-    Returns the time per generation and K's largest difference from the
-    library's K (d["K"])."""
-    import math
-    L, H = c["L"], c["H"]
-    dev = d["K"].device
-    jj = torch.arange(L // 2, device=dev, dtype=torch.float32)
-    z = torch.polar(torch.ones_like(jj), -2.0 * math.pi * jj / L)
-    lam, C, B, P, Q = (d[k] for k in ("Lambda", "C", "B", "P", "Q"))
-    dt = torch.exp(d["log_dt"])
-
-    def generate():
-        Ks = []
-        for h0 in range(0, H, chunk):
-            hs = slice(h0, min(H, h0 + chunk))
-            lm = torch.cat([lam[hs], lam[hs].conj()], dim=1)                       # [hc, N]
-            V = torch.stack([C[hs] * B[hs], C[hs] * P[hs], Q[hs].conj() * B[hs], Q[hs].conj() * P[hs]], 1)
-            V = torch.cat([V, V.conj()], dim=2)                                      # [hc, 4, N]
-            g = (2.0 / dt[hs])[:, None] * ((1 - z) / (1 + z))[None, :]              # [hc, L/2]
-            r = 1.0 / (g[:, :, None] - lm[:, None, :])                              # [hc, L/2, N]
-            k = torch.einsum("hjn,hvn->hvj", r, V)                                  # [hc, 4, L/2]
-            kh = (2.0 / (1 + z))[None, :] * (k[:, 0] - k[:, 1] * k[:, 2] / (1 + k[:, 3]))
-            nyq = dt[hs] * (C[hs] * B[hs]).real.sum(1)
-            kh = torch.cat([kh, nyq.to(kh.dtype)[:, None]], dim=1)                   # [hc, L/2 + 1]
-            Ks.append(torch.fft.irfft(kh, n=L))
-        return torch.cat(Ks, 0)
-
+    line): torch_dplr_kernel on the same device and parameters, timed with
+    CUDA events, and K's largest per-channel difference from the library's K
+    (d["K"])."""
+    L = c["L"]
     for _ in range(warmup):
-        generate()
+        torch_dplr_kernel(torch, d, L, chunk)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
-        generate()
+        torch_dplr_kernel(torch, d, L, chunk)
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / steps
-    K = generate()
+    K = torch_dplr_kernel(torch, d, L, chunk)
     err = float(((K - d["K"]).abs().max(dim=1).values / d["K"].abs().max(dim=1).values).max())
     torch.cuda.empty_cache()
     return {"torch_generation_us": us, "library_generation_us": lib_gen_us,

@@ -115,3 +115,21 @@ def test_peak_file_is_read_or_falls_back(tmp_path, monkeypatch):
     for bad in ("not json", json.dumps({"bf16_tflops": 1643.0}), json.dumps({"hbm_gbs": "n/a"}), json.dumps([1, 2])):
         f.write_text(bad)
         assert bench.peaks()[2] == "fallback"
+
+
+def test_torch_formulation_of_the_kernel_matches_the_oracle():
+    """The bench's context timing of the pages' formulation (torch complex64
+    Cauchy sums, Woodbury, 2/(1+z), irfft) computes the kernel the oracle
+    does: on the CPU, at the small workload, every output within the
+    parity bound."""
+    import numpy as np
+    import torch
+    import bench
+    import s4inputs
+    from oracle import workloads
+    inp = s4inputs.make_inputs(1)
+    d = {k: torch.from_numpy(np.ascontiguousarray(inp[k])) for k in ("Lambda", "P", "Q", "B", "C", "log_dt")}
+    K = bench.torch_dplr_kernel(torch, d, inp["L"], chunk=3).numpy()
+    Kr = workloads.dplr_kernel(inp)
+    err = max(np.abs(K[h] - Kr[h]).max() / np.abs(Kr[h]).max() for h in range(inp["H"]))
+    assert err <= 1e-4, err
