@@ -159,3 +159,23 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(s4.S4Error) as e:
         s4.fft_conv(u, K, D, workspace=ws)
     assert e.value.status == 3
+
+
+@pytest.mark.parametrize("Bt,H,L", [(3, 100, 16384), (3, 200, 4096)])
+def test_more_row_pairs_than_resident_units_with_an_unpaired_row(Bt, H, L):
+    """Each persistent CTA (cluster at L = 16384) runs several row pairs, and
+    with an odd batch every other pair has no second row: at L = 16384 the
+    L2 prefetch of a following pair skips that row, at L = 4096 the staged
+    copy zero-fills it. Every output of rows from late pairs (paired and
+    unpaired) against the oracle's direct sum."""
+    rng = np.random.default_rng(1700 + L)
+    u = rng.standard_normal((Bt, H, L), dtype=np.float32)
+    K = (rng.standard_normal((H, L)) * np.exp(-np.arange(L) / (L / 4))).astype(np.float32)
+    D = rng.standard_normal(H).astype(np.float32)
+    yg = _conv(u, K, D)
+    rows = [(2, H - 1), (0, H - 1), (1, H - 1), (2, H // 2 + 1), (2, 3 * H // 4), (0, H // 2)]
+    ur = np.stack([u[b, h] for b, h in rows]).astype(np.float64)
+    yr = ssm.causal_conv_rows_at(ur, np.array([h for _, h in rows]), K.astype(np.float64), D.astype(np.float64),
+                                 np.arange(L))
+    for i, (b, h) in enumerate(rows):
+        assert rel_l2(yg[b, h], yr[i]) <= 4 * Y_TOL, (b, h)
