@@ -38,8 +38,9 @@ def test_random_kernel_full_outputs(L, Bt, H):
 @pytest.mark.parametrize("Bt,H", [(1, 1), (3, 2), (6, 3)])
 def test_cluster_of_two_full_outputs(Bt, H):
     """L = 16384 (the transform split four ways over a cluster of two CTAs):
-    every output, unpaired rows, several channels, and more row pairs than
-    one cluster takes in a single pass."""
+    every output, unpaired rows, several channels (at most nine row pairs,
+    one per cluster; the test of more row pairs than resident units below
+    gives each cluster several)."""
     L = 16384
     rng = np.random.default_rng(1600 + Bt)
     u = rng.standard_normal((Bt, H, L), dtype=np.float32)
